@@ -1,0 +1,188 @@
+/*
+ * salsc.h -- C ABI of the SALS latent-space sparse attention library (B200, sm_100a).
+ *
+ * The method is "SALS: Sparse Attention in Latent Space for KV cache
+ * Compression" (arXiv 2510.24273v1).  Its technical-framework section has four
+ * stages: (1) project keys and values into a low-dimensional latent space
+ * with a low-rank matrix, (2) select the important tokens in that space with
+ * a RoPE-free query-key interaction, (3) reconstruct only the selected
+ * tokens, (4) run standard attention on them; its abstract explains that
+ * RoPE can only be applied after reconstruction.  The attention formula
+ * softmax(Q K^T / sqrt(d)) is the one printed in the VL-Cache OpenReview
+ * response to reviewer KiPr, "On Weakness 1".
+ *
+ * Conventions for every entry point
+ *   - All tensors are row-major and contiguous; every data pointer is a CUDA
+ *     device pointer owned by the caller, unless its name ends in _host.
+ *   - Nothing allocates, frees or synchronises.  Work is enqueued on the
+ *     given stream (NULL = legacy default stream) and is asynchronous.  The
+ *     library keeps no state between calls; concurrent calls on different
+ *     workspaces are safe.
+ *   - Argument errors are reported synchronously by the return value before
+ *     anything is enqueued.  SALSC_ERR_CUDA means a launch failed; the CUDA
+ *     error string is available from salsc_last_cuda_error() on that thread.
+ *   - No C++ exception crosses this boundary.
+ *
+ * Storage types: SALSC_F32 (IEEE binary32) or SALSC_BF16 (bfloat16).  All
+ * arithmetic accumulates in fp32; outputs are rounded once to the storage
+ * type, round-to-nearest-even.
+ */
+#ifndef SALSC_H
+#define SALSC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SALSC_OK = 0,
+  SALSC_ERR_INVALID_ARG = 1, /* a shape, pointer or option is invalid */
+  SALSC_ERR_UNSUPPORTED = 2, /* valid but no kernel for this shape/dtype */
+  SALSC_ERR_WORKSPACE = 3,   /* workspace missing, misaligned or too small */
+  SALSC_ERR_CUDA = 4         /* a CUDA launch or runtime call failed */
+} salsc_status;
+
+typedef enum { SALSC_F32 = 0, SALSC_BF16 = 1 } salsc_dtype;
+
+/* Same type as cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st* salsc_stream;
+
+/*
+ * Stage 1, low-rank projection (prefill compression):
+ *     Kc = K . Pk     Vc = V . Pv
+ * SALS technical framework, stage 1 ("project K and V into a low-dimensional
+ * latent space with a low-rank matrix"); keys are projected before RoPE
+ * (abstract: the selection interaction is RoPE-free).
+ *
+ *   K, V     [n_tokens][hidden]   keys (pre-RoPE) and values; either may be
+ *                                 NULL to skip that half (its Kc/Vc and P are
+ *                                 then ignored)
+ *   Pk, Pv   [hidden][rank]       projections (orthonormal columns expected,
+ *                                 not checked)
+ *   Kc, Vc   [n_tokens][rank]     outputs, storage dtype
+ *   hidden = n_kv_heads * head_dim.
+ * Requirements: n_tokens >= 0, hidden >= 16 and rank >= 16 multiples of 16
+ * for SALSC_BF16 (multiples of 4 for SALSC_F32); 16-byte aligned pointers.
+ * Errors: INVALID_ARG on bad sizes, null required pointers or misalignment;
+ * CUDA on launch failure.  Accumulation is fp32; one rounding to the dtype.
+ */
+salsc_status salsc_compress(const void* K, const void* V, const void* Pk, const void* Pv,
+                            void* Kc, void* Vc, int64_t n_tokens, int32_t hidden, int32_t rank,
+                            salsc_dtype dtype, salsc_stream stream);
+
+/*
+ * Shapes of one decode layer-step.  B sequences share one layer's
+ * projections; sequence b owns latent rows seq_offsets[b] .. seq_offsets[b+1]-1
+ * of Kc/Vc (a packed ragged cache), so n_b = seq_offsets[b+1]-seq_offsets[b].
+ * Cached token t of sequence b sits at RoPE position t.
+ *
+ * Query head h belongs to KV head (selection unit) u = h / (n_q_heads /
+ * n_kv_heads); unit u uses rows u*head_dim .. u*head_dim+head_dim-1 of Pk and
+ * Pv.  With n_q_heads == n_kv_heads (MHA) every head is its own unit.
+ */
+typedef struct {
+  int32_t batch;      /* B >= 1 */
+  int32_t n_q_heads;  /* Hq, a multiple of n_kv_heads */
+  int32_t n_kv_heads; /* Hkv = U, selection units per sequence */
+  int32_t head_dim;   /* d, even; 64 or 128 supported */
+  int32_t rank;       /* r, latent width; multiple of 64 (bf16) or 4 (f32), r <= 512 */
+  int32_t top_k;      /* k >= 1 tokens kept per unit (k_b = min(k, n_b)) */
+  const int64_t* seq_offsets_host; /* [B+1] on the host, for planning; [0] == 0, strictly increasing */
+  const int64_t* seq_offsets_dev;  /* [B+1] the same values in device memory */
+  const int32_t* q_pos_dev;        /* [B] query positions in device memory, or NULL for n_b */
+  double rope_base;                /* RoPE base (10000, 500000, ...) > 1 */
+  float softmax_scale;             /* 0 -> 1/sqrt(head_dim) */
+  salsc_dtype dtype;               /* storage type of q, Kc, Vc, Pk, Pv and out */
+} salsc_decode_desc;
+
+/*
+ * Bytes of device workspace salsc_decode_step needs for this shape (0 if the
+ * descriptor is invalid).  It depends on the shapes and seq_offsets_host only.
+ */
+size_t salsc_decode_workspace_size(const salsc_decode_desc* desc);
+
+/*
+ * Initialise a workspace: clears its device-side status word.  Call once per
+ * workspace before the first salsc_decode_step (stream-ordered, no sync).
+ * Errors: INVALID_ARG (bad desc), WORKSPACE (NULL, not 256-byte aligned or
+ * smaller than salsc_decode_workspace_size), CUDA.
+ */
+salsc_status salsc_decode_prepare(const salsc_decode_desc* desc, void* ws, size_t ws_bytes,
+                                  salsc_stream stream);
+
+/*
+ * One decode layer-step, stages 2-4 of the SALS technical framework:
+ *
+ *   for every sequence b and unit u:
+ *     s[t]  = sum_{h in u} (q[b,h] . Pk_u) . Kc_b[t]        (RoPE-free, all t < n_b)
+ *     S     = the k_b tokens with the largest s (ties -> lower t)
+ *     for every query head h of u:
+ *       K_t   = RoPE(Kc_b[t] . Pk_u^T, t),  V_t = Vc_b[t] . Pv_u^T    (t in S only)
+ *       l_t   = RoPE(q[b,h], q_pos[b]) . K_t * softmax_scale
+ *       out[b,h] = sum_{t in S} softmax(l)_t V_t
+ *
+ * RoPE is the rotate-half form on pairs (i, i + d/2) with angle
+ * pos * rope_base^(-2i/d).
+ *
+ *   q        [B][Hq][d]        current queries, before RoPE, storage dtype
+ *   Kc, Vc   [N][r]            latent cache, N = seq_offsets[B]
+ *   Pk, Pv   [Hkv*d][r]        projections
+ *   out      [B][Hq][d]        attention output, storage dtype
+ *   idx_out  [B][U][k] int32   selected token indices within each sequence,
+ *                              unordered, -1 in slots >= k_b; may be NULL
+ *   ws       workspace of at least salsc_decode_workspace_size bytes,
+ *            prepared once with salsc_decode_prepare; 256-byte aligned
+ * No allocation, no host synchronisation: safe to capture in a CUDA graph.
+ * Errors: INVALID_ARG (desc or null pointer), UNSUPPORTED (shape without a
+ * kernel), WORKSPACE, CUDA.
+ */
+salsc_status salsc_decode_step(const salsc_decode_desc* desc, const void* q, const void* Kc,
+                               const void* Vc, const void* Pk, const void* Pv, void* out,
+                               int32_t* idx_out, void* ws, size_t ws_bytes, salsc_stream stream);
+
+/*
+ * Number of kernels one decode layer-step launches, in order: latent query,
+ * latent scoring, top-k, attention over the kept tokens, split merge.
+ */
+#define SALSC_DECODE_KERNELS 5
+
+/*
+ * salsc_decode_step with timing marks: the same work, plus
+ * cudaEventRecord(events[i], stream) just before kernel i and
+ * events[SALSC_DECODE_KERNELS] after the last, so that
+ * cudaEventElapsedTime(events[i], events[i+1]) is kernel i's time on the
+ * stream.  events: SALSC_DECODE_KERNELS + 1 cudaEvent_t handles created by
+ * the caller (cast to void*); n_events must equal that count.
+ * Errors: as salsc_decode_step; INVALID_ARG for a missing or short event list.
+ */
+salsc_status salsc_decode_step_timed(const salsc_decode_desc* desc, const void* q, const void* Kc,
+                                     const void* Vc, const void* Pk, const void* Pv, void* out,
+                                     int32_t* idx_out, void* ws, size_t ws_bytes,
+                                     salsc_stream stream, void* const* events, int32_t n_events);
+
+/*
+ * Device-side anomaly flags recorded in a workspace since salsc_decode_prepare
+ * (bit 0: a selected index fell outside its sequence; bit 1: a pipeline wait
+ * gave up after its iteration limit).  Copies one word to *flags_host and
+ * synchronises the stream.  Returns INVALID_ARG/WORKSPACE/CUDA on failure.
+ */
+salsc_status salsc_decode_read_flags(void* ws, size_t ws_bytes, uint32_t* flags_host,
+                                     salsc_stream stream);
+
+/* Static description of a status code. */
+const char* salsc_status_string(salsc_status status);
+
+/* Text of the last CUDA error seen by this library on the calling thread. */
+const char* salsc_last_cuda_error(void);
+
+/* Library version string. */
+const char* salsc_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SALSC_H */

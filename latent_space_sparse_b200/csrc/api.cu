@@ -1,0 +1,266 @@
+// api.cu -- the extern "C" boundary of libsalsc: validation, planning,
+// workspace layout and the launch sequence of one decode layer-step.
+//
+// Method: "SALS: Sparse Attention in Latent Space for KV cache Compression",
+// technical framework, stages 1-4.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "common.cuh"
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "no error";
+
+salsc_status cuda_fail(cudaError_t e) {
+  snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "%s: %s", cudaGetErrorName(e),
+           cudaGetErrorString(e));
+  return SALSC_ERR_CUDA;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+constexpr int kScoreTile = 128;
+constexpr int kTopkSliceTarget = 8192;  // keys per top-k CTA before the cluster grows
+constexpr int kTopkMaxCluster = 8;
+constexpr int kAttendTargetCtas = 2 * 148;
+
+// Validate the descriptor and derive the plan.  Returns SALSC_OK or the error.
+salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
+  if (!D || !D->seq_offsets_host) return SALSC_ERR_INVALID_ARG;
+  if (D->batch < 1 || D->n_q_heads < 1 || D->n_kv_heads < 1 || D->head_dim < 2 || D->rank < 1 ||
+      D->top_k < 1)
+    return SALSC_ERR_INVALID_ARG;
+  if (D->n_q_heads % D->n_kv_heads != 0 || D->head_dim % 2 != 0) return SALSC_ERR_INVALID_ARG;
+  if (D->dtype != SALSC_F32 && D->dtype != SALSC_BF16) return SALSC_ERR_INVALID_ARG;
+  if (!(D->rope_base > 1.0) || !isfinite(D->rope_base)) return SALSC_ERR_INVALID_ARG;
+  if (!(D->softmax_scale >= 0.0f) || !isfinite(D->softmax_scale)) return SALSC_ERR_INVALID_ARG;
+  if (D->seq_offsets_host[0] != 0) return SALSC_ERR_INVALID_ARG;
+  int64_t n_max = 0;
+  int n_tiles = 0;
+  for (int b = 0; b < D->batch; ++b) {
+    const int64_t nb = D->seq_offsets_host[b + 1] - D->seq_offsets_host[b];
+    if (nb < 1 || nb > (int64_t)INT32_MAX) return SALSC_ERR_INVALID_ARG;
+    if (nb > n_max) n_max = nb;
+    n_tiles += (int)((nb + kScoreTile - 1) / kScoreTile);
+  }
+  // shapes with kernels
+  if (D->head_dim != 64 && D->head_dim != 128) return SALSC_ERR_UNSUPPORTED;
+  if (D->rank > salsc::kMaxRank) return SALSC_ERR_UNSUPPORTED;
+  if (D->dtype == SALSC_BF16 && D->rank % 64 != 0) return SALSC_ERR_UNSUPPORTED;
+  if (D->dtype == SALSC_F32 && D->rank % 4 != 0) return SALSC_ERR_UNSUPPORTED;
+  if (D->rank > D->n_kv_heads * D->head_dim) return SALSC_ERR_INVALID_ARG;
+
+  salsc::DecodePlan p{};
+  p.B = D->batch;
+  p.Hq = D->n_q_heads;
+  p.U = D->n_kv_heads;
+  p.G = p.Hq / p.U;
+  p.d = D->head_dim;
+  p.r = D->rank;
+  p.k = D->top_k;
+  p.dtype = D->dtype;
+  p.N = D->seq_offsets_host[D->batch];
+  p.n_max = n_max;
+  p.score_tile = kScoreTile;
+  p.n_score_tiles = n_tiles;
+  int c = 1;
+  while (c < kTopkMaxCluster && (n_max + c - 1) / c > kTopkSliceTarget) c *= 2;
+  p.topk_cluster = c;
+  p.topk_slice = (int)((n_max + c - 1) / c);
+  const int64_t k_eff = D->top_k < n_max ? D->top_k : n_max;
+  const int units = p.B * p.U;
+  int splits = (kAttendTargetCtas + units - 1) / units;
+  if (splits > 64) splits = 64;
+  int chunk = (int)((k_eff + splits - 1) / splits);
+  if (chunk < 64) chunk = 64;
+  chunk = (chunk + 15) / 16 * 16;
+  splits = (int)((k_eff + chunk - 1) / chunk);  // never more than before: chunk only grew
+  if (splits < 1) splits = 1;
+  p.splits = splits;
+  p.chunk = chunk;
+  p.scale = D->softmax_scale != 0.0f ? D->softmax_scale : (float)(1.0 / sqrt((double)p.d));
+  p.rope_base = D->rope_base;
+
+  size_t off = 0;
+  p.off_flags = off;
+  off = align_up(off + 16, salsc::kWsAlign);
+  p.off_qlat = off;
+  off = align_up(off + sizeof(float) * (size_t)p.B * p.U * p.r, salsc::kWsAlign);
+  p.off_qsplit = off;
+  off = align_up(off + sizeof(__nv_bfloat16) * (size_t)p.B * 2 * p.U * p.r, salsc::kWsAlign);
+  p.off_scores = off;
+  off = align_up(off + sizeof(float) * (size_t)p.N * p.U, salsc::kWsAlign);
+  p.off_idx = off;
+  off = align_up(off + sizeof(int32_t) * (size_t)p.B * p.U * p.k, salsc::kWsAlign);
+  p.off_part = off;
+  off = align_up(off + sizeof(float) * (size_t)p.B * p.Hq * p.splits * (p.r + 2), salsc::kWsAlign);
+  p.total = off;
+  *P = p;
+  return SALSC_OK;
+}
+
+salsc_status check_ws(const salsc::DecodePlan& p, void* ws, size_t ws_bytes) {
+  if (!ws || ((uintptr_t)ws % salsc::kWsAlign) != 0 || ws_bytes < p.total)
+    return SALSC_ERR_WORKSPACE;
+  return SALSC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* salsc_status_string(salsc_status st) {
+  switch (st) {
+    case SALSC_OK: return "ok";
+    case SALSC_ERR_INVALID_ARG: return "invalid argument";
+    case SALSC_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case SALSC_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case SALSC_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+const char* salsc_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* salsc_version(void) { return "salsc 0.1 (sm_100a)"; }
+
+size_t salsc_decode_workspace_size(const salsc_decode_desc* desc) {
+  salsc::DecodePlan p;
+  if (make_plan(desc, &p) != SALSC_OK) return 0;
+  return p.total;
+}
+
+salsc_status salsc_decode_prepare(const salsc_decode_desc* desc, void* ws, size_t ws_bytes,
+                                  salsc_stream stream) {
+  salsc::DecodePlan p;
+  salsc_status st = make_plan(desc, &p);
+  if (st != SALSC_OK) return st;
+  if ((st = check_ws(p, ws, ws_bytes)) != SALSC_OK) return st;
+  cudaError_t e = cudaMemsetAsync((char*)ws + p.off_flags, 0, 16, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return SALSC_OK;
+}
+
+salsc_status salsc_decode_read_flags(void* ws, size_t ws_bytes, uint32_t* flags_host,
+                                     salsc_stream stream) {
+  if (!flags_host) return SALSC_ERR_INVALID_ARG;
+  if (!ws || ((uintptr_t)ws % salsc::kWsAlign) != 0 || ws_bytes < 16) return SALSC_ERR_WORKSPACE;
+  cudaError_t e = cudaMemcpyAsync(flags_host, ws, sizeof(uint32_t), cudaMemcpyDeviceToHost,
+                                  (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return SALSC_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+salsc_status decode_step_impl(const salsc_decode_desc* desc, const void* q, const void* Kc,
+                              const void* Vc, const void* Pk, const void* Pv, void* out,
+                              int32_t* idx_out, void* ws, size_t ws_bytes, salsc_stream stream,
+                              void* const* events, int32_t n_events) {
+  salsc::DecodePlan p;
+  salsc_status st = make_plan(desc, &p);
+  if (st != SALSC_OK) return st;
+  if (!desc->seq_offsets_dev || !q || !Kc || !Vc || !Pk || !Pv || !out)
+    return SALSC_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(Pk) || !aligned16(Pv) ||
+      !aligned16(out) || ((uintptr_t)idx_out & 3u))
+    return SALSC_ERR_INVALID_ARG;
+  if (events) {
+    if (n_events != SALSC_DECODE_KERNELS + 1) return SALSC_ERR_INVALID_ARG;
+    for (int i = 0; i < n_events; ++i)
+      if (!events[i]) return SALSC_ERR_INVALID_ARG;
+  }
+  if ((st = check_ws(p, ws, ws_bytes)) != SALSC_OK) return st;
+
+  char* w = (char*)ws;
+  salsc::DecodeArgs a;
+  a.q = q;
+  a.Kc = Kc;
+  a.Vc = Vc;
+  a.Pk = Pk;
+  a.Pv = Pv;
+  a.out = out;
+  a.idx = idx_out ? idx_out : (int32_t*)(w + p.off_idx);
+  a.seq_off = desc->seq_offsets_dev;
+  a.q_pos = desc->q_pos_dev;
+  a.flags = (uint32_t*)(w + p.off_flags);
+  a.qlat = (float*)(w + p.off_qlat);
+  a.qsplit = (__nv_bfloat16*)(w + p.off_qsplit);
+  a.scores = (float*)(w + p.off_scores);
+  a.part = (float*)(w + p.off_part);
+
+  cudaStream_t s = (cudaStream_t)stream;
+  typedef cudaError_t (*launcher)(const salsc::DecodePlan&, const salsc::DecodeArgs&, cudaStream_t);
+  const launcher seq[SALSC_DECODE_KERNELS] = {salsc::launch_latent_q, salsc::launch_score,
+                                              salsc::launch_topk, salsc::launch_attend,
+                                              salsc::launch_combine};
+  cudaError_t e;
+  // Inside stream capture an event record must be an external node to
+  // record at replay time.
+  unsigned rec_flags = cudaEventRecordDefault;
+  if (events) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if ((e = cudaStreamIsCapturing(s, &cs)) != cudaSuccess) return cuda_fail(e);
+    if (cs == cudaStreamCaptureStatusActive) rec_flags = cudaEventRecordExternal;
+  }
+  for (int i = 0; i < SALSC_DECODE_KERNELS; ++i) {
+    if (events &&
+        (e = cudaEventRecordWithFlags((cudaEvent_t)events[i], s, rec_flags)) != cudaSuccess)
+      return cuda_fail(e);
+    if ((e = seq[i](p, a, s)) != cudaSuccess) return cuda_fail(e);
+  }
+  if (events && (e = cudaEventRecordWithFlags((cudaEvent_t)events[SALSC_DECODE_KERNELS], s,
+                                              rec_flags)) != cudaSuccess)
+    return cuda_fail(e);
+  return SALSC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+salsc_status salsc_decode_step(const salsc_decode_desc* desc, const void* q, const void* Kc,
+                               const void* Vc, const void* Pk, const void* Pv, void* out,
+                               int32_t* idx_out, void* ws, size_t ws_bytes, salsc_stream stream) {
+  return decode_step_impl(desc, q, Kc, Vc, Pk, Pv, out, idx_out, ws, ws_bytes, stream, nullptr, 0);
+}
+
+salsc_status salsc_decode_step_timed(const salsc_decode_desc* desc, const void* q, const void* Kc,
+                                     const void* Vc, const void* Pk, const void* Pv, void* out,
+                                     int32_t* idx_out, void* ws, size_t ws_bytes,
+                                     salsc_stream stream, void* const* events, int32_t n_events) {
+  if (!events) return SALSC_ERR_INVALID_ARG;
+  return decode_step_impl(desc, q, Kc, Vc, Pk, Pv, out, idx_out, ws, ws_bytes, stream, events,
+                          n_events);
+}
+
+salsc_status salsc_compress(const void* K, const void* V, const void* Pk, const void* Pv, void* Kc,
+                            void* Vc, int64_t n_tokens, int32_t hidden, int32_t rank,
+                            salsc_dtype dtype, salsc_stream stream) {
+  if (dtype != SALSC_F32 && dtype != SALSC_BF16) return SALSC_ERR_INVALID_ARG;
+  if (n_tokens < 0 || hidden < 1 || rank < 1) return SALSC_ERR_INVALID_ARG;
+  const int q = dtype == SALSC_BF16 ? 16 : 4;
+  if (hidden % q != 0 || rank % q != 0) return SALSC_ERR_INVALID_ARG;
+  if (!K && !V) return SALSC_ERR_INVALID_ARG;
+  if (K && (!Pk || !Kc || !aligned16(K) || !aligned16(Pk) || !aligned16(Kc)))
+    return SALSC_ERR_INVALID_ARG;
+  if (V && (!Pv || !Vc || !aligned16(V) || !aligned16(Pv) || !aligned16(Vc)))
+    return SALSC_ERR_INVALID_ARG;
+  if (n_tokens == 0) return SALSC_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e;
+  if (K && (e = salsc::launch_compress(K, Pk, Kc, n_tokens, hidden, rank, dtype, s)) != cudaSuccess)
+    return cuda_fail(e);
+  if (V && (e = salsc::launch_compress(V, Pv, Vc, n_tokens, hidden, rank, dtype, s)) != cudaSuccess)
+    return cuda_fail(e);
+  return SALSC_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,122 @@
+// common.cuh -- internal definitions shared by the salsc CUDA sources.
+//
+// Nothing here is part of the public ABI (include/salsc.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "salsc.h"
+
+namespace salsc {
+
+// Device-side anomaly flags (first word of the workspace).
+enum : uint32_t {
+  FLAG_BAD_INDEX = 1u << 0,  // a selected index fell outside its sequence
+  FLAG_WAIT_TIMEOUT = 1u << 1,  // a bounded pipeline wait gave up
+};
+
+constexpr int kMaxRank = 512;
+constexpr int kMaxHeadDim = 128;
+constexpr size_t kWsAlign = 256;
+
+// Host-side plan of one decode layer-step, derived from the descriptor only.
+struct DecodePlan {
+  int B, Hq, U, G, d, r, k;
+  salsc_dtype dtype;
+  int64_t N, n_max;
+  int n_score_tiles;    // sum_b ceil(n_b / score tile)
+  int score_tile;       // tokens per scoring CTA
+  int topk_cluster;     // CTAs per selection unit in the top-k kernel
+  int topk_slice;       // max keys per top-k CTA
+  int splits;           // attention CTAs per unit
+  int chunk;            // selected tokens per attention CTA
+  float scale;
+  double rope_base;
+  // workspace layout (byte offsets)
+  size_t off_flags, off_qlat, off_qsplit, off_scores, off_idx, off_part, total;
+};
+
+// Raw pointers of one decode call, passed to the launchers.
+struct DecodeArgs {
+  const void* q;
+  const void* Kc;
+  const void* Vc;
+  const void* Pk;
+  const void* Pv;
+  void* out;
+  int32_t* idx;  // [B][U][k] (caller's or workspace)
+  const int64_t* seq_off;
+  const int32_t* q_pos;
+  uint32_t* flags;
+  float* qlat;                 // [B][U][r]
+  __nv_bfloat16* qsplit;       // [B][2U][r] hi rows then lo rows
+  float* scores;               // packed per (b,u)
+  float* part;                 // [B][Hq][splits][r+2]
+};
+
+// Launchers (each returns the cudaError_t of its launch).
+cudaError_t launch_latent_q(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_score(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_topk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_attend(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_combine(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_compress(const void* X, const void* P, void* Y, int64_t n, int hid, int r,
+                            salsc_dtype dt, cudaStream_t s);
+
+// Raise a kernel's dynamic shared-memory limit once per device (not on every
+// launch, so that launches inside CUDA-graph capture make no attribute calls).
+constexpr int kMaxDevices = 64;
+template <typename K>
+cudaError_t ensure_smem(K* kernel, size_t bytes, int (&done)[kMaxDevices]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if ((int)bytes <= done[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done[dev] = (int)bytes;
+  return e;
+}
+
+// ---------------------------------------------------------------- device helpers
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Locate the tile `tile` of a ragged batch where sequence b has
+// ceil(n_b / tile_len) tiles; returns b and the first token of the tile.
+__device__ __forceinline__ void find_tile(const int64_t* __restrict__ seq_off, int B, int tile_len,
+                                          int tile, int& b_out, int64_t& t0_out) {
+  int acc = 0;
+  for (int b = 0; b < B; ++b) {
+    const int64_t nb = seq_off[b + 1] - seq_off[b];
+    const int nt = (int)((nb + tile_len - 1) / tile_len);
+    if (tile < acc + nt) {
+      b_out = b;
+      t0_out = (int64_t)(tile - acc) * tile_len;
+      return;
+    }
+    acc += nt;
+  }
+  b_out = -1;
+  t0_out = 0;
+}
+
+}  // namespace salsc

@@ -1,0 +1,237 @@
+"""ctypes binding of libsalsc (include/salsc.h): argument marshalling only.
+
+Every function here passes raw device pointers, sizes and the current CUDA
+stream to the C ABI; all arithmetic happens in the library's kernels.  The
+library must have been built (``python -m latent_space_sparse_b200.build``);
+importing this module without it raises, and nothing falls back to the CPU.
+Tensors are torch CUDA tensors (torch supplies device memory and streams).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "csrc", "libsalsc.so")
+
+SALSC_OK, SALSC_ERR_INVALID_ARG, SALSC_ERR_UNSUPPORTED, SALSC_ERR_WORKSPACE, SALSC_ERR_CUDA = range(5)
+SALSC_F32, SALSC_BF16 = 0, 1
+FLAG_BAD_INDEX, FLAG_WAIT_TIMEOUT = 1, 2
+WS_ALIGN = 256
+
+EXPORTS = (
+    "salsc_compress", "salsc_decode_workspace_size", "salsc_decode_prepare", "salsc_decode_step",
+    "salsc_decode_step_timed", "salsc_decode_read_flags", "salsc_status_string", "salsc_last_cuda_error", "salsc_version",
+)
+
+
+class SalscError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        msg = f"{what}: {status_string(status)}"
+        if status == SALSC_ERR_CUDA:
+            msg += f" ({_lib().salsc_last_cuda_error().decode()})"
+        super().__init__(msg)
+        self.status = status
+
+
+class DecodeDesc(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("n_q_heads", ctypes.c_int32),
+        ("n_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("rank", ctypes.c_int32),
+        ("top_k", ctypes.c_int32),
+        ("seq_offsets_host", ctypes.POINTER(ctypes.c_int64)),
+        ("seq_offsets_dev", ctypes.c_void_p),
+        ("q_pos_dev", ctypes.c_void_p),
+        ("rope_base", ctypes.c_double),
+        ("softmax_scale", ctypes.c_float),
+        ("dtype", ctypes.c_int),
+    ]
+
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m latent_space_sparse_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        dp = ctypes.POINTER(DecodeDesc)
+        lib.salsc_compress.restype = ctypes.c_int
+        lib.salsc_compress.argtypes = [vp, vp, vp, vp, vp, vp, i64, i32, i32, ctypes.c_int, vp]
+        lib.salsc_decode_workspace_size.restype = sz
+        lib.salsc_decode_workspace_size.argtypes = [dp]
+        lib.salsc_decode_prepare.restype = ctypes.c_int
+        lib.salsc_decode_prepare.argtypes = [dp, vp, sz, vp]
+        lib.salsc_decode_step.restype = ctypes.c_int
+        lib.salsc_decode_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.salsc_decode_step_timed.restype = ctypes.c_int
+        lib.salsc_decode_step_timed.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
+                                                ctypes.POINTER(ctypes.c_void_p), i32]
+        lib.salsc_decode_read_flags.restype = ctypes.c_int
+        lib.salsc_decode_read_flags.argtypes = [vp, sz, ctypes.POINTER(ctypes.c_uint32), vp]
+        lib.salsc_status_string.restype = ctypes.c_char_p
+        lib.salsc_status_string.argtypes = [ctypes.c_int]
+        lib.salsc_last_cuda_error.restype = ctypes.c_char_p
+        lib.salsc_last_cuda_error.argtypes = []
+        lib.salsc_version.restype = ctypes.c_char_p
+        lib.salsc_version.argtypes = []
+        _LIB = lib
+    return _LIB
+
+
+def load():
+    """Load the library (raises ImportError if it was not built)."""
+    return _lib()
+
+
+def status_string(status: int) -> str:
+    return _lib().salsc_status_string(status).decode()
+
+
+def version() -> str:
+    return _lib().salsc_version().decode()
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return SALSC_BF16
+    if t == torch.float32:
+        return SALSC_F32
+    raise TypeError(f"unsupported storage dtype {t}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(st: int, what: str):
+    if st != SALSC_OK:
+        raise SalscError(st, what)
+
+
+def salsc_compress(K, V, Pk, Pv, Kc, Vc, stream=None):
+    """Kc = K . Pk and Vc = V . Pv on the current stream; K or V may be None."""
+    x = K if K is not None else V
+    n, hid = x.shape
+    r = (Pk if K is not None else Pv).shape[1]
+    st = _lib().salsc_compress(_ptr(K), _ptr(V), _ptr(Pk), _ptr(Pv), _ptr(Kc), _ptr(Vc), n, hid, r,
+                               _dtype_code(x.dtype), _stream(stream))
+    _check(st, "salsc_compress")
+
+
+def make_desc(batch, n_q_heads, n_kv_heads, head_dim, rank, top_k, seq_offsets_host,
+              seq_offsets_dev=None, q_pos_dev=None, rope_base=10000.0, softmax_scale=0.0,
+              dtype=torch.bfloat16):
+    """Build a DecodeDesc; ``seq_offsets_host`` must be a contiguous CPU int64 tensor kept alive
+    by the caller (the descriptor points into it)."""
+    assert seq_offsets_host.dtype == torch.int64 and not seq_offsets_host.is_cuda
+    assert seq_offsets_host.is_contiguous()
+    return DecodeDesc(
+        batch, n_q_heads, n_kv_heads, head_dim, rank, top_k,
+        ctypes.cast(seq_offsets_host.data_ptr(), ctypes.POINTER(ctypes.c_int64)),
+        None if seq_offsets_dev is None else seq_offsets_dev.data_ptr(),
+        None if q_pos_dev is None else q_pos_dev.data_ptr(),
+        float(rope_base), float(softmax_scale), _dtype_code(dtype))
+
+
+def salsc_decode_workspace_size(desc: DecodeDesc) -> int:
+    return int(_lib().salsc_decode_workspace_size(ctypes.byref(desc)))
+
+
+def salsc_decode_prepare(desc: DecodeDesc, ws, stream=None):
+    st = _lib().salsc_decode_prepare(ctypes.byref(desc), _ptr(ws), ws.numel() * ws.element_size(),
+                                     _stream(stream))
+    _check(st, "salsc_decode_prepare")
+
+
+def salsc_decode_step(desc: DecodeDesc, q, Kc, Vc, Pk, Pv, out, idx_out, ws, stream=None):
+    st = _lib().salsc_decode_step(ctypes.byref(desc), _ptr(q), _ptr(Kc), _ptr(Vc), _ptr(Pk),
+                                  _ptr(Pv), _ptr(out), _ptr(idx_out), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream))
+    _check(st, "salsc_decode_step")
+
+
+DECODE_KERNELS = ("latent_q", "score", "topk", "attend", "combine")
+
+
+def salsc_decode_step_timed(desc: DecodeDesc, q, Kc, Vc, Pk, Pv, out, idx_out, ws, events,
+                            stream=None):
+    """salsc_decode_step plus an event record before each kernel and after the last
+    (``events``: len(DECODE_KERNELS)+1 torch.cuda.Event(enable_timing=True))."""
+    for e in events:  # torch creates the CUDA event lazily
+        if e.cuda_event == 0:
+            e.record(stream if stream is not None else torch.cuda.current_stream())
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    st = _lib().salsc_decode_step_timed(ctypes.byref(desc), _ptr(q), _ptr(Kc), _ptr(Vc), _ptr(Pk),
+                                        _ptr(Pv), _ptr(out), _ptr(idx_out), _ptr(ws),
+                                        ws.numel() * ws.element_size(), _stream(stream), arr,
+                                        len(events))
+    _check(st, "salsc_decode_step_timed")
+
+
+def salsc_decode_read_flags(ws, stream=None) -> int:
+    v = ctypes.c_uint32(0)
+    st = _lib().salsc_decode_read_flags(_ptr(ws), ws.numel() * ws.element_size(), ctypes.byref(v),
+                                        _stream(stream))
+    _check(st, "salsc_decode_read_flags")
+    return int(v.value)
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    """A uint8 device buffer of ``nbytes`` starting on a 256-byte boundary."""
+    buf = torch.empty(nbytes + WS_ALIGN, dtype=torch.uint8, device=device)
+    shift = (-buf.data_ptr()) % WS_ALIGN
+    return buf[shift:shift + nbytes]
+
+
+class Decoder:
+    """Descriptor + workspace for one decode shape (marshalling only).
+
+    ``seq_lens`` fixes the ragged layout of the latent cache; q/Kc/Vc/Pk/Pv/out
+    are passed per call.  q_pos (CUDA int32 [B]) defaults to n_b.
+    """
+
+    def __init__(self, batch, n_q_heads, n_kv_heads, head_dim, rank, top_k, seq_lens,
+                 rope_base=10000.0, softmax_scale=0.0, dtype=torch.bfloat16, device="cuda",
+                 q_pos=None):
+        lens = [int(x) for x in seq_lens]
+        offs = [0]
+        for n in lens:
+            offs.append(offs[-1] + n)
+        self.seq_offsets_host = torch.tensor(offs, dtype=torch.int64)
+        self.seq_offsets_dev = self.seq_offsets_host.to(device)
+        self.q_pos = None if q_pos is None else q_pos.to(device=device, dtype=torch.int32).contiguous()
+        self.shape = dict(batch=batch, n_q_heads=n_q_heads, n_kv_heads=n_kv_heads,
+                          head_dim=head_dim, rank=rank, top_k=top_k)
+        self.dtype = dtype
+        self.desc = make_desc(batch, n_q_heads, n_kv_heads, head_dim, rank, top_k,
+                              self.seq_offsets_host, self.seq_offsets_dev, self.q_pos, rope_base,
+                              softmax_scale, dtype)
+        nbytes = salsc_decode_workspace_size(self.desc)
+        if nbytes == 0:
+            raise SalscError(SALSC_ERR_INVALID_ARG, "salsc_decode_workspace_size")
+        self.ws = alloc_workspace(nbytes, device)
+        salsc_decode_prepare(self.desc, self.ws)
+
+    def step(self, q, Kc, Vc, Pk, Pv, out=None, idx_out=None, stream=None):
+        if out is None:
+            out = torch.empty_like(q)
+        salsc_decode_step(self.desc, q, Kc, Vc, Pk, Pv, out, idx_out, self.ws, stream)
+        return out
+
+    def flags(self, stream=None) -> int:
+        return salsc_decode_read_flags(self.ws, stream)

@@ -86,3 +86,31 @@ def compress_inputs(w: Workload, rows: int, seed: int | None = None) -> dict:
     pv = orthonormal(rng, hid, r)
     return {"K": _cast(k, w.dtype), "V": _cast(v, w.dtype), "Pk": _cast(pk, w.dtype),
             "Pv": _cast(pv, w.dtype)}
+
+
+def decode_inputs_device(w: Workload, layer: int, device, seq_lens=None) -> dict:
+    """The same recipe drawn on the GPU with a seeded torch generator.
+
+    Used for the extra layer buffer sets of the benchmark (fast to draw);
+    parity tests use :func:`decode_inputs`, whose values the oracle sees.
+    """
+    lens = tuple(int(n) for n in (seq_lens if seq_lens is not None else w.seq_lens))
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed * 1000 + layer)
+    n = sum(lens)
+    hid, r = w.hidden, w.rank
+    f32 = dict(device=device, dtype=torch.float32, generator=g)
+    dt = _TORCH_DT[w.dtype]
+    kc = torch.randn(n, w.low_rank, **f32) @ torch.randn(w.low_rank, r, **f32)
+    kc += 0.05 * torch.randn(n, r, **f32)
+    out = {
+        "Kc": kc.to(dt),
+        "Vc": torch.randn(n, r, **f32).to(dt),
+        "q": torch.randn(len(lens), w.n_q_heads, w.head_dim, **f32).to(dt),
+        "Pk": torch.linalg.qr(torch.randn(hid, r, **f32))[0].to(dt).contiguous(),
+        "Pv": torch.linalg.qr(torch.randn(hid, r, **f32))[0].to(dt).contiguous(),
+    }
+    offs = torch.zeros(len(lens) + 1, dtype=torch.int64)
+    offs[1:] = torch.cumsum(torch.tensor(lens, dtype=torch.int64), 0)
+    out["seq_offsets"] = offs
+    return out

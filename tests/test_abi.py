@@ -1,0 +1,119 @@
+"""The C-ABI library loads, exports every declared symbol and validates
+arguments on the host.  No test here launches a kernel: every call below
+returns its error before any CUDA work is enqueued."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from latent_space_sparse_b200 import salsc
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "salsc.h")).read()
+    return sorted(set(re.findall(r"\b(salsc_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declarations_are_the_binding_exports():
+    assert declared_symbols() == sorted(salsc.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = salsc.load()
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert salsc.version().startswith("salsc")
+
+
+def test_status_strings():
+    for code in range(5):
+        assert salsc.status_string(code)
+    assert salsc.status_string(salsc.SALSC_ERR_WORKSPACE).startswith("workspace")
+
+
+def desc(offs, **kw):
+    a = dict(batch=len(offs) - 1, n_q_heads=32, n_kv_heads=8, head_dim=128, rank=256, top_k=64,
+             rope_base=10000.0, softmax_scale=0.0, dtype=torch.bfloat16)
+    a.update(kw)
+    host = torch.tensor(offs, dtype=torch.int64)
+    d = salsc.make_desc(a["batch"], a["n_q_heads"], a["n_kv_heads"], a["head_dim"], a["rank"],
+                        a["top_k"], host, None, None, a["rope_base"], a["softmax_scale"], a["dtype"])
+    d._keep = host
+    return d
+
+
+def test_workspace_size_valid_shapes_grow_with_tokens():
+    small = salsc.salsc_decode_workspace_size(desc([0, 1000]))
+    big = salsc.salsc_decode_workspace_size(desc([0, 1000, 40000]))
+    assert 0 < small < big
+    assert small % 256 == 0
+
+
+@pytest.mark.parametrize("kw,offs", [
+    (dict(n_q_heads=30), [0, 10]),             # Hq not a multiple of Hkv
+    (dict(head_dim=127), [0, 10]),             # odd head dim
+    (dict(top_k=0), [0, 10]),                  # k < 1
+    (dict(rank=2048), [0, 10]),                # r > hidden / unsupported
+    (dict(rope_base=1.0), [0, 10]),            # base must exceed 1
+    (dict(softmax_scale=-1.0), [0, 10]),       # negative scale
+    ({}, [0, 10, 10]),                         # empty sequence
+    ({}, [1, 10]),                             # offsets must start at 0
+    (dict(head_dim=96, n_kv_heads=8), [0, 10]),  # no kernel for d = 96
+    (dict(rank=96), [0, 10]),                  # bf16 rank must be a multiple of 64
+])
+def test_invalid_descriptors_have_no_workspace(kw, offs):
+    assert salsc.salsc_decode_workspace_size(desc(offs, **kw)) == 0
+
+
+def call_step(d, q=1 << 20, kc=1 << 21, vc=1 << 22, pk=1 << 23, pv=1 << 24, out=1 << 25,
+              idx=None, ws=1 << 26, ws_bytes=16):
+    lib = salsc.load()
+    vp = ctypes.c_void_p
+    return lib.salsc_decode_step(ctypes.byref(d), vp(q), vp(kc), vp(vc), vp(pk), vp(pv), vp(out),
+                                 vp(idx), vp(ws), ws_bytes, None)
+
+
+def test_step_rejects_bad_arguments_before_launch():
+    d = desc([0, 100])
+    # no device offsets
+    assert call_step(d) == salsc.SALSC_ERR_INVALID_ARG
+    d.seq_offsets_dev = 1 << 27
+    assert call_step(d, q=0) == salsc.SALSC_ERR_INVALID_ARG           # null q
+    assert call_step(d, out=0) == salsc.SALSC_ERR_INVALID_ARG         # null out
+    assert call_step(d, kc=(1 << 21) + 2) == salsc.SALSC_ERR_INVALID_ARG  # misaligned
+    assert call_step(d, ws=0) == salsc.SALSC_ERR_WORKSPACE            # no workspace
+    assert call_step(d, ws=(1 << 26) + 64) == salsc.SALSC_ERR_WORKSPACE  # misaligned workspace
+    assert call_step(d, ws_bytes=16) == salsc.SALSC_ERR_WORKSPACE     # too small
+    bad = desc([0, 100], top_k=0)
+    bad.seq_offsets_dev = 1 << 27
+    assert call_step(bad) == salsc.SALSC_ERR_INVALID_ARG
+
+
+def test_prepare_rejects_short_workspace():
+    lib = salsc.load()
+    d = desc([0, 100])
+    need = salsc.salsc_decode_workspace_size(d)
+    st = lib.salsc_decode_prepare(ctypes.byref(d), ctypes.c_void_p(1 << 26), need - 1, None)
+    assert st == salsc.SALSC_ERR_WORKSPACE
+    st = lib.salsc_decode_prepare(ctypes.byref(d), None, need, None)
+    assert st == salsc.SALSC_ERR_WORKSPACE
+
+
+def test_compress_validation_before_launch():
+    lib = salsc.load()
+    vp = ctypes.c_void_p
+    a, b, c = vp(1 << 20), vp(1 << 21), vp(1 << 22)
+    # both halves missing
+    assert lib.salsc_compress(None, None, a, b, c, c, 10, 64, 16, salsc.SALSC_BF16, None) == 1
+    # hidden not a multiple of 16 (bf16)
+    assert lib.salsc_compress(a, None, b, None, c, None, 10, 40, 16, salsc.SALSC_BF16, None) == 1
+    # negative rows
+    assert lib.salsc_compress(a, None, b, None, c, None, -1, 64, 16, salsc.SALSC_BF16, None) == 1
+    # missing projection for a present half
+    assert lib.salsc_compress(a, None, None, None, c, None, 10, 64, 16, salsc.SALSC_BF16, None) == 1
+    # zero rows is a valid no-op (nothing is enqueued)
+    assert lib.salsc_compress(a, None, b, None, c, None, 0, 64, 16, salsc.SALSC_BF16, None) == 0

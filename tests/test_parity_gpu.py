@@ -1,0 +1,201 @@
+"""CUDA path vs the fp64 oracle on the same seeded inputs (needs a B200).
+
+Every call goes through the C ABI (libsalsc via the ctypes binding).  Rules
+(tests/parity.py): top-k sets identical up to swaps inside the tie band
+1e-4*max|s| of the k-th score; outputs within 2e-2 (bf16) / 1e-4 (fp32) of
+the oracle output's max-abs, against the oracle's attention over the GPU's
+own kept set, and against the plain oracle when the sets are identical.
+Full-size workloads are checked on sampled sequences: the oracle runs on
+those sequences alone, which is the same computation (a ragged batch
+decomposes into its sequences; pinned in test_oracle_pins).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from latent_space_sparse_b200 import salsc, synth, workloads as W
+from tests.parity import TOL, check_topk, max_rel_err, problem_of
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def gpu_decode(w, x, top_k=None, q_pos=None):
+    offs = x["seq_offsets"].numpy()
+    lens = np.diff(offs)
+    k = top_k or w.top_k
+    dec = salsc.Decoder(len(lens), w.n_q_heads, w.n_kv_heads, w.head_dim, w.rank, k, lens,
+                        rope_base=w.rope_base, dtype=synth.torch_dtype(w.dtype), device=DEV,
+                        q_pos=None if q_pos is None else torch.as_tensor(q_pos))
+    t = {n: x[n].to(DEV) for n in ("q", "Kc", "Vc", "Pk", "Pv")}
+    idx = torch.full((len(lens), w.n_kv_heads, k), -7, dtype=torch.int32, device=DEV)
+    out = dec.step(t["q"], t["Kc"], t["Vc"], t["Pk"], t["Pv"], idx_out=idx)
+    torch.cuda.synchronize()
+    assert dec.flags() == 0
+    return out.float().cpu().numpy(), idx.cpu().numpy()
+
+
+def sub_inputs(x, seqs):
+    """Inputs of the chosen sequences only (for the oracle)."""
+    offs = x["seq_offsets"].numpy()
+    rows = np.concatenate([np.arange(offs[b], offs[b + 1]) for b in seqs])
+    lens = [offs[b + 1] - offs[b] for b in seqs]
+    so = np.zeros(len(seqs) + 1, dtype=np.int64)
+    so[1:] = np.cumsum(lens)
+    return {"q": x["q"][list(seqs)], "Kc": x["Kc"][rows], "Vc": x["Vc"][rows], "Pk": x["Pk"],
+            "Pv": x["Pv"], "seq_offsets": torch.from_numpy(so)}
+
+
+def check(w, x, seqs=None, top_k=None, q_pos=None):
+    out, idx = gpu_decode(w, x, top_k, q_pos)
+    if seqs is not None:
+        x = sub_inputs(x, seqs)
+        out, idx = out[list(seqs)], idx[list(seqs)]
+        q_pos = None if q_pos is None else np.asarray(q_pos)[list(seqs)]
+    p = problem_of(w, x["seq_offsets"].numpy(), q_pos, top_k)
+    ora = oracle.decode(p, x["q"], x["Kc"], x["Vc"], x["Pk"], x["Pv"])
+    swaps = check_topk(p, idx, ora)
+    given = oracle.attend_given_idx(p, x["q"], x["Kc"], x["Vc"], x["Pk"], x["Pv"], idx)
+    err = max_rel_err(out, given["out"])
+    assert err <= TOL[w.dtype], f"output error {err:.3e} vs oracle on the GPU's kept set"
+    if swaps == 0:
+        err2 = max_rel_err(out, ora["out"])
+        assert err2 <= TOL[w.dtype], f"output error {err2:.3e} vs oracle"
+    return swaps, idx, ora
+
+
+# ------------------------------------------------------------ whole workloads
+
+def test_tiny_f32():
+    w = W.TINY_F32
+    check(w, synth.decode_inputs(w))
+
+
+def test_llama2_4k_b1():
+    w = W.LLAMA2_4K_B1
+    check(w, synth.decode_inputs(w))
+
+
+def test_llama2_4k_b16_reduced():
+    w = W.LLAMA2_4K_B16
+    check(w, synth.decode_inputs(w, seq_lens=(1024, 777, 1500)))
+
+
+def test_mistral_gqa_reduced():
+    w = W.MISTRAL_32K_B4
+    check(w, synth.decode_inputs(w, seq_lens=(4096, 2500)))
+
+
+def test_llama31_ragged_reduced():
+    # k = 4096 exceeds two of the lengths: k_b = n_b there
+    w = W.LLAMA31_RAGGED_128K
+    check(w, synth.decode_inputs(w, seq_lens=(1000, 3000, 5000, 8191)))
+
+
+@pytest.mark.parametrize("w,seqs", [
+    (W.LLAMA2_4K_B16, (0, 15)),
+    (W.MISTRAL_32K_B4, (0, 3)),
+    (W.LLAMA31_RAGGED_128K, (0, 3)),
+])
+def test_full_size_sampled_sequences(w, seqs):
+    check(w, synth.decode_inputs(w), seqs=seqs)
+
+
+# ------------------------------------------------------------ edge cases
+
+def test_single_token_sequences_and_k_above_n():
+    w = W.MISTRAL_32K_B4
+    x = synth.decode_inputs(w, seq_lens=(1, 2, 130, 1))
+    check(w, x, top_k=64)
+
+
+def test_k_equals_one():
+    w = W.LLAMA2_4K_B1
+    check(w, synth.decode_inputs(w, seq_lens=(700,)), top_k=1)
+
+
+def test_all_equal_scores_take_lowest_indices():
+    w = W.MISTRAL_32K_B4
+    x = synth.decode_inputs(w, seq_lens=(600, 333))
+    x["Kc"][:] = x["Kc"][0]  # every cached latent key identical: every score ties
+    swaps, idx, ora = check(w, x, top_k=100)
+    for b, nb in enumerate((600, 333)):
+        for u in range(w.n_kv_heads):
+            np.testing.assert_array_equal(np.sort(idx[b, u, :100]), np.arange(100))
+
+
+def test_large_query_positions():
+    w = W.LLAMA31_RAGGED_128K
+    x = synth.decode_inputs(w, seq_lens=(2000, 900))
+    check(w, x, top_k=256, q_pos=np.array([131071, 77777], dtype=np.int32))
+
+
+def test_head_dim_64_gqa_bf16():
+    w = W.Workload(name="gqa_d64", batch=2, n_q_heads=8, n_kv_heads=2, head_dim=64, rank=64,
+                   top_k=40, seq_lens=(300, 129), dtype="bf16", rope_base=10000.0, low_rank=8,
+                   seed=99)
+    check(w, synth.decode_inputs(w))
+
+
+def test_small_rank_f32():
+    w = W.Workload(name="f32_r16", batch=3, n_q_heads=6, n_kv_heads=3, head_dim=64, rank=16,
+                   top_k=9, seq_lens=(50, 17, 200), dtype="f32", rope_base=500000.0, low_rank=4,
+                   seed=98)
+    check(w, synth.decode_inputs(w))
+
+
+def test_repeated_steps_are_deterministic():
+    w = W.MISTRAL_32K_B4
+    x = synth.decode_inputs(w, seq_lens=(3000, 1000))
+    a_out, a_idx = gpu_decode(w, x)
+    b_out, b_idx = gpu_decode(w, x)
+    np.testing.assert_array_equal(a_idx, b_idx)
+    np.testing.assert_array_equal(a_out, b_out)
+
+
+# ------------------------------------------------------------ compression
+
+def test_compress_tiny_f32():
+    w = W.TINY_F32
+    x = synth.compress_inputs(w, rows=512)
+    K, V, Pk, Pv = (x[n].to(DEV) for n in ("K", "V", "Pk", "Pv"))
+    Kc = torch.empty(512, w.rank, device=DEV)
+    Vc = torch.empty_like(Kc)
+    salsc.salsc_compress(K, V, Pk, Pv, Kc, Vc)
+    torch.cuda.synchronize()
+    for got, X, P in ((Kc, x["K"], x["Pk"]), (Vc, x["V"], x["Pv"])):
+        ref = oracle.compress(X, P)
+        assert max_rel_err(got.cpu().numpy(), ref) <= TOL["f32"]
+
+
+def test_compress_llama2_prefill_sampled_rows():
+    w = W.LLAMA2_4K_B16
+    rows = w.compress_rows
+    x = synth.compress_inputs(w, rows=rows)
+    K, V, Pk, Pv = (x[n].to(DEV) for n in ("K", "V", "Pk", "Pv"))
+    Kc = torch.empty(rows, w.rank, dtype=torch.bfloat16, device=DEV)
+    Vc = torch.empty_like(Kc)
+    salsc.salsc_compress(K, V, Pk, Pv, Kc, Vc)
+    torch.cuda.synchronize()
+    sample = np.random.default_rng(0).choice(rows, 256, replace=False)
+    sample = np.concatenate([sample, [0, rows - 1]])
+    for got, X, P in ((Kc, x["K"], x["Pk"]), (Vc, x["V"], x["Pv"])):
+        ref = oracle.compress(X[sample], P)
+        g = got[torch.from_numpy(sample).to(DEV)].float().cpu().numpy()
+        assert max_rel_err(g, ref) <= TOL["bf16"]
+        # one rounding of an fp32 accumulation: almost every entry is the
+        # correctly rounded bf16 value or its neighbour
+        exact = oracle.round_storage(ref, "bf16")
+        assert np.mean(g == exact) > 0.9
+
+
+def test_compress_one_half_only():
+    w = W.TINY_F32
+    x = synth.compress_inputs(w, rows=100)
+    V, Pv = x["V"].to(DEV), x["Pv"].to(DEV)
+    Vc = torch.empty(100, w.rank, device=DEV)
+    salsc.salsc_compress(None, V, None, Pv, None, Vc)
+    torch.cuda.synchronize()
+    assert max_rel_err(Vc.cpu().numpy(), oracle.compress(x["V"], x["Pv"])) <= TOL["f32"]
