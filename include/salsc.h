@@ -164,6 +164,39 @@ salsc_status salsc_decode_step_timed(const salsc_decode_desc* desc, const void* 
                                      salsc_stream stream, void* const* events, int32_t n_events);
 
 /*
+ * Decode step whose scratch is a fixed array inside the library, for callers
+ * that cannot allocate device memory (no counterpart in the SALS paper).
+ *
+ * Some callers cannot hand the library a workspace: a plugin inside a host
+ * application whose memory manager owns every device allocation, or a
+ * serving loop that must never call cudaMalloc.  This entry point computes
+ * exactly what salsc_decode_step computes, with the same arguments minus the
+ * workspace, and allocates nothing (no cudaMalloc/cudaFree, no allocating
+ * library routine).  The caller still owns q, Kc, Vc, Pk, Pv, out and idx_out.
+ *
+ *   - Limit: the shape's salsc_decode_workspace_size(desc) must not exceed
+ *     SALSC_STATIC_WORKSPACE_BYTES (16 MiB; enough for every workload in the
+ *     test-suite, e.g. 4 x 32768 tokens x 8 KV heads).  Larger shapes return
+ *     SALSC_ERR_WORKSPACE and enqueue nothing.
+ *   - Every GPU that loads this part of the library keeps the 16 MiB array
+ *     until the process exits.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents; each call clears the part that must start at zero.  Calls
+ *     that overlap on the GPU (different streams, or different host threads
+ *     without ordering) race on the array: serialise them.
+ *   - The anomaly flags of this variant are not readable by the caller.
+ * Errors: as salsc_decode_step; WORKSPACE when the shape needs more scratch.
+ */
+#define SALSC_STATIC_WORKSPACE_BYTES (16u << 20)
+salsc_status salsc_decode_step_static_ws(const salsc_decode_desc* desc, const void* q,
+                                         const void* Kc, const void* Vc, const void* Pk,
+                                         const void* Pv, void* out, int32_t* idx_out,
+                                         salsc_stream stream);
+
+/*
  * Device-side anomaly flags recorded in a workspace since salsc_decode_prepare
  * (bit 0: a selected index fell outside its sequence; bit 1: a pipeline wait
  * gave up after its iteration limit).  Copies one word to *flags_host and

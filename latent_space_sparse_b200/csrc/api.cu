@@ -111,6 +111,8 @@ salsc_status check_ws(const salsc::DecodePlan& p, void* ws, size_t ws_bytes) {
 
 }  // namespace
 
+salsc_status salsc::record_cuda_error(cudaError_t e) { return cuda_fail(e); }
+
 extern "C" {
 
 const char* salsc_status_string(salsc_status st) {

@@ -56,6 +56,9 @@ struct DecodeArgs {
   float* part;                 // [B][Hq][splits][r+2]
 };
 
+// Record a CUDA error for salsc_last_cuda_error() and return SALSC_ERR_CUDA.
+salsc_status record_cuda_error(cudaError_t e);
+
 // Launchers (each returns the cudaError_t of its launch).
 cudaError_t launch_latent_q(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_score(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);

@@ -23,7 +23,7 @@ WS_ALIGN = 256
 
 EXPORTS = (
     "salsc_compress", "salsc_decode_workspace_size", "salsc_decode_prepare", "salsc_decode_step",
-    "salsc_decode_step_timed", "salsc_decode_read_flags", "salsc_status_string", "salsc_last_cuda_error", "salsc_version",
+    "salsc_decode_step_timed", "salsc_decode_step_static_ws", "salsc_decode_read_flags", "salsc_status_string", "salsc_last_cuda_error", "salsc_version",
 )
 
 
@@ -76,6 +76,8 @@ def _lib():
         lib.salsc_decode_step_timed.restype = ctypes.c_int
         lib.salsc_decode_step_timed.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
                                                 ctypes.POINTER(ctypes.c_void_p), i32]
+        lib.salsc_decode_step_static_ws.restype = ctypes.c_int
+        lib.salsc_decode_step_static_ws.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
         lib.salsc_decode_read_flags.restype = ctypes.c_int
         lib.salsc_decode_read_flags.argtypes = [vp, sz, ctypes.POINTER(ctypes.c_uint32), vp]
         lib.salsc_status_string.restype = ctypes.c_char_p
@@ -181,6 +183,18 @@ def salsc_decode_step_timed(desc: DecodeDesc, q, Kc, Vc, Pk, Pv, out, idx_out, w
                                         ws.numel() * ws.element_size(), _stream(stream), arr,
                                         len(events))
     _check(st, "salsc_decode_step_timed")
+
+
+STATIC_WORKSPACE_BYTES = 16 << 20
+
+
+def salsc_decode_step_static_ws(desc: DecodeDesc, q, Kc, Vc, Pk, Pv, out, idx_out, stream=None):
+    """salsc_decode_step with the library's fixed internal scratch: no workspace argument,
+    nothing allocated (for callers that cannot allocate device memory)."""
+    st = _lib().salsc_decode_step_static_ws(ctypes.byref(desc), _ptr(q), _ptr(Kc), _ptr(Vc),
+                                            _ptr(Pk), _ptr(Pv), _ptr(out), _ptr(idx_out),
+                                            _stream(stream))
+    _check(st, "salsc_decode_step_static_ws")
 
 
 def salsc_decode_read_flags(ws, stream=None) -> int:
