@@ -62,6 +62,7 @@ salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
   p.d = D->head_dim;
   p.r = D->rank;
   p.k = D->top_k;
+  p.npad = (2 * p.U + 15) / 16 * 16;
   p.dtype = D->dtype;
   p.N = D->seq_offsets_host[D->batch];
   p.n_max = n_max;
@@ -72,16 +73,32 @@ salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
   p.topk_cluster = c;
   p.topk_slice = (int)((n_max + c - 1) / c);
   const int64_t k_eff = D->top_k < n_max ? D->top_k : n_max;
-  const int units = p.B * p.U;
-  int splits = (kAttendTargetCtas + units - 1) / units;
-  if (splits > 64) splits = 64;
-  int chunk = (int)((k_eff + splits - 1) / splits);
-  if (chunk < 64) chunk = 64;
-  chunk = (chunk + 15) / 16 * 16;
-  splits = (int)((k_eff + chunk - 1) / chunk);  // never more than before: chunk only grew
-  if (splits < 1) splits = 1;
-  p.splits = splits;
-  p.chunk = chunk;
+  p.attend_tc = salsc::attend_tc_supported(p);
+  if (p.attend_tc) {
+    // one partial slot per tile of 128 kept tokens
+    p.chunk = 128;
+    p.splits = (int)((k_eff + 127) / 128);
+    int64_t tiles = 0;
+    for (int b = 0; b < D->batch; ++b) {
+      const int64_t nb = D->seq_offsets_host[b + 1] - D->seq_offsets_host[b];
+      const int64_t kb = nb < D->top_k ? nb : D->top_k;
+      tiles += (int64_t)p.U * ((kb + 127) / 128);
+    }
+    if (tiles > INT32_MAX) return SALSC_ERR_UNSUPPORTED;
+    p.att_tiles = (int)tiles;
+  } else {
+    const int units = p.B * p.U;
+    int splits = (kAttendTargetCtas + units - 1) / units;
+    if (splits > 64) splits = 64;
+    int chunk = (int)((k_eff + splits - 1) / splits);
+    if (chunk < 64) chunk = 64;
+    chunk = (chunk + 15) / 16 * 16;
+    splits = (int)((k_eff + chunk - 1) / chunk);  // never more than before: chunk only grew
+    if (splits < 1) splits = 1;
+    p.splits = splits;
+    p.chunk = chunk;
+    p.att_tiles = 0;
+  }
   p.scale = D->softmax_scale != 0.0f ? D->softmax_scale : (float)(1.0 / sqrt((double)p.d));
   p.rope_base = D->rope_base;
 
@@ -91,7 +108,7 @@ salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
   p.off_qlat = off;
   off = align_up(off + sizeof(float) * (size_t)p.B * p.U * p.r, salsc::kWsAlign);
   p.off_qsplit = off;
-  off = align_up(off + sizeof(__nv_bfloat16) * (size_t)p.B * 2 * p.U * p.r, salsc::kWsAlign);
+  off = align_up(off + sizeof(__nv_bfloat16) * (size_t)p.B * p.npad * p.r, salsc::kWsAlign);
   p.off_scores = off;
   off = align_up(off + sizeof(float) * (size_t)p.N * p.U, salsc::kWsAlign);
   p.off_idx = off;

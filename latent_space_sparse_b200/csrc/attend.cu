@@ -205,45 +205,73 @@ attend_simt_kernel(const T* __restrict__ q, const T* __restrict__ Kc, const T* _
   }
 }
 
-// Merge the splits of one head and apply the deferred value projection:
-// out_h = (sum_s e^{m_s - M} acc_s / sum_s e^{m_s - M} l_s) . Pv_u^T
+// Merge the partial results of one head and apply the deferred value
+// projection:
+//   out_h = (sum_s e^{m_s - M} acc_s / sum_s e^{m_s - M} l_s) . Pv_u^T
+// Only the first ceil(k_b / chunk) slots of a head hold results.
 template <typename T>
 __global__ void __launch_bounds__(128)
 combine_kernel(const float* __restrict__ part, const T* __restrict__ Pv, T* __restrict__ out,
-               int Hq, int U, int G, int d, int r, int splits) {
+               const int64_t* __restrict__ seq_off, int Hq, int U, int G, int d, int r,
+               int splits, int chunk, int k) {
+  extern __shared__ float w_s[];  // [splits]
   __shared__ float accf[kMaxRank];
-  __shared__ float w_s[64];
   __shared__ float inv_l;
   const int bh = blockIdx.x;
-  const int h = bh % Hq, u = h / G;
+  const int b = bh / Hq, h = bh % Hq, u = h / G;
+  const int64_t nb = seq_off[b + 1] - seq_off[b];
+  const int64_t kb = nb < k ? nb : k;
+  const int ns = (int)((kb + chunk - 1) / chunk);
   const float* pp = part + (size_t)bh * splits * (r + 2);
-  if (threadIdx.x == 0) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (warp == 0) {
     float M = -INFINITY;
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, pp[(size_t)s * (r + 2)]);
+    for (int s = lane; s < ns; s += 32) M = fmaxf(M, pp[(size_t)s * (r + 2)]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float L = 0.f;
-    for (int s = 0; s < splits; ++s) {
+    for (int s = lane; s < ns; s += 32) {
       const float m = pp[(size_t)s * (r + 2)];
       const float w = (m == -INFINITY) ? 0.f : expf(m - M);
-      if (s < 64) w_s[s] = w;
+      w_s[s] = w;
       L += w * pp[(size_t)s * (r + 2) + 1];
     }
-    inv_l = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (lane == 0) inv_l = L > 0.f ? 1.f / L : 0.f;
   }
   __syncthreads();
   for (int c = threadIdx.x; c < r; c += blockDim.x) {
     float a = 0.f;
-    for (int s = 0; s < splits; ++s) a = fmaf(w_s[s], pp[(size_t)s * (r + 2) + 2 + c], a);
+    for (int s = 0; s < ns; ++s) a = fmaf(w_s[s], pp[(size_t)s * (r + 2) + 2 + c], a);
     accf[c] = a * inv_l;
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int i = warp; i < d; i += blockDim.x / 32) {
+  // one output element per thread: a dot product over its row of Pv_u
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
     const T* pv = Pv + ((size_t)u * d + i) * r;
     float a = 0.f;
-    for (int c = lane; c < r; c += 32) a = fmaf(accf[c], to_f32(pv[c]), a);
+    if (sizeof(T) == 2) {
+      for (int c0 = 0; c0 < r; c0 += 8) {
+        const uint4 v = *(const uint4*)(pv + c0);
+        const __nv_bfloat162* h2 = (const __nv_bfloat162*)&v;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-    if (lane == 0) out[(size_t)bh * d + i] = from_f32<T>(a);
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __bfloat1622float2(h2[j]);
+          a = fmaf(accf[c0 + 2 * j], f.x, a);
+          a = fmaf(accf[c0 + 2 * j + 1], f.y, a);
+        }
+      }
+    } else {
+      for (int c0 = 0; c0 < r; c0 += 4) {
+        const float4 v = *(const float4*)(pv + c0);
+        a = fmaf(accf[c0], v.x, a);
+        a = fmaf(accf[c0 + 1], v.y, a);
+        a = fmaf(accf[c0 + 2], v.z, a);
+        a = fmaf(accf[c0 + 3], v.w, a);
+      }
+    }
+    out[(size_t)bh * d + i] = from_f32<T>(a);
   }
 }
 
@@ -257,7 +285,8 @@ size_t attend_smem(const DecodePlan& p, size_t elem) {
 }  // namespace
 
 cudaError_t launch_attend(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
-  if (p.G * p.r > kAccPer * kThreads || p.splits > 64) return cudaErrorInvalidConfiguration;
+  if (p.attend_tc) return launch_attend_tc(p, a, s);
+  if (p.G * p.r > kAccPer * kThreads) return cudaErrorInvalidConfiguration;
   dim3 grid(p.splits, p.B * p.U);
   if (p.dtype == SALSC_BF16) {
     static int done[kMaxDevices] = {};
@@ -284,13 +313,22 @@ cudaError_t launch_attend(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
 }
 
 cudaError_t launch_combine(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
-  if (p.dtype == SALSC_BF16)
-    combine_kernel<__nv_bfloat16><<<p.B * p.Hq, 128, 0, s>>>(
-        a.part, (const __nv_bfloat16*)a.Pv, (__nv_bfloat16*)a.out, p.Hq, p.U, p.G, p.d, p.r,
-        p.splits);
-  else
-    combine_kernel<float><<<p.B * p.Hq, 128, 0, s>>>(a.part, (const float*)a.Pv, (float*)a.out,
-                                                     p.Hq, p.U, p.G, p.d, p.r, p.splits);
+  const size_t smem = sizeof(float) * (size_t)p.splits;
+  if (p.dtype == SALSC_BF16) {
+    static int done[kMaxDevices] = {};
+    cudaError_t e = ensure_smem(combine_kernel<__nv_bfloat16>, smem, done);
+    if (e != cudaSuccess) return e;
+    combine_kernel<__nv_bfloat16><<<p.B * p.Hq, 128, smem, s>>>(
+        a.part, (const __nv_bfloat16*)a.Pv, (__nv_bfloat16*)a.out, a.seq_off, p.Hq, p.U, p.G, p.d,
+        p.r, p.splits, p.chunk, p.k);
+  } else {
+    static int done[kMaxDevices] = {};
+    cudaError_t e = ensure_smem(combine_kernel<float>, smem, done);
+    if (e != cudaSuccess) return e;
+    combine_kernel<float><<<p.B * p.Hq, 128, smem, s>>>(a.part, (const float*)a.Pv, (float*)a.out,
+                                                       a.seq_off, p.Hq, p.U, p.G, p.d, p.r,
+                                                       p.splits, p.chunk, p.k);
+  }
   return cudaGetLastError();
 }
 

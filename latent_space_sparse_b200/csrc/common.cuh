@@ -24,14 +24,17 @@ constexpr size_t kWsAlign = 256;
 // Host-side plan of one decode layer-step, derived from the descriptor only.
 struct DecodePlan {
   int B, Hq, U, G, d, r, k;
+  int npad;             // rows of the split latent query per sequence: 2U rounded up to 16
   salsc_dtype dtype;
   int64_t N, n_max;
   int n_score_tiles;    // sum_b ceil(n_b / score tile)
   int score_tile;       // tokens per scoring CTA
   int topk_cluster;     // CTAs per selection unit in the top-k kernel
   int topk_slice;       // max keys per top-k CTA
-  int splits;           // attention CTAs per unit
-  int chunk;            // selected tokens per attention CTA
+  int splits;           // partial-result slots per head (attention CTAs or tiles per unit)
+  int chunk;            // kept tokens per slot
+  bool attend_tc;       // tensor-core attention path (tiles of 128 kept tokens)
+  int att_tiles;        // sum over units of ceil(k_b / 128) (tensor-core path)
   float scale;
   double rope_base;
   // workspace layout (byte offsets)
@@ -51,7 +54,7 @@ struct DecodeArgs {
   const int32_t* q_pos;
   uint32_t* flags;
   float* qlat;                 // [B][U][r]
-  __nv_bfloat16* qsplit;       // [B][2U][r] hi rows then lo rows
+  __nv_bfloat16* qsplit;       // [B][npad][r]: row 2u = hi(q_lat[u]), 2u+1 = lo, rest zero
   float* scores;               // packed per (b,u)
   float* part;                 // [B][Hq][splits][r+2]
 };
@@ -65,6 +68,8 @@ cudaError_t launch_score(const DecodePlan& p, const DecodeArgs& a, cudaStream_t 
 cudaError_t launch_topk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_attend(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
+bool attend_tc_supported(const DecodePlan& p);
+cudaError_t launch_attend_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_compress(const void* X, const void* P, void* Y, int64_t n, int hid, int r,
                             salsc_dtype dt, cudaStream_t s);
 
@@ -121,5 +126,36 @@ __device__ __forceinline__ void find_tile(const int64_t* __restrict__ seq_off, i
   b_out = -1;
   t0_out = 0;
 }
+
+// Walks consecutive fixed-length tiles of a ragged batch: each sequence has
+// ceil(n_b / tile_len) tiles; sequence offsets are read only when the cursor
+// enters a new sequence.
+struct TileCursor {
+  const int64_t* seq_off;
+  int B, tile_len;
+  int b;
+  int64_t t0, off, nb;
+  __device__ __forceinline__ void start(const int64_t* so, int B_, int len, int tile) {
+    seq_off = so;
+    B = B_;
+    tile_len = len;
+    find_tile(so, B_, len, tile, b, t0);
+    load();
+  }
+  __device__ __forceinline__ void load() {
+    if (b >= 0 && b < B) {
+      off = seq_off[b];
+      nb = seq_off[b + 1] - off;
+    }
+  }
+  __device__ __forceinline__ void next() {
+    t0 += tile_len;
+    if (t0 >= nb) {
+      ++b;
+      t0 = 0;
+      load();
+    }
+  }
+};
 
 }  // namespace salsc

@@ -7,8 +7,8 @@
 // by linearity) and each unit needs one latent query q_lat = qsum . Pk_u.
 //
 // Output: q_lat fp32 [B][U][r], and the same values split into bf16 hi/lo
-// parts [B][2U][r] (rows 0..U-1 = hi, U..2U-1 = lo, hi + lo = q_lat to
-// about 2^-16 relative) for the tensor-core scoring kernel.
+// parts [B][npad][r] (row 2u = hi, row 2u+1 = lo, hi + lo = q_lat to about
+// 2^-16 relative; rows 2U..npad-1 zero) for the tensor-core scoring kernel.
 #include "common.cuh"
 
 namespace salsc {
@@ -20,7 +20,8 @@ constexpr int kBatchChunk = 16;
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 latent_q_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __restrict__ qlat,
-                __nv_bfloat16* __restrict__ qsplit, int B, int Hq, int U, int G, int d, int r) {
+                __nv_bfloat16* __restrict__ qsplit, int B, int Hq, int U, int G, int d, int r,
+                int npad) {
   __shared__ float qsum[kBatchChunk * kMaxHeadDim];
   const int u = blockIdx.x;
   const int c = blockIdx.y * kThreads + threadIdx.x;
@@ -51,8 +52,12 @@ latent_q_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __rest
         qlat[((size_t)b * U + u) * r + c] = v;
         const __nv_bfloat16 hi = __float2bfloat16_rn(v);
         const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-        qsplit[((size_t)b * 2 * U + u) * r + c] = hi;
-        qsplit[((size_t)b * 2 * U + U + u) * r + c] = lo;
+        qsplit[((size_t)b * npad + 2 * u) * r + c] = hi;
+        qsplit[((size_t)b * npad + 2 * u + 1) * r + c] = lo;
+        // the padding rows are cleared by the last unit's CTAs
+        if (u == U - 1)
+          for (int row = 2 * U; row < npad; ++row)
+            qsplit[((size_t)b * npad + row) * r + c] = __float2bfloat16_rn(0.f);
       }
     }
   }
@@ -65,10 +70,11 @@ cudaError_t launch_latent_q(const DecodePlan& p, const DecodeArgs& a, cudaStream
   if (p.dtype == SALSC_BF16)
     latent_q_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(
         (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.Pk, a.qlat, a.qsplit, p.B, p.Hq, p.U,
-        p.G, p.d, p.r);
+        p.G, p.d, p.r, p.npad);
   else
     latent_q_kernel<float><<<grid, kThreads, 0, s>>>((const float*)a.q, (const float*)a.Pk, a.qlat,
-                                                     a.qsplit, p.B, p.Hq, p.U, p.G, p.d, p.r);
+                                                     a.qsplit, p.B, p.Hq, p.U, p.G, p.d, p.r,
+                                                     p.npad);
   return cudaGetLastError();
 }
 

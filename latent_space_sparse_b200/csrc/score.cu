@@ -6,7 +6,7 @@
 //
 // Scores are written fp32, packed per (b,u): unit (b,u)'s n_b scores start at
 // seq_off[b]*U + u*n_b.
-#include "common.cuh"
+#include "tc.cuh"
 
 namespace salsc {
 namespace {
@@ -55,9 +55,261 @@ score_simt_kernel(const T* __restrict__ Kc, const float* __restrict__ qlat,
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Tensor-core path (bf16 storage, r % 64 == 0, 2U <= 256).
+//
+// Per 128-token tile of one sequence: D[128 x npad] = Kc_tile[128 x r] .
+// Qs[npad x r]^T on tcgen05, where Qs holds the hi and lo bf16 parts of each
+// unit's fp32 latent query (rows 2u, 2u+1) so that hi + lo carries the query
+// to ~16 bits and the score error stays far below the top-k tie band.  Kc is
+// exact in bf16; the tensor core multiplies exactly and accumulates in fp32.
+//
+// Warp roles (192 threads): warp 0 lane 0 = TMA producer of 16 KiB Kc
+// k-blocks [128 rows x 64] into a `stages`-deep ring (plus the sequence's Qs
+// when the sequence changes); warp 1 = TMEM owner and (lane 0) MMA issuer,
+// accumulating into one of two TMEM buffers; warps 2-5 = epilogue: TMEM ->
+// registers, s_u = D[:, 2u] + D[:, 2u+1], coalesced fp32 stores.
+// Each CTA owns a contiguous range of tiles (persistent, grid <= #SMs), so
+// Qs is reloaded only at sequence boundaries.
+constexpr int kTcThreads = 192;
+constexpr int kTileM = 128;
+constexpr uint32_t kStageBytes = kTileM * 64 * 2;  // one [128 x 64] bf16 k-block
+
+struct ScoreTcParams {
+  const int64_t* seq_off;
+  float* scores;
+  uint32_t* flags;
+  int B, U, npad, r, n_tiles, stages, tmem_cols;
+};
+
+__global__ void __launch_bounds__(kTcThreads)
+score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
+                const __grid_constant__ CUtensorMap tmap_q, const ScoreTcParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const int KB = P.r / 64;
+  const int S = P.stages;
+  const uint32_t b_kblock_bytes = (uint32_t)P.npad * 128u;
+  uint8_t* a_ring = smem;
+  uint8_t* b_buf = a_ring + (size_t)S * kStageBytes;
+  uint64_t* bars = (uint64_t*)(b_buf + (size_t)KB * b_kblock_bytes);
+  uint32_t* tmem_slot = (uint32_t*)(bars + 2 * S + 6);
+  const uint32_t bar0 = tc::smem_u32(bars);
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 8u * (S + s); };
+  const uint32_t bfull = bar0 + 8u * (2 * S), bempty = bar0 + 8u * (2 * S + 1);
+  auto tfull = [&](int a) { return bar0 + 8u * (2 * S + 2 + a); };
+  auto tempty = [&](int a) { return bar0 + 8u * (2 * S + 4 + a); };
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int t_begin = (int)((int64_t)blockIdx.x * P.n_tiles / gridDim.x);
+  const int t_end = (int)((int64_t)(blockIdx.x + 1) * P.n_tiles / gridDim.x);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      tc::mbar_init(full(s), 1);
+      tc::mbar_init(empty(s), 1);
+    }
+    tc::mbar_init(bfull, 1);
+    tc::mbar_init(bempty, 1);
+    for (int a = 0; a < 2; ++a) {
+      tc::mbar_init(tfull(a), 1);
+      tc::mbar_init(tempty(a), 128);
+    }
+    tc::mbar_fence_init();
+    tc::tma_prefetch_desc(&tmap_kc);
+    tc::tma_prefetch_desc(&tmap_q);
+  }
+  if (warp == 1) tc::tmem_alloc(tc::smem_u32(tmem_slot), (uint32_t)P.tmem_cols);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    uint32_t it = 0, bpar = 0;
+    int cur_b = -1;
+    bool ok = true;
+    TileCursor cur;
+    cur.start(P.seq_off, P.B, kTileM, t_begin);
+    for (int tile = t_begin; tile < t_end && ok; ++tile, cur.next()) {
+      const int b = cur.b;
+      if (b != cur_b) {
+        if (cur_b >= 0) {
+          ok = tc::mbar_wait(bempty, bpar, P.flags);
+          bpar ^= 1u;
+          if (!ok) break;
+        }
+        tc::mbar_expect_tx(bfull, (uint32_t)KB * b_kblock_bytes);
+        for (int kb = 0; kb < KB; ++kb)
+          tc::tma_load_2d(tc::smem_u32(b_buf + (size_t)kb * b_kblock_bytes), &tmap_q, kb * 64,
+                          b * P.npad, bfull);
+        cur_b = b;
+      }
+      const int row0 = (int)(cur.off + cur.t0);
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const int s = (int)(it % (uint32_t)S);
+        const uint32_t ph = (it / (uint32_t)S) & 1u;
+        if (!tc::mbar_wait(empty(s), ph ^ 1u, P.flags)) {
+          ok = false;
+          break;
+        }
+        tc::mbar_expect_tx(full(s), kStageBytes);
+        tc::tma_load_2d(tc::smem_u32(a_ring + (size_t)s * kStageBytes), &tmap_kc, kb * 64, row0,
+                        full(s));
+      }
+    }
+    // every issued load has landed before the CTA may exit
+    for (uint32_t j = it > (uint32_t)S ? it - (uint32_t)S : 0u; j < it; ++j)
+      tc::mbar_wait(full((int)(j % (uint32_t)S)), (j / (uint32_t)S) & 1u, P.flags);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    const uint32_t idesc = tc::idesc_bf16_f32(kTileM, P.npad);
+    uint32_t it = 0, bpar = 0;
+    int cur_b = -1, nseq = 0, i = 0;
+    bool ok = true;
+    TileCursor cur;
+    cur.start(P.seq_off, P.B, kTileM, t_begin);
+    for (int tile = t_begin; tile < t_end && ok; ++tile, ++i, cur.next()) {
+      const int b = cur.b;
+      if (b != cur_b) {
+        if (!tc::mbar_wait(bfull, bpar, P.flags)) break;
+        bpar ^= 1u;
+        cur_b = b;
+        ++nseq;
+      }
+      const int acc = i & 1;
+      if (!tc::mbar_wait(tempty(acc), (((uint32_t)i >> 1) & 1u) ^ 1u, P.flags)) break;
+      tc::fence_after_sync();
+      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * P.npad);
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const int s = (int)(it % (uint32_t)S);
+        const uint32_t ph = (it / (uint32_t)S) & 1u;
+        if (!tc::mbar_wait(full(s), ph, P.flags)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t a_addr = tc::smem_u32(a_ring + (size_t)s * kStageBytes);
+        const uint32_t b_addr = tc::smem_u32(b_buf + (size_t)kb * b_kblock_bytes);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          tc::mma_bf16(d_tmem, tc::sdesc_kmajor_sw128(a_addr + 32u * k),
+                       tc::sdesc_kmajor_sw128(b_addr + 32u * k), idesc, (kb | k) != 0);
+        tc::mma_commit(empty(s));
+      }
+      if (!ok) break;
+      tc::mma_commit(tfull(acc));
+      // last tile of this sequence in the CTA's range: the sequence's Qs is then free
+      const bool last_of_seq = tile + 1 == t_end || cur.t0 + kTileM >= cur.nb;
+      if (last_of_seq) tc::mma_commit(bempty);
+    }
+    // the last release of Qs lands before the CTA may exit
+    if (ok && nseq > 0) tc::mbar_wait(bempty, (uint32_t)(nseq - 1) & 1u, P.flags);
+  } else if (warp >= 2) {
+    // ---------------- epilogue: TMEM -> scores
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    int i = 0;
+    TileCursor cur;
+    cur.start(P.seq_off, P.B, kTileM, t_begin);
+    for (int tile = t_begin; tile < t_end; ++tile, ++i, cur.next()) {
+      const int acc = i & 1;
+      // warp-uniform wait: the TMEM loads below need a converged warp
+      const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(tfull(acc), ((uint32_t)i >> 1) & 1u,
+                                                            P.flags));
+      if (!ok) break;
+      tc::fence_after_sync();
+      const int64_t off = cur.off;
+      const int64_t nb = cur.nb;
+      const int64_t t = cur.t0 + row;
+      float* sbase = P.scores + off * P.U + t;
+      for (int c0 = 0; c0 < 2 * P.U; c0 += 16) {
+        uint32_t v[16];
+        tc::tmem_ld16(lane_addr + (uint32_t)(acc * P.npad + c0), v);
+        tc::tmem_ld_wait();
+        if (t < nb) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int u = c0 / 2 + j;
+            if (u < P.U) sbase[(int64_t)u * nb] = __uint_as_float(v[2 * j]) + __uint_as_float(v[2 * j + 1]);
+          }
+        }
+      }
+      tc::fence_before_sync();
+      tc::mbar_arrive(tempty(acc));
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem_base, (uint32_t)P.tmem_cols);
+  }
+}
+
+int num_sms() {
+  static int cached[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
+cudaError_t launch_score_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
+  const int KB = p.r / 64;
+  const size_t b_bytes = (size_t)KB * p.npad * 128;
+  // Small query blocks (GQA): two CTAs per SM with a 4-deep ring each; large
+  // ones (MHA, 64 KiB of Qs) one CTA per SM with an 8-deep ring.
+  int stages, ctas_per_sm;
+  if (b_bytes <= 16384) {
+    stages = 4;
+    ctas_per_sm = 2;
+  } else {
+    stages = (int)((200u * 1024u - b_bytes) / kStageBytes);
+    if (stages > 8) stages = 8;
+    ctas_per_sm = 1;
+  }
+  if (stages < 2) return cudaErrorInvalidConfiguration;
+  const size_t smem = 1024 + (size_t)stages * kStageBytes + b_bytes + (2 * stages + 6) * 8 + 16;
+  CUtensorMap tk, tq;
+  if (!make_tmap_bf16_2d(&tk, a.Kc, (uint64_t)p.N, (uint64_t)p.r, kTileM, 64) ||
+      !make_tmap_bf16_2d(&tq, a.qsplit, (uint64_t)p.B * p.npad, (uint64_t)p.r, p.npad, 64))
+    return cudaErrorInvalidValue;
+  static int done[kMaxDevices] = {};
+  cudaError_t e = ensure_smem(score_tc_kernel, smem, done);
+  if (e != cudaSuccess) return e;
+  ScoreTcParams P;
+  P.seq_off = a.seq_off;
+  P.scores = a.scores;
+  P.flags = a.flags;
+  P.B = p.B;
+  P.U = p.U;
+  P.npad = p.npad;
+  P.r = p.r;
+  P.n_tiles = p.n_score_tiles;
+  P.stages = stages;
+  int cols = 32;
+  while (cols < 2 * p.npad) cols *= 2;
+  P.tmem_cols = cols;
+  const int max_ctas = num_sms() * ctas_per_sm;
+  const int grid = p.n_score_tiles < max_ctas ? p.n_score_tiles : max_ctas;
+  score_tc_kernel<<<grid, kTcThreads, smem, s>>>(tk, tq, P);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_score(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
+  if (p.dtype == SALSC_BF16 && p.r % 64 == 0 && p.npad <= 256) return launch_score_tc(p, a, s);
   const size_t smem = sizeof(float) * (size_t)p.U * p.r;
   if (p.dtype == SALSC_BF16) {
     static int done[kMaxDevices] = {};
