@@ -243,6 +243,7 @@ combine_kernel(const float* __restrict__ part, const T* __restrict__ Pv, T* __re
   __syncthreads();
   for (int c = threadIdx.x; c < r; c += blockDim.x) {
     float a = 0.f;
+#pragma unroll 8
     for (int s = 0; s < ns; ++s) a = fmaf(w_s[s], pp[(size_t)s * (r + 2) + 2 + c], a);
     accf[c] = a * inv_l;
   }
@@ -252,6 +253,7 @@ combine_kernel(const float* __restrict__ part, const T* __restrict__ Pv, T* __re
     const T* pv = Pv + ((size_t)u * d + i) * r;
     float a = 0.f;
     if (sizeof(T) == 2) {
+#pragma unroll 8
       for (int c0 = 0; c0 < r; c0 += 8) {
         const uint4 v = *(const uint4*)(pv + c0);
         const __nv_bfloat162* h2 = (const __nv_bfloat162*)&v;
@@ -263,6 +265,7 @@ combine_kernel(const float* __restrict__ part, const T* __restrict__ Pv, T* __re
         }
       }
     } else {
+#pragma unroll 8
       for (int c0 = 0; c0 < r; c0 += 4) {
         const float4 v = *(const float4*)(pv + c0);
         a = fmaf(accf[c0], v.x, a);

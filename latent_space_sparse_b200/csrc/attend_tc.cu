@@ -1,37 +1,50 @@
-// attend_tc.cu -- selective reconstruction on tcgen05, RoPE, softmax and the
-// latent value sum over the kept tokens (bf16 storage, d in {64, 128},
+// attend_tc.cu -- selective reconstruction, RoPE, softmax and the latent
+// value sum over the kept tokens, on tcgen05 (bf16 storage, d in {64, 128},
 // r <= 256, G in {1, 2, 4, 8}).
 //
-// SALS technical framework, stages 3-4, with RoPE after reconstruction
-// (abstract).  Work unit: a tile of 128 kept tokens of one selection unit
-// (b, u).  For each tile:
-//   1. gather the 128 latent key rows Kc_b[idx] into shared memory in the
-//      128-byte-swizzled K-major layout (cp.async, 16 B per copy);
-//   2. K_sel[128 x d] = Kc_tile . Pk_u^T on tcgen05 into TMEM (fp32; Pk_u is
-//      loaded once per unit by TMA and stays in shared memory);
-//   3. one thread per token row reads its K_sel row from TMEM, rotates each
-//      pair (i, i+d/2) by t * base^(-2i/d) (angle reduced modulo 2 pi in fp64)
-//      and dots it with each rotated query head of the unit;
-//   4. softmax inside the tile (max m and normaliser l per head);
-//   5. the tile's latent value rows Vc_b[idx] are gathered into the buffer the
-//      MMA has finished with, and acc[r] = sum_t p_t Vc_b[t] is formed on the
-//      CUDA cores in fp32.
-// Each tile writes its own (m, l, acc) per head; the combine kernel merges
-// the tiles of a unit and applies Pv_u^T.  The Kc gather of the next tile
-// and the Vc gather of the current one overlap steps 3-4.
+// SALS technical framework, stages 3-4, with RoPE applied after
+// reconstruction (abstract).  Work unit: a tile of 128 kept tokens of one
+// selection unit (b, u):
+//   1. TMA gather4 brings the 128 latent key rows Kc_b[idx] into shared memory
+//      (128-byte swizzled, K-major);
+//   2. tcgen05: K_sel[128 x d] = Kc_tile . Pk_u^T into TMEM (fp32; Pk_u comes
+//      by TMA once per unit and stays in shared memory);
+//   3. the same rows of Vc are gathered into the buffer the MMA has finished
+//      with;
+//   4. eight epilogue warps (one thread per token row and half of the RoPE
+//      pairs) read K_sel from TMEM, rotate pair (i, i+d/2) by the angle
+//      t * base^(-2i/d) and dot it with every rotated query head of the unit;
+//      the tile's softmax (max m, normaliser l) follows, and the weights p are
+//      written to shared memory as bf16 hi + lo parts;
+//   5. tcgen05: acc^T[r x 2G] = Vc_tile^T . [p_hi p_lo] into TMEM (Vc_tile read
+//      as an MN-major operand, so the latent value rows need no transpose);
+//   6. the epilogue reads acc[c] = D[c][2g] + D[c][2g+1] and writes the
+//      tile's (m, l, acc) per head; the combine kernel merges tiles.
+// Warp roles (320 threads): warps 0-7 epilogue, warp 8 TMEM owner and MMA
+// issuer, warp 9 gather issuer.  Each CTA walks a contiguous range of tiles;
+// the two tile buffers alternate (Kc(i) -> Vc(i) -> Kc(i+2)), so the
+// reconstruction of tile i+1 runs during the epilogue of tile i.
+//
+// The RoPE angle uses an exact fixed-point phase: F_i = round(2^64 *
+// theta_i / 2 pi), and the top 32 bits of t * F_i (mod 2^64) are t * theta_i
+// modulo one turn, to 2^-32 of a turn, for any 32-bit position t.
 #include "tc.cuh"
 
 namespace salsc {
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
+constexpr int kThreads = 320;
 constexpr int kTile = 128;
+constexpr int kPRows = 16;  // rows of the p operand (2G <= 16)
+constexpr uint32_t kEpiBar = 1;
 constexpr double kTwoPi = 6.283185307179586476925286766559;
 
 struct AttendTcParams {
   const __nv_bfloat16* q;
-  const __nv_bfloat16* Kc;
-  const __nv_bfloat16* Vc;
   const int32_t* idx;
   const int64_t* seq_off;
   const int32_t* q_pos;
@@ -83,280 +96,386 @@ struct UnitTileCursor {
   }
 };
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
+struct Smem {
+  uint8_t* pk;       // Pk_u: KB k-blocks of [D rows x 128 B]
+  uint8_t* buf[2];   // tile buffers: KB k-blocks of [128 rows x 128 B]
+  uint8_t* pbuf[2];  // p operand: 2 k-blocks of [16 rows x 128 B]
+  uint64_t* fturn;   // [D/2] fixed-point turns per token position
+  double* theta;     // [D/2]
+  float* qr;         // [G][D] rotated queries
+  float* pd;         // [2][G][128] partial dot products of the two pair halves
+  float* lg;         // [G][128] logits, then softmax weights
+  float* stat;       // [G][2] (m, l)
+  int* tok;          // [2][128] token index per row (-1: no token), gather warp only
+  uint64_t* bars;
+  uint32_t* tmem_slot;
+};
 
-// Byte offset of element column c of row m in a [128 x r] tile stored as
-// r/64 k-blocks of [128 rows x 128 B] with the 128-byte swizzle.
-__device__ __forceinline__ uint32_t swz_offset(int m, int c) {
-  const int kb = c >> 6, chunk = (c >> 3) & 7;
-  return (uint32_t)(kb * 16384 + (m >> 3) * 1024 + (m & 7) * 128 + ((chunk ^ (m & 7)) << 4) +
-                    (c & 7) * 2);
-}
-
-// Copy the rows tok[0..127] of `src` ([N][r] bf16, rows relative to `off`)
-// into `buf`; rows with tok < 0 are zero-filled.  Thread e copies 16-byte
-// chunks e, e+128, ...: consecutive threads cover consecutive bytes of a row.
-__device__ __forceinline__ void gather_rows(uint8_t* buf, const __nv_bfloat16* src, int64_t off,
-                                            const int* tok, int r) {
-  const int cpr = r / 8;  // 16-byte chunks per row
-  const uint32_t base = tc::smem_u32(buf);
-  for (int e = threadIdx.x; e < kTile * cpr; e += kThreads) {
-    const int m = e / cpr, cc = e % cpr;
-    const int t = tok[m];
-    const __nv_bfloat16* s = t >= 0 ? src + (off + t) * r + cc * 8 : src;
-    cp_async16(base + swz_offset(m, cc * 8), s, t >= 0 ? 16u : 0u);
-  }
-  cp_async_commit();
-}
+// barrier indices
+enum { B_PK = 0, B_KFULL = 1, B_VFULL = 3, B_KDONE = 5, B_PDONE = 7, B_PREADY = 9,
+       B_TKFREE = 11, B_TOFREE = 13, B_COUNT = 15 };
 
 template <int G, int D>
 __global__ void __launch_bounds__(kThreads, 1)
-attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk, const AttendTcParams P) {
+attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
+                 const __grid_constant__ CUtensorMap tmap_kc,
+                 const __grid_constant__ CUtensorMap tmap_vc, const AttendTcParams P) {
   constexpr int HALF = D / 2;
+  constexpr int QPAIRS = HALF / 2;  // RoPE pairs per epilogue thread
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int KB = P.r / 64;
+  const int n_chunks = (P.r + 127) / 128;  // M = 128 slices of the latent width
   const uint32_t pk_bytes = (uint32_t)KB * D * 128;
   const uint32_t buf_bytes = (uint32_t)KB * 16384;
-  uint8_t* pk = smem;
-  uint8_t* bufs[2] = {pk + pk_bytes, pk + pk_bytes + buf_bytes};
-  double* theta = (double*)(pk + pk_bytes + 2 * buf_bytes);
-  float* qr = (float*)(theta + HALF);     // [G][D]
-  float* lg = qr + G * D;                 // [G][128]
-  float* stat = lg + G * kTile;           // [G][2]
-  int* tok = (int*)(stat + 2 * G);        // [2][128]
-  uint64_t* bars = (uint64_t*)(((uintptr_t)(tok + 2 * kTile) + 7) & ~(uintptr_t)7);
-  uint32_t* tmem_slot = (uint32_t*)(bars + 2);
-  const uint32_t pk_full = tc::smem_u32(bars), mma_done = pk_full + 8;
+  Smem S;
+  S.pk = base;
+  S.buf[0] = base + pk_bytes;
+  S.buf[1] = S.buf[0] + buf_bytes;
+  S.pbuf[0] = S.buf[1] + buf_bytes;
+  S.pbuf[1] = S.pbuf[0] + 4096;
+  S.fturn = (uint64_t*)(S.pbuf[1] + 4096);
+  S.theta = (double*)(S.fturn + HALF);
+  S.qr = (float*)(S.theta + HALF);
+  S.pd = S.qr + G * D;
+  S.lg = S.pd + 2 * G * kTile;
+  S.stat = S.lg + G * kTile;
+  S.tok = (int*)(S.stat + 2 * G);
+  S.bars = (uint64_t*)(((uintptr_t)(S.tok + 2 * kTile) + 7) & ~(uintptr_t)7);
+  S.tmem_slot = (uint32_t*)(S.bars + B_COUNT);
+  const uint32_t bar0 = tc::smem_u32(S.bars);
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int t_begin = (int)((int64_t)blockIdx.x * P.n_tiles / gridDim.x);
   const int t_end = (int)((int64_t)(blockIdx.x + 1) * P.n_tiles / gridDim.x);
+  const int n = t_end - t_begin;
+  // TMEM columns: K_sel [2][D], then acc [2][n_chunks * 16]
+  const uint32_t o_col0 = 2 * D;
+  const uint32_t o_cols = (uint32_t)n_chunks * 16;
 
   if (tid == 0) {
-    tc::mbar_init(pk_full, 1);
-    tc::mbar_init(mma_done, 1);
+    for (int i = 0; i < B_COUNT; ++i) tc::mbar_init(bar(i), 1);
     tc::mbar_fence_init();
     tc::tma_prefetch_desc(&tmap_pk);
+    tc::tma_prefetch_desc(&tmap_kc);
+    tc::tma_prefetch_desc(&tmap_vc);
   }
-  if (warp == 0) tc::tmem_alloc(tc::smem_u32(tmem_slot), 2 * D);
-  for (int i = tid; i < HALF; i += kThreads) theta[i] = pow(P.base, -2.0 * (double)i / (double)D);
+  if (warp == kMmaWarp) tc::tmem_alloc(tc::smem_u32(S.tmem_slot), 512);
+  for (int i = tid; i < HALF; i += kThreads) {
+    const double th = pow(P.base, -2.0 * (double)i / (double)D);
+    S.theta[i] = th;
+    S.fturn[i] = __double2ull_rn(th / kTwoPi * 18446744073709551616.0);
+  }
+  // the p operand's unused rows (2G..15) stay zero
+  for (int e = tid; e < 2 * 4096 / 4; e += kThreads) ((uint32_t*)S.pbuf[0])[e] = 0u;
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  const uint32_t tmem_base = *tmem_slot;
-  const uint32_t idesc = tc::idesc_bf16_f32(kTile, D);
+  const uint32_t tmem_base = *S.tmem_slot;
 
-  // token index of every row of a tile (thread m = row m), then the gather
-  auto prepare_tok = [&](const UnitTileCursor& c, int* tk) {
-    const int64_t j = (int64_t)c.slot * kTile + tid;
-    int t = -1;
-    if (j < c.kb) {
-      t = P.idx[((int64_t)c.b * P.U + c.u) * P.k + j];
-      if (t < 0 || t >= c.nb) {
-        atomicOr(P.flags, FLAG_BAD_INDEX);
-        t = -1;
+  if (warp == kLoadWarp) {
+    // ======================= gather issuer (all 32 lanes) ======================
+    // Lane l owns rows 4l..4l+3 of every tile: it resolves their token indices
+    // and issues the gather4 copies of those rows for every k-block.
+    UnitTileCursor cur;
+    cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
+    UnitTileCursor ahead = cur;  // tile i+2 when loading Kc(i+2)
+    auto issue = [&](const UnitTileCursor& c, int bi, const CUtensorMap* map, int b_full,
+                     bool resolve) {
+      int rows[4];
+      int* tk = S.tok + bi * kTile;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int m = 4 * lane + j;
+        int t;
+        if (resolve) {
+          const int64_t jj = (int64_t)c.slot * kTile + m;
+          t = -1;
+          if (jj < c.kb) {
+            t = P.idx[((int64_t)c.b * P.U + c.u) * P.k + jj];
+            if (t < 0 || t >= c.nb) {
+              atomicOr(P.flags, FLAG_BAD_INDEX);
+              t = -1;
+            }
+          }
+          tk[m] = t;
+        } else {
+          t = tk[m];
+        }
+        // rows without a token read the sequence's first row; their weight is 0
+        rows[j] = (int)(c.off + (t < 0 ? 0 : t));
+      }
+      if (lane == 0) tc::mbar_expect_tx(bar(b_full + bi), (uint32_t)kTile * P.r * 2);
+      __syncwarp();
+      const uint32_t dst0 = tc::smem_u32(S.buf[bi]) + (uint32_t)(lane >> 1) * 1024u +
+                            (uint32_t)(lane & 1) * 512u;
+      for (int kb = 0; kb < KB; ++kb)
+        tc::tma_gather4(dst0 + kb * 16384u, map, kb * 64, rows[0], rows[1], rows[2], rows[3],
+                        bar(b_full + bi));
+    };
+    for (int i = 0; i < 2 && i < n; ++i) {
+      issue(ahead, i, &tmap_kc, B_KFULL, true);
+      ahead.next();
+    }
+    bool ok = true;
+    for (int i = 0; i < n && ok; ++i, cur.next()) {
+      const int bi = i & 1;
+      const uint32_t ph = ((uint32_t)i >> 1) & 1u;
+      // the reconstruction is done with Kc(i): bring Vc(i) into the same buffer
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(B_KDONE + bi), ph, P.flags));
+      if (!ok) break;
+      issue(cur, bi, &tmap_vc, B_VFULL, false);
+      if (i + 2 < n) {
+        // the value MMA is done with Vc(i): bring Kc(i+2)
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(B_PDONE + bi), ph, P.flags));
+        if (!ok) break;
+        issue(ahead, bi, &tmap_kc, B_KFULL, true);
+        ahead.next();
       }
     }
-    tk[tid] = t;
-    __syncthreads();
-  };
-
-  UnitTileCursor cur, nxt;
-  cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
-  nxt = cur;
-  if (t_begin < t_end) {
-    prepare_tok(cur, tok);
-    gather_rows(bufs[0], P.Kc, cur.off, tok, P.r);
-  }
-  int cur_b = -1, cur_u = -1;
-  uint32_t pk_phase = 0, mma_phase = 0;
-  bool ok = true;
-  for (int i = 0; t_begin + i < t_end && ok; ++i, cur.next()) {
-    const int bi = i & 1;
-    int* tk = tok + bi * kTile;
-    // ---- new unit: Pk_u by TMA, rotated queries of the unit's heads
-    const bool new_unit = cur.b != cur_b || cur.u != cur_u;
-    if (new_unit) {
-      if (tid == 0) {
-        tc::mbar_expect_tx(pk_full, pk_bytes);
-        for (int kb = 0; kb < KB; ++kb)
-          tc::tma_load_2d(tc::smem_u32(pk + (size_t)kb * D * 128), &tmap_pk, kb * 64, cur.u * D,
-                          pk_full);
-      }
-      const double qpos = P.q_pos ? (double)P.q_pos[cur.b] : (double)cur.nb;
-      for (int e = tid; e < G * HALF; e += kThreads) {
-        const int g = e / HALF, ii = e % HALF;
-        const __nv_bfloat16* qh = P.q + ((int64_t)cur.b * P.Hq + cur.u * G + g) * D;
-        const double a = qpos * theta[ii];
-        const double n = rint(a * (1.0 / kTwoPi));
-        float s, c;
-        sincosf((float)fma(-n, kTwoPi, a), &s, &c);
-        const float x0 = __bfloat162float(qh[ii]), x1 = __bfloat162float(qh[ii + HALF]);
-        qr[g * D + ii] = x0 * c - x1 * s;
-        qr[g * D + ii + HALF] = x1 * c + x0 * s;
-      }
-      cur_b = cur.b;
-      cur_u = cur.u;
-    }
-    // ---- Kc tile of this step has landed
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
-    __syncthreads();
-    // ---- K_sel = Kc_tile . Pk_u^T on the tensor cores
-    if (tid == 0) {
-      bool ready = true;
-      if (new_unit) {
-        ready = tc::mbar_wait(pk_full, pk_phase, P.flags);
-        pk_phase ^= 1u;
-      }
-      if (ready) {
+  } else if (warp == kMmaWarp) {
+    // ======================= MMA issuer (lane 0) =======================
+    if (lane == 0) {
+      const uint32_t idesc_k = tc::idesc_bf16_f32(kTile, D);
+      const uint32_t idesc_v = tc::idesc_bf16_f32_amn(128, kPRows);
+      UnitTileCursor cur;
+      cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
+      int cur_b = -1, cur_u = -1;
+      uint32_t pk_phase = 0;
+      bool ok = true;
+      auto issue_pv = [&](int j) -> bool {
+        const int bj = j & 1;
+        const uint32_t ph = ((uint32_t)j >> 1) & 1u;
+        if (!tc::mbar_wait(bar(B_PREADY + bj), ph, P.flags)) return false;
+        if (!tc::mbar_wait(bar(B_VFULL + bj), ph, P.flags)) return false;
+        if (!tc::mbar_wait(bar(B_TOFREE + bj), ph ^ 1u, P.flags)) return false;
         tc::fence_after_sync();
-        const uint32_t a0 = tc::smem_u32(bufs[bi]), b0 = tc::smem_u32(pk);
-        const uint32_t d_tmem = tmem_base + (uint32_t)(bi * D);
+        const uint32_t v0 = tc::smem_u32(S.buf[bj]), p0 = tc::smem_u32(S.pbuf[bj]);
+        for (int ch = 0; ch < n_chunks; ++ch) {
+          const uint32_t d_tmem = tmem_base + o_col0 + (uint32_t)bj * o_cols + (uint32_t)ch * 16;
+#pragma unroll
+          for (int ks = 0; ks < kTile / 16; ++ks) {
+            // A = Vc_tile^T: latent columns ch*128.. (MN), tokens ks*16.. (K)
+            const uint64_t ad = tc::sdesc_mnmajor_sw128(
+                v0 + (uint32_t)ch * 2 * 16384 + (uint32_t)(ks * 2) * 1024, 16384, 1024);
+            // B = p rows (hi/lo per head), tokens ks*16..: K-major k-block ks/4
+            const uint64_t bd =
+                tc::sdesc_kmajor_sw128(p0 + (uint32_t)(ks >> 2) * 2048 + (uint32_t)(ks & 3) * 32);
+            tc::mma_bf16(d_tmem, ad, bd, idesc_v, ks != 0);
+          }
+        }
+        tc::mma_commit(bar(B_PDONE + bj));
+        return true;
+      };
+      for (int i = 0; i < n && ok; ++i, cur.next()) {
+        const int bi = i & 1;
+        const uint32_t ph = ((uint32_t)i >> 1) & 1u;
+        if (cur.b != cur_b || cur.u != cur_u) {
+          // Pk_u of the new unit; the previous reconstruction must be done with Pk
+          if (i > 0 &&
+              !tc::mbar_wait(bar(B_KDONE + ((i - 1) & 1)), ((uint32_t)(i - 1) >> 1) & 1u,
+                             P.flags)) {
+            ok = false;
+            break;
+          }
+          tc::mbar_expect_tx(bar(B_PK), pk_bytes);
+          for (int kb = 0; kb < KB; ++kb)
+            tc::tma_load_2d(tc::smem_u32(S.pk + (size_t)kb * D * 128), &tmap_pk, kb * 64,
+                            cur.u * D, bar(B_PK));
+          if (!tc::mbar_wait(bar(B_PK), pk_phase, P.flags)) {
+            ok = false;
+            break;
+          }
+          pk_phase ^= 1u;
+          cur_b = cur.b;
+          cur_u = cur.u;
+        }
+        if (!tc::mbar_wait(bar(B_KFULL + bi), ph, P.flags) ||
+            !tc::mbar_wait(bar(B_TKFREE + bi), ph ^ 1u, P.flags)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t a0 = tc::smem_u32(S.buf[bi]), b0 = tc::smem_u32(S.pk);
+        const uint32_t d_tmem = tmem_base + (uint32_t)bi * D;
         for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             tc::mma_bf16(d_tmem, tc::sdesc_kmajor_sw128(a0 + kb * 16384 + 32 * k),
-                         tc::sdesc_kmajor_sw128(b0 + kb * D * 128 + 32 * k), idesc,
+                         tc::sdesc_kmajor_sw128(b0 + kb * D * 128 + 32 * k), idesc_k,
                          (kb | k) != 0);
-        tc::mma_commit(mma_done);
-      } else {
-        tc::mbar_arrive(mma_done);  // release the waiters; the flag reports the failure
+        tc::mma_commit(bar(B_KDONE + bi));
+        if (i > 0 && !issue_pv(i - 1)) ok = false;
       }
+      if (ok && n > 0) issue_pv(n - 1);
     }
-    ok = __syncthreads_and(tc::mbar_wait(mma_done, mma_phase, P.flags));
-    mma_phase ^= 1u;
-    if (!ok) break;
-    tc::fence_after_sync();
-    // ---- the MMA is done with the Kc tile: gather the same rows of Vc into it,
-    //      and the next tile's Kc rows into the other buffer
-    gather_rows(bufs[bi], P.Vc, cur.off, tk, P.r);
-    const bool has_next = t_begin + i + 1 < t_end;
-    if (has_next) {
-      nxt = cur;
-      nxt.next();
-      prepare_tok(nxt, tok + (bi ^ 1) * kTile);
-      gather_rows(bufs[bi ^ 1], P.Kc, nxt.off, tok + (bi ^ 1) * kTile, P.r);
-    }
-    // ---- logits: one thread per kept token (TMEM lane = row)
-    {
-      const int t = tk[tid];
+  } else {
+    // ======================= epilogue (warps 0-7) =======================
+    const int quarter = warp & 3, half = warp >> 2;
+    const int m = quarter * 32 + lane;  // token row = TMEM lane
+    UnitTileCursor cur;
+    cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
+    int cur_b = -1, cur_u = -1;
+    for (int i = 0; i < n; ++i, cur.next()) {
+      const int bi = i & 1;
+      const uint32_t ph = ((uint32_t)i >> 1) & 1u;
+      if (cur.b != cur_b || cur.u != cur_u) {
+        // rotated queries of the unit's heads (angles reduced in fp64)
+        const double qpos = P.q_pos ? (double)P.q_pos[cur.b] : (double)cur.nb;
+        for (int e = tid; e < G * HALF; e += kEpiThreads) {
+          const int g = e / HALF, ii = e % HALF;
+          const __nv_bfloat16* qh = P.q + ((int64_t)cur.b * P.Hq + cur.u * G + g) * D;
+          const double a = qpos * S.theta[ii];
+          const double nt = rint(a * (1.0 / kTwoPi));
+          float s, c;
+          sincosf((float)fma(-nt, kTwoPi, a), &s, &c);
+          const float x0 = __bfloat162float(qh[ii]), x1 = __bfloat162float(qh[ii + HALF]);
+          S.qr[g * D + ii] = x0 * c - x1 * s;
+          S.qr[g * D + ii + HALF] = x1 * c + x0 * s;
+        }
+        cur_b = cur.b;
+        cur_u = cur.u;
+        tc::named_sync(kEpiBar, kEpiThreads);
+      }
+      // ---- K_sel row m, pairs [half*QPAIRS, (half+1)*QPAIRS)
+      const bool ok =
+          __all_sync(0xffffffffu, tc::mbar_wait(bar(B_KDONE + bi), ph, P.flags));
+      tc::fence_after_sync();
+      // this row's token (resolved again here rather than read from the
+      // gather warp's table, so no cross-warp ordering is needed)
+      int t = -1;
+      {
+        const int64_t jj = (int64_t)cur.slot * kTile + m;
+        if (jj < cur.kb) {
+          t = P.idx[((int64_t)cur.b * P.U + cur.u) * P.k + jj];
+          if (t < 0 || t >= cur.nb) t = -1;
+        }
+      }
       float dot[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) dot[g] = 0.f;
-      const uint32_t row_addr = tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(bi * D);
-      const double pos = (double)(t < 0 ? 0 : t);
+      if (ok) {
+        const uint32_t row_addr =
+            tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)bi * D;
+        const uint32_t tu = (uint32_t)(t < 0 ? 0 : t);
 #pragma unroll 1
-      for (int i0 = 0; i0 < HALF; i0 += 16) {
-        uint32_t v0[16], v1[16];
-        tc::tmem_ld16(row_addr + i0, v0);
-        tc::tmem_ld16(row_addr + HALF + i0, v1);
-        tc::tmem_ld_wait();
+        for (int i0 = half * QPAIRS; i0 < (half + 1) * QPAIRS; i0 += 16) {
+          uint32_t v0[16], v1[16];
+          tc::tmem_ld16(row_addr + i0, v0);
+          tc::tmem_ld16(row_addr + HALF + i0, v1);
+          tc::tmem_ld_wait();
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const int ii = i0 + jj;
-          const double a = pos * theta[ii];
-          const double n = rint(a * (1.0 / kTwoPi));
-          float s, c;
-          __sincosf((float)fma(-n, kTwoPi, a), &s, &c);
-          const float x0 = __uint_as_float(v0[jj]), x1 = __uint_as_float(v1[jj]);
-          const float k0 = x0 * c - x1 * s;
-          const float k1 = x1 * c + x0 * s;
+          for (int jj = 0; jj < 16; ++jj) {
+            const int ii = i0 + jj;
+            const uint64_t F = S.fturn[ii];
+            const uint32_t turn = __umulhi(tu, (uint32_t)F) + tu * (uint32_t)(F >> 32);
+            float s, c;
+            __sincosf((float)(int32_t)turn * (float)(kTwoPi / 4294967296.0), &s, &c);
+            const float x0 = __uint_as_float(v0[jj]), x1 = __uint_as_float(v1[jj]);
+            const float k0 = x0 * c - x1 * s;
+            const float k1 = x1 * c + x0 * s;
 #pragma unroll
-          for (int g = 0; g < G; ++g)
-            dot[g] = fmaf(qr[g * D + ii], k0, fmaf(qr[g * D + ii + HALF], k1, dot[g]));
+            for (int g = 0; g < G; ++g)
+              dot[g] = fmaf(S.qr[g * D + ii], k0, fmaf(S.qr[g * D + ii + HALF], k1, dot[g]));
+          }
         }
       }
 #pragma unroll
-      for (int g = 0; g < G; ++g) lg[g * kTile + tid] = t >= 0 ? dot[g] * P.scale : -INFINITY;
-    }
-    tc::fence_before_sync();
-    __syncthreads();
-    // ---- softmax inside the tile: warp w takes heads w, w+4, ...
-    for (int g = warp; g < G; g += kThreads / 32) {
-      float v[4], mx = -INFINITY;
+      for (int g = 0; g < G; ++g) S.pd[(half * G + g) * kTile + m] = dot[g];
+      tc::fence_before_sync();
+      tc::named_sync(kEpiBar, kEpiThreads);
+      if (tid == 0) tc::mbar_arrive(bar(B_TKFREE + bi));  // K_sel[bi] may be overwritten
+      if (tid < kTile) {  // half 0: m == tid
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        v[q] = lg[g * kTile + lane + 32 * q];
-        mx = fmaxf(mx, v[q]);
+        for (int g = 0; g < G; ++g)
+          S.lg[g * kTile + tid] =
+              t >= 0 ? (S.pd[g * kTile + tid] + S.pd[(G + g) * kTile + tid]) * P.scale : -INFINITY;
       }
+      tc::named_sync(kEpiBar, kEpiThreads);
+      // ---- softmax inside the tile: warp w takes head w
+      if (warp < G) {
+        const int g = warp;
+        float v[4], mx = -INFINITY;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      float sum = 0.f;
+        for (int q = 0; q < 4; ++q) {
+          v[q] = S.lg[g * kTile + lane + 32 * q];
+          mx = fmaxf(mx, v[q]);
+        }
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float p = v[q] == -INFINITY ? 0.f : expf(v[q] - mx);
-        lg[g * kTile + lane + 32 * q] = p;
-        sum += p;
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float sum = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float p = v[q] == -INFINITY ? 0.f : expf(v[q] - mx);
+          S.lg[g * kTile + lane + 32 * q] = p;
+          sum += p;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (lane == 0) {
+          S.stat[2 * g] = mx;
+          S.stat[2 * g + 1] = sum;
+        }
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      if (lane == 0) {
-        stat[2 * g] = mx;
-        stat[2 * g + 1] = sum;
-      }
-    }
-    // ---- the Vc rows have landed (the next tile's Kc group may still be in flight)
-    if (has_next)
-      cp_async_wait<1>();
-    else
-      cp_async_wait<0>();
-    __syncthreads();
-    // ---- acc[g][c] = sum_m p[g][m] * Vc_tile[m][c]; thread owns column pairs
-    const uint8_t* vb = bufs[bi];
-    for (int cp = tid; cp < P.r / 2; cp += kThreads) {
-      const int c = 2 * cp;
-      float acc0[G], acc1[G];
-#pragma unroll
-      for (int g = 0; g < G; ++g) acc0[g] = acc1[g] = 0.f;
-#pragma unroll 4
-      for (int m = 0; m < kTile; ++m) {
-        const __nv_bfloat162 v = *(const __nv_bfloat162*)(vb + swz_offset(m, c));
-        const float2 f = __bfloat1622float2(v);
+      tc::named_sync(kEpiBar, kEpiThreads);
+      // ---- p as bf16 hi/lo rows 2g, 2g+1 of the value MMA's B operand
+      if (tid < kTile) {
+        const int mm = tid;
+        uint8_t* pb = S.pbuf[bi] + (mm >> 6) * 2048;
+        const int col = mm & 63, chunk = col >> 3, within = col & 7;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          const float p = lg[g * kTile + m];
-          acc0[g] = fmaf(p, f.x, acc0[g]);
-          acc1[g] = fmaf(p, f.y, acc1[g]);
+          const float p = S.lg[g * kTile + mm];
+          const __nv_bfloat16 hi = __float2bfloat16_rn(p);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(p - __bfloat162float(hi));
+          const int r0 = 2 * g, r1 = 2 * g + 1;
+          *(__nv_bfloat16*)(pb + (r0 >> 3) * 1024 + (r0 & 7) * 128 + ((chunk ^ (r0 & 7)) << 4) +
+                            within * 2) = hi;
+          *(__nv_bfloat16*)(pb + (r1 >> 3) * 1024 + (r1 & 7) * 128 + ((chunk ^ (r1 & 7)) << 4) +
+                            within * 2) = lo;
         }
       }
+      tc::fence_proxy_async_smem();
+      tc::named_sync(kEpiBar, kEpiThreads);
+      if (tid == 0) tc::mbar_arrive(bar(B_PREADY + bi));
+      // ---- acc from TMEM: warp (quarter, half) reads latent columns half*128 + quarter*32 + lane
+      const bool ok2 = __all_sync(0xffffffffu, tc::mbar_wait(bar(B_PDONE + bi), ph, P.flags));
+      tc::fence_after_sync();
+      if (ok2 && half < n_chunks) {
+        uint32_t v[16];
+        tc::tmem_ld16(tmem_base + ((uint32_t)(quarter * 32) << 16) + o_col0 +
+                          (uint32_t)bi * o_cols + (uint32_t)half * 16,
+                      v);
+        tc::tmem_ld_wait();
+        const int c = half * 128 + quarter * 32 + lane;
+        if (c < P.r) {
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float* pp = P.part +
-                    (((int64_t)cur.b * P.Hq + cur.u * G + g) * P.n_slots + cur.slot) * (P.r + 2);
-        *(float2*)(pp + 2 + c) = make_float2(acc0[g], acc1[g]);
+          for (int g = 0; g < G; ++g) {
+            float* pp = P.part +
+                        (((int64_t)cur.b * P.Hq + cur.u * G + g) * P.n_slots + cur.slot) *
+                            (P.r + 2);
+            pp[2 + c] = __uint_as_float(v[2 * g]) + __uint_as_float(v[2 * g + 1]);
+          }
+        }
       }
+      if (tid < G) {
+        float* pp = P.part +
+                    (((int64_t)cur.b * P.Hq + cur.u * G + tid) * P.n_slots + cur.slot) * (P.r + 2);
+        pp[0] = S.stat[2 * tid];
+        pp[1] = S.stat[2 * tid + 1];
+      }
+      tc::fence_before_sync();
+      tc::named_sync(kEpiBar, kEpiThreads);
+      if (tid == 0) tc::mbar_arrive(bar(B_TOFREE + bi));
     }
-    if (tid < G) {
-      float* pp = P.part +
-                  (((int64_t)cur.b * P.Hq + cur.u * G + tid) * P.n_slots + cur.slot) * (P.r + 2);
-      pp[0] = stat[2 * tid];
-      pp[1] = stat[2 * tid + 1];
-    }
-    __syncthreads();
   }
-  cp_async_wait<0>();
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem_base, 2 * D);
+    tc::tmem_dealloc(tmem_base, 512);
   }
 }
 
@@ -373,20 +492,25 @@ int num_sms_att() {
 }
 
 template <int G, int D>
+size_t smem_bytes(int r) {
+  const int KB = r / 64;
+  return 1024 + (size_t)KB * D * 128 + 2 * (size_t)KB * 16384 + 2 * 4096 + 8 * (D / 2) * 2 +
+         4 * (G * D + 2 * G * kTile + G * kTile + 2 * G + 2 * kTile) + 8 + 8 * B_COUNT + 16;
+}
+
+template <int G, int D>
 cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
-  const int KB = p.r / 64;
-  const size_t smem = 1024 + (size_t)KB * D * 128 + 2 * (size_t)KB * 16384 + 8 * (D / 2) +
-                      4 * (G * D + G * kTile + 2 * G + 2 * kTile) + 64;
-  CUtensorMap tpk;
-  if (!make_tmap_bf16_2d(&tpk, a.Pk, (uint64_t)p.U * D, (uint64_t)p.r, D, 64))
+  const size_t smem = smem_bytes<G, D>(p.r);
+  CUtensorMap tpk, tkc, tvc;
+  if (!make_tmap_bf16_2d(&tpk, a.Pk, (uint64_t)p.U * D, (uint64_t)p.r, D, 64) ||
+      !make_tmap_bf16_2d(&tkc, a.Kc, (uint64_t)p.N, (uint64_t)p.r, 1, 64) ||
+      !make_tmap_bf16_2d(&tvc, a.Vc, (uint64_t)p.N, (uint64_t)p.r, 1, 64))
     return cudaErrorInvalidValue;
   static int done[kMaxDevices] = {};
   cudaError_t e = ensure_smem(attend_tc_kernel<G, D>, smem, done);
   if (e != cudaSuccess) return e;
   AttendTcParams P;
   P.q = (const __nv_bfloat16*)a.q;
-  P.Kc = (const __nv_bfloat16*)a.Kc;
-  P.Vc = (const __nv_bfloat16*)a.Vc;
   P.idx = a.idx;
   P.seq_off = a.seq_off;
   P.q_pos = a.q_pos;
@@ -402,7 +526,7 @@ cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s)
   P.scale = p.scale;
   P.base = p.rope_base;
   const int grid = p.att_tiles < num_sms_att() ? p.att_tiles : num_sms_att();
-  attend_tc_kernel<G, D><<<grid, kThreads, smem, s>>>(tpk, P);
+  attend_tc_kernel<G, D><<<grid, kThreads, smem, s>>>(tpk, tkc, tvc, P);
   return cudaGetLastError();
 }
 
@@ -410,7 +534,7 @@ cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s)
 
 bool attend_tc_supported(const DecodePlan& p) {
   return p.dtype == SALSC_BF16 && p.r % 64 == 0 && p.r <= 256 && (p.d == 64 || p.d == 128) &&
-         (p.G == 1 || p.G == 2 || p.G == 4 || p.G == 8);
+         (p.G == 1 || p.G == 2 || p.G == 4 || p.G == 8) && p.N <= INT32_MAX;
 }
 
 cudaError_t launch_attend_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {

@@ -14,17 +14,36 @@
 namespace salsc {
 namespace {
 
-constexpr int kThreads = 128;  // one latent column per thread
-constexpr int kBatchChunk = 16;
+constexpr int kThreads = 128;  // 4 warps; each warp takes a quarter of the head dim
+constexpr int kCols = 64;      // latent columns per CTA: 2 per lane
+constexpr int kBatchChunk = 8;
 
+template <typename T>
+__device__ __forceinline__ float2 load2(const T* p);
+template <>
+__device__ __forceinline__ float2 load2<float>(const float* p) {
+  return *(const float2*)p;
+}
+template <>
+__device__ __forceinline__ float2 load2<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat1622float2(*(const __nv_bfloat162*)p);
+}
+
+// CTA (u, column block): q_lat[b, u, c] = sum_i qsum[b, i] * Pk[u*d + i, c] for
+// its 64 columns.  Each warp reads a quarter of the d rows of Pk_u (coalesced
+// 128-byte rows, all loads independent), and the four partial sums are
+// added in shared memory.
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 latent_q_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __restrict__ qlat,
                 __nv_bfloat16* __restrict__ qsplit, int B, int Hq, int U, int G, int d, int r,
                 int npad) {
-  __shared__ float qsum[kBatchChunk * kMaxHeadDim];
+  __shared__ float qsum[kBatchChunk][kMaxHeadDim];
+  __shared__ float2 red[4][kBatchChunk][32];
   const int u = blockIdx.x;
-  const int c = blockIdx.y * kThreads + threadIdx.x;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int c = blockIdx.y * kCols + 2 * lane;
+  const int rows = d / 4, i0 = warp * rows;
   for (int b0 = 0; b0 < B; b0 += kBatchChunk) {
     const int nb = min(kBatchChunk, B - b0);
     __syncthreads();
@@ -33,32 +52,50 @@ latent_q_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __rest
       float s = 0.f;
       if (bb < nb)
         for (int g = 0; g < G; ++g) s += to_f32(q[((size_t)(b0 + bb) * Hq + u * G + g) * d + i]);
-      qsum[bb * d + i] = s;
+      qsum[bb][i] = s;
     }
     __syncthreads();
+    float2 acc[kBatchChunk];
+#pragma unroll
+    for (int bb = 0; bb < kBatchChunk; ++bb) acc[bb] = make_float2(0.f, 0.f);
     if (c < r) {
-      float acc[kBatchChunk];
+      const T* pcol = Pk + ((size_t)u * d + i0) * r + c;
+#pragma unroll 8
+      for (int i = 0; i < rows; ++i) {
+        const float2 pk = load2<T>(pcol + (size_t)i * r);
 #pragma unroll
-      for (int bb = 0; bb < kBatchChunk; ++bb) acc[bb] = 0.f;
-      const T* pcol = Pk + (size_t)u * d * r + c;
-      for (int i = 0; i < d; ++i) {
-        const float pk = to_f32(pcol[(size_t)i * r]);
+        for (int bb = 0; bb < kBatchChunk; ++bb) {
+          const float qv = qsum[bb][i0 + i];
+          acc[bb].x = fmaf(qv, pk.x, acc[bb].x);
+          acc[bb].y = fmaf(qv, pk.y, acc[bb].y);
+        }
+      }
+    }
 #pragma unroll
-        for (int bb = 0; bb < kBatchChunk; ++bb) acc[bb] = fmaf(qsum[bb * d + i], pk, acc[bb]);
+    for (int bb = 0; bb < kBatchChunk; ++bb) red[warp][bb][lane] = acc[bb];
+    __syncthreads();
+    // warp w finishes batch rows w, w+4
+    for (int bb = warp; bb < nb; bb += 4) {
+      if (c >= r) continue;
+      float2 v = red[0][bb][lane];
+#pragma unroll
+      for (int w = 1; w < 4; ++w) {
+        v.x += red[w][bb][lane].x;
+        v.y += red[w][bb][lane].y;
       }
-      for (int bb = 0; bb < nb; ++bb) {
-        const int b = b0 + bb;
-        const float v = acc[bb];
-        qlat[((size_t)b * U + u) * r + c] = v;
-        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-        qsplit[((size_t)b * npad + 2 * u) * r + c] = hi;
-        qsplit[((size_t)b * npad + 2 * u + 1) * r + c] = lo;
-        // the padding rows are cleared by the last unit's CTAs
-        if (u == U - 1)
-          for (int row = 2 * U; row < npad; ++row)
-            qsplit[((size_t)b * npad + row) * r + c] = __float2bfloat16_rn(0.f);
-      }
+      const int b = b0 + bb;
+      *(float2*)(qlat + ((size_t)b * U + u) * r + c) = v;
+      const __nv_bfloat16 hx = __float2bfloat16_rn(v.x), hy = __float2bfloat16_rn(v.y);
+      const __nv_bfloat16 lx = __float2bfloat16_rn(v.x - __bfloat162float(hx));
+      const __nv_bfloat16 ly = __float2bfloat16_rn(v.y - __bfloat162float(hy));
+      *(__nv_bfloat162*)(qsplit + ((size_t)b * npad + 2 * u) * r + c) = __halves2bfloat162(hx, hy);
+      *(__nv_bfloat162*)(qsplit + ((size_t)b * npad + 2 * u + 1) * r + c) =
+          __halves2bfloat162(lx, ly);
+      // the padding rows are cleared by the last unit's CTAs
+      if (u == U - 1)
+        for (int row = 2 * U; row < npad; ++row)
+          *(__nv_bfloat162*)(qsplit + ((size_t)b * npad + row) * r + c) =
+              __halves2bfloat162(__float2bfloat16_rn(0.f), __float2bfloat16_rn(0.f));
     }
   }
 }
@@ -66,7 +103,7 @@ latent_q_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __rest
 }  // namespace
 
 cudaError_t launch_latent_q(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
-  dim3 grid(p.U, (p.r + kThreads - 1) / kThreads);
+  dim3 grid(p.U, (p.r + kCols - 1) / kCols);
   if (p.dtype == SALSC_BF16)
     latent_q_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(
         (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.Pk, a.qlat, a.qsplit, p.B, p.Hq, p.U,
