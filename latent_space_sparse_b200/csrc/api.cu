@@ -115,6 +115,8 @@ salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
   off = align_up(off + sizeof(int32_t) * (size_t)p.B * p.U * p.k, salsc::kWsAlign);
   p.off_part = off;
   off = align_up(off + sizeof(float) * (size_t)p.B * p.Hq * p.splits * (p.r + 2), salsc::kWsAlign);
+  p.off_count = off;
+  off = align_up(off + sizeof(int) * (size_t)p.B * p.U, salsc::kWsAlign);
   p.total = off;
   *P = p;
   return SALSC_OK;
@@ -214,12 +216,14 @@ salsc_status decode_step_impl(const salsc_decode_desc* desc, const void* q, cons
   a.qsplit = (__nv_bfloat16*)(w + p.off_qsplit);
   a.scores = (float*)(w + p.off_scores);
   a.part = (float*)(w + p.off_part);
+  a.unit_count = (int*)(w + p.off_count);
 
   cudaStream_t s = (cudaStream_t)stream;
   typedef cudaError_t (*launcher)(const salsc::DecodePlan&, const salsc::DecodeArgs&, cudaStream_t);
   const launcher seq[SALSC_DECODE_KERNELS] = {salsc::launch_latent_q, salsc::launch_score,
                                               salsc::launch_topk, salsc::launch_attend,
                                               salsc::launch_combine};
+  // the tensor-core attention merges its own tiles (no separate merge kernel)
   cudaError_t e;
   // Inside stream capture an event record must be an external node to
   // record at replay time.

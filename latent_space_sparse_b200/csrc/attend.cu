@@ -208,73 +208,116 @@ attend_simt_kernel(const T* __restrict__ q, const T* __restrict__ Kc, const T* _
 // Merge the partial results of one head and apply the deferred value
 // projection:
 //   out_h = (sum_s e^{m_s - M} acc_s / sum_s e^{m_s - M} l_s) . Pv_u^T
-// Only the first ceil(k_b / chunk) slots of a head hold results.
+// Slot s of head h holds (m, l, acc[r]) or is empty (m = -inf, acc unused).
+// Only the first ceil(k_b / chunk) slots of a head are looked at.  The Pv_u
+// rows are requested first (they depend on nothing), then the slot
+// statistics, then the used slots' accumulators: three overlapping memory
+// latencies in all.
+constexpr int kCombThreads = 256;
 template <typename T>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kCombThreads)
 combine_kernel(const float* __restrict__ part, const T* __restrict__ Pv, T* __restrict__ out,
                const int64_t* __restrict__ seq_off, int Hq, int U, int G, int d, int r,
                int splits, int chunk, int k) {
-  extern __shared__ float w_s[];  // [splits]
+  constexpr int kPer = sizeof(T) == 2 ? 8 : 4;         // row elements per 16-byte load
+  constexpr int kRows = kMaxHeadDim / (kCombThreads / 32);  // Pv rows per warp (16)
   __shared__ float accf[kMaxRank];
-  __shared__ float inv_l;
+  __shared__ float w_s[128];
+  __shared__ int seg[128];
+  __shared__ int s_nseg;
+  __shared__ float s_inv;
   const int bh = blockIdx.x;
   const int b = bh / Hq, h = bh % Hq, u = h / G;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = kCombThreads / 32;
+  const int nl = r / kPer;  // 16-byte pieces per Pv row
+  // ---- Pv_u rows i = warp + nwarps*j, lane's piece of the row (rows of up to 256 bf16 or
+  //      128 fp32 are loaded here; longer rows are finished below)
+  uint4 pv[kRows];
+#pragma unroll
+  for (int j = 0; j < kRows; ++j) {
+    const int i = warp + nwarps * j;
+    pv[j] = (i < d && lane < nl) ? *(const uint4*)(Pv + ((size_t)u * d + i) * r + lane * kPer)
+                                 : make_uint4(0u, 0u, 0u, 0u);
+  }
   const int64_t nb = seq_off[b + 1] - seq_off[b];
   const int64_t kb = nb < k ? nb : k;
   const int ns = (int)((kb + chunk - 1) / chunk);
   const float* pp = part + (size_t)bh * splits * (r + 2);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (warp == 0) {
-    float M = -INFINITY;
-    for (int s = lane; s < ns; s += 32) M = fmaxf(M, pp[(size_t)s * (r + 2)]);
+    float mv[4], lv[4], M = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int sl = lane + 32 * q;
+      mv[q] = sl < ns ? pp[(size_t)sl * (r + 2)] : -INFINITY;
+      lv[q] = sl < ns ? pp[(size_t)sl * (r + 2) + 1] : 0.f;
+      M = fmaxf(M, mv[q]);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float L = 0.f;
-    for (int s = lane; s < ns; s += 32) {
-      const float m = pp[(size_t)s * (r + 2)];
-      const float w = (m == -INFINITY) ? 0.f : expf(m - M);
-      w_s[s] = w;
-      L += w * pp[(size_t)s * (r + 2) + 1];
+    int cnt = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float wv = mv[q] == -INFINITY ? 0.f : expf(mv[q] - M);
+      L += wv * lv[q];
+      const bool used = wv != 0.f;
+      const uint32_t mk = __ballot_sync(0xffffffffu, used);
+      if (used) {
+        const int pos = cnt + __popc(mk & ((1u << lane) - 1u));
+        seg[pos] = lane + 32 * q;
+        w_s[pos] = wv;
+      }
+      cnt += __popc(mk);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (lane == 0) inv_l = L > 0.f ? 1.f / L : 0.f;
+    if (lane == 0) {
+      s_nseg = cnt;
+      s_inv = L > 0.f ? 1.f / L : 0.f;
+    }
   }
   __syncthreads();
-  for (int c = threadIdx.x; c < r; c += blockDim.x) {
+  const int nseg = s_nseg;
+  for (int c = threadIdx.x; c < r; c += kCombThreads) {
     float a = 0.f;
-#pragma unroll 8
-    for (int s = 0; s < ns; ++s) a = fmaf(w_s[s], pp[(size_t)s * (r + 2) + 2 + c], a);
-    accf[c] = a * inv_l;
+    for (int q0 = 0; q0 < nseg; q0 += 8) {
+      float v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        v[q] = q0 + q < nseg ? pp[(size_t)seg[q0 + q] * (r + 2) + 2 + c] : 0.f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (q0 + q < nseg) a = fmaf(w_s[q0 + q], v[q], a);
+    }
+    accf[c] = a * s_inv;
   }
   __syncthreads();
-  // one output element per thread: a dot product over its row of Pv_u
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    const T* pv = Pv + ((size_t)u * d + i) * r;
-    float a = 0.f;
-    if (sizeof(T) == 2) {
-#pragma unroll 8
-      for (int c0 = 0; c0 < r; c0 += 8) {
-        const uint4 v = *(const uint4*)(pv + c0);
+  // ---- out[i] = accf . Pv_u[i]
+#pragma unroll
+  for (int j = 0; j < kRows; ++j) {
+    const int i = warp + nwarps * j;
+    float o = 0.f;
+    for (int piece = lane; piece < nl; piece += 32) {
+      uint4 v = pv[j];
+      if (piece >= 32) v = *(const uint4*)(Pv + ((size_t)u * d + i) * r + piece * kPer);
+      const int c0 = piece * kPer;
+      if (sizeof(T) == 2) {
         const __nv_bfloat162* h2 = (const __nv_bfloat162*)&v;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 f = __bfloat1622float2(h2[j]);
-          a = fmaf(accf[c0 + 2 * j], f.x, a);
-          a = fmaf(accf[c0 + 2 * j + 1], f.y, a);
+        for (int jj = 0; jj < 4; ++jj) {
+          const float2 f = __bfloat1622float2(h2[jj]);
+          o = fmaf(accf[c0 + 2 * jj], f.x, fmaf(accf[c0 + 2 * jj + 1], f.y, o));
         }
-      }
-    } else {
-#pragma unroll 8
-      for (int c0 = 0; c0 < r; c0 += 4) {
-        const float4 v = *(const float4*)(pv + c0);
-        a = fmaf(accf[c0], v.x, a);
-        a = fmaf(accf[c0 + 1], v.y, a);
-        a = fmaf(accf[c0 + 2], v.z, a);
-        a = fmaf(accf[c0 + 3], v.w, a);
+      } else {
+        const float4 f = *(const float4*)&v;
+        o = fmaf(accf[c0], f.x, fmaf(accf[c0 + 1], f.y, fmaf(accf[c0 + 2], f.z,
+                 fmaf(accf[c0 + 3], f.w, o))));
       }
     }
-    out[(size_t)bh * d + i] = from_f32<T>(a);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) o += __shfl_xor_sync(0xffffffffu, o, off);
+    if (lane == 0 && i < d) out[(size_t)bh * d + i] = from_f32<T>(o);
   }
 }
 
@@ -316,22 +359,15 @@ cudaError_t launch_attend(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
 }
 
 cudaError_t launch_combine(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
-  const size_t smem = sizeof(float) * (size_t)p.splits;
-  if (p.dtype == SALSC_BF16) {
-    static int done[kMaxDevices] = {};
-    cudaError_t e = ensure_smem(combine_kernel<__nv_bfloat16>, smem, done);
-    if (e != cudaSuccess) return e;
-    combine_kernel<__nv_bfloat16><<<p.B * p.Hq, 128, smem, s>>>(
+  if (p.splits > 128) return cudaErrorInvalidConfiguration;
+  if (p.dtype == SALSC_BF16)
+    combine_kernel<__nv_bfloat16><<<p.B * p.Hq, kCombThreads, 0, s>>>(
         a.part, (const __nv_bfloat16*)a.Pv, (__nv_bfloat16*)a.out, a.seq_off, p.Hq, p.U, p.G, p.d,
         p.r, p.splits, p.chunk, p.k);
-  } else {
-    static int done[kMaxDevices] = {};
-    cudaError_t e = ensure_smem(combine_kernel<float>, smem, done);
-    if (e != cudaSuccess) return e;
-    combine_kernel<float><<<p.B * p.Hq, 128, smem, s>>>(a.part, (const float*)a.Pv, (float*)a.out,
-                                                       a.seq_off, p.Hq, p.U, p.G, p.d, p.r,
-                                                       p.splits, p.chunk, p.k);
-  }
+  else
+    combine_kernel<float><<<p.B * p.Hq, kCombThreads, 0, s>>>(a.part, (const float*)a.Pv, (float*)a.out,
+                                                     a.seq_off, p.Hq, p.U, p.G, p.d, p.r,
+                                                     p.splits, p.chunk, p.k);
   return cudaGetLastError();
 }
 

@@ -5,7 +5,7 @@
 // SALS technical framework, stages 3-4, with RoPE applied after
 // reconstruction (abstract).  Work unit: a tile of 128 kept tokens of one
 // selection unit (b, u):
-//   1. TMA gather4 brings the 128 latent key rows Kc_b[idx] into shared memory
+//   1. cp.async brings the 128 latent key rows Kc_b[idx] into shared memory
 //      (128-byte swizzled, K-major);
 //   2. tcgen05: K_sel[128 x d] = Kc_tile . Pk_u^T into TMEM (fp32; Pk_u comes
 //      by TMA once per unit and stays in shared memory);
@@ -19,9 +19,14 @@
 //   5. tcgen05: acc^T[r x 2G] = Vc_tile^T . [p_hi p_lo] into TMEM (Vc_tile read
 //      as an MN-major operand, so the latent value rows need no transpose);
 //   6. the epilogue reads acc[c] = D[c][2g] + D[c][2g+1] and writes the
-//      tile's (m, l, acc) per head; the combine kernel merges tiles.
-// Warp roles (320 threads): warps 0-7 epilogue, warp 8 TMEM owner and MMA
-// issuer, warp 9 gather issuer.  Each CTA walks a contiguous range of tiles;
+//      tile's (m, l, acc) per head;
+//   7. consecutive tiles of one unit in a CTA are folded into a running
+//      (m, l, acc) per head (online softmax rescaling); each CTA publishes one
+//      partial per unit segment at the slot of the segment's first tile and
+//      marks its other slots empty.  The combine kernel merges the few
+//      segments of a unit and applies the deferred Pv_u^T.
+// Warp roles (352 threads): warps 0-7 epilogue, warp 8 TMEM owner and MMA
+// issuer, warps 9-10 row gathers (one per tile buffer).  Each CTA walks a contiguous range of tiles;
 // the two tile buffers alternate (Kc(i) -> Vc(i) -> Kc(i+2)), so the
 // reconstruction of tile i+1 runs during the epilogue of tile i.
 //
@@ -36,8 +41,8 @@ namespace {
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kMmaWarp = 8;
-constexpr int kLoadWarp = 9;
-constexpr int kThreads = 320;
+constexpr int kLoadWarp0 = 9;  // gathers of the even tiles (buffer 0); warp 10: odd tiles
+constexpr int kThreads = 352;
 constexpr int kTile = 128;
 constexpr int kPRows = 16;  // rows of the p operand (2G <= 16)
 constexpr uint32_t kEpiBar = 1;
@@ -45,6 +50,11 @@ constexpr double kTwoPi = 6.283185307179586476925286766559;
 
 struct AttendTcParams {
   const __nv_bfloat16* q;
+  const __nv_bfloat16* Kc;
+  const __nv_bfloat16* Vc;
+  const __nv_bfloat16* Pv;
+  __nv_bfloat16* out;
+  int* unit_count;
   const int32_t* idx;
   const int64_t* seq_off;
   const int32_t* q_pos;
@@ -96,20 +106,6 @@ struct UnitTileCursor {
   }
 };
 
-struct Smem {
-  uint8_t* pk;       // Pk_u: KB k-blocks of [D rows x 128 B]
-  uint8_t* buf[2];   // tile buffers: KB k-blocks of [128 rows x 128 B]
-  uint8_t* pbuf[2];  // p operand: 2 k-blocks of [16 rows x 128 B]
-  uint64_t* fturn;   // [D/2] fixed-point turns per token position
-  double* theta;     // [D/2]
-  float* qr;         // [G][D] rotated queries
-  float* pd;         // [2][G][128] partial dot products of the two pair halves
-  float* lg;         // [G][128] logits, then softmax weights
-  float* stat;       // [G][2] (m, l)
-  int* tok;          // [2][128] token index per row (-1: no token), gather warp only
-  uint64_t* bars;
-  uint32_t* tmem_slot;
-};
 
 // barrier indices
 enum { B_PK = 0, B_KFULL = 1, B_VFULL = 3, B_KDONE = 5, B_PDONE = 7, B_PREADY = 9,
@@ -128,23 +124,29 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
   const int n_chunks = (P.r + 127) / 128;  // M = 128 slices of the latent width
   const uint32_t pk_bytes = (uint32_t)KB * D * 128;
   const uint32_t buf_bytes = (uint32_t)KB * 16384;
-  Smem S;
-  S.pk = base;
-  S.buf[0] = base + pk_bytes;
-  S.buf[1] = S.buf[0] + buf_bytes;
-  S.pbuf[0] = S.buf[1] + buf_bytes;
-  S.pbuf[1] = S.pbuf[0] + 4096;
-  S.fturn = (uint64_t*)(S.pbuf[1] + 4096);
-  S.theta = (double*)(S.fturn + HALF);
-  S.qr = (float*)(S.theta + HALF);
-  S.pd = S.qr + G * D;
-  S.lg = S.pd + 2 * G * kTile;
-  S.stat = S.lg + G * kTile;
-  S.tok = (int*)(S.stat + 2 * G);
-  S.bars = (uint64_t*)(((uintptr_t)(S.tok + 2 * kTile) + 7) & ~(uintptr_t)7);
-  S.tmem_slot = (uint32_t*)(S.bars + B_COUNT);
-  const uint32_t bar0 = tc::smem_u32(S.bars);
-  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  // shared-memory layout (plain locals: nothing here may live in local memory)
+  uint8_t* const s_pk = base;                                // Pk_u: KB x [D rows x 128 B]
+  uint8_t* const s_buf0 = base + pk_bytes;                   // tile buffers: KB x [128 x 128 B]
+  uint8_t* const s_buf1 = s_buf0 + buf_bytes;
+  uint8_t* const s_pbuf0 = s_buf1 + buf_bytes;               // p operand: 2 x [16 x 128 B]
+  uint8_t* const s_pbuf1 = s_pbuf0 + 4096;
+  (void)tmap_kc;
+  (void)tmap_vc;
+  uint64_t* const s_fturn = (uint64_t*)(s_pbuf1 + 4096);    // [D/2] fixed-point turns
+  double* const s_theta = (double*)(s_fturn + HALF);         // [D/2]
+  float* const s_qr = (float*)(s_theta + HALF);              // [G][D/2] rotated (q_i, q_i+d/2)
+  float* const s_pd = s_qr + G * D;                          // [2][G][128] half-pair dots
+  float* const s_lg = s_pd + 2 * G * kTile;                  // [G][128] logits -> weights
+  float* const s_stat = s_lg + G * kTile;                    // [G][2] (m, l)
+  int* const s_tok = (int*)(s_stat + 2 * G);                 // [2][128] token per row
+  int* const s_last = s_tok + 2 * kTile;                     // [1] this tile closes its unit
+  float* const s_run = (float*)(s_last + 2);                 // [G][2] segment's running (m, l)
+  float* const s_ab = s_run + 2 * G;                         // [G][2] rescale factors
+  int* const s_segs = (int*)(s_ab + 2 * G);                  // [128] segment start slots
+  uint64_t* const s_bars = (uint64_t*)(((uintptr_t)(s_segs + kTile) + 7) & ~(uintptr_t)7);
+  uint32_t* const s_tmem_slot = (uint32_t*)(s_bars + B_COUNT);
+  const uint32_t bar0 = tc::smem_u32(s_bars);
+  auto bar = [bar0](int i) { return bar0 + 8u * (uint32_t)i; };
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int t_begin = (int)((int64_t)blockIdx.x * P.n_tiles / gridDim.x);
@@ -158,81 +160,82 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     for (int i = 0; i < B_COUNT; ++i) tc::mbar_init(bar(i), 1);
     tc::mbar_fence_init();
     tc::tma_prefetch_desc(&tmap_pk);
-    tc::tma_prefetch_desc(&tmap_kc);
-    tc::tma_prefetch_desc(&tmap_vc);
   }
-  if (warp == kMmaWarp) tc::tmem_alloc(tc::smem_u32(S.tmem_slot), 512);
+  if (warp == kMmaWarp) tc::tmem_alloc(tc::smem_u32(s_tmem_slot), 512);
   for (int i = tid; i < HALF; i += kThreads) {
     const double th = pow(P.base, -2.0 * (double)i / (double)D);
-    S.theta[i] = th;
-    S.fturn[i] = __double2ull_rn(th / kTwoPi * 18446744073709551616.0);
+    s_theta[i] = th;
+    s_fturn[i] = __double2ull_rn(th / kTwoPi * 18446744073709551616.0);
   }
   // the p operand's unused rows (2G..15) stay zero
-  for (int e = tid; e < 2 * 4096 / 4; e += kThreads) ((uint32_t*)S.pbuf[0])[e] = 0u;
+  for (int e = tid; e < 2 * 4096 / 4; e += kThreads) ((uint32_t*)s_pbuf0)[e] = 0u;
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  const uint32_t tmem_base = *S.tmem_slot;
+  const uint32_t tmem_base = *s_tmem_slot;
 
-  if (warp == kLoadWarp) {
-    // ======================= gather issuer (all 32 lanes) ======================
-    // Lane l owns rows 4l..4l+3 of every tile: it resolves their token indices
-    // and issues the gather4 copies of those rows for every k-block.
+  if (warp >= kLoadWarp0) {
+    // ======================= gather warps =======================
+    // Warp 9 + bi fills buffer bi: the latent key rows of tiles bi, bi+2, ...
+    // (cp.async, 16 B per lane, whole rows per instruction so every row read
+    // is coalesced), then the same rows of Vc once the reconstruction is done
+    // with them.  Each gather completes (wait + proxy fence) before its
+    // barrier is released, so the tensor core sees the data.
+    const int bi = warp - kLoadWarp0;
+    int* tk = s_tok + bi * kTile;
+    uint8_t* buf = bi ? s_buf1 : s_buf0;
+    const uint32_t buf_s = tc::smem_u32(buf);
+    const int cpr = P.r / 8;              // 16-byte chunks per row
+    const int rows_per = 32 / cpr;        // rows per warp instruction (r <= 256)
+    const int lrow = lane / cpr, lchunk = lane % cpr;
     UnitTileCursor cur;
     cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
-    UnitTileCursor ahead = cur;  // tile i+2 when loading Kc(i+2)
-    auto issue = [&](const UnitTileCursor& c, int bi, const CUtensorMap* map, int b_full,
-                     bool resolve) {
-      int rows[4];
-      int* tk = S.tok + bi * kTile;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int m = 4 * lane + j;
-        int t;
-        if (resolve) {
-          const int64_t jj = (int64_t)c.slot * kTile + m;
-          t = -1;
-          if (jj < c.kb) {
-            t = P.idx[((int64_t)c.b * P.U + c.u) * P.k + jj];
-            if (t < 0 || t >= c.nb) {
-              atomicOr(P.flags, FLAG_BAD_INDEX);
-              t = -1;
-            }
-          }
-          tk[m] = t;
-        } else {
-          t = tk[m];
-        }
-        // rows without a token read the sequence's first row; their weight is 0
-        rows[j] = (int)(c.off + (t < 0 ? 0 : t));
+    if (bi == 1) cur.next();
+    auto gather = [=](const __nv_bfloat16* src, int64_t off) {
+      for (int m0 = 0; m0 < kTile; m0 += rows_per) {
+        const int m = m0 + lrow;
+        const int t = tk[m];
+        const __nv_bfloat16* sp = src + (off + (t < 0 ? 0 : t)) * P.r + lchunk * 8;
+        const int c = lchunk * 8;
+        const uint32_t dst = buf_s + (uint32_t)((c >> 6) * 16384 + (m >> 3) * 1024 + (m & 7) * 128 +
+                                                ((((c >> 3) & 7) ^ (m & 7)) << 4));
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(sp) : "memory");
       }
-      if (lane == 0) tc::mbar_expect_tx(bar(b_full + bi), (uint32_t)kTile * P.r * 2);
+      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+      tc::fence_proxy_async_smem();
       __syncwarp();
-      const uint32_t dst0 = tc::smem_u32(S.buf[bi]) + (uint32_t)(lane >> 1) * 1024u +
-                            (uint32_t)(lane & 1) * 512u;
-      for (int kb = 0; kb < KB; ++kb)
-        tc::tma_gather4(dst0 + kb * 16384u, map, kb * 64, rows[0], rows[1], rows[2], rows[3],
-                        bar(b_full + bi));
     };
-    for (int i = 0; i < 2 && i < n; ++i) {
-      issue(ahead, i, &tmap_kc, B_KFULL, true);
-      ahead.next();
-    }
     bool ok = true;
-    for (int i = 0; i < n && ok; ++i, cur.next()) {
-      const int bi = i & 1;
+    for (int i = bi; i < n && ok; i += 2) {
       const uint32_t ph = ((uint32_t)i >> 1) & 1u;
-      // the reconstruction is done with Kc(i): bring Vc(i) into the same buffer
+      // the buffer is free once the value MMA of tile i-2 is done
+      if (i >= 2) {
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(B_PDONE + bi), ph ^ 1u, P.flags));
+        if (!ok) break;
+      }
+      // token of every row (lane l resolves rows l, l+32, ...)
+      for (int m = lane; m < kTile; m += 32) {
+        const int64_t jj = (int64_t)cur.slot * kTile + m;
+        int t = -1;
+        if (jj < cur.kb) {
+          t = P.idx[((int64_t)cur.b * P.U + cur.u) * P.k + jj];
+          if (t < 0 || t >= cur.nb) {
+            atomicOr(P.flags, FLAG_BAD_INDEX);
+            t = -1;
+          }
+        }
+        tk[m] = t;
+      }
+      __syncwarp();
+      gather(P.Kc, cur.off);
+      if (lane == 0) tc::mbar_arrive(bar(B_KFULL + bi));
+      // the reconstruction is done with the key rows: bring the value rows
       ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(B_KDONE + bi), ph, P.flags));
       if (!ok) break;
-      issue(cur, bi, &tmap_vc, B_VFULL, false);
-      if (i + 2 < n) {
-        // the value MMA is done with Vc(i): bring Kc(i+2)
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(B_PDONE + bi), ph, P.flags));
-        if (!ok) break;
-        issue(ahead, bi, &tmap_kc, B_KFULL, true);
-        ahead.next();
-      }
+      gather(P.Vc, cur.off);
+      if (lane == 0) tc::mbar_arrive(bar(B_VFULL + bi));
+      cur.next();
+      cur.next();
     }
   } else if (warp == kMmaWarp) {
     // ======================= MMA issuer (lane 0) =======================
@@ -244,14 +247,14 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       int cur_b = -1, cur_u = -1;
       uint32_t pk_phase = 0;
       bool ok = true;
-      auto issue_pv = [&](int j) -> bool {
+      auto issue_pv = [=](int j) -> bool {
         const int bj = j & 1;
         const uint32_t ph = ((uint32_t)j >> 1) & 1u;
         if (!tc::mbar_wait(bar(B_PREADY + bj), ph, P.flags)) return false;
         if (!tc::mbar_wait(bar(B_VFULL + bj), ph, P.flags)) return false;
         if (!tc::mbar_wait(bar(B_TOFREE + bj), ph ^ 1u, P.flags)) return false;
         tc::fence_after_sync();
-        const uint32_t v0 = tc::smem_u32(S.buf[bj]), p0 = tc::smem_u32(S.pbuf[bj]);
+        const uint32_t v0 = tc::smem_u32((bj ? s_buf1 : s_buf0)), p0 = tc::smem_u32((bj ? s_pbuf1 : s_pbuf0));
         for (int ch = 0; ch < n_chunks; ++ch) {
           const uint32_t d_tmem = tmem_base + o_col0 + (uint32_t)bj * o_cols + (uint32_t)ch * 16;
 #pragma unroll
@@ -281,7 +284,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
           }
           tc::mbar_expect_tx(bar(B_PK), pk_bytes);
           for (int kb = 0; kb < KB; ++kb)
-            tc::tma_load_2d(tc::smem_u32(S.pk + (size_t)kb * D * 128), &tmap_pk, kb * 64,
+            tc::tma_load_2d(tc::smem_u32(s_pk + (size_t)kb * D * 128), &tmap_pk, kb * 64,
                             cur.u * D, bar(B_PK));
           if (!tc::mbar_wait(bar(B_PK), pk_phase, P.flags)) {
             ok = false;
@@ -297,7 +300,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
           break;
         }
         tc::fence_after_sync();
-        const uint32_t a0 = tc::smem_u32(S.buf[bi]), b0 = tc::smem_u32(S.pk);
+        const uint32_t a0 = tc::smem_u32((bi ? s_buf1 : s_buf0)), b0 = tc::smem_u32(s_pk);
         const uint32_t d_tmem = tmem_base + (uint32_t)bi * D;
         for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
@@ -317,6 +320,14 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     UnitTileCursor cur;
     cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
     int cur_b = -1, cur_u = -1;
+    float acc_run[G];  // this thread's latent column of the segment's running sum
+#pragma unroll
+    for (int g = 0; g < G; ++g) acc_run[g] = 0.f;
+    int seg_tiles = 0;
+    if (tid < G) {
+      s_run[2 * tid] = -INFINITY;
+      s_run[2 * tid + 1] = 0.f;
+    }
     for (int i = 0; i < n; ++i, cur.next()) {
       const int bi = i & 1;
       const uint32_t ph = ((uint32_t)i >> 1) & 1u;
@@ -326,13 +337,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
         for (int e = tid; e < G * HALF; e += kEpiThreads) {
           const int g = e / HALF, ii = e % HALF;
           const __nv_bfloat16* qh = P.q + ((int64_t)cur.b * P.Hq + cur.u * G + g) * D;
-          const double a = qpos * S.theta[ii];
+          const double a = qpos * s_theta[ii];
           const double nt = rint(a * (1.0 / kTwoPi));
           float s, c;
           sincosf((float)fma(-nt, kTwoPi, a), &s, &c);
           const float x0 = __bfloat162float(qh[ii]), x1 = __bfloat162float(qh[ii + HALF]);
-          S.qr[g * D + ii] = x0 * c - x1 * s;
-          S.qr[g * D + ii + HALF] = x1 * c + x0 * s;
+          *(float2*)(s_qr + g * D + 2 * ii) = make_float2(x0 * c - x1 * s, x1 * c + x0 * s);
         }
         cur_b = cur.b;
         cur_u = cur.u;
@@ -342,16 +352,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       const bool ok =
           __all_sync(0xffffffffu, tc::mbar_wait(bar(B_KDONE + bi), ph, P.flags));
       tc::fence_after_sync();
-      // this row's token (resolved again here rather than read from the
-      // gather warp's table, so no cross-warp ordering is needed)
-      int t = -1;
-      {
-        const int64_t jj = (int64_t)cur.slot * kTile + m;
-        if (jj < cur.kb) {
-          t = P.idx[((int64_t)cur.b * P.U + cur.u) * P.k + jj];
-          if (t < 0 || t >= cur.nb) t = -1;
-        }
-      }
+      // this row's token: written by the gather warp before it released the
+      // Kc barrier of this tile, which is acquired here (its phase is complete)
+      tc::mbar_wait(bar(B_KFULL + bi), ph, P.flags);
+      const int t = s_tok[bi * kTile + m];
       float dot[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) dot[g] = 0.f;
@@ -368,7 +372,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) {
             const int ii = i0 + jj;
-            const uint64_t F = S.fturn[ii];
+            const uint64_t F = s_fturn[ii];
             const uint32_t turn = __umulhi(tu, (uint32_t)F) + tu * (uint32_t)(F >> 32);
             float s, c;
             __sincosf((float)(int32_t)turn * (float)(kTwoPi / 4294967296.0), &s, &c);
@@ -376,21 +380,23 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
             const float k0 = x0 * c - x1 * s;
             const float k1 = x1 * c + x0 * s;
 #pragma unroll
-            for (int g = 0; g < G; ++g)
-              dot[g] = fmaf(S.qr[g * D + ii], k0, fmaf(S.qr[g * D + ii + HALF], k1, dot[g]));
+            for (int g = 0; g < G; ++g) {
+              const float2 qv = *(const float2*)(s_qr + g * D + 2 * ii);
+              dot[g] = fmaf(qv.x, k0, fmaf(qv.y, k1, dot[g]));
+            }
           }
         }
       }
 #pragma unroll
-      for (int g = 0; g < G; ++g) S.pd[(half * G + g) * kTile + m] = dot[g];
+      for (int g = 0; g < G; ++g) s_pd[(half * G + g) * kTile + m] = dot[g];
       tc::fence_before_sync();
       tc::named_sync(kEpiBar, kEpiThreads);
       if (tid == 0) tc::mbar_arrive(bar(B_TKFREE + bi));  // K_sel[bi] may be overwritten
       if (tid < kTile) {  // half 0: m == tid
 #pragma unroll
         for (int g = 0; g < G; ++g)
-          S.lg[g * kTile + tid] =
-              t >= 0 ? (S.pd[g * kTile + tid] + S.pd[(G + g) * kTile + tid]) * P.scale : -INFINITY;
+          s_lg[g * kTile + tid] =
+              t >= 0 ? (s_pd[g * kTile + tid] + s_pd[(G + g) * kTile + tid]) * P.scale : -INFINITY;
       }
       tc::named_sync(kEpiBar, kEpiThreads);
       // ---- softmax inside the tile: warp w takes head w
@@ -399,7 +405,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
         float v[4], mx = -INFINITY;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          v[q] = S.lg[g * kTile + lane + 32 * q];
+          v[q] = s_lg[g * kTile + lane + 32 * q];
           mx = fmaxf(mx, v[q]);
         }
 #pragma unroll
@@ -408,25 +414,25 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float p = v[q] == -INFINITY ? 0.f : expf(v[q] - mx);
-          S.lg[g * kTile + lane + 32 * q] = p;
+          s_lg[g * kTile + lane + 32 * q] = p;
           sum += p;
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
         if (lane == 0) {
-          S.stat[2 * g] = mx;
-          S.stat[2 * g + 1] = sum;
+          s_stat[2 * g] = mx;
+          s_stat[2 * g + 1] = sum;
         }
       }
       tc::named_sync(kEpiBar, kEpiThreads);
       // ---- p as bf16 hi/lo rows 2g, 2g+1 of the value MMA's B operand
       if (tid < kTile) {
         const int mm = tid;
-        uint8_t* pb = S.pbuf[bi] + (mm >> 6) * 2048;
+        uint8_t* pb = (bi ? s_pbuf1 : s_pbuf0) + (mm >> 6) * 2048;
         const int col = mm & 63, chunk = col >> 3, within = col & 7;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          const float p = S.lg[g * kTile + mm];
+          const float p = s_lg[g * kTile + mm];
           const __nv_bfloat16 hi = __float2bfloat16_rn(p);
           const __nv_bfloat16 lo = __float2bfloat16_rn(p - __bfloat162float(hi));
           const int r0 = 2 * g, r1 = 2 * g + 1;
@@ -439,35 +445,72 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       tc::fence_proxy_async_smem();
       tc::named_sync(kEpiBar, kEpiThreads);
       if (tid == 0) tc::mbar_arrive(bar(B_PREADY + bi));
-      // ---- acc from TMEM: warp (quarter, half) reads latent columns half*128 + quarter*32 + lane
+      // ---- fold this tile into the unit segment's running (m, l, acc): heads' scale factors
+      if (tid < G) {
+        const float mt = s_stat[2 * tid], lt = s_stat[2 * tid + 1];
+        const float mr = s_run[2 * tid], lr = s_run[2 * tid + 1];
+        const float mx = fmaxf(mr, mt);
+        float al = 0.f, be = 0.f;
+        if (mx != -INFINITY) {
+          al = mr == -INFINITY ? 0.f : expf(mr - mx);
+          be = mt == -INFINITY ? 0.f : expf(mt - mx);
+        }
+        s_ab[2 * tid] = al;
+        s_ab[2 * tid + 1] = be;
+        s_run[2 * tid] = mx;
+        s_run[2 * tid + 1] = lr * al + lt * be;
+      }
+      // ---- this tile's acc from TMEM: warp (quarter, half) holds latent column
+      //      c = half*128 + quarter*32 + lane
       const bool ok2 = __all_sync(0xffffffffu, tc::mbar_wait(bar(B_PDONE + bi), ph, P.flags));
       tc::fence_after_sync();
+      uint32_t v[16];
       if (ok2 && half < n_chunks) {
-        uint32_t v[16];
         tc::tmem_ld16(tmem_base + ((uint32_t)(quarter * 32) << 16) + o_col0 +
                           (uint32_t)bi * o_cols + (uint32_t)half * 16,
                       v);
         tc::tmem_ld_wait();
-        const int c = half * 128 + quarter * 32 + lane;
-        if (c < P.r) {
-#pragma unroll
-          for (int g = 0; g < G; ++g) {
-            float* pp = P.part +
-                        (((int64_t)cur.b * P.Hq + cur.u * G + g) * P.n_slots + cur.slot) *
-                            (P.r + 2);
-            pp[2 + c] = __uint_as_float(v[2 * g]) + __uint_as_float(v[2 * g + 1]);
-          }
-        }
-      }
-      if (tid < G) {
-        float* pp = P.part +
-                    (((int64_t)cur.b * P.Hq + cur.u * G + tid) * P.n_slots + cur.slot) * (P.r + 2);
-        pp[0] = S.stat[2 * tid];
-        pp[1] = S.stat[2 * tid + 1];
       }
       tc::fence_before_sync();
       tc::named_sync(kEpiBar, kEpiThreads);
       if (tid == 0) tc::mbar_arrive(bar(B_TOFREE + bi));
+      if (ok2 && half < n_chunks) {
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+          acc_run[g] = acc_run[g] * s_ab[2 * g] +
+                       (__uint_as_float(v[2 * g]) + __uint_as_float(v[2 * g + 1])) * s_ab[2 * g + 1];
+      }
+      // ---- end of this CTA's segment of the unit: publish it, and merge the
+      //      unit if every tile has arrived
+      UnitTileCursor nx = cur;
+      nx.next();
+      const bool seg_end = i + 1 == n || nx.b != cur.b || nx.u != cur.u;
+      ++seg_tiles;
+      if (seg_end) {
+        const int s0 = cur.slot + 1 - seg_tiles;  // first slot of the segment
+        const int c = half * 128 + quarter * 32 + lane;
+        if (half < n_chunks && c < P.r) {
+#pragma unroll
+          for (int g = 0; g < G; ++g)
+            P.part[(((int64_t)cur.b * P.Hq + cur.u * G + g) * P.n_slots + s0) * (P.r + 2) + 2 + c] =
+                acc_run[g];
+        }
+        for (int e = tid; e < G * seg_tiles; e += kEpiThreads) {
+          const int g = e / seg_tiles, sl = s0 + e % seg_tiles;
+          float* pp = P.part + (((int64_t)cur.b * P.Hq + cur.u * G + g) * P.n_slots + sl) * (P.r + 2);
+          pp[0] = sl == s0 ? s_run[2 * g] : -INFINITY;  // only the segment's first slot is used
+          pp[1] = sl == s0 ? s_run[2 * g + 1] : 0.f;
+        }
+        // a new segment starts with the next tile
+        seg_tiles = 0;
+#pragma unroll
+        for (int g = 0; g < G; ++g) acc_run[g] = 0.f;
+        if (tid < G) {
+          s_run[2 * tid] = -INFINITY;
+          s_run[2 * tid + 1] = 0.f;
+        }
+        tc::named_sync(kEpiBar, kEpiThreads);
+      }
     }
   }
   tc::fence_before_sync();
@@ -495,7 +538,8 @@ template <int G, int D>
 size_t smem_bytes(int r) {
   const int KB = r / 64;
   return 1024 + (size_t)KB * D * 128 + 2 * (size_t)KB * 16384 + 2 * 4096 + 8 * (D / 2) * 2 +
-         4 * (G * D + 2 * G * kTile + G * kTile + 2 * G + 2 * kTile) + 8 + 8 * B_COUNT + 16;
+         4 * (G * D + 2 * G * kTile + G * kTile + 2 * G + 2 * kTile + 2 + 4 * G + kTile) + 8 +
+         8 * B_COUNT + 16;
 }
 
 template <int G, int D>
@@ -511,6 +555,11 @@ cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s)
   if (e != cudaSuccess) return e;
   AttendTcParams P;
   P.q = (const __nv_bfloat16*)a.q;
+  P.Kc = (const __nv_bfloat16*)a.Kc;
+  P.Vc = (const __nv_bfloat16*)a.Vc;
+  P.Pv = (const __nv_bfloat16*)a.Pv;
+  P.out = (__nv_bfloat16*)a.out;
+  P.unit_count = a.unit_count;
   P.idx = a.idx;
   P.seq_off = a.seq_off;
   P.q_pos = a.q_pos;
@@ -533,8 +582,10 @@ cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s)
 }  // namespace
 
 bool attend_tc_supported(const DecodePlan& p) {
+  const int64_t k_eff = p.k < p.n_max ? p.k : p.n_max;
   return p.dtype == SALSC_BF16 && p.r % 64 == 0 && p.r <= 256 && (p.d == 64 || p.d == 128) &&
-         (p.G == 1 || p.G == 2 || p.G == 4 || p.G == 8) && p.N <= INT32_MAX;
+         (p.G == 1 || p.G == 2 || p.G == 4 || p.G == 8) && p.N <= INT32_MAX &&
+         (k_eff + kTile - 1) / kTile <= kTile;  // the merge keeps <= 128 tile weights per head
 }
 
 cudaError_t launch_attend_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {

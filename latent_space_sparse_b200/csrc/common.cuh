@@ -38,7 +38,7 @@ struct DecodePlan {
   float scale;
   double rope_base;
   // workspace layout (byte offsets)
-  size_t off_flags, off_qlat, off_qsplit, off_scores, off_idx, off_part, total;
+  size_t off_flags, off_qlat, off_qsplit, off_scores, off_idx, off_part, off_count, total;
 };
 
 // Raw pointers of one decode call, passed to the launchers.
@@ -57,6 +57,7 @@ struct DecodeArgs {
   __nv_bfloat16* qsplit;       // [B][npad][r]: row 2u = hi(q_lat[u]), 2u+1 = lo, rest zero
   float* scores;               // packed per (b,u)
   float* part;                 // [B][Hq][splits][r+2]
+  int* unit_count;             // [B][U] tiles finished per selection unit (tensor-core path)
 };
 
 // Record a CUDA error for salsc_last_cuda_error() and return SALSC_ERR_CUDA.

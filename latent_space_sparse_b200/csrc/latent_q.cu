@@ -30,45 +30,63 @@ __device__ __forceinline__ float2 load2<__nv_bfloat16>(const __nv_bfloat16* p) {
 }
 
 // CTA (u, column block): q_lat[b, u, c] = sum_i qsum[b, i] * Pk[u*d + i, c] for
-// its 64 columns.  Each warp reads a quarter of the d rows of Pk_u (coalesced
-// 128-byte rows, all loads independent), and the four partial sums are
-// added in shared memory.
+// its 64 columns.  Warp w owns rows i0..i0+d/4 of Pk_u and of the query sums:
+// every load of a thread (its queries and its Pk elements) is issued before
+// any arithmetic, so the kernel costs about one memory latency.  The four
+// warps' partial sums are added in shared memory.
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 latent_q_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __restrict__ qlat,
-                __nv_bfloat16* __restrict__ qsplit, int B, int Hq, int U, int G, int d, int r,
-                int npad) {
-  __shared__ float qsum[kBatchChunk][kMaxHeadDim];
+                __nv_bfloat16* __restrict__ qsplit, int* __restrict__ unit_count, int B, int Hq,
+                int U, int G, int d, int r, int npad) {
+  constexpr int kRowsMax = kMaxHeadDim / 4;  // Pk rows per warp
+  __shared__ float qsum[4][kBatchChunk][kRowsMax];
   __shared__ float2 red[4][kBatchChunk][32];
+  if (blockIdx.y == 0 && unit_count)
+    for (int b = threadIdx.x; b < B; b += kThreads) unit_count[b * U + blockIdx.x] = 0;
   const int u = blockIdx.x;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int c = blockIdx.y * kCols + 2 * lane;
   const int rows = d / 4, i0 = warp * rows;
   for (int b0 = 0; b0 < B; b0 += kBatchChunk) {
     const int nb = min(kBatchChunk, B - b0);
-    __syncthreads();
-    for (int e = threadIdx.x; e < kBatchChunk * d; e += kThreads) {
-      const int bb = e / d, i = e % d;
-      float s = 0.f;
-      if (bb < nb)
-        for (int g = 0; g < G; ++g) s += to_f32(q[((size_t)(b0 + bb) * Hq + u * G + g) * d + i]);
-      qsum[bb][i] = s;
+    // ---- issue all loads: Pk rows of this warp, and the queries this lane sums
+    float2 pk[kRowsMax];
+#pragma unroll
+    for (int i = 0; i < kRowsMax; ++i)
+      pk[i] = (i < rows && c < r) ? load2<T>(Pk + ((size_t)u * d + i0 + i) * r + c)
+                                  : make_float2(0.f, 0.f);
+    // lane covers (bb, row) pairs lane, lane+32, ... of the warp's kBatchChunk x rows block
+    constexpr int kPairs = kBatchChunk * kRowsMax / 32;
+    float qs[kPairs];
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) {
+      const int e = lane + 32 * j;
+      const int bb = e / rows, i = e % rows;
+      float sacc = 0.f;
+      if (bb < nb && e < kBatchChunk * rows) {
+        const T* qp = q + ((size_t)(b0 + bb) * Hq + u * G) * d + i0 + i;
+        for (int g = 0; g < G; ++g) sacc += to_f32(qp[(size_t)g * d]);
+      }
+      qs[j] = sacc;
     }
-    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) {
+      const int e = lane + 32 * j;
+      if (e < kBatchChunk * rows) qsum[warp][e / rows][e % rows] = qs[j];
+    }
+    __syncwarp();
     float2 acc[kBatchChunk];
 #pragma unroll
     for (int bb = 0; bb < kBatchChunk; ++bb) acc[bb] = make_float2(0.f, 0.f);
-    if (c < r) {
-      const T* pcol = Pk + ((size_t)u * d + i0) * r + c;
-#pragma unroll 8
-      for (int i = 0; i < rows; ++i) {
-        const float2 pk = load2<T>(pcol + (size_t)i * r);
 #pragma unroll
-        for (int bb = 0; bb < kBatchChunk; ++bb) {
-          const float qv = qsum[bb][i0 + i];
-          acc[bb].x = fmaf(qv, pk.x, acc[bb].x);
-          acc[bb].y = fmaf(qv, pk.y, acc[bb].y);
-        }
+    for (int i = 0; i < kRowsMax; ++i) {
+      if (i >= rows) break;
+#pragma unroll
+      for (int bb = 0; bb < kBatchChunk; ++bb) {
+        const float qv = qsum[warp][bb][i];
+        acc[bb].x = fmaf(qv, pk[i].x, acc[bb].x);
+        acc[bb].y = fmaf(qv, pk[i].y, acc[bb].y);
       }
     }
 #pragma unroll
@@ -97,6 +115,7 @@ latent_q_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __rest
           *(__nv_bfloat162*)(qsplit + ((size_t)b * npad + row) * r + c) =
               __halves2bfloat162(__float2bfloat16_rn(0.f), __float2bfloat16_rn(0.f));
     }
+    __syncthreads();
   }
 }
 
@@ -106,12 +125,12 @@ cudaError_t launch_latent_q(const DecodePlan& p, const DecodeArgs& a, cudaStream
   dim3 grid(p.U, (p.r + kCols - 1) / kCols);
   if (p.dtype == SALSC_BF16)
     latent_q_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(
-        (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.Pk, a.qlat, a.qsplit, p.B, p.Hq, p.U,
-        p.G, p.d, p.r, p.npad);
+        (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.Pk, a.qlat, a.qsplit, a.unit_count, p.B,
+        p.Hq, p.U, p.G, p.d, p.r, p.npad);
   else
     latent_q_kernel<float><<<grid, kThreads, 0, s>>>((const float*)a.q, (const float*)a.Pk, a.qlat,
-                                                     a.qsplit, p.B, p.Hq, p.U, p.G, p.d, p.r,
-                                                     p.npad);
+                                                     a.qsplit, a.unit_count, p.B, p.Hq, p.U, p.G,
+                                                     p.d, p.r, p.npad);
   return cudaGetLastError();
 }
 
