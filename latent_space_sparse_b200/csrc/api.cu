@@ -72,6 +72,7 @@ salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
   while (c < kTopkMaxCluster && (n_max + c - 1) / c > kTopkSliceTarget) c *= 2;
   p.topk_cluster = c;
   p.topk_slice = (int)((n_max + c - 1) / c);
+  if ((size_t)p.topk_slice * 4 > 200u * 1024u) return SALSC_ERR_UNSUPPORTED;  // slice in smem
   const int64_t k_eff = D->top_k < n_max ? D->top_k : n_max;
   p.attend_tc = salsc::attend_tc_supported(p);
   if (p.attend_tc) {

@@ -209,18 +209,15 @@ attend_simt_kernel(const T* __restrict__ q, const T* __restrict__ Kc, const T* _
 // projection:
 //   out_h = (sum_s e^{m_s - M} acc_s / sum_s e^{m_s - M} l_s) . Pv_u^T
 // Slot s of head h holds (m, l, acc[r]) or is empty (m = -inf, acc unused).
-// Only the first ceil(k_b / chunk) slots of a head are looked at.  The Pv_u
-// rows are requested first (they depend on nothing), then the slot
-// statistics, then the used slots' accumulators: three overlapping memory
-// latencies in all.
+// Only the first ceil(k_b / chunk) slots of a head are looked at.  The code
+// is kept short: each CTA lives for a few microseconds on an otherwise idle
+// SM, so a cold instruction cache would dominate a heavily unrolled version.
 constexpr int kCombThreads = 256;
 template <typename T>
 __global__ void __launch_bounds__(kCombThreads)
 combine_kernel(const float* __restrict__ part, const T* __restrict__ Pv, T* __restrict__ out,
                const int64_t* __restrict__ seq_off, int Hq, int U, int G, int d, int r,
                int splits, int chunk, int k) {
-  constexpr int kPer = sizeof(T) == 2 ? 8 : 4;         // row elements per 16-byte load
-  constexpr int kRows = kMaxHeadDim / (kCombThreads / 32);  // Pv rows per warp (16)
   __shared__ float accf[kMaxRank];
   __shared__ float w_s[128];
   __shared__ int seg[128];
@@ -229,30 +226,20 @@ combine_kernel(const float* __restrict__ part, const T* __restrict__ Pv, T* __re
   const int bh = blockIdx.x;
   const int b = bh / Hq, h = bh % Hq, u = h / G;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nwarps = kCombThreads / 32;
-  const int nl = r / kPer;  // 16-byte pieces per Pv row
-  // ---- Pv_u rows i = warp + nwarps*j, lane's piece of the row (rows of up to 256 bf16 or
-  //      128 fp32 are loaded here; longer rows are finished below)
-  uint4 pv[kRows];
-#pragma unroll
-  for (int j = 0; j < kRows; ++j) {
-    const int i = warp + nwarps * j;
-    pv[j] = (i < d && lane < nl) ? *(const uint4*)(Pv + ((size_t)u * d + i) * r + lane * kPer)
-                                 : make_uint4(0u, 0u, 0u, 0u);
-  }
-  const int64_t nb = seq_off[b + 1] - seq_off[b];
-  const int64_t kb = nb < k ? nb : k;
-  const int ns = (int)((kb + chunk - 1) / chunk);
   const float* pp = part + (size_t)bh * splits * (r + 2);
   if (warp == 0) {
+    const int64_t nb = seq_off[b + 1] - seq_off[b];
+    const int64_t kb = nb < k ? nb : k;
+    const int ns = (int)((kb + chunk - 1) / chunk);
     float mv[4], lv[4], M = -INFINITY;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int sl = lane + 32 * q;
       mv[q] = sl < ns ? pp[(size_t)sl * (r + 2)] : -INFINITY;
       lv[q] = sl < ns ? pp[(size_t)sl * (r + 2) + 1] : 0.f;
-      M = fmaxf(M, mv[q]);
     }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) M = fmaxf(M, mv[q]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float L = 0.f;
@@ -281,27 +268,19 @@ combine_kernel(const float* __restrict__ part, const T* __restrict__ Pv, T* __re
   const int nseg = s_nseg;
   for (int c = threadIdx.x; c < r; c += kCombThreads) {
     float a = 0.f;
-    for (int q0 = 0; q0 < nseg; q0 += 8) {
-      float v[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        v[q] = q0 + q < nseg ? pp[(size_t)seg[q0 + q] * (r + 2) + 2 + c] : 0.f;
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        if (q0 + q < nseg) a = fmaf(w_s[q0 + q], v[q], a);
-    }
+    for (int q = 0; q < nseg; ++q) a = fmaf(w_s[q], pp[(size_t)seg[q] * (r + 2) + 2 + c], a);
     accf[c] = a * s_inv;
   }
   __syncthreads();
-  // ---- out[i] = accf . Pv_u[i]
-#pragma unroll
-  for (int j = 0; j < kRows; ++j) {
-    const int i = warp + nwarps * j;
+  // out[i] = accf . Pv_u[i]: warp w takes rows w, w+8, ...; each lane a 16-byte piece
+  constexpr int kPer = sizeof(T) == 2 ? 8 : 4;
+  const int nl = r / kPer;
+  for (int i = warp; i < d; i += kCombThreads / 32) {
+    const T* pv = Pv + ((size_t)u * d + i) * r;
     float o = 0.f;
     for (int piece = lane; piece < nl; piece += 32) {
-      uint4 v = pv[j];
-      if (piece >= 32) v = *(const uint4*)(Pv + ((size_t)u * d + i) * r + piece * kPer);
       const int c0 = piece * kPer;
+      const uint4 v = *(const uint4*)(pv + c0);
       if (sizeof(T) == 2) {
         const __nv_bfloat162* h2 = (const __nv_bfloat162*)&v;
 #pragma unroll
@@ -317,7 +296,7 @@ combine_kernel(const float* __restrict__ part, const T* __restrict__ Pv, T* __re
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) o += __shfl_xor_sync(0xffffffffu, o, off);
-    if (lane == 0 && i < d) out[(size_t)bh * d + i] = from_f32<T>(o);
+    if (lane == 0) out[(size_t)bh * d + i] = from_f32<T>(o);
   }
 }
 

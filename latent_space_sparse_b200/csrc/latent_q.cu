@@ -14,7 +14,7 @@
 namespace salsc {
 namespace {
 
-constexpr int kThreads = 128;  // 4 warps; each warp takes a quarter of the head dim
+constexpr int kThreads = 256;  // 8 warps; each warp takes d/8 rows of Pk_u
 constexpr int kCols = 64;      // latent columns per CTA: 2 per lane
 constexpr int kBatchChunk = 8;
 
@@ -30,74 +30,67 @@ __device__ __forceinline__ float2 load2<__nv_bfloat16>(const __nv_bfloat16* p) {
 }
 
 // CTA (u, column block): q_lat[b, u, c] = sum_i qsum[b, i] * Pk[u*d + i, c] for
-// its 64 columns.  Warp w owns rows i0..i0+d/4 of Pk_u and of the query sums:
-// every load of a thread (its queries and its Pk elements) is issued before
-// any arithmetic, so the kernel costs about one memory latency.  The four
-// warps' partial sums are added in shared memory.
+// its 64 columns.  Each warp owns d/8 rows of Pk_u; its Pk loads are issued
+// first, the query sums are formed by the whole CTA meanwhile, and the eight
+// warps' partial sums are added in shared memory.  Small loops keep the code
+// short (the kernel is too brief to amortise a cold instruction cache).
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 latent_q_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __restrict__ qlat,
                 __nv_bfloat16* __restrict__ qsplit, int* __restrict__ unit_count, int B, int Hq,
                 int U, int G, int d, int r, int npad) {
-  constexpr int kRowsMax = kMaxHeadDim / 4;  // Pk rows per warp
-  __shared__ float qsum[4][kBatchChunk][kRowsMax];
-  __shared__ float2 red[4][kBatchChunk][32];
+  constexpr int kRowsMax = kMaxHeadDim / 8;  // Pk rows per warp
+  __shared__ float qsum[kBatchChunk][kMaxHeadDim];
+  __shared__ float2 red[8][kBatchChunk][32];
   if (blockIdx.y == 0 && unit_count)
     for (int b = threadIdx.x; b < B; b += kThreads) unit_count[b * U + blockIdx.x] = 0;
   const int u = blockIdx.x;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int c = blockIdx.y * kCols + 2 * lane;
-  const int rows = d / 4, i0 = warp * rows;
+  const int rows = d / 8, i0 = warp * rows;
   for (int b0 = 0; b0 < B; b0 += kBatchChunk) {
     const int nb = min(kBatchChunk, B - b0);
-    // ---- issue all loads: Pk rows of this warp, and the queries this lane sums
     float2 pk[kRowsMax];
 #pragma unroll
     for (int i = 0; i < kRowsMax; ++i)
       pk[i] = (i < rows && c < r) ? load2<T>(Pk + ((size_t)u * d + i0 + i) * r + c)
                                   : make_float2(0.f, 0.f);
-    // lane covers (bb, row) pairs lane, lane+32, ... of the warp's kBatchChunk x rows block
-    constexpr int kPairs = kBatchChunk * kRowsMax / 32;
-    float qs[kPairs];
-#pragma unroll
-    for (int j = 0; j < kPairs; ++j) {
-      const int e = lane + 32 * j;
-      const int bb = e / rows, i = e % rows;
+    // query group sums: thread e covers (bb, i) = e, e+256, ...
+    for (int e = threadIdx.x; e < nb * d; e += kThreads) {
+      const int bb = e / d, i = e % d;
+      const T* qp = q + ((size_t)(b0 + bb) * Hq + u * G) * d + i;
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
       float sacc = 0.f;
-      if (bb < nb && e < kBatchChunk * rows) {
-        const T* qp = q + ((size_t)(b0 + bb) * Hq + u * G) * d + i0 + i;
-        for (int g = 0; g < G; ++g) sacc += to_f32(qp[(size_t)g * d]);
-      }
-      qs[j] = sacc;
-    }
+      for (int g0 = 0; g0 < G; g0 += 4) {
 #pragma unroll
-    for (int j = 0; j < kPairs; ++j) {
-      const int e = lane + 32 * j;
-      if (e < kBatchChunk * rows) qsum[warp][e / rows][e % rows] = qs[j];
+        for (int g = 0; g < 4; ++g) v[g] = g0 + g < G ? to_f32(qp[(size_t)(g0 + g) * d]) : 0.f;
+        sacc += (v[0] + v[1]) + (v[2] + v[3]);
+      }
+      qsum[bb][i] = sacc;
     }
-    __syncwarp();
+    __syncthreads();
     float2 acc[kBatchChunk];
 #pragma unroll
     for (int bb = 0; bb < kBatchChunk; ++bb) acc[bb] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < kRowsMax; ++i) {
-      if (i >= rows) break;
+      if (i < rows) {
 #pragma unroll
-      for (int bb = 0; bb < kBatchChunk; ++bb) {
-        const float qv = qsum[warp][bb][i];
-        acc[bb].x = fmaf(qv, pk[i].x, acc[bb].x);
-        acc[bb].y = fmaf(qv, pk[i].y, acc[bb].y);
+        for (int bb = 0; bb < kBatchChunk; ++bb) {
+          const float qv = qsum[bb][i0 + i];
+          acc[bb].x = fmaf(qv, pk[i].x, acc[bb].x);
+          acc[bb].y = fmaf(qv, pk[i].y, acc[bb].y);
+        }
       }
     }
 #pragma unroll
     for (int bb = 0; bb < kBatchChunk; ++bb) red[warp][bb][lane] = acc[bb];
     __syncthreads();
-    // warp w finishes batch rows w, w+4
-    for (int bb = warp; bb < nb; bb += 4) {
-      if (c >= r) continue;
+    // warp w finishes batch row w
+    if (warp < nb && c < r) {
+      const int bb = warp;
       float2 v = red[0][bb][lane];
-#pragma unroll
-      for (int w = 1; w < 4; ++w) {
+      for (int w = 1; w < 8; ++w) {
         v.x += red[w][bb][lane].x;
         v.y += red[w][bb][lane].y;
       }

@@ -1,18 +1,23 @@
-// topk.cu -- exact per-unit top-k by cluster-wide radix select.
+// topk.cu -- exact per-unit top-k by radix select in shared memory.
 //
 // SALS keeps only the most important tokens of each unit (page section "key
 // designs": Top-K selection).  k_b = min(k, n_b) tokens with the largest
 // score are kept; among equal scores the lower token index wins; slots
 // k_b..k-1 are set to -1.
 //
-// Design: a thread-block cluster of C CTAs owns one unit.  Each CTA loads a
-// contiguous slice of the unit's scores into shared memory once, as 32-bit
-// keys whose unsigned order is the float order.  Four 8-bit radix passes find
-// the exact k_b-th largest key T: each CTA histograms its slice, the C
-// histograms are summed through distributed shared memory, and every CTA
-// picks the same digit.  A final ordered compaction writes the keys > T and
-// the lowest-index keys == T; slice ranks give a global index order, so the
-// result is deterministic.  No full sort, no global-memory scratch.
+// Design: C CTAs (a thread-block cluster when C > 1) own one unit.  Each CTA
+// loads a contiguous slice of the unit's scores into shared memory once, as
+// 32-bit keys whose unsigned order is the float order, and the unit's key
+// range [kmin, kmax] is found.  A radix select on rel = key - kmin with
+// 11-bit digits, starting at the top bit of the range (at most three
+// passes), finds the exact k_b-th largest key T: each CTA histograms its
+// slice into 2048 bins (keys spread over the bins, so the shared-memory
+// atomics barely contend), the C histograms are summed through distributed
+// shared memory, and every CTA picks the same digit with a block-wide scan.  The final compaction gives every warp a contiguous segment of the
+// slice: one counting pass, one prefix over warps (and cluster ranks), one
+// writing pass with warp ballots.  Output order is the index order of the
+// keys > T followed by the lowest-index keys == T, so the result is
+// deterministic.  No full sort, no global-memory scratch.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -22,8 +27,9 @@ namespace cg = cooperative_groups;
 namespace salsc {
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
+constexpr int kBatch = 32;  // keys a thread loads before converting them
 
 // Unsigned key with the same order as the float; -0 and +0 map to one key.
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -32,20 +38,65 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+constexpr int kBins = 2048;  // 11-bit digits
+constexpr int kDigit = 11;
+
+// Block-wide search for the digit that holds the target rank: `cnt` holds the
+// histogram (ascending bins); bins are scanned from the top.  Thread t looks
+// at bins 2047-2t and 2046-2t.  Returns through s_digit / s_above.
+__device__ __forceinline__ void find_digit(const uint32_t* cnt, uint32_t target, int nbins,
+                                           uint32_t* wsum, uint32_t* s_digit, uint32_t* s_above) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b0 = kBins - 1 - 2 * tid, b1 = b0 - 1;
+  const uint32_t c0 = b0 < nbins ? cnt[b0] : 0u, c1 = b1 < nbins ? cnt[b1] : 0u;
+  const uint32_t mine = c0 + c1;
+  uint32_t incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t v = wsum[lane];
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += t;
+    }
+    wsum[32 + lane] = x - v;  // exclusive prefix of the warps above
+  }
+  __syncthreads();
+  const uint32_t above0 = wsum[32 + warp] + incl - mine;  // keys in bins above b0
+  if (above0 < target && target <= above0 + c0) {
+    *s_digit = (uint32_t)b0;
+    *s_above = above0;
+  } else if (above0 + c0 < target && target <= above0 + c0 + c1) {
+    *s_digit = (uint32_t)b1;
+    *s_above = above0 + c0;
+  }
+}
+
+template <bool kCluster>
 __global__ void __launch_bounds__(kThreads)
-topk_cluster_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_off,
-                    int32_t* __restrict__ idx_out, int U, int k) {
+topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_off,
+            int32_t* __restrict__ idx_out, int U, int k) {
   cg::cluster_group cluster = cg::this_cluster();
-  const int C = (int)cluster.num_blocks();
-  const int rank = (int)cluster.block_rank();
+  const int C = kCluster ? (int)cluster.num_blocks() : 1;
+  const int rank = kCluster ? (int)cluster.block_rank() : 0;
   const int unit = blockIdx.x / C;
   const int b = unit / U, u = unit % U;
 
   extern __shared__ uint32_t keys[];
-  __shared__ uint32_t hist[2][256];
-  __shared__ uint32_t total[256];
+  __shared__ uint32_t hist[2][kBins];
+  __shared__ uint32_t total[kBins];
+  __shared__ uint32_t wsum[64];
+  __shared__ uint32_t mm[2];      // this CTA's (min key, max key), read by the cluster
   __shared__ uint32_t counts[2];  // this CTA's (#keys > T, #keys == T), read by the cluster
-  __shared__ uint32_t wtot[kWarps][2];
+  __shared__ uint32_t wcnt[kWarps][2];
+  __shared__ uint32_t wbase[kWarps][2];
   __shared__ uint32_t s_digit, s_above, s_base_gt, s_base_eq;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -56,150 +107,212 @@ topk_cluster_kernel(const float* __restrict__ scores, const int64_t* __restrict_
   const int64_t lo = nb * rank / C, hi = nb * (rank + 1) / C;
   const int n_loc = (int)(hi - lo);
 
-  for (int i = tid; i < n_loc; i += kThreads) keys[i] = order_key(s[lo + i]);
-
-  // Radix select: T = the kb-th largest key; `remaining` ends as the number
-  // of keys equal to T that are kept.
-  uint32_t prefix = 0u, mask = 0u, remaining = (uint32_t)kb;
-  const bool take_all = kb == nb;
-  if (take_all) {
-    remaining = 0u;  // every finite score has key > 0
-    __syncthreads();
-  } else {
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      uint32_t* h = hist[pass & 1];
-      for (int i = tid; i < 256; i += kThreads) h[i] = 0u;
-      __syncthreads();
-      for (int i = tid; i < n_loc; i += kThreads) {
-        const uint32_t key = keys[i];
-        if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
-      }
-      cluster.sync();
-      if (tid < 256) {
-        uint32_t t = 0u;
-        for (int q = 0; q < C; ++q) t += cluster.map_shared_rank(h, q)[tid];
-        total[tid] = t;
-      }
-      __syncthreads();
-      if (warp == 0) {
-        // lane L covers bins 255-8L .. 248-8L, in descending order
-        uint32_t v[8], sum = 0u;
+  // ---- keys of the slice (loads of a batch issued before their stores) and their range
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  for (int base = 0; base < n_loc; base += kThreads * kBatch) {
+    float v[kBatch];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          v[j] = total[255 - 8 * lane - j];
-          sum += v[j];
-        }
-        uint32_t incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += t;
-        }
-        uint32_t run = incl - sum;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (run < remaining && remaining <= run + v[j]) {
-            s_digit = (uint32_t)(255 - 8 * lane - j);
-            s_above = run;
-          }
-          run += v[j];
-        }
-      }
-      __syncthreads();
-      prefix |= s_digit << shift;
-      mask |= 255u << shift;
-      remaining -= s_above;
+    for (int j = 0; j < kBatch; ++j) {
+      const int i = base + j * kThreads + tid;
+      v[j] = i < n_loc ? s[lo + i] : 0.f;
     }
-  }
-  const uint32_t T = prefix;
-  const uint32_t need_eq = remaining;
-  const uint32_t n_gt_total = (uint32_t)kb - need_eq;
-
-  // Local counts, then this CTA's offsets from the lower ranks.
-  uint32_t my_gt = 0u, my_eq = 0u;
-  for (int i = tid; i < n_loc; i += kThreads) {
-    const uint32_t key = keys[i];
-    my_gt += key > T;
-    my_eq += key == T;
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int i = base + j * kThreads + tid;
+      if (i < n_loc) {
+        const uint32_t key = order_key(v[j]);
+        keys[i] = key;
+        kmin = min(kmin, key);
+        kmax = max(kmax, key);
+      }
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    my_gt += __shfl_xor_sync(0xffffffffu, my_gt, o);
-    my_eq += __shfl_xor_sync(0xffffffffu, my_eq, o);
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
   }
   if (lane == 0) {
-    wtot[warp][0] = my_gt;
-    wtot[warp][1] = my_eq;
+    wcnt[warp][0] = kmin;
+    wcnt[warp][1] = kmax;
   }
   __syncthreads();
-  if (tid == 0) {
-    uint32_t g = 0u, e = 0u;
-    for (int w = 0; w < kWarps; ++w) {
-      g += wtot[w][0];
-      e += wtot[w][1];
+  if (warp == 0) {
+    uint32_t a = wcnt[lane][0], z = wcnt[lane][1];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      a = min(a, __shfl_xor_sync(0xffffffffu, a, o));
+      z = max(z, __shfl_xor_sync(0xffffffffu, z, o));
     }
-    counts[0] = g;
-    counts[1] = e;
+    if (lane == 0) {
+      mm[0] = a;
+      mm[1] = z;
+    }
   }
-  cluster.sync();
-  if (tid == 0) {
-    uint32_t g = 0u, e = 0u;
-    for (int q = 0; q < rank; ++q) {
-      const uint32_t* rc = cluster.map_shared_rank(counts, q);
-      g += rc[0];
-      e += rc[1];
+  if (kCluster) {
+    cluster.sync();
+    if (tid == 0) {
+      uint32_t a = 0xffffffffu, z = 0u;
+      for (int q = 0; q < C; ++q) {
+        const uint32_t* r = cluster.map_shared_rank(mm, q);
+        a = min(a, r[0]);
+        z = max(z, r[1]);
+      }
+      wsum[0] = a;
+      wsum[1] = z;
     }
-    s_base_gt = g;
-    s_base_eq = e;
+  } else if (tid == 0) {
+    wsum[0] = mm[0];
+    wsum[1] = mm[1];
+  }
+  __syncthreads();
+  kmin = wsum[0];
+  kmax = wsum[1];
+  __syncthreads();
+
+  // ---- radix select on rel = key - kmin, 11-bit digits from the top bit of the range:
+  //      T = kmin + prefix is the kb-th largest key; `remaining` ends as the number
+  //      of keys equal to T that are kept
+  uint64_t prefix = 0u;
+  uint32_t remaining = (uint32_t)kb;
+  uint32_t T = 0u;
+  const int n_iter = (n_loc + kThreads - 1) / kThreads;
+  if (kb == nb) {
+    remaining = 0u;  // keep everything: every finite score has key > 0
+  } else {
+    const uint32_t range = kmax - kmin;
+    int hi_bit = range == 0u ? 0 : 32 - __clz(range);  // bits of rel still to resolve: [0, hi_bit)
+    int pass = 0;
+    while (hi_bit > 0) {
+      const int width = hi_bit < kDigit ? hi_bit : kDigit;
+      const int lo_bit = hi_bit - width;
+      uint32_t* h = hist[pass & 1];
+      for (int i = tid; i < kBins; i += kThreads) h[i] = 0u;
+      __syncthreads();
+      for (int it = 0; it < n_iter; ++it) {
+        const int i = it * kThreads + tid;
+        if (i < n_loc) {
+          const uint64_t rel = (uint64_t)(keys[i] - kmin);
+          if ((rel >> hi_bit) == (prefix >> hi_bit))
+            atomicAdd(&h[(uint32_t)(rel >> lo_bit) & ((1u << width) - 1u)], 1u);
+        }
+      }
+      const uint32_t* cnt = h;
+      if (kCluster) {
+        cluster.sync();
+        for (int i = tid; i < kBins; i += kThreads) {
+          uint32_t t = 0u;
+          for (int q = 0; q < C; ++q) t += cluster.map_shared_rank(h, q)[i];
+          total[i] = t;
+        }
+        cnt = total;
+      }
+      __syncthreads();
+      find_digit(cnt, remaining, 1 << width, wsum, &s_digit, &s_above);
+      __syncthreads();
+      prefix |= (uint64_t)s_digit << lo_bit;
+      remaining -= s_above;
+      hi_bit = lo_bit;
+      ++pass;
+    }
+    T = kmin + (uint32_t)prefix;
+  }
+  const uint32_t need_eq = remaining;
+  const uint32_t n_gt_total = (uint32_t)kb - need_eq;
+
+  // ---- compaction: warp w owns keys [w*seg, min((w+1)*seg, n_loc))
+  const int seg = (n_loc + kWarps - 1) / kWarps;
+  const int s0 = warp * seg, s1 = min(s0 + seg, n_loc);
+  uint32_t cgt = 0u, ceq = 0u;
+  for (int i = s0 + lane; i < s1; i += 32) {
+    const uint32_t key = keys[i];
+    cgt += key > T;
+    ceq += key == T;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    cgt += __shfl_xor_sync(0xffffffffu, cgt, o);
+    ceq += __shfl_xor_sync(0xffffffffu, ceq, o);
+  }
+  if (lane == 0) {
+    wcnt[warp][0] = cgt;
+    wcnt[warp][1] = ceq;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t g = wcnt[lane][0], e = wcnt[lane][1];
+    uint32_t ig = g, ie = e;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t tg = __shfl_up_sync(0xffffffffu, ig, o);
+      const uint32_t te = __shfl_up_sync(0xffffffffu, ie, o);
+      if (lane >= o) {
+        ig += tg;
+        ie += te;
+      }
+    }
+    wbase[lane][0] = ig - g;
+    wbase[lane][1] = ie - e;
+    if (lane == 31) {
+      counts[0] = ig;
+      counts[1] = ie;
+    }
+  }
+  if (kCluster) {
+    cluster.sync();
+    if (tid == 0) {
+      uint32_t g = 0u, e = 0u;
+      for (int q = 0; q < rank; ++q) {
+        const uint32_t* rc = cluster.map_shared_rank(counts, q);
+        g += rc[0];
+        e += rc[1];
+      }
+      s_base_gt = g;
+      s_base_eq = e;
+    }
+  } else if (tid == 0) {
+    s_base_gt = 0u;
+    s_base_eq = 0u;
   }
   __syncthreads();
 
   int32_t* out = idx_out + ((int64_t)b * U + u) * k;
-  uint32_t run_gt = s_base_gt, run_eq = s_base_eq;
+  uint32_t run_gt = s_base_gt + wbase[warp][0], run_eq = s_base_eq + wbase[warp][1];
   const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int c0 = 0; c0 < n_loc; c0 += kThreads) {
-    const int i = c0 + tid;
-    const bool valid = i < n_loc;
+  for (int c0 = s0; c0 < s1; c0 += 32) {
+    const int i = c0 + lane;
+    const bool valid = i < s1;
     const uint32_t key = valid ? keys[i] : 0u;
     const bool g = valid && key > T;
     const bool e = valid && key == T && need_eq > 0u;
     const uint32_t bg = __ballot_sync(0xffffffffu, g);
     const uint32_t be = __ballot_sync(0xffffffffu, e);
-    if (lane == 0) {
-      wtot[warp][0] = __popc(bg);
-      wtot[warp][1] = __popc(be);
-    }
-    __syncthreads();
-    uint32_t og = 0u, oe = 0u, tg = 0u, te = 0u;
-    for (int w = 0; w < kWarps; ++w) {
-      if (w < warp) {
-        og += wtot[w][0];
-        oe += wtot[w][1];
-      }
-      tg += wtot[w][0];
-      te += wtot[w][1];
-    }
-    if (g) out[run_gt + og + __popc(bg & lt_mask)] = (int32_t)(lo + i);
+    if (g) out[run_gt + __popc(bg & lt_mask)] = (int32_t)(lo + i);
     if (e) {
-      const uint32_t er = run_eq + oe + __popc(be & lt_mask);
+      const uint32_t er = run_eq + __popc(be & lt_mask);
       if (er < need_eq) out[n_gt_total + er] = (int32_t)(lo + i);
     }
-    run_gt += tg;
-    run_eq += te;
-    __syncthreads();
+    run_gt += __popc(bg);
+    run_eq += __popc(be);
   }
   if (rank == 0)
     for (int64_t j = kb + tid; j < k; j += kThreads) out[j] = -1;
-  cluster.sync();  // no CTA leaves while another may still read its counts
+  if (kCluster) cluster.sync();  // no CTA leaves while another may still read its counts
 }
 
 }  // namespace
 
 cudaError_t launch_topk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
   const size_t smem = sizeof(uint32_t) * (size_t)p.topk_slice;
+  if (p.topk_cluster == 1) {
+    static int done[kMaxDevices] = {};
+    cudaError_t e = ensure_smem(topk_kernel<false>, smem, done);
+    if (e != cudaSuccess) return e;
+    topk_kernel<false><<<p.B * p.U, kThreads, smem, s>>>(a.scores, a.seq_off, a.idx, p.U, p.k);
+    return cudaGetLastError();
+  }
   static int done[kMaxDevices] = {};
-  cudaError_t e = ensure_smem(topk_cluster_kernel, smem, done);
+  cudaError_t e = ensure_smem(topk_kernel<true>, smem, done);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(p.B * p.U * p.topk_cluster));
@@ -213,7 +326,7 @@ cudaError_t launch_topk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, topk_cluster_kernel, (const float*)a.scores, a.seq_off, a.idx,
+  return cudaLaunchKernelEx(&cfg, topk_kernel<true>, (const float*)a.scores, a.seq_off, a.idx,
                             p.U, p.k);
 }
 
