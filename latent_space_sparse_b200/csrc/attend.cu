@@ -61,6 +61,8 @@ attend_simt_kernel(const T* __restrict__ q, const T* __restrict__ Kc, const T* _
   const int64_t nb = seq_off[b + 1] - off;
   const int64_t kb = nb < k ? nb : k;
   const double qpos = q_pos ? (double)q_pos[b] : (double)nb;
+  allow_dependent_launch();
+  grid_dependency_wait();  // the kept indices come from the previous kernel
 
   for (int i = tid; i < half; i += kThreads) theta[i] = pow(base, -2.0 * (double)i / (double)d);
   for (int e = tid; e < d * r; e += kThreads) pk[e] = Pk[(size_t)u * d * r + e];
@@ -227,6 +229,8 @@ combine_kernel(const float* __restrict__ part, const T* __restrict__ Pv, T* __re
   const int b = bh / Hq, h = bh % Hq, u = h / G;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const float* pp = part + (size_t)bh * splits * (r + 2);
+  allow_dependent_launch();
+  grid_dependency_wait();  // the partial results come from the previous kernel
   if (warp == 0) {
     const int64_t nb = seq_off[b + 1] - seq_off[b];
     const int64_t kb = nb < k ? nb : k;
@@ -319,20 +323,23 @@ cudaError_t launch_attend(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
     const size_t smem = attend_smem(p, 2);
     cudaError_t e = ensure_smem(kern, smem, done);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, smem, s>>>((const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.Kc,
-                                      (const __nv_bfloat16*)a.Vc, (const __nv_bfloat16*)a.Pk, a.idx,
-                                      a.seq_off, a.q_pos, a.part, a.flags, p.Hq, p.U, p.G, p.d, p.r,
-                                      p.k, p.chunk, p.splits, p.scale, p.rope_base);
+    e = launch_k(kern, grid, dim3(kThreads), smem, s, true, (const __nv_bfloat16*)a.q,
+                 (const __nv_bfloat16*)a.Kc, (const __nv_bfloat16*)a.Vc,
+                 (const __nv_bfloat16*)a.Pk, (const int32_t*)a.idx, (const int64_t*)a.seq_off,
+                 (const int32_t*)a.q_pos, a.part, a.flags, p.Hq, p.U, p.G, p.d, p.r, p.k, p.chunk,
+                 p.splits, p.scale, p.rope_base);
+    if (e != cudaSuccess) return e;
   } else {
     static int done[kMaxDevices] = {};
     auto kern = attend_simt_kernel<float>;
     const size_t smem = attend_smem(p, 4);
     cudaError_t e = ensure_smem(kern, smem, done);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, smem, s>>>((const float*)a.q, (const float*)a.Kc, (const float*)a.Vc,
-                                      (const float*)a.Pk, a.idx, a.seq_off, a.q_pos, a.part,
-                                      a.flags, p.Hq, p.U, p.G, p.d, p.r, p.k, p.chunk, p.splits,
-                                      p.scale, p.rope_base);
+    e = launch_k(kern, grid, dim3(kThreads), smem, s, true, (const float*)a.q,
+                 (const float*)a.Kc, (const float*)a.Vc, (const float*)a.Pk, (const int32_t*)a.idx,
+                 (const int64_t*)a.seq_off, (const int32_t*)a.q_pos, a.part, a.flags, p.Hq, p.U,
+                 p.G, p.d, p.r, p.k, p.chunk, p.splits, p.scale, p.rope_base);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
@@ -340,14 +347,13 @@ cudaError_t launch_attend(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
 cudaError_t launch_combine(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
   if (p.splits > 128) return cudaErrorInvalidConfiguration;
   if (p.dtype == SALSC_BF16)
-    combine_kernel<__nv_bfloat16><<<p.B * p.Hq, kCombThreads, 0, s>>>(
-        a.part, (const __nv_bfloat16*)a.Pv, (__nv_bfloat16*)a.out, a.seq_off, p.Hq, p.U, p.G, p.d,
-        p.r, p.splits, p.chunk, p.k);
-  else
-    combine_kernel<float><<<p.B * p.Hq, kCombThreads, 0, s>>>(a.part, (const float*)a.Pv, (float*)a.out,
-                                                     a.seq_off, p.Hq, p.U, p.G, p.d, p.r,
-                                                     p.splits, p.chunk, p.k);
-  return cudaGetLastError();
+    return launch_k(combine_kernel<__nv_bfloat16>, dim3(p.B * p.Hq), dim3(kCombThreads), 0, s,
+                    true, (const float*)a.part, (const __nv_bfloat16*)a.Pv,
+                    (__nv_bfloat16*)a.out, (const int64_t*)a.seq_off, p.Hq, p.U, p.G, p.d, p.r,
+                    p.splits, p.chunk, p.k);
+  return launch_k(combine_kernel<float>, dim3(p.B * p.Hq), dim3(kCombThreads), 0, s, true,
+                  (const float*)a.part, (const float*)a.Pv, (float*)a.out,
+                  (const int64_t*)a.seq_off, p.Hq, p.U, p.G, p.d, p.r, p.splits, p.chunk, p.k);
 }
 
 }  // namespace salsc

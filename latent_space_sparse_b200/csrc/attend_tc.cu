@@ -5,7 +5,7 @@
 // SALS technical framework, stages 3-4, with RoPE applied after
 // reconstruction (abstract).  Work unit: a tile of 128 kept tokens of one
 // selection unit (b, u):
-//   1. cp.async brings the 128 latent key rows Kc_b[idx] into shared memory
+//   1. TMA gather4 brings the 128 latent key rows Kc_b[idx] into shared memory
 //      (128-byte swizzled, K-major);
 //   2. tcgen05: K_sel[128 x d] = Kc_tile . Pk_u^T into TMEM (fp32; Pk_u comes
 //      by TMA once per unit and stays in shared memory);
@@ -25,8 +25,9 @@
 //      partial per unit segment at the slot of the segment's first tile and
 //      marks its other slots empty.  The combine kernel merges the few
 //      segments of a unit and applies the deferred Pv_u^T.
-// Warp roles (352 threads): warps 0-7 epilogue, warp 8 TMEM owner and MMA
-// issuer, warps 9-10 row gathers (one per tile buffer).  Each CTA walks a contiguous range of tiles;
+// Warp roles (544 threads): warps 0-7 epilogue, warp 8 TMEM owner and MMA
+// issuer, warps 9-12 and 13-16 row gathers (one group of four per tile
+// buffer; latent keys by TMA gather4, latent values by cp.async).  Each CTA walks a contiguous range of tiles;
 // the two tile buffers alternate (Kc(i) -> Vc(i) -> Kc(i+2)), so the
 // reconstruction of tile i+1 runs during the epilogue of tile i.
 //
@@ -41,8 +42,10 @@ namespace {
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kMmaWarp = 8;
-constexpr int kLoadWarp0 = 9;  // gathers of the even tiles (buffer 0); warp 10: odd tiles
-constexpr int kThreads = 352;
+constexpr int kLoadWarp0 = 9;  // warps 9-12 fill buffer 0 (even tiles), 13-16 buffer 1
+constexpr int kGatherWarps = 4;
+constexpr int kGatherThreads = kGatherWarps * 32;
+constexpr int kThreads = (kLoadWarp0 + 2 * kGatherWarps) * 32;  // 544
 constexpr int kTile = 128;
 constexpr int kPRows = 16;  // rows of the p operand (2G <= 16)
 constexpr uint32_t kEpiBar = 1;
@@ -130,7 +133,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
   uint8_t* const s_buf1 = s_buf0 + buf_bytes;
   uint8_t* const s_pbuf0 = s_buf1 + buf_bytes;               // p operand: 2 x [16 x 128 B]
   uint8_t* const s_pbuf1 = s_pbuf0 + 4096;
-  (void)tmap_kc;
   (void)tmap_vc;
   uint64_t* const s_fturn = (uint64_t*)(s_pbuf1 + 4096);    // [D/2] fixed-point turns
   double* const s_theta = (double*)(s_fturn + HALF);         // [D/2]
@@ -149,6 +151,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
   auto bar = [bar0](int i) { return bar0 + 8u * (uint32_t)i; };
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  allow_dependent_launch();
   const int t_begin = (int)((int64_t)blockIdx.x * P.n_tiles / gridDim.x);
   const int t_end = (int)((int64_t)(blockIdx.x + 1) * P.n_tiles / gridDim.x);
   const int n = t_end - t_begin;
@@ -160,6 +163,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     for (int i = 0; i < B_COUNT; ++i) tc::mbar_init(bar(i), 1);
     tc::mbar_fence_init();
     tc::tma_prefetch_desc(&tmap_pk);
+    tc::tma_prefetch_desc(&tmap_kc);
   }
   if (warp == kMmaWarp) tc::tmem_alloc(tc::smem_u32(s_tmem_slot), 512);
   for (int i = tid; i < HALF; i += kThreads) {
@@ -176,46 +180,31 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
 
   if (warp >= kLoadWarp0) {
     // ======================= gather warps =======================
-    // Warp 9 + bi fills buffer bi: the latent key rows of tiles bi, bi+2, ...
-    // (cp.async, 16 B per lane, whole rows per instruction so every row read
-    // is coalesced), then the same rows of Vc once the reconstruction is done
-    // with them.  Each gather completes (wait + proxy fence) before its
-    // barrier is released, so the tensor core sees the data.
-    const int bi = warp - kLoadWarp0;
+    // Group bi (4 warps, 128 threads) fills buffer bi with tiles bi, bi+2, ...:
+    // the latent key rows by TMA gather4 (thread t: row group t % 32, k-block
+    // t / 32), then, once the reconstruction is done with them, the same rows
+    // of Vc by 16-byte cp.async (two request paths of the SM in parallel).
+    const int bi = (warp - kLoadWarp0) / kGatherWarps;
+    const int gt = tid - (kLoadWarp0 + bi * kGatherWarps) * 32;  // 0..127
+    const uint32_t gbar = 2 + bi;                                 // named barrier of the group
     int* tk = s_tok + bi * kTile;
     uint8_t* buf = bi ? s_buf1 : s_buf0;
     const uint32_t buf_s = tc::smem_u32(buf);
-    const int cpr = P.r / 8;              // 16-byte chunks per row
-    const int rows_per = 32 / cpr;        // rows per warp instruction (r <= 256)
-    const int lrow = lane / cpr, lchunk = lane % cpr;
+    const int cpr = P.r / 8;  // 16-byte chunks per row
     UnitTileCursor cur;
     cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
     if (bi == 1) cur.next();
-    auto gather = [=](const __nv_bfloat16* src, int64_t off) {
-      for (int m0 = 0; m0 < kTile; m0 += rows_per) {
-        const int m = m0 + lrow;
-        const int t = tk[m];
-        const __nv_bfloat16* sp = src + (off + (t < 0 ? 0 : t)) * P.r + lchunk * 8;
-        const int c = lchunk * 8;
-        const uint32_t dst = buf_s + (uint32_t)((c >> 6) * 16384 + (m >> 3) * 1024 + (m & 7) * 128 +
-                                                ((((c >> 3) & 7) ^ (m & 7)) << 4));
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(sp) : "memory");
-      }
-      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-      tc::fence_proxy_async_smem();
-      __syncwarp();
-    };
+    grid_dependency_wait();  // the kept indices come from the previous kernel
     bool ok = true;
     for (int i = bi; i < n && ok; i += 2) {
       const uint32_t ph = ((uint32_t)i >> 1) & 1u;
       // the buffer is free once the value MMA of tile i-2 is done
       if (i >= 2) {
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(B_PDONE + bi), ph ^ 1u, P.flags));
-        if (!ok) break;
+        ok = tc::mbar_wait(bar(B_PDONE + bi), ph ^ 1u, P.flags);
       }
-      // token of every row (lane l resolves rows l, l+32, ...)
-      for (int m = lane; m < kTile; m += 32) {
-        const int64_t jj = (int64_t)cur.slot * kTile + m;
+      // token of row gt
+      {
+        const int64_t jj = (int64_t)cur.slot * kTile + gt;
         int t = -1;
         if (jj < cur.kb) {
           t = P.idx[((int64_t)cur.b * P.U + cur.u) * P.k + jj];
@@ -224,16 +213,39 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
             t = -1;
           }
         }
-        tk[m] = t;
+        tk[gt] = t;
       }
-      __syncwarp();
-      gather(P.Kc, cur.off);
-      if (lane == 0) tc::mbar_arrive(bar(B_KFULL + bi));
+      if (gt == 0) tc::mbar_expect_tx(bar(B_KFULL + bi), (uint32_t)kTile * P.r * 2);
+      tc::named_sync(gbar, kGatherThreads);
+      // latent key rows: gather4 of rows 4g..4g+3, k-block kb
+      {
+        const int g = gt % 32;
+        int rows[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int t = tk[4 * g + j];
+          rows[j] = (int)(cur.off + (t < 0 ? 0 : t));  // no token: weight 0, any valid row
+        }
+        for (int kb = gt / 32; kb < KB; kb += kGatherThreads / 32)
+          tc::tma_gather4(buf_s + kb * 16384u + (uint32_t)(g >> 1) * 1024u + (uint32_t)(g & 1) * 512u,
+                          &tmap_kc, kb * 64, rows[0], rows[1], rows[2], rows[3],
+                          bar(B_KFULL + bi));
+      }
       // the reconstruction is done with the key rows: bring the value rows
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(bar(B_KDONE + bi), ph, P.flags));
-      if (!ok) break;
-      gather(P.Vc, cur.off);
-      if (lane == 0) tc::mbar_arrive(bar(B_VFULL + bi));
+      if (!tc::mbar_wait(bar(B_KDONE + bi), ph, P.flags)) break;
+      for (int e = gt; e < kTile * cpr; e += kGatherThreads) {
+        const int m = e / cpr, cc = e % cpr;
+        const int t = tk[m];
+        const __nv_bfloat16* sp = P.Vc + (cur.off + (t < 0 ? 0 : t)) * P.r + cc * 8;
+        const int c = cc * 8;
+        const uint32_t dst = buf_s + (uint32_t)((c >> 6) * 16384 + (m >> 3) * 1024 + (m & 7) * 128 +
+                                                ((((c >> 3) & 7) ^ (m & 7)) << 4));
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(sp) : "memory");
+      }
+      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+      tc::fence_proxy_async_smem();
+      tc::named_sync(gbar, kGatherThreads);
+      if (gt == 0) tc::mbar_arrive(bar(B_VFULL + bi));
       cur.next();
       cur.next();
     }
@@ -364,13 +376,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
             tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)bi * D;
         const uint32_t tu = (uint32_t)(t < 0 ? 0 : t);
 #pragma unroll 1
-        for (int i0 = half * QPAIRS; i0 < (half + 1) * QPAIRS; i0 += 16) {
-          uint32_t v0[16], v1[16];
-          tc::tmem_ld16(row_addr + i0, v0);
-          tc::tmem_ld16(row_addr + HALF + i0, v1);
+        for (int i0 = half * QPAIRS; i0 < (half + 1) * QPAIRS; i0 += 8) {
+          uint32_t v0[8], v1[8];
+          tc::tmem_ld8(row_addr + i0, v0);
+          tc::tmem_ld8(row_addr + HALF + i0, v1);
           tc::tmem_ld_wait();
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
+          for (int jj = 0; jj < 8; ++jj) {
             const int ii = i0 + jj;
             const uint64_t F = s_fturn[ii];
             const uint32_t turn = __umulhi(tu, (uint32_t)F) + tu * (uint32_t)(F >> 32);
@@ -575,8 +587,8 @@ cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s)
   P.scale = p.scale;
   P.base = p.rope_base;
   const int grid = p.att_tiles < num_sms_att() ? p.att_tiles : num_sms_att();
-  attend_tc_kernel<G, D><<<grid, kThreads, smem, s>>>(tpk, tkc, tvc, P);
-  return cudaGetLastError();
+  return launch_k(attend_tc_kernel<G, D>, dim3(grid), dim3(kThreads), smem, s, true, tpk, tkc, tvc,
+                  P);
 }
 
 }  // namespace

@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "salsc.h"
 
 namespace salsc {
@@ -87,6 +89,37 @@ cudaError_t ensure_smem(K* kernel, size_t bytes, int (&done)[kMaxDevices]) {
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e == cudaSuccess) done[dev] = (int)bytes;
   return e;
+}
+
+// Launch `kernel` on `s`; with `pdl` the launch may begin while the previous
+// kernel on the stream is still running (programmatic dependent launch): the
+// kernel must execute grid_dependency_wait() before it reads anything the
+// previous kernel writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                     bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Wait until the kernels this one depends on have finished and their writes
+// are visible (no-op when the kernel was launched without PDL).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Let the next kernel on the stream be scheduled now (it still waits, with
+// grid_dependency_wait, for this kernel to finish before reading its output).
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- device helpers

@@ -42,6 +42,7 @@ latent_q_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __rest
   constexpr int kRowsMax = kMaxHeadDim / 8;  // Pk rows per warp
   __shared__ float qsum[kBatchChunk][kMaxHeadDim];
   __shared__ float2 red[8][kBatchChunk][32];
+  allow_dependent_launch();
   if (blockIdx.y == 0 && unit_count)
     for (int b = threadIdx.x; b < B; b += kThreads) unit_count[b * U + blockIdx.x] = 0;
   const int u = blockIdx.x;

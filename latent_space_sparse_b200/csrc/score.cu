@@ -27,6 +27,8 @@ score_simt_kernel(const T* __restrict__ Kc, const float* __restrict__ qlat,
   if (b < 0) return;
   const int64_t off = seq_off[b];
   const int64_t nb = seq_off[b + 1] - off;
+  allow_dependent_launch();
+  grid_dependency_wait();  // q_lat comes from the previous kernel
   for (int e = threadIdx.x; e < U * r; e += kThreads) sq[e] = qlat[(size_t)b * U * r + e];
   __syncthreads();
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -105,6 +107,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int t_begin = (int)((int64_t)blockIdx.x * P.n_tiles / gridDim.x);
   const int t_end = (int)((int64_t)(blockIdx.x + 1) * P.n_tiles / gridDim.x);
+  allow_dependent_launch();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -141,6 +144,17 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
           ok = tc::mbar_wait(bempty, bpar, P.flags);
           bpar ^= 1u;
           if (!ok) break;
+        } else {
+          // the latent cache streams in already; the split query comes from the
+          // previous kernel
+          if (tile == t_begin) {
+            for (int kb = 0; kb < KB && kb < S; ++kb) {
+              tc::mbar_expect_tx(full(kb), kStageBytes);
+              tc::tma_load_2d(tc::smem_u32(a_ring + (size_t)kb * kStageBytes), &tmap_kc, kb * 64,
+                              (int)(cur.off + cur.t0), full(kb));
+            }
+          }
+          grid_dependency_wait();
         }
         tc::mbar_expect_tx(bfull, (uint32_t)KB * b_kblock_bytes);
         for (int kb = 0; kb < KB; ++kb)
@@ -152,6 +166,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
       for (int kb = 0; kb < KB; ++kb, ++it) {
         const int s = (int)(it % (uint32_t)S);
         const uint32_t ph = (it / (uint32_t)S) & 1u;
+        if (tile == t_begin && kb < S) continue;  // issued before the dependency wait
         if (!tc::mbar_wait(empty(s), ph ^ 1u, P.flags)) {
           ok = false;
           break;
@@ -302,8 +317,7 @@ cudaError_t launch_score_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream
   P.tmem_cols = cols;
   const int max_ctas = num_sms() * ctas_per_sm;
   const int grid = p.n_score_tiles < max_ctas ? p.n_score_tiles : max_ctas;
-  score_tc_kernel<<<grid, kTcThreads, smem, s>>>(tk, tq, P);
-  return cudaGetLastError();
+  return launch_k(score_tc_kernel, dim3(grid), dim3(kTcThreads), smem, s, true, tk, tq, P);
 }
 
 }  // namespace
@@ -316,15 +330,19 @@ cudaError_t launch_score(const DecodePlan& p, const DecodeArgs& a, cudaStream_t 
     auto k = score_simt_kernel<__nv_bfloat16>;
     cudaError_t e = ensure_smem(k, smem, done);
     if (e != cudaSuccess) return e;
-    k<<<p.n_score_tiles, kThreads, smem, s>>>((const __nv_bfloat16*)a.Kc, a.qlat, a.seq_off,
-                                              a.scores, p.B, p.U, p.r, p.score_tile);
+    e = launch_k(k, dim3(p.n_score_tiles), dim3(kThreads), smem, s, true,
+                 (const __nv_bfloat16*)a.Kc, (const float*)a.qlat, (const int64_t*)a.seq_off,
+                 a.scores, p.B, p.U, p.r, p.score_tile);
+    if (e != cudaSuccess) return e;
   } else {
     static int done[kMaxDevices] = {};
     auto k = score_simt_kernel<float>;
     cudaError_t e = ensure_smem(k, smem, done);
     if (e != cudaSuccess) return e;
-    k<<<p.n_score_tiles, kThreads, smem, s>>>((const float*)a.Kc, a.qlat, a.seq_off, a.scores,
-                                              p.B, p.U, p.r, p.score_tile);
+    e = launch_k(k, dim3(p.n_score_tiles), dim3(kThreads), smem, s, true, (const float*)a.Kc,
+                 (const float*)a.qlat, (const int64_t*)a.seq_off, a.scores, p.B, p.U, p.r,
+                 p.score_tile);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

@@ -100,10 +100,12 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
   __shared__ uint32_t s_digit, s_above, s_base_gt, s_base_eq;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  allow_dependent_launch();
   const int64_t off = seq_off[b];
   const int64_t nb = seq_off[b + 1] - off;
   const int64_t kb = nb < k ? nb : k;
   const float* s = scores + off * U + (int64_t)u * nb;
+  grid_dependency_wait();  // the scores come from the previous kernel
   const int64_t lo = nb * rank / C, hi = nb * (rank + 1) / C;
   const int n_loc = (int)(hi - lo);
 
@@ -308,8 +310,8 @@ cudaError_t launch_topk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s
     static int done[kMaxDevices] = {};
     cudaError_t e = ensure_smem(topk_kernel<false>, smem, done);
     if (e != cudaSuccess) return e;
-    topk_kernel<false><<<p.B * p.U, kThreads, smem, s>>>(a.scores, a.seq_off, a.idx, p.U, p.k);
-    return cudaGetLastError();
+    return launch_k(topk_kernel<false>, dim3(p.B * p.U), dim3(kThreads), smem, s, true,
+                    (const float*)a.scores, (const int64_t*)a.seq_off, a.idx, p.U, p.k);
   }
   static int done[kMaxDevices] = {};
   cudaError_t e = ensure_smem(topk_kernel<true>, smem, done);
@@ -319,13 +321,15 @@ cudaError_t launch_topk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)p.topk_cluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, topk_kernel<true>, (const float*)a.scores, a.seq_off, a.idx,
                             p.U, p.k);
 }
