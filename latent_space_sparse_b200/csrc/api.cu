@@ -63,6 +63,7 @@ salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
   p.r = D->rank;
   p.k = D->top_k;
   p.npad = (2 * p.U + 15) / 16 * 16;
+  if (p.G > 8) return SALSC_ERR_UNSUPPORTED;  // the merge handles up to 8 query heads per unit
   p.dtype = D->dtype;
   p.N = D->seq_offsets_host[D->batch];
   p.n_max = n_max;

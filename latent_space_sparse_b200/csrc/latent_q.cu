@@ -41,7 +41,9 @@ latent_q_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __rest
                 int U, int G, int d, int r, int npad) {
   constexpr int kRowsMax = kMaxHeadDim / 8;  // Pk rows per warp
   __shared__ float qsum[kBatchChunk][kMaxHeadDim];
-  __shared__ float2 red[8][kBatchChunk][32];
+  // per warp: its Pk rows during the row loop, then its partial sums
+  static_assert(kBatchChunk <= kRowsMax, "partial sums reuse the Pk staging rows");
+  __shared__ float2 wbuf[8][kRowsMax][32];
   allow_dependent_launch();
   if (blockIdx.y == 0 && unit_count)
     for (int b = threadIdx.x; b < B; b += kThreads) unit_count[b * U + blockIdx.x] = 0;
@@ -70,30 +72,35 @@ latent_q_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __rest
       qsum[bb][i] = sacc;
     }
     __syncthreads();
+    // the Pk values go through shared memory so that the row loop stays rolled:
+    // code executed once per SM costs a cold instruction fetch per instruction
+#pragma unroll
+    for (int i = 0; i < kRowsMax; ++i) wbuf[warp][i][lane] = pk[i];
+    __syncwarp();
     float2 acc[kBatchChunk];
 #pragma unroll
     for (int bb = 0; bb < kBatchChunk; ++bb) acc[bb] = make_float2(0.f, 0.f);
+#pragma unroll 1
+    for (int i = 0; i < rows; ++i) {
+      const float2 pv = wbuf[warp][i][lane];
 #pragma unroll
-    for (int i = 0; i < kRowsMax; ++i) {
-      if (i < rows) {
-#pragma unroll
-        for (int bb = 0; bb < kBatchChunk; ++bb) {
-          const float qv = qsum[bb][i0 + i];
-          acc[bb].x = fmaf(qv, pk[i].x, acc[bb].x);
-          acc[bb].y = fmaf(qv, pk[i].y, acc[bb].y);
-        }
+      for (int bb = 0; bb < kBatchChunk; ++bb) {
+        const float qv = qsum[bb][i0 + i];
+        acc[bb].x = fmaf(qv, pv.x, acc[bb].x);
+        acc[bb].y = fmaf(qv, pv.y, acc[bb].y);
       }
     }
+    __syncwarp();
 #pragma unroll
-    for (int bb = 0; bb < kBatchChunk; ++bb) red[warp][bb][lane] = acc[bb];
+    for (int bb = 0; bb < kBatchChunk; ++bb) wbuf[warp][bb][lane] = acc[bb];
     __syncthreads();
     // warp w finishes batch row w
     if (warp < nb && c < r) {
       const int bb = warp;
-      float2 v = red[0][bb][lane];
+      float2 v = wbuf[0][bb][lane];
       for (int w = 1; w < 8; ++w) {
-        v.x += red[w][bb][lane].x;
-        v.y += red[w][bb][lane].y;
+        v.x += wbuf[w][bb][lane].x;
+        v.y += wbuf[w][bb][lane].y;
       }
       const int b = b0 + bb;
       *(float2*)(qlat + ((size_t)b * U + u) * r + c) = v;
