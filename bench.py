@@ -41,6 +41,13 @@ from latent_space_sparse_b200 import synth, workloads  # noqa: E402
 
 METRIC = "latent-sparse decode µs/layer-step at 4K/32K ctx; achieved HBM GB/s vs peak"
 UNIT = "us/layer-step"
+
+# DRAM bytes (read + write) of one launch, from an ncu capture of the named
+# kernel on the named workload (the summary under profiles/ gives the command).
+# An entry is removed whenever its kernel changes after the capture.
+PROFILED_TRAFFIC: dict[tuple[str, str], float] = {
+    ("mistral_7b_gqa32x8_d128_r256_n32768_b4_k2048_bf16", "attend"): 54.45248e6 + 0.402944e6,
+}
 DEFAULT_WORKLOAD = workloads.MISTRAL_32K_B4.name
 THROTTLE_BITS = {
     0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -138,49 +145,79 @@ def make_layers(w, L, device):
     return layers
 
 
+def distinct_rows(w, idx):
+    """Distinct selected token rows of each sequence (union over its units)."""
+    return sum(np.unique(idx[b].reshape(-1)[idx[b].reshape(-1) >= 0]).size
+               for b in range(w.batch))
+
+
 def algorithmic_bytes(w, idx_list, elem):
     """Algorithmic HBM bytes of one layer-step per layer: Kc once, the distinct
     kept Vc rows of each sequence, Pk and Pv once, q and out."""
     N, r, hid = w.n_tokens, w.rank, w.hidden
-    offs = w.seq_offsets()
-    per_layer = []
-    for idx in idx_list:  # [B][U][k] int32 on the host
-        vrows = 0
-        for b in range(w.batch):
-            sel = idx[b].reshape(-1)
-            vrows += np.unique(sel[sel >= 0]).size
-        per_layer.append(N * r * elem + vrows * r * elem + 2 * hid * r * elem
-                         + 2 * w.batch * w.n_q_heads * w.head_dim * elem)
-    return per_layer
+    return [N * r * elem + distinct_rows(w, idx) * r * elem + 2 * hid * r * elem
+            + 2 * w.batch * w.n_q_heads * w.head_dim * elem for idx in idx_list]
+
+
+def kernel_bytes(w, idx_list, elem):
+    """Algorithmic bytes of one launch of each kernel (mean over layers): what
+    the kernel must read and write at least once, counting no re-reads.
+
+    latent_q: q, Pk, q_lat (fp32) and its hi/lo bf16 split.
+    score:    Kc, the hi/lo latent queries, the fp32 scores.
+    topk:     the fp32 scores, the int32 indices.
+    attend:   the distinct selected Kc and Vc rows of each sequence, Pk, q,
+              the indices (its fp32 per-segment partials are not counted).
+    combine:  Pv and out (the partials it reads are not counted)."""
+    B, U, r, k, N = w.batch, w.n_kv_heads, w.rank, w.top_k, w.n_tokens
+    hid, qo = w.hidden, w.batch * w.n_q_heads * w.head_dim * elem
+    npad = (2 * U + 15) // 16 * 16
+    split = B * npad * r * 2
+    rows = float(np.mean([distinct_rows(w, idx) for idx in idx_list]))
+    return {
+        "latent_q": qo + hid * r * elem + B * U * r * 4 + split,
+        "score": N * r * elem + split + N * U * 4,
+        "topk": N * U * 4 + B * U * k * 4,
+        "attend": 2 * rows * r * elem + hid * r * elem + qo + B * U * k * 4,
+        "combine": hid * r * elem + qo,
+    }
 
 
 # ------------------------------------------------------------------ oracle timing
 
-def oracle_sample(w, units: int, n_threads: int):
-    """Time the oracle on the first `units` selection units of sequence 0."""
+def oracle_inputs(w, units: int):
+    """The first `units` selection units of sequence 0 as their own problem."""
     import oracle
     x = synth.decode_inputs(w, seq_lens=(w.seq_lens[0],))
     G = w.group
     units = min(units, w.n_kv_heads)
-    # the first `units` KV heads of sequence 0 as their own problem
     p = oracle.Problem(1, units * G, units, w.head_dim, w.rank, w.top_k,
                        np.array([0, w.seq_lens[0]], dtype=np.int64), w.rope_base)
-    q = x["q"][:, :units * G]
-    Pk = x["Pk"][:units * w.head_dim]
-    Pv = x["Pv"][:units * w.head_dim]
+    return (p, x["q"][:, :units * G], x["Kc"], x["Vc"], x["Pk"][:units * w.head_dim],
+            x["Pv"][:units * w.head_dim]), units
+
+
+def oracle_time(inputs, n_threads: int) -> float:
+    import oracle
     t0 = time.perf_counter()
-    oracle.decode(p, q, x["Kc"], x["Vc"], Pk, Pv, n_threads=n_threads)
-    return time.perf_counter() - t0, units
+    oracle.decode(*inputs, n_threads=n_threads)
+    return time.perf_counter() - t0
 
 
-def cpu_baseline(w, n_threads):
+def cpu_baseline(w, n_threads, min_seconds: float = 10.0):
+    """The oracle on all units of sequence 0, repeated for at least
+    `min_seconds`, scaled to one layer-step of the whole batch."""
     total_units = w.batch * w.n_kv_heads
-    sec, units = oracle_sample(w, max(1, min(w.n_kv_heads, n_threads)), n_threads)
+    inputs, units = oracle_inputs(w, w.n_kv_heads)
+    secs = []
+    while sum(secs) < min_seconds:
+        secs.append(oracle_time(inputs, n_threads))
     scale = total_units / units
-    return {"value": sec * scale * 1e6, "unit": UNIT, "cores": n_threads, "kind": "oracle",
-            "sample": f"oracle.decode of {units} of {total_units} selection units "
-                      f"(sequence 0, n={w.seq_lens[0]}), {sec:.2f} s, scaled x{scale:g} "
-                      f"to one layer-step"}
+    mean = statistics.mean(secs)
+    return {"value": mean * scale * 1e6, "unit": UNIT, "cores": n_threads, "kind": "oracle",
+            "sample": f"oracle.decode of sequence 0 ({units} of {total_units} selection units, "
+                      f"n={w.seq_lens[0]}), {len(secs)} runs in {sum(secs):.1f} s, mean "
+                      f"{mean:.3f} s scaled x{scale:g} to one layer-step"}
 
 
 def run_reference(args, w):
@@ -190,10 +227,10 @@ def run_reference(args, w):
         return
     import oracle
     n_threads = oracle.default_threads()
-    units = max(1, min(w.n_kv_heads, n_threads))
+    inputs, units = oracle_inputs(w, max(1, min(w.n_kv_heads, n_threads)))
     for _ in range(args.warmup):
-        oracle_sample(w, units, n_threads)
-    secs = [oracle_sample(w, units, n_threads)[0] for _ in range(args.steps)]
+        oracle_time(inputs, n_threads)
+    secs = [oracle_time(inputs, n_threads) for _ in range(args.steps)]
     scale = w.batch * w.n_kv_heads / units
     value = statistics.mean(secs) * scale * 1e6
     line = {
@@ -324,18 +361,12 @@ def main():
     step_bytes = algorithmic_bytes(w, idx_host, elem)
     bytes_layer = float(np.mean(step_bytes))
     peak, peak_kind = measured_peaks()
-    kc_bytes = w.n_tokens * w.rank * elem
-    kern_bytes = {"score": kc_bytes}
+    kbytes = kernel_bytes(w, idx_host, elem)
     name = salsc.DECODE_KERNELS[dominant]
-    roofline = None
-    if name in kern_bytes:
-        ach = kern_bytes[name] / (per_kernel_us[dominant] * 1e-6) / 1e9
-        roofline = {"kernel": name, "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
-                    "frac": ach / peak, "traffic": None, "peak_kind": peak_kind,
-                    "algorithmic_bytes_per_launch": kern_bytes[name]}
-    else:
-        roofline = {"kernel": name, "bound": "hbm", "achieved": None, "peak": peak, "unit": "GB/s",
-                    "frac": None, "traffic": None, "peak_kind": peak_kind}
+    ach = kbytes[name] / (per_kernel_us[dominant] * 1e-6) / 1e9
+    roofline = {"kernel": name, "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
+                "frac": ach / peak, "traffic": PROFILED_TRAFFIC.get((w.name, name)),
+                "peak_kind": peak_kind, "algorithmic_bytes_per_launch": kbytes[name]}
     step_gbs = bytes_layer / (us_layer * 1e-6) / 1e9
 
     # ---- end to end through the public API with host buffers
@@ -376,6 +407,8 @@ def main():
                           "achieved": step_gbs, "peak": peak, "unit": "GB/s",
                           "frac": step_gbs / peak, "frac_of_8tbs": step_gbs / 8000.0},
         "per_kernel_us": {n: float(v) for n, v in zip(salsc.DECODE_KERNELS, per_kernel_us)},
+        "per_kernel_gbs": {n: kbytes[n] / (v * 1e-6) / 1e9
+                           for n, v in zip(salsc.DECODE_KERNELS, per_kernel_us)},
         "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": qbytes,
                 "d2h_bytes_per_step": obytes, "steps": e2e_steps,
                 "how": "eager salsc_decode_step per layer; q copied in from pinned host memory "
