@@ -45,9 +45,7 @@ UNIT = "us/layer-step"
 # DRAM bytes (read + write) of one launch, from an ncu capture of the named
 # kernel on the named workload (the summary under profiles/ gives the command).
 # An entry is removed whenever its kernel changes after the capture.
-PROFILED_TRAFFIC: dict[tuple[str, str], float] = {
-    ("mistral_7b_gqa32x8_d128_r256_n32768_b4_k2048_bf16", "attend"): 54.45248e6 + 0.402944e6,
-}
+PROFILED_TRAFFIC: dict[tuple[str, str], float] = {}
 DEFAULT_WORKLOAD = workloads.MISTRAL_32K_B4.name
 THROTTLE_BITS = {
     0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",

@@ -110,6 +110,22 @@ struct UnitTileCursor {
 };
 
 
+// Token of row `row` of the cursor's tile, or -1 past the unit's k_b kept
+// tokens; an index outside [0, n_b) raises FLAG_BAD_INDEX and reads as -1.
+__device__ __forceinline__ int row_token(const AttendTcParams& P, const UnitTileCursor& c,
+                                         int row) {
+  const int64_t jj = (int64_t)c.slot * kTile + row;
+  int t = -1;
+  if (jj < c.kb) {
+    t = P.idx[((int64_t)c.b * P.U + c.u) * P.k + jj];
+    if (t < 0 || t >= c.nb) {
+      atomicOr(P.flags, FLAG_BAD_INDEX);
+      t = -1;
+    }
+  }
+  return t;
+}
+
 // barrier indices
 enum { B_PK = 0, B_KFULL = 1, B_VFULL = 3, B_KDONE = 5, B_PDONE = 7, B_PREADY = 9,
        B_TKFREE = 11, B_TOFREE = 13, B_COUNT = 15 };
@@ -133,7 +149,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
   uint8_t* const s_buf1 = s_buf0 + buf_bytes;
   uint8_t* const s_pbuf0 = s_buf1 + buf_bytes;               // p operand: 2 x [16 x 128 B]
   uint8_t* const s_pbuf1 = s_pbuf0 + 4096;
-  (void)tmap_vc;
   uint64_t* const s_fturn = (uint64_t*)(s_pbuf1 + 4096);    // [D/2] fixed-point turns
   double* const s_theta = (double*)(s_fturn + HALF);         // [D/2]
   float* const s_qr = (float*)(s_theta + HALF);              // [G][D/2] rotated (q_i, q_i+d/2)
@@ -164,6 +179,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     tc::mbar_fence_init();
     tc::tma_prefetch_desc(&tmap_pk);
     tc::tma_prefetch_desc(&tmap_kc);
+    tc::tma_prefetch_desc(&tmap_vc);
   }
   if (warp == kMmaWarp) tc::tmem_alloc(tc::smem_u32(s_tmem_slot), 512);
   for (int i = tid; i < HALF; i += kThreads) {
@@ -181,74 +197,60 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
   if (warp >= kLoadWarp0) {
     // ======================= gather warps =======================
     // Group bi (4 warps, 128 threads) fills buffer bi with tiles bi, bi+2, ...:
-    // the latent key rows by TMA gather4 (thread t: row group t % 32, k-block
-    // t / 32), then, once the reconstruction is done with them, the same rows
-    // of Vc by 16-byte cp.async (two request paths of the SM in parallel).
+    // first the latent key rows Kc_b[idx], then, once the reconstruction is
+    // done with them, the same rows of Vc, both by TMA gather4 (thread t: row
+    // group t % 32, k-block t / 32).  The next tile's token of row t is loaded
+    // while the current tile is in flight.
     const int bi = (warp - kLoadWarp0) / kGatherWarps;
     const int gt = tid - (kLoadWarp0 + bi * kGatherWarps) * 32;  // 0..127
     const uint32_t gbar = 2 + bi;                                 // named barrier of the group
     int* tk = s_tok + bi * kTile;
-    uint8_t* buf = bi ? s_buf1 : s_buf0;
-    const uint32_t buf_s = tc::smem_u32(buf);
-    const int cpr = P.r / 8;  // 16-byte chunks per row
+    const uint32_t buf_s = tc::smem_u32(bi ? s_buf1 : s_buf0);
+    const uint32_t tile_bytes = (uint32_t)kTile * P.r * 2;
+    const int g4 = gt % 32;
     UnitTileCursor cur;
     cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
     if (bi == 1) cur.next();
     grid_dependency_wait();  // the kept indices come from the previous kernel
+    int t_next = bi < n ? row_token(P, cur, gt) : -1;
+    int last_v = -1;  // last tile whose value rows were requested
     bool ok = true;
     for (int i = bi; i < n && ok; i += 2) {
       const uint32_t ph = ((uint32_t)i >> 1) & 1u;
+      const int64_t off = cur.off;
       // the buffer is free once the value MMA of tile i-2 is done
       if (i >= 2) {
         ok = tc::mbar_wait(bar(B_PDONE + bi), ph ^ 1u, P.flags);
       }
-      // token of row gt
-      {
-        const int64_t jj = (int64_t)cur.slot * kTile + gt;
-        int t = -1;
-        if (jj < cur.kb) {
-          t = P.idx[((int64_t)cur.b * P.U + cur.u) * P.k + jj];
-          if (t < 0 || t >= cur.nb) {
-            atomicOr(P.flags, FLAG_BAD_INDEX);
-            t = -1;
-          }
-        }
-        tk[gt] = t;
-      }
-      if (gt == 0) tc::mbar_expect_tx(bar(B_KFULL + bi), (uint32_t)kTile * P.r * 2);
+      tk[gt] = t_next;
+      if (gt == 0) tc::mbar_expect_tx(bar(B_KFULL + bi), tile_bytes);
       tc::named_sync(gbar, kGatherThreads);
-      // latent key rows: gather4 of rows 4g..4g+3, k-block kb
-      {
-        const int g = gt % 32;
-        int rows[4];
+      int rows[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int t = tk[4 * g + j];
-          rows[j] = (int)(cur.off + (t < 0 ? 0 : t));  // no token: weight 0, any valid row
-        }
-        for (int kb = gt / 32; kb < KB; kb += kGatherThreads / 32)
-          tc::tma_gather4(buf_s + kb * 16384u + (uint32_t)(g >> 1) * 1024u + (uint32_t)(g & 1) * 512u,
-                          &tmap_kc, kb * 64, rows[0], rows[1], rows[2], rows[3],
-                          bar(B_KFULL + bi));
+      for (int j = 0; j < 4; ++j) {
+        const int t = tk[4 * g4 + j];
+        rows[j] = (int)(off + (t < 0 ? 0 : t));  // no token: weight 0, any valid row
       }
+      for (int kb = gt / 32; kb < KB; kb += kGatherThreads / 32)
+        tc::tma_gather4(buf_s + kb * 16384u + (uint32_t)(g4 >> 1) * 1024u + (uint32_t)(g4 & 1) * 512u,
+                        &tmap_kc, kb * 64, rows[0], rows[1], rows[2], rows[3], bar(B_KFULL + bi));
+      // next tile of this group: its tokens arrive during this tile
+      cur.next();
+      cur.next();
+      t_next = i + 2 < n ? row_token(P, cur, gt) : -1;
       // the reconstruction is done with the key rows: bring the value rows
       if (!tc::mbar_wait(bar(B_KDONE + bi), ph, P.flags)) break;
-      for (int e = gt; e < kTile * cpr; e += kGatherThreads) {
-        const int m = e / cpr, cc = e % cpr;
-        const int t = tk[m];
-        const __nv_bfloat16* sp = P.Vc + (cur.off + (t < 0 ? 0 : t)) * P.r + cc * 8;
-        const int c = cc * 8;
-        const uint32_t dst = buf_s + (uint32_t)((c >> 6) * 16384 + (m >> 3) * 1024 + (m & 7) * 128 +
-                                                ((((c >> 3) & 7) ^ (m & 7)) << 4));
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(sp) : "memory");
-      }
-      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-      tc::fence_proxy_async_smem();
+      if (gt == 0) tc::mbar_expect_tx(bar(B_VFULL + bi), tile_bytes);
       tc::named_sync(gbar, kGatherThreads);
-      if (gt == 0) tc::mbar_arrive(bar(B_VFULL + bi));
-      cur.next();
-      cur.next();
+      for (int kb = gt / 32; kb < KB; kb += kGatherThreads / 32)
+        tc::tma_gather4(buf_s + kb * 16384u + (uint32_t)(g4 >> 1) * 1024u + (uint32_t)(g4 & 1) * 512u,
+                        &tmap_vc, kb * 64, rows[0], rows[1], rows[2], rows[3], bar(B_VFULL + bi));
+      last_v = i;
     }
+    // this group's copies have all landed before the CTA may exit (a no-op
+    // unless a wait above gave up)
+    if (gt == 0 && last_v >= 0)
+      tc::mbar_wait(bar(B_VFULL + bi), ((uint32_t)last_v >> 1) & 1u, P.flags);
   } else if (warp == kMmaWarp) {
     // ======================= MMA issuer (lane 0) =======================
     if (lane == 0) {
