@@ -64,6 +64,8 @@ def parse_args():
     ap.add_argument("--layers", type=int, default=32)
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle timing on the host cores")
+    ap.add_argument("--no-compress", action="store_true",
+                    help="skip the prefill compression GEMM timing")
     return ap.parse_args()
 
 
@@ -74,6 +76,55 @@ def measured_peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def measured_bf16_peak():
+    """Burst bf16 dense GEMM TFLOP/s (a kernel timed alone)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
+def bench_compress(salsc, dev, reps: int = 20, warmup: int = 3):
+    """The prefill compression GEMM of the LLaMA2-7B-shaped batch (16 x 4096
+    rows of K and V, hidden 4096, r 512), both halves in one salsc_compress
+    call, timed alone with CUDA events; torch.matmul (cuBLAS) on the same
+    operands is timed beside it as a library reference point."""
+    w = workloads.LLAMA2_4K_B16
+    n, hid, r = w.compress_rows, w.hidden, w.rank
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed)
+    K = torch.randn(n, hid, device=dev, generator=g).to(torch.bfloat16)
+    V = torch.randn(n, hid, device=dev, generator=g).to(torch.bfloat16)
+    Pk = torch.linalg.qr(torch.randn(hid, r, device=dev, generator=g))[0].to(torch.bfloat16)
+    Pv = torch.linalg.qr(torch.randn(hid, r, device=dev, generator=g))[0].to(torch.bfloat16)
+    Kc = torch.empty(n, r, dtype=torch.bfloat16, device=dev)
+    Vc = torch.empty_like(Kc)
+    flop = 2 * 2 * n * hid * r
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        for i in range(reps):
+            ev[i].record()
+            fn()
+            ev[i + 1].record()
+        torch.cuda.synchronize(dev)
+        ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(reps)]
+        return statistics.median(ms)
+
+    ms = timed(lambda: salsc.salsc_compress(K, V, Pk, Pv, Kc, Vc))
+    ms_lib = timed(lambda: (torch.matmul(K, Pk, out=Kc), torch.matmul(V, Pv, out=Vc)))
+    peak, kind = measured_bf16_peak()
+    tf = flop / (ms * 1e-3) / 1e12
+    return {"workload": f"{w.name} prefill: 2 x [{n} x {hid}] . [{hid} x {r}] bf16",
+            "us": ms * 1e3, "achieved": tf, "peak": peak, "unit": "TFLOP/s", "bound": "tensor",
+            "frac": tf / peak, "peak_kind": kind,
+            "torch_matmul_us": ms_lib * 1e3,
+            "torch_matmul_tflops": flop / (ms_lib * 1e-3) / 1e12}
 
 
 # ------------------------------------------------------------------ clocks
@@ -412,6 +463,8 @@ def main():
                 "how": "eager salsc_decode_step per layer; q copied in from pinned host memory "
                        "and out copied back every step; host waits for each step"},
     }
+    if not args.no_compress:
+        line["compress"] = bench_compress(salsc, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         line["cpu_baseline"] = cpu_baseline(w, oracle.default_threads())

@@ -281,6 +281,14 @@ salsc_status salsc_compress(const void* K, const void* V, const void* Pk, const 
   if (n_tokens == 0) return SALSC_OK;
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e;
+  if (salsc::compress_tc_supported(hidden, rank, dtype)) {
+    // both halves in one tensor-core launch
+    const void* X[2] = {K ? K : V, V};
+    const void* Pm[2] = {K ? Pk : Pv, Pv};
+    void* Y[2] = {K ? Kc : Vc, Vc};
+    e = salsc::launch_compress_tc(X, Pm, Y, (K && V) ? 2 : 1, n_tokens, hidden, rank, s);
+    return e == cudaSuccess ? SALSC_OK : cuda_fail(e);
+  }
   if (K && (e = salsc::launch_compress(K, Pk, Kc, n_tokens, hidden, rank, dtype, s)) != cudaSuccess)
     return cuda_fail(e);
   if (V && (e = salsc::launch_compress(V, Pv, Vc, n_tokens, hidden, rank, dtype, s)) != cudaSuccess)

@@ -75,6 +75,10 @@ bool attend_tc_supported(const DecodePlan& p);
 cudaError_t launch_attend_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_compress(const void* X, const void* P, void* Y, int64_t n, int hid, int r,
                             salsc_dtype dt, cudaStream_t s);
+bool compress_tc_supported(int hid, int r, salsc_dtype dt);
+// Tensor-core compression of n_mats (1 or 2) matrices X[i] . Pm[i] -> Y[i] in one launch.
+cudaError_t launch_compress_tc(const void* const X[2], const void* const Pm[2], void* const Y[2],
+                               int n_mats, int64_t n, int hid, int r, cudaStream_t s);
 
 // Raise a kernel's dynamic shared-memory limit once per device (not on every
 // launch, so that launches inside CUDA-graph capture make no attribute calls).

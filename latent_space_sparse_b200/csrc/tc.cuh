@@ -55,8 +55,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity completes.  Gives up after
-// `limit_ns` of wall time, sets FLAG_WAIT_TIMEOUT and returns false, so that a
-// broken pipeline ends the kernel instead of hanging the GPU.
+// kWaitLimitNs of wall time, sets FLAG_WAIT_TIMEOUT in *flags (unless flags is
+// null) and returns false, so that a broken pipeline ends the kernel instead of
+// hanging the GPU.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t* flags) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -64,7 +65,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 255u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
-      atomicOr(flags, FLAG_WAIT_TIMEOUT);
+      if (flags) atomicOr(flags, FLAG_WAIT_TIMEOUT);
       return false;
     }
   }
@@ -154,6 +155,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 // Instruction descriptor: bf16 A stored MN-major, bf16 B K-major, fp32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32_amn(int M, int N) {
   return idesc_bf16_f32(M, N) | (1u << 15);
+}
+
+// Instruction descriptor: bf16 A K-major, bf16 B stored MN-major, fp32 D.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) {
+  return idesc_bf16_f32(M, N) | (1u << 16);
 }
 
 // Shared-memory descriptor of an MN-major operand in the 128-byte swizzled

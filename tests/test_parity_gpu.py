@@ -199,3 +199,40 @@ def test_compress_one_half_only():
     salsc.salsc_compress(None, V, None, Pv, None, Vc)
     torch.cuda.synchronize()
     assert max_rel_err(Vc.cpu().numpy(), oracle.compress(x["V"], x["Pv"])) <= TOL["f32"]
+
+
+@pytest.mark.parametrize("rows,hid,r", [
+    (1000, 1024, 256),   # 256-column tiles, two 128-row sub-tiles, ragged last row block
+    (300, 512, 512),     # two latent column tiles
+    (130, 256, 128),     # 128-column tiles, one sub-tile
+    (77, 128, 64),       # 64-column tiles, fewer rows than one block
+    (513, 208, 192),     # hidden not a multiple of 64 (zero-filled K tail), 64-column tiles
+])
+def test_compress_tensor_core_shapes(rows, hid, r):
+    w = W.Workload(name="cmp", batch=1, n_q_heads=1, n_kv_heads=1, head_dim=hid, rank=r,
+                   top_k=1, seq_lens=(rows,), dtype="bf16", rope_base=10000.0, low_rank=16,
+                   seed=rows + hid + r)
+    x = synth.compress_inputs(w, rows=rows)
+    K, V, Pk, Pv = (x[n].to(DEV) for n in ("K", "V", "Pk", "Pv"))
+    Kc = torch.full((rows, r), float("nan"), dtype=torch.bfloat16, device=DEV)
+    Vc = torch.full_like(Kc, float("nan"))
+    salsc.salsc_compress(K, V, Pk, Pv, Kc, Vc)
+    torch.cuda.synchronize()
+    for got, X, P in ((Kc, x["K"], x["Pk"]), (Vc, x["V"], x["Pv"])):
+        ref = oracle.compress(X, P)
+        g = got.float().cpu().numpy()
+        assert np.isfinite(g).all()
+        assert max_rel_err(g, ref) <= TOL["bf16"]
+        assert np.mean(g == oracle.round_storage(ref, "bf16")) > 0.9
+
+
+def test_compress_tensor_core_one_half_only():
+    w = W.LLAMA2_4K_B1
+    rows = 700
+    x = synth.compress_inputs(w, rows=rows)
+    K, Pk = x["K"].to(DEV), x["Pk"].to(DEV)
+    Kc = torch.zeros(rows, w.rank, dtype=torch.bfloat16, device=DEV)
+    salsc.salsc_compress(K, None, Pk, None, Kc, None)
+    torch.cuda.synchronize()
+    ref = oracle.compress(x["K"], x["Pk"])
+    assert max_rel_err(Kc.float().cpu().numpy(), ref) <= TOL["bf16"]
