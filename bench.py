@@ -410,6 +410,7 @@ def main():
     step_bytes = algorithmic_bytes(w, idx_host, elem)
     bytes_layer = float(np.mean(step_bytes))
     peak, peak_kind = measured_peaks()
+    launches = salsc.salsc_decode_launch_count(dec.desc)
     kbytes = kernel_bytes(w, idx_host, elem)
     name = salsc.DECODE_KERNELS[dominant]
     ach = kbytes[name] / (per_kernel_us[dominant] * 1e-6) / 1e9
@@ -450,7 +451,7 @@ def main():
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic", "config": config_of(args, w),
         "clocks": clocks.summary(),
-        "gpu_launches": nk * L * args.steps,
+        "gpu_launches": launches * L * args.steps,
         "roofline": roofline,
         "step_roofline": {"bound": "hbm", "algorithmic_bytes_per_layer_step": bytes_layer,
                           "achieved": step_gbs, "peak": peak, "unit": "GB/s",

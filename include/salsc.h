@@ -145,9 +145,17 @@ salsc_status salsc_decode_step(const salsc_decode_desc* desc, const void* q, con
 
 /*
  * Number of kernels one decode layer-step launches, in order: latent query,
- * latent scoring, top-k, attention over the kept tokens, split merge.
+ * latent scoring, top-k, attention over the kept tokens, split merge (with
+ * the deferred value projection).
  */
 #define SALSC_DECODE_KERNELS 5
+
+/*
+ * Number of kernels salsc_decode_step launches for this descriptor
+ * (SALSC_DECODE_KERNELS for every supported shape), or -1 when the
+ * descriptor is invalid or unsupported.
+ */
+int32_t salsc_decode_launch_count(const salsc_decode_desc* desc);
 
 /*
  * salsc_decode_step with timing marks: the same work, plus

@@ -101,6 +101,7 @@ salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
     p.chunk = chunk;
     p.att_tiles = 0;
   }
+  if (!salsc::combine_supported(p)) return SALSC_ERR_UNSUPPORTED;
   p.scale = D->softmax_scale != 0.0f ? D->softmax_scale : (float)(1.0 / sqrt((double)p.d));
   p.rope_base = D->rope_base;
 
@@ -116,9 +117,8 @@ salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
   p.off_idx = off;
   off = align_up(off + sizeof(int32_t) * (size_t)p.B * p.U * p.k, salsc::kWsAlign);
   p.off_part = off;
-  off = align_up(off + sizeof(float) * (size_t)p.B * p.Hq * p.splits * (p.r + 2), salsc::kWsAlign);
-  p.off_count = off;
-  off = align_up(off + sizeof(int) * (size_t)p.B * p.U, salsc::kWsAlign);
+  off = align_up(off + sizeof(float) * (size_t)p.B * p.Hq * p.splits * salsc::part_row(p.r),
+                 salsc::kWsAlign);
   p.total = off;
   *P = p;
   return SALSC_OK;
@@ -150,6 +150,12 @@ const char* salsc_status_string(salsc_status st) {
 const char* salsc_last_cuda_error(void) { return g_last_cuda_error; }
 
 const char* salsc_version(void) { return "salsc 0.1 (sm_100a)"; }
+
+int32_t salsc_decode_launch_count(const salsc_decode_desc* desc) {
+  salsc::DecodePlan p;
+  if (make_plan(desc, &p) != SALSC_OK) return -1;
+  return SALSC_DECODE_KERNELS;
+}
 
 size_t salsc_decode_workspace_size(const salsc_decode_desc* desc) {
   salsc::DecodePlan p;
@@ -218,7 +224,6 @@ salsc_status decode_step_impl(const salsc_decode_desc* desc, const void* q, cons
   a.qsplit = (__nv_bfloat16*)(w + p.off_qsplit);
   a.scores = (float*)(w + p.off_scores);
   a.part = (float*)(w + p.off_part);
-  a.unit_count = (int*)(w + p.off_count);
 
   cudaStream_t s = (cudaStream_t)stream;
   typedef cudaError_t (*launcher)(const salsc::DecodePlan&, const salsc::DecodeArgs&, cudaStream_t);

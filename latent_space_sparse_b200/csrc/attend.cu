@@ -196,142 +196,14 @@ attend_simt_kernel(const T* __restrict__ q, const T* __restrict__ Kc, const T* _
     const int e = tid + j * kThreads;
     if (e < G * r) {
       const int g = e / r, c = e % r;
-      float* pp = part + (((size_t)b * Hq + u * G + g) * splits + split) * (r + 2);
-      pp[2 + c] = acc[j];
+      float* pp = part + (((size_t)b * Hq + u * G + g) * splits + split) * part_row(r);
+      pp[kPartAcc + c] = acc[j];
     }
   }
   if (tid < G) {
-    float* pp = part + (((size_t)b * Hq + u * G + tid) * splits + split) * (r + 2);
+    float* pp = part + (((size_t)b * Hq + u * G + tid) * splits + split) * part_row(r);
     pp[0] = m_s[tid];
     pp[1] = l_s[tid];
-  }
-}
-
-// Merge the partial results of a selection unit and apply the deferred value
-// projection:
-//   out_h = (sum_s e^{m_s - M} acc_s / sum_s e^{m_s - M} l_s) . Pv_u^T
-// Slot s of head h holds (m, l, acc[r]) or is empty (m = -inf, acc unused);
-// only the first ceil(k_b / chunk) slots are looked at.  CTA (b, u, slice)
-// merges the slots of the unit's G heads and produces output rows
-// slice*32 .. slice*32+31 of each head: every CTA reads only its 32 rows of
-// Pv_u, so the projection's loads are spread over many SMs.  Eight threads
-// share one row (4 x 16-byte loads each) and add their partial dots with
-// shuffles.
-constexpr int kCombThreads = 256;
-constexpr int kCombRows = 32;  // output rows per CTA
-constexpr int kCombHeads = 8;  // heads per unit handled (G <= 8)
-template <typename T>
-__global__ void __launch_bounds__(kCombThreads)
-combine_kernel(const float* __restrict__ part, const T* __restrict__ Pv, T* __restrict__ out,
-               const int64_t* __restrict__ seq_off, int Hq, int U, int G, int d, int r,
-               int splits, int chunk, int k) {
-  __shared__ float accf[kCombHeads][kMaxRank];
-  __shared__ float w_s[kCombHeads][128];
-  __shared__ int seg[128];
-  __shared__ int s_nseg;
-  __shared__ float s_inv[kCombHeads];
-  const int n_slices = (d + kCombRows - 1) / kCombRows;
-  const int slice = blockIdx.x % n_slices;
-  const int bu = blockIdx.x / n_slices;
-  const int b = bu / U, u = bu % U;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  allow_dependent_launch();
-  grid_dependency_wait();  // the partial results come from the previous kernel
-  const int64_t nb = seq_off[b + 1] - seq_off[b];
-  const int64_t kb = nb < k ? nb : k;
-  const int ns = (int)((kb + chunk - 1) / chunk);
-  // ---- slot weights of each head (warp g); the used slots are the same for every head
-  for (int g = warp; g < G; g += kCombThreads / 32) {
-    const float* pp = part + ((size_t)(b * Hq + u * G + g)) * splits * (r + 2);
-    float mv[4], lv[4], M = -INFINITY;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int sl = lane + 32 * q;
-      mv[q] = sl < ns ? pp[(size_t)sl * (r + 2)] : -INFINITY;
-      lv[q] = sl < ns ? pp[(size_t)sl * (r + 2) + 1] : 0.f;
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) M = fmaxf(M, mv[q]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.f;
-    int cnt = 0;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float wv = mv[q] == -INFINITY ? 0.f : expf(mv[q] - M);
-      L += wv * lv[q];
-      const bool used = mv[q] != -INFINITY;
-      const uint32_t mk = __ballot_sync(0xffffffffu, used);
-      if (used) {
-        const int pos = cnt + __popc(mk & ((1u << lane) - 1u));
-        if (g == 0) seg[pos] = lane + 32 * q;
-        w_s[g][pos] = wv;
-      }
-      cnt += __popc(mk);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (lane == 0) {
-      if (g == 0) s_nseg = cnt;
-      s_inv[g] = L > 0.f ? 1.f / L : 0.f;
-    }
-  }
-  __syncthreads();
-  const int nseg = s_nseg;
-  for (int e = threadIdx.x; e < G * r; e += kCombThreads) {
-    const int g = e / r, c = e % r;
-    const float* pp = part + ((size_t)(b * Hq + u * G + g)) * splits * (r + 2) + 2 + c;
-    float a = 0.f;
-    for (int q = 0; q < nseg; ++q) a = fmaf(w_s[g][q], pp[(size_t)seg[q] * (r + 2)], a);
-    accf[g][c] = a * s_inv[g];
-  }
-  __syncthreads();
-  // ---- rows slice*32 + row of Pv_u; thread group of 8 per row, 4 pieces of 16 B each
-  constexpr int kPer = 16 / sizeof(T);  // elements per 16-byte piece
-  const int row = threadIdx.x / 8, sub = threadIdx.x % 8;
-  const int i = slice * kCombRows + row;
-  float o[kCombHeads];
-#pragma unroll
-  for (int g = 0; g < kCombHeads; ++g) o[g] = 0.f;
-  if (i < d) {
-    const T* pv = Pv + ((size_t)u * d + i) * r;
-    // rolled loop over the thread's 16-byte pieces: short code (see latent_q.cu)
-#pragma unroll 1
-    for (int c = sub * kPer; c < r; c += 8 * kPer) {
-      const uint4 v = *(const uint4*)(pv + c);
-      float f[kPer];
-      if (sizeof(T) == 2) {
-        const __nv_bfloat162* h2 = (const __nv_bfloat162*)&v;
-#pragma unroll
-        for (int jj = 0; jj < kPer / 2; ++jj) {
-          const float2 t2 = __bfloat1622float2(h2[jj]);
-          f[2 * jj] = t2.x;
-          f[2 * jj + 1] = t2.y;
-        }
-      } else {
-        const float* t4 = (const float*)&v;
-#pragma unroll
-        for (int jj = 0; jj < kPer; ++jj) f[jj] = t4[jj];
-      }
-#pragma unroll
-      for (int g = 0; g < kCombHeads; ++g) {
-        if (g < G) {
-#pragma unroll
-          for (int jj = 0; jj < kPer; ++jj) o[g] = fmaf(accf[g][c + jj], f[jj], o[g]);
-        }
-      }
-    }
-  }
-#pragma unroll
-  for (int g = 0; g < kCombHeads; ++g) {
-    o[g] += __shfl_xor_sync(0xffffffffu, o[g], 4);
-    o[g] += __shfl_xor_sync(0xffffffffu, o[g], 2);
-    o[g] += __shfl_xor_sync(0xffffffffu, o[g], 1);
-  }
-  if (sub == 0 && i < d) {
-#pragma unroll
-    for (int g = 0; g < kCombHeads; ++g)
-      if (g < G) out[((size_t)b * Hq + u * G + g) * d + i] = from_f32<T>(o[g]);
   }
 }
 
@@ -373,19 +245,6 @@ cudaError_t launch_attend(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
-}
-
-cudaError_t launch_combine(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
-  if (p.splits > 128 || p.G > kCombHeads) return cudaErrorInvalidConfiguration;
-  const int n_slices = (p.d + kCombRows - 1) / kCombRows;
-  const dim3 grid(p.B * p.U * n_slices);
-  if (p.dtype == SALSC_BF16)
-    return launch_k(combine_kernel<__nv_bfloat16>, grid, dim3(kCombThreads), 0, s, true,
-                    (const float*)a.part, (const __nv_bfloat16*)a.Pv, (__nv_bfloat16*)a.out,
-                    (const int64_t*)a.seq_off, p.Hq, p.U, p.G, p.d, p.r, p.splits, p.chunk, p.k);
-  return launch_k(combine_kernel<float>, grid, dim3(kCombThreads), 0, s, true,
-                  (const float*)a.part, (const float*)a.Pv, (float*)a.out,
-                  (const int64_t*)a.seq_off, p.Hq, p.U, p.G, p.d, p.r, p.splits, p.chunk, p.k);
 }
 
 }  // namespace salsc

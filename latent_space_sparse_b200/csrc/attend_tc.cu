@@ -9,8 +9,8 @@
 //      (128-byte swizzled, K-major);
 //   2. tcgen05: K_sel[128 x d] = Kc_tile . Pk_u^T into TMEM (fp32; Pk_u comes
 //      by TMA once per unit and stays in shared memory);
-//   3. the same rows of Vc are gathered into the buffer the MMA has finished
-//      with;
+//   3. the same rows of Vc are gathered (TMA gather4) into the buffer the
+//      MMA has finished with;
 //   4. eight epilogue warps (one thread per token row and half of the RoPE
 //      pairs) read K_sel from TMEM, rotate pair (i, i+d/2) by the angle
 //      t * base^(-2i/d) and dot it with every rotated query head of the unit;
@@ -22,12 +22,14 @@
 //      tile's (m, l, acc) per head;
 //   7. consecutive tiles of one unit in a CTA are folded into a running
 //      (m, l, acc) per head (online softmax rescaling); each CTA publishes one
-//      partial per unit segment at the slot of the segment's first tile and
-//      marks its other slots empty.  The combine kernel merges the few
-//      segments of a unit and applies the deferred Pv_u^T.
+//      partial per unit segment, at the slot of the segment's first tile.  A
+//      segment starts at a unit's first tile and at every CTA's first tile,
+//      so the combine kernel finds the used slots from the tile partition
+//      alone; it merges the few segments of a unit and applies the deferred
+//      Pv_u^T.
 // Warp roles (544 threads): warps 0-7 epilogue, warp 8 TMEM owner and MMA
 // issuer, warps 9-12 and 13-16 row gathers (one group of four per tile
-// buffer; latent keys by TMA gather4, latent values by cp.async).  Each CTA walks a contiguous range of tiles;
+// buffer; latent key and value rows by TMA gather4).  Each CTA walks a contiguous range of tiles;
 // the two tile buffers alternate (Kc(i) -> Vc(i) -> Kc(i+2)), so the
 // reconstruction of tile i+1 runs during the epilogue of tile i.
 //
@@ -55,9 +57,6 @@ struct AttendTcParams {
   const __nv_bfloat16* q;
   const __nv_bfloat16* Kc;
   const __nv_bfloat16* Vc;
-  const __nv_bfloat16* Pv;
-  __nv_bfloat16* out;
-  int* unit_count;
   const int32_t* idx;
   const int64_t* seq_off;
   const int32_t* q_pos;
@@ -156,11 +155,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
   float* const s_lg = s_pd + 2 * G * kTile;                  // [G][128] logits -> weights
   float* const s_stat = s_lg + G * kTile;                    // [G][2] (m, l)
   int* const s_tok = (int*)(s_stat + 2 * G);                 // [2][128] token per row
-  int* const s_last = s_tok + 2 * kTile;                     // [1] this tile closes its unit
-  float* const s_run = (float*)(s_last + 2);                 // [G][2] segment's running (m, l)
+  float* const s_run = (float*)(s_tok + 2 * kTile);          // [G][2] segment's running (m, l)
   float* const s_ab = s_run + 2 * G;                         // [G][2] rescale factors
-  int* const s_segs = (int*)(s_ab + 2 * G);                  // [128] segment start slots
-  uint64_t* const s_bars = (uint64_t*)(((uintptr_t)(s_segs + kTile) + 7) & ~(uintptr_t)7);
+  uint64_t* const s_bars = (uint64_t*)(((uintptr_t)(s_ab + 2 * G) + 7) & ~(uintptr_t)7);
   uint32_t* const s_tmem_slot = (uint32_t*)(s_bars + B_COUNT);
   const uint32_t bar0 = tc::smem_u32(s_bars);
   auto bar = [bar0](int i) { return bar0 + 8u * (uint32_t)i; };
@@ -494,8 +491,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
           acc_run[g] = acc_run[g] * s_ab[2 * g] +
                        (__uint_as_float(v[2 * g]) + __uint_as_float(v[2 * g + 1])) * s_ab[2 * g + 1];
       }
-      // ---- end of this CTA's segment of the unit: publish it, and merge the
-      //      unit if every tile has arrived
+      // ---- end of this CTA's segment of the unit: publish it
       UnitTileCursor nx = cur;
       nx.next();
       const bool seg_end = i + 1 == n || nx.b != cur.b || nx.u != cur.u;
@@ -503,17 +499,16 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       if (seg_end) {
         const int s0 = cur.slot + 1 - seg_tiles;  // first slot of the segment
         const int c = half * 128 + quarter * 32 + lane;
+        const int64_t row0 = ((int64_t)cur.b * P.Hq + cur.u * G) * P.n_slots + s0;
         if (half < n_chunks && c < P.r) {
 #pragma unroll
           for (int g = 0; g < G; ++g)
-            P.part[(((int64_t)cur.b * P.Hq + cur.u * G + g) * P.n_slots + s0) * (P.r + 2) + 2 + c] =
-                acc_run[g];
+            P.part[(row0 + (int64_t)g * P.n_slots) * part_row(P.r) + kPartAcc + c] = acc_run[g];
         }
-        for (int e = tid; e < G * seg_tiles; e += kEpiThreads) {
-          const int g = e / seg_tiles, sl = s0 + e % seg_tiles;
-          float* pp = P.part + (((int64_t)cur.b * P.Hq + cur.u * G + g) * P.n_slots + sl) * (P.r + 2);
-          pp[0] = sl == s0 ? s_run[2 * g] : -INFINITY;  // only the segment's first slot is used
-          pp[1] = sl == s0 ? s_run[2 * g + 1] : 0.f;
+        if (tid < G) {
+          float* pp = P.part + (row0 + (int64_t)tid * P.n_slots) * part_row(P.r);
+          pp[0] = s_run[2 * tid];
+          pp[1] = s_run[2 * tid + 1];
         }
         // a new segment starts with the next tile
         seg_tiles = 0;
@@ -552,7 +547,7 @@ template <int G, int D>
 size_t smem_bytes(int r) {
   const int KB = r / 64;
   return 1024 + (size_t)KB * D * 128 + 2 * (size_t)KB * 16384 + 2 * 4096 + 8 * (D / 2) * 2 +
-         4 * (G * D + 2 * G * kTile + G * kTile + 2 * G + 2 * kTile + 2 + 4 * G + kTile) + 8 +
+         4 * (G * D + 2 * G * kTile + G * kTile + 2 * G + 2 * kTile + 4 * G) + 8 +
          8 * B_COUNT + 16;
 }
 
@@ -571,9 +566,6 @@ cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s)
   P.q = (const __nv_bfloat16*)a.q;
   P.Kc = (const __nv_bfloat16*)a.Kc;
   P.Vc = (const __nv_bfloat16*)a.Vc;
-  P.Pv = (const __nv_bfloat16*)a.Pv;
-  P.out = (__nv_bfloat16*)a.out;
-  P.unit_count = a.unit_count;
   P.idx = a.idx;
   P.seq_off = a.seq_off;
   P.q_pos = a.q_pos;
@@ -588,18 +580,21 @@ cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s)
   P.n_tiles = p.att_tiles;
   P.scale = p.scale;
   P.base = p.rope_base;
-  const int grid = p.att_tiles < num_sms_att() ? p.att_tiles : num_sms_att();
-  return launch_k(attend_tc_kernel<G, D>, dim3(grid), dim3(kThreads), smem, s, true, tpk, tkc, tvc,
-                  P);
+  return launch_k(attend_tc_kernel<G, D>, dim3(attend_tc_grid(p)), dim3(kThreads), smem, s, true,
+                  tpk, tkc, tvc, P);
 }
 
 }  // namespace
+
+int attend_tc_grid(const DecodePlan& p) {
+  return p.att_tiles < num_sms_att() ? p.att_tiles : num_sms_att();
+}
 
 bool attend_tc_supported(const DecodePlan& p) {
   const int64_t k_eff = p.k < p.n_max ? p.k : p.n_max;
   return p.dtype == SALSC_BF16 && p.r % 64 == 0 && p.r <= 256 && (p.d == 64 || p.d == 128) &&
          (p.G == 1 || p.G == 2 || p.G == 4 || p.G == 8) && p.N <= INT32_MAX &&
-         (k_eff + kTile - 1) / kTile <= kTile;  // the merge keeps <= 128 tile weights per head
+         (k_eff + kTile - 1) / kTile <= kTile;  // the merge takes <= 128 slots per unit
 }
 
 cudaError_t launch_attend_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {

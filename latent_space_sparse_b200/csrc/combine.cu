@@ -1,0 +1,284 @@
+// combine.cu -- merge of a unit's split partials and the deferred value
+// projection.
+//
+// The attention kernels split the kept tokens of a selection unit (b, u)
+// over several slots; slot s of query head h holds (m, l, acc[r]): the
+// running maximum logit, the softmax normaliser and the unnormalised latent
+// value sum of its tokens.  The merge is the exact online-softmax combination
+//   M = max_s m_s,  w_s = e^{m_s - M},  L = sum_s w_s l_s,
+//   acc = sum_s w_s acc_s / L,
+// and the output is out_h = acc . Pv_u^T (SALS technical framework, stage 4:
+// the value projection is applied once, after the weighted sum of latent
+// rows, which is exact by associativity).
+//
+// CTA (b, u, slice) produces output rows slice*16 .. slice*16+15 of the G
+// heads of unit u.  Its loads are whole-row bulk copies into shared memory,
+// so that they are in flight together while the code stays short (the
+// kernel runs once per SM and layer-step; every instruction it executes once
+// is a cold instruction fetch): the 32 rows of Pv_u are copied before the
+// dependency wait (Pv is a weight, not an output of the attention kernel),
+// the used partial rows after it.  Used slots: with the tensor-core
+// attention, a slot holds a partial when a CTA's contiguous range of tiles
+// starts there or the unit starts there, which follows from the tile
+// partition; with the CUDA-core attention every slot of the unit is used.
+// The sums run over slots in slot order, so the result is deterministic.
+#include "tc.cuh"
+
+namespace salsc {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kRows = 16;                      // output rows per CTA
+constexpr int kTpr = kThreads / kRows;         // threads per output row
+constexpr int kColsPer = kMaxRank / kThreads;  // latent columns per thread (r <= 512)
+constexpr uint32_t kRowBuf = 32u * 1024u;      // bytes of partial rows per batch
+constexpr int kMaxSegs = 128;
+
+struct CombineParams {
+  const float* part;
+  const void* Pv;
+  void* out;
+  const int64_t* seq_off;
+  uint32_t* flags;
+  int B, Hq, U, d, r, k, n_slots, chunk;
+  int seg_grid, seg_tiles;  // tensor-core tile partition (seg_grid = 0: every slot used)
+};
+
+template <typename T, int G>
+__global__ void __launch_bounds__(kThreads)
+combine_kernel(const CombineParams P) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int rowf = part_row(P.r);  // floats per partial row
+  T* const pv_s = (T*)smem;                                                 // [16][r]
+  float* const rows_s = (float*)(smem + (size_t)kRows * P.r * sizeof(T));  // batch of rows
+  float* const acc_s = rows_s + kRowBuf / 4;                                // [G][r]
+  float* const w_s = acc_s + G * P.r;                                       // [G][32]
+  __shared__ int s_seg[kMaxSegs];
+  __shared__ int s_nseg, s_ok;
+  __shared__ float s_scale[G], s_L[G], s_M[G];
+  __shared__ __align__(8) uint64_t s_bar[2];
+  const uint32_t bar_pv = tc::smem_u32(&s_bar[0]), bar_rows = tc::smem_u32(&s_bar[1]);
+
+  const int n_slices = P.d / kRows;
+  const int slice = blockIdx.x % n_slices;
+  const int bu = blockIdx.x / n_slices;
+  const int b = bu / P.U, u = bu % P.U;
+  const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+  const uint32_t pv_bytes = (uint32_t)(kRows * P.r * sizeof(T));
+  if (tid == 0) {
+    tc::mbar_init(bar_pv, 1);
+    tc::mbar_init(bar_rows, 1);
+    tc::mbar_fence_init();
+    // the 16 rows of Pv_u: a weight, copied before the dependency wait
+    tc::mbar_expect_tx(bar_pv, pv_bytes);
+    tc::bulk_load(tc::smem_u32(pv_s),
+                  (const T*)P.Pv + ((int64_t)u * P.d + (int64_t)slice * kRows) * P.r, pv_bytes,
+                  bar_pv);
+  }
+  allow_dependent_launch();
+  grid_dependency_wait();  // the partials come from the attention kernel
+  if (warp == 0) {
+    // slots of unit (b, u) and, with the tile partition, the unit's first tile:
+    // every lane reads one sequence's offsets, a warp scan sums the tiles
+    int64_t before = 0;  // tiles of the sequences before b
+    int tb = 0;
+    for (int b0 = 0; b0 <= b; b0 += 32) {
+      const int bb = b0 + lane;
+      int64_t t = 0;
+      if (bb <= b && bb < P.B) {
+        const int64_t n2 = P.seq_off[bb + 1] - P.seq_off[bb];
+        const int64_t k2 = n2 < P.k ? n2 : P.k;
+        t = (k2 + P.chunk - 1) / P.chunk;
+        if (bb == b) tb = (int)t;
+      }
+      int64_t x = bb < b ? t : 0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+      before += x;
+    }
+    tb = __reduce_max_sync(0xffffffffu, tb);  // set by the lane of sequence b only
+    const int64_t unit_tile0 = before * P.U + (int64_t)u * tb;
+    int cnt = 0;
+    for (int s0 = 0; s0 < tb; s0 += 32) {
+      const int sl = s0 + lane;
+      bool used = sl < tb;
+      if (used && sl > 0 && P.seg_grid > 0) {
+        const int64_t t = unit_tile0 + sl;
+        const int64_t c = (t * P.seg_grid + P.seg_tiles - 1) / P.seg_tiles;  // first CTA at or after t
+        used = c < P.seg_grid && c * P.seg_tiles / P.seg_grid == t;
+      }
+      const uint32_t mk = __ballot_sync(0xffffffffu, used);
+      if (used) s_seg[cnt + __popc(mk & ((1u << lane) - 1u))] = sl;
+      cnt += __popc(mk);
+    }
+    if (lane == 0) s_nseg = cnt;
+    if (lane < G) {
+      s_M[lane] = -INFINITY;
+      s_L[lane] = 0.f;
+    }
+  }
+  __syncthreads();
+  const int nseg = s_nseg;
+  // this thread's latent columns tid, tid + 256 for every head
+  float acc[G][kColsPer];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int j = 0; j < kColsPer; ++j) acc[g][j] = 0.f;
+  int bs = (int)(kRowBuf / (uint32_t)(rowf * 4)) / G;  // slots per batch
+  if (bs * G > 32) bs = 32 / G;  // one row copy per lane of warp 0
+  const float* part_u = P.part + ((int64_t)b * P.Hq + (int64_t)u * G) * P.n_slots * rowf;
+  uint32_t phase = 0;
+  bool ok = true;
+  for (int q0 = 0; q0 < nseg; q0 += bs, phase ^= 1u) {
+    const int nq = nseg - q0 < bs ? nseg - q0 : bs;
+    if (warp == 0) {
+      // lane e copies row e = (head e / nq, slot q0 + e % nq); one warp waits
+      if (lane == 0) tc::mbar_expect_tx(bar_rows, (uint32_t)(G * nq * rowf * 4));
+      __syncwarp();
+      if (lane < G * nq) {
+        const int g = lane / nq, j = lane % nq;
+        tc::bulk_load(tc::smem_u32(rows_s + (size_t)lane * rowf),
+                      part_u + ((int64_t)g * P.n_slots + s_seg[q0 + j]) * rowf,
+                      (uint32_t)(rowf * 4), bar_rows);
+      }
+      ok = tc::mbar_wait(bar_rows, phase, P.flags) && ok;
+    }
+    __syncthreads();
+    // weights of this batch: warp g, lane j
+    if (warp < G) {
+      const int g = warp;
+      const float m = lane < nq ? rows_s[(size_t)(g * nq + lane) * rowf] : -INFINITY;
+      const float l = lane < nq ? rows_s[(size_t)(g * nq + lane) * rowf + 1] : 0.f;
+      float mb = m;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+      const float Mo = s_M[g], Mn = fmaxf(Mo, mb);
+      const float sc = Mo == -INFINITY ? 0.f : expf(Mo - Mn);
+      const float w = m == -INFINITY ? 0.f : expf(m - Mn);
+      float wl = w * l;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) wl += __shfl_xor_sync(0xffffffffu, wl, o);
+      if (lane < nq) w_s[g * 32 + lane] = w;
+      __syncwarp();
+      if (lane == 0) {
+        s_scale[g] = sc;
+        s_L[g] = s_L[g] * sc + wl;
+        s_M[g] = Mn;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kColsPer; ++j) {
+      const int c = tid + j * kThreads;
+      if (c < P.r) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float a = acc[g][j] * s_scale[g];
+          for (int q = 0; q < nq; ++q)
+            a = fmaf(w_s[g * 32 + q], rows_s[(size_t)(g * nq + q) * rowf + kPartAcc + c], a);
+          acc[g][j] = a;
+        }
+      }
+    }
+    __syncthreads();  // the row buffer is refilled by the next batch
+  }
+#pragma unroll
+  for (int j = 0; j < kColsPer; ++j) {
+    const int c = tid + j * kThreads;
+    if (c < P.r) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) acc_s[g * P.r + c] = s_L[g] > 0.f ? acc[g][j] / s_L[g] : 0.f;
+    }
+  }
+  if (warp == 0) {
+    ok = tc::mbar_wait(bar_pv, 0, P.flags) && ok;
+    if (lane == 0) s_ok = ok;
+  }
+  __syncthreads();
+  // out row i = slice*16 + tid/16: the row's 16 threads take interleaved
+  // groups of 4 latent columns, then add up with shuffles
+  const int i = tid / kTpr, part = tid % kTpr;
+  float o[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) o[g] = 0.f;
+  const T* pvr = pv_s + (size_t)i * P.r;
+#pragma unroll 2
+  for (int c = part * 4; c < P.r; c += 4 * kTpr) {
+    float f[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) f[e] = to_f32(pvr[c + e]);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float4 a4 = *(const float4*)(acc_s + g * P.r + c);
+      o[g] = fmaf(a4.x, f[0], fmaf(a4.y, f[1], fmaf(a4.z, f[2], fmaf(a4.w, f[3], o[g]))));
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int off = kTpr / 2; off > 0; off >>= 1) o[g] += __shfl_xor_sync(0xffffffffu, o[g], off);
+  if (part == 0 && s_ok) {
+    T* out = (T*)P.out + ((int64_t)b * P.Hq + (int64_t)u * G) * P.d + slice * kRows + i;
+#pragma unroll
+    for (int g = 0; g < G; ++g) out[(int64_t)g * P.d] = from_f32<T>(o[g]);
+  }
+}
+
+size_t combine_smem(const DecodePlan& p) {
+  const size_t elem = p.dtype == SALSC_BF16 ? 2 : 4;
+  return (size_t)kRows * p.r * elem + kRowBuf + sizeof(float) * (size_t)p.G * (p.r + 32);
+}
+
+template <typename T, int G>
+cudaError_t launch_tg(const CombineParams& P, const DecodePlan& p, cudaStream_t s) {
+  static int done[kMaxDevices] = {};
+  const size_t smem = combine_smem(p);
+  cudaError_t e = ensure_smem(combine_kernel<T, G>, smem, done);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)(p.B * p.U * (p.d / kRows)));
+  return launch_k(combine_kernel<T, G>, grid, dim3(kThreads), smem, s, true, P);
+}
+
+template <typename T>
+cudaError_t launch_t(const CombineParams& P, const DecodePlan& p, cudaStream_t s) {
+  switch (p.G) {
+    case 1: return launch_tg<T, 1>(P, p, s);
+    case 2: return launch_tg<T, 2>(P, p, s);
+    case 4: return launch_tg<T, 4>(P, p, s);
+    case 8: return launch_tg<T, 8>(P, p, s);
+  }
+  return cudaErrorInvalidConfiguration;
+}
+
+}  // namespace
+
+bool combine_supported(const DecodePlan& p) {
+  // one row of partials per head fits the row buffer; the used slots of a unit
+  // fit the segment list
+  return (p.G == 1 || p.G == 2 || p.G == 4 || p.G == 8) && p.r <= kMaxRank && p.d % kRows == 0 &&
+         (uint32_t)(p.G * part_row(p.r) * 4) <= kRowBuf && p.splits <= kMaxSegs;
+}
+
+cudaError_t launch_combine(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
+  if (!combine_supported(p)) return cudaErrorInvalidConfiguration;
+  CombineParams P;
+  P.part = a.part;
+  P.Pv = a.Pv;
+  P.out = a.out;
+  P.seq_off = a.seq_off;
+  P.flags = a.flags;
+  P.B = p.B;
+  P.Hq = p.Hq;
+  P.U = p.U;
+  P.d = p.d;
+  P.r = p.r;
+  P.k = p.k;
+  P.n_slots = p.splits;
+  P.chunk = p.chunk;
+  P.seg_grid = p.attend_tc ? attend_tc_grid(p) : 0;
+  P.seg_tiles = p.att_tiles;
+  return p.dtype == SALSC_BF16 ? launch_t<__nv_bfloat16>(P, p, s) : launch_t<float>(P, p, s);
+}
+
+}  // namespace salsc

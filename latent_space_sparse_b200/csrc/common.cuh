@@ -20,6 +20,12 @@ enum : uint32_t {
 };
 
 constexpr int kMaxRank = 512;
+
+// Split partials: one row of part_row(r) floats per (sequence, query head,
+// slot): m, l, two unused words, then acc[r] at kPartAcc, so that every row
+// starts on a 16-byte boundary (rows are copied whole with cp.async.bulk).
+constexpr int kPartAcc = 4;
+__host__ __device__ constexpr int part_row(int r) { return r + kPartAcc; }
 constexpr int kMaxHeadDim = 128;
 constexpr size_t kWsAlign = 256;
 
@@ -40,7 +46,7 @@ struct DecodePlan {
   float scale;
   double rope_base;
   // workspace layout (byte offsets)
-  size_t off_flags, off_qlat, off_qsplit, off_scores, off_idx, off_part, off_count, total;
+  size_t off_flags, off_qlat, off_qsplit, off_scores, off_idx, off_part, total;
 };
 
 // Raw pointers of one decode call, passed to the launchers.
@@ -58,8 +64,7 @@ struct DecodeArgs {
   float* qlat;                 // [B][U][r]
   __nv_bfloat16* qsplit;       // [B][npad][r]: row 2u = hi(q_lat[u]), 2u+1 = lo, rest zero
   float* scores;               // packed per (b,u)
-  float* part;                 // [B][Hq][splits][r+2]
-  int* unit_count;             // [B][U] tiles finished per selection unit (tensor-core path)
+  float* part;                 // [B][Hq][splits][part_row(r)]
 };
 
 // Record a CUDA error for salsc_last_cuda_error() and return SALSC_ERR_CUDA.
@@ -72,6 +77,8 @@ cudaError_t launch_topk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s
 cudaError_t launch_attend(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 bool attend_tc_supported(const DecodePlan& p);
+int attend_tc_grid(const DecodePlan& p);  // CTAs of the tensor-core attention (tile partition)
+bool combine_supported(const DecodePlan& p);
 cudaError_t launch_attend_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_compress(const void* X, const void* P, void* Y, int64_t n, int hid, int r,
                             salsc_dtype dt, cudaStream_t s);

@@ -7,15 +7,21 @@
 //
 // Design: C CTAs (a thread-block cluster when C > 1) own one unit.  Each CTA
 // loads a contiguous slice of the unit's scores into shared memory once, as
-// 32-bit keys whose unsigned order is the float order, and the unit's key
-// range [kmin, kmax] is found.  A radix select on rel = key - kmin with
-// 11-bit digits, starting at the top bit of the range (at most three
-// passes), finds the exact k_b-th largest key T: each CTA histograms its
-// slice into 2048 bins (keys spread over the bins, so the shared-memory
-// atomics barely contend), the C histograms are summed through distributed
-// shared memory, and every CTA picks the same digit with a block-wide scan.  The final compaction gives every warp a contiguous segment of the
-// slice: one counting pass, one prefix over warps (and cluster ranks), one
-// writing pass with warp ballots.  Output order is the index order of the
+// 32-bit keys whose unsigned order is the float order, and the unit's score
+// range [min, max] is found.  Each CTA histograms its slice into 2048 bins of
+// equal width over that range (the bin is a monotone function of the score,
+// and scores spread over many bins, so the shared-memory atomics barely
+// contend); the C histograms are summed through distributed shared memory and
+// every CTA finds, with a block-wide scan, the bin that holds the k_b-th
+// largest score.  The pairs (key, index) of that bin are few for any smooth
+// score distribution: they are gathered from the cluster, and the one whose
+// rank (score descending, index ascending) is the number still needed gives
+// the exact threshold T.  When that bin holds more than kCand pairs (heavily
+// repeated or extreme scores), a radix select on rel = key - kmin with 11-bit
+// digits, starting at the top bit of the key range (at most three passes),
+// finds T instead.  The final compaction gives every warp a contiguous
+// segment of the slice: one counting pass, one prefix over warps (and cluster
+// ranks), one writing pass with warp ballots.  Output order is the index order of the
 // keys > T followed by the lowest-index keys == T, so the result is
 // deterministic.  No full sort, no global-memory scratch.
 #include <cooperative_groups.h>
@@ -30,6 +36,7 @@ namespace {
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBatch = 32;  // keys a thread loads before converting them
+constexpr int kMaxCluster = 8;  // largest cluster of CTAs per unit
 
 // Unsigned key with the same order as the float; -0 and +0 map to one key.
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -38,8 +45,22 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Float whose order_key is `key` (-0 comes back as +0).
+__device__ __forceinline__ float key_float(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
 constexpr int kBins = 2048;  // 11-bit digits
 constexpr int kDigit = 11;
+constexpr int kCand = 1024;  // most candidates the boundary bin may hold for the fast path
+
+// Bin of a key in the linear partition of [fmin, fmax] into kBins bins: a
+// composition of monotone roundings, so a larger score never lands in a lower
+// bin and equal scores share a bin.
+__device__ __forceinline__ int linear_bin(uint32_t key, float fmin, float scale) {
+  const float x = (key_float(key) - fmin) * scale;
+  return min(kBins - 1, (int)x);
+}
 
 // Block-wide search for the digit that holds the target rank: `cnt` holds the
 // histogram (ascending bins); bins are scanned from the top.  Thread t looks
@@ -97,9 +118,13 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
   __shared__ uint32_t counts[2];  // this CTA's (#keys > T, #keys == T), read by the cluster
   __shared__ uint32_t wcnt[kWarps][2];
   __shared__ uint32_t wbase[kWarps][2];
-  __shared__ uint32_t s_digit, s_above, s_base_gt, s_base_eq;
+  __shared__ uint32_t s_digit, s_above, s_base_gt, s_base_eq, s_ncand;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // shared memory of cluster rank q (this CTA's own when not a cluster)
+  auto remote = [&](uint32_t* ptr, int q) -> uint32_t* {
+    return kCluster ? cluster.map_shared_rank(ptr, q) : ptr;
+  };
   allow_dependent_launch();
   const int64_t off = seq_off[b];
   const int64_t nb = seq_off[b + 1] - off;
@@ -155,10 +180,13 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
     cluster.sync();
     if (tid == 0) {
       uint32_t a = 0xffffffffu, z = 0u;
-      for (int q = 0; q < C; ++q) {
-        const uint32_t* r = cluster.map_shared_rank(mm, q);
-        a = min(a, r[0]);
-        z = max(z, r[1]);
+#pragma unroll
+      for (int q = 0; q < kMaxCluster; ++q) {
+        if (q < C) {
+          const uint32_t* r = remote(mm, q);
+          a = min(a, r[0]);
+          z = max(z, r[1]);
+        }
       }
       wsum[0] = a;
       wsum[1] = z;
@@ -179,9 +207,95 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
   uint32_t remaining = (uint32_t)kb;
   uint32_t T = 0u;
   const int n_iter = (n_loc + kThreads - 1) / kThreads;
+  bool resolved = false;
   if (kb == nb) {
     remaining = 0u;  // keep everything: every finite score has key > 0
+    resolved = true;
   } else {
+    // ---- linear pass: bins of equal width over [min score, max score]
+    const float fmin = key_float(kmin), fmax = key_float(kmax);
+    const float frange = fmax - fmin;
+    const float scale = (float)kBins / frange;
+    if (isfinite(frange) && frange > 0.f && isfinite(scale)) {
+      uint32_t* h = hist[0];
+      for (int i = tid; i < kBins; i += kThreads) h[i] = 0u;
+      __syncthreads();
+      for (int it = 0; it < n_iter; ++it) {
+        const int i = it * kThreads + tid;
+        if (i < n_loc) atomicAdd(&h[linear_bin(keys[i], fmin, scale)], 1u);
+      }
+      const uint32_t* cnt = h;
+      if (kCluster) {
+        cluster.sync();
+        for (int i = tid; i < kBins; i += kThreads) {
+          uint32_t t = 0u;
+#pragma unroll
+          for (int q = 0; q < kMaxCluster; ++q)
+            if (q < C) t += remote(h, q)[i];
+          total[i] = t;
+        }
+        cnt = total;
+      }
+      __syncthreads();
+      find_digit(cnt, (uint32_t)kb, kBins, wsum, &s_digit, &s_above);
+      __syncthreads();
+      const int bstar = (int)s_digit;
+      const uint32_t need = (uint32_t)kb - s_above;  // 1 <= need <= cnt[bstar]
+      const uint32_t n_cand = cnt[bstar];
+      if (n_cand <= (uint32_t)kCand) {
+        // ---- the boundary bin's (key, index) pairs: a short list per CTA ...
+        uint32_t* loc = hist[1];  // [kCand] keys, then [kCand] indices
+        if (tid == 0) s_ncand = 0u;
+        __syncthreads();
+        for (int it = 0; it < n_iter; ++it) {
+          const int i = it * kThreads + tid;
+          if (i < n_loc && linear_bin(keys[i], fmin, scale) == bstar) {
+            const uint32_t pos = atomicAdd(&s_ncand, 1u);
+            loc[pos] = keys[i];
+            loc[kCand + pos] = (uint32_t)(lo + i);
+          }
+        }
+        if (kCluster) cluster.sync(); else __syncthreads();
+        // ... merged in rank order into `total`: [n_cand] keys, then [n_cand] indices
+        uint32_t base = 0u;
+#pragma unroll
+        for (int q = 0; q < kMaxCluster; ++q) {
+          if (q < C) {
+            uint32_t* rl = remote(loc, q);
+            const uint32_t nq = *remote(&s_ncand, q);
+            for (uint32_t j = tid; j < nq; j += kThreads) {
+              total[base + j] = rl[j];
+              total[kCand + base + j] = rl[kCand + j];
+            }
+            base += nq;
+          }
+        }
+        __syncthreads();
+        // ---- the need-th best pair (score descending, index ascending) is the threshold
+        for (uint32_t t = tid; t < n_cand; t += kThreads) {
+          const uint32_t kt = total[t], it_ = total[kCand + t];
+          uint32_t better = 0u, eq_le = 0u;
+          for (uint32_t j = 0; j < n_cand; ++j) {
+            const uint32_t kj = total[j], ij = total[kCand + j];
+            better += (kj > kt) || (kj == kt && ij < it_);
+            eq_le += (kj == kt) && (ij <= it_);
+          }
+          if (better == need - 1u) {
+            s_digit = kt;     // T
+            s_above = eq_le;  // keys equal to T that are kept
+          }
+        }
+        __syncthreads();
+        T = s_digit;
+        remaining = s_above;
+        resolved = true;
+      } else if (kCluster) {
+        cluster.sync();  // the other CTAs have read this pass's histogram before it is reused
+      }
+    }
+  }
+  if (!resolved) {
+    // ---- fallback: radix select over the keys' bits
     const uint32_t range = kmax - kmin;
     int hi_bit = range == 0u ? 0 : 32 - __clz(range);  // bits of rel still to resolve: [0, hi_bit)
     int pass = 0;
@@ -204,7 +318,9 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
         cluster.sync();
         for (int i = tid; i < kBins; i += kThreads) {
           uint32_t t = 0u;
-          for (int q = 0; q < C; ++q) t += cluster.map_shared_rank(h, q)[i];
+#pragma unroll
+          for (int q = 0; q < kMaxCluster; ++q)
+            if (q < C) t += remote(h, q)[i];
           total[i] = t;
         }
         cnt = total;
@@ -264,10 +380,13 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
     cluster.sync();
     if (tid == 0) {
       uint32_t g = 0u, e = 0u;
-      for (int q = 0; q < rank; ++q) {
-        const uint32_t* rc = cluster.map_shared_rank(counts, q);
-        g += rc[0];
-        e += rc[1];
+#pragma unroll
+      for (int q = 0; q < kMaxCluster; ++q) {
+        if (q < rank) {
+          const uint32_t* rc = remote(counts, q);
+          g += rc[0];
+          e += rc[1];
+        }
       }
       s_base_gt = g;
       s_base_eq = e;

@@ -23,7 +23,7 @@ WS_ALIGN = 256
 
 EXPORTS = (
     "salsc_compress", "salsc_decode_workspace_size", "salsc_decode_prepare", "salsc_decode_step",
-    "salsc_decode_step_timed", "salsc_decode_step_static_ws", "salsc_decode_read_flags", "salsc_status_string", "salsc_last_cuda_error", "salsc_version",
+    "salsc_decode_step_timed", "salsc_decode_step_static_ws", "salsc_decode_launch_count", "salsc_decode_read_flags", "salsc_status_string", "salsc_last_cuda_error", "salsc_version",
 )
 
 
@@ -73,6 +73,8 @@ def _lib():
         lib.salsc_decode_prepare.argtypes = [dp, vp, sz, vp]
         lib.salsc_decode_step.restype = ctypes.c_int
         lib.salsc_decode_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.salsc_decode_launch_count.restype = ctypes.c_int32
+        lib.salsc_decode_launch_count.argtypes = [dp]
         lib.salsc_decode_step_timed.restype = ctypes.c_int
         lib.salsc_decode_step_timed.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
                                                 ctypes.POINTER(ctypes.c_void_p), i32]
@@ -168,6 +170,14 @@ def salsc_decode_step(desc: DecodeDesc, q, Kc, Vc, Pk, Pv, out, idx_out, ws, str
 
 
 DECODE_KERNELS = ("latent_q", "score", "topk", "attend", "combine")
+
+
+def salsc_decode_launch_count(desc: DecodeDesc) -> int:
+    """Kernels one salsc_decode_step launches for this descriptor (4 or 5)."""
+    n = _lib().salsc_decode_launch_count(ctypes.byref(desc))
+    if n < 0:
+        raise ValueError("salsc_decode_launch_count: invalid or unsupported descriptor")
+    return n
 
 
 def salsc_decode_step_timed(desc: DecodeDesc, q, Kc, Vc, Pk, Pv, out, idx_out, ws, events,

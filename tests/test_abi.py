@@ -53,6 +53,13 @@ def test_workspace_size_valid_shapes_grow_with_tokens():
     assert small % 256 == 0
 
 
+def test_launch_count():
+    for kw in (dict(rank=256), dict(rank=512), dict(dtype=torch.float32)):
+        assert salsc.salsc_decode_launch_count(desc([0, 1000], **kw)) == 5
+    with pytest.raises(ValueError):
+        salsc.salsc_decode_launch_count(desc([0, 10], top_k=0))
+
+
 @pytest.mark.parametrize("kw,offs", [
     (dict(n_q_heads=30), [0, 10]),             # Hq not a multiple of Hkv
     (dict(head_dim=127), [0, 10]),             # odd head dim
