@@ -50,6 +50,7 @@ salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
   // shapes with kernels
   if (D->head_dim != 64 && D->head_dim != 128) return SALSC_ERR_UNSUPPORTED;
   if (D->rank > salsc::kMaxRank) return SALSC_ERR_UNSUPPORTED;
+  if (D->n_kv_heads > salsc::kMaxUnits) return SALSC_ERR_UNSUPPORTED;
   if (D->dtype == SALSC_BF16 && D->rank % 64 != 0) return SALSC_ERR_UNSUPPORTED;
   if (D->dtype == SALSC_F32 && D->rank % 4 != 0) return SALSC_ERR_UNSUPPORTED;
   if (D->rank > D->n_kv_heads * D->head_dim) return SALSC_ERR_INVALID_ARG;
@@ -114,6 +115,8 @@ salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
   off = align_up(off + sizeof(__nv_bfloat16) * (size_t)p.B * p.npad * p.r, salsc::kWsAlign);
   p.off_scores = off;
   off = align_up(off + sizeof(float) * (size_t)p.N * p.U, salsc::kWsAlign);
+  p.off_krange = off;
+  off = align_up(off + sizeof(uint32_t) * 2 * (size_t)p.B * p.U, salsc::kWsAlign);
   p.off_idx = off;
   off = align_up(off + sizeof(int32_t) * (size_t)p.B * p.U * p.k, salsc::kWsAlign);
   p.off_part = off;
@@ -223,6 +226,7 @@ salsc_status decode_step_impl(const salsc_decode_desc* desc, const void* q, cons
   a.qlat = (float*)(w + p.off_qlat);
   a.qsplit = (__nv_bfloat16*)(w + p.off_qsplit);
   a.scores = (float*)(w + p.off_scores);
+  a.krange = (uint32_t*)(w + p.off_krange);
   a.part = (float*)(w + p.off_part);
 
   cudaStream_t s = (cudaStream_t)stream;

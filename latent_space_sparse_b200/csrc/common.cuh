@@ -27,6 +27,7 @@ constexpr int kMaxRank = 512;
 constexpr int kPartAcc = 4;
 __host__ __device__ constexpr int part_row(int r) { return r + kPartAcc; }
 constexpr int kMaxHeadDim = 128;
+constexpr int kMaxUnits = 256;  // KV heads per layer
 constexpr size_t kWsAlign = 256;
 
 // Host-side plan of one decode layer-step, derived from the descriptor only.
@@ -46,7 +47,7 @@ struct DecodePlan {
   float scale;
   double rope_base;
   // workspace layout (byte offsets)
-  size_t off_flags, off_qlat, off_qsplit, off_scores, off_idx, off_part, total;
+  size_t off_flags, off_qlat, off_qsplit, off_scores, off_krange, off_idx, off_part, total;
 };
 
 // Raw pointers of one decode call, passed to the launchers.
@@ -64,6 +65,7 @@ struct DecodeArgs {
   float* qlat;                 // [B][U][r]
   __nv_bfloat16* qsplit;       // [B][npad][r]: row 2u = hi(q_lat[u]), 2u+1 = lo, rest zero
   float* scores;               // packed per (b,u)
+  uint32_t* krange;            // [B][U][2] (min, max) order key of each unit's scores
   float* part;                 // [B][Hq][splits][part_row(r)]
 };
 
@@ -151,6 +153,13 @@ __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
+}
+
+// Unsigned key with the same order as the float; -0 and +0 map to one key.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
 // Locate the tile `tile` of a ragged batch where sequence b has

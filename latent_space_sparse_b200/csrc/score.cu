@@ -18,9 +18,10 @@ constexpr int kThreads = 256;
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 score_simt_kernel(const T* __restrict__ Kc, const float* __restrict__ qlat,
-                  const int64_t* __restrict__ seq_off, float* __restrict__ scores, int B, int U,
-                  int r, int tile_len) {
+                  const int64_t* __restrict__ seq_off, float* __restrict__ scores,
+                  uint32_t* __restrict__ krange, int B, int U, int r, int tile_len) {
   extern __shared__ float sq[];  // [U][r]
+  __shared__ uint32_t s_kr[kMaxUnits][2];  // this CTA's (min, max) score key per unit
   int b;
   int64_t t0;
   find_tile(seq_off, B, tile_len, blockIdx.x, b, t0);
@@ -30,6 +31,10 @@ score_simt_kernel(const T* __restrict__ Kc, const float* __restrict__ qlat,
   allow_dependent_launch();
   grid_dependency_wait();  // q_lat comes from the previous kernel
   for (int e = threadIdx.x; e < U * r; e += kThreads) sq[e] = qlat[(size_t)b * U * r + e];
+  for (int e = threadIdx.x; e < U; e += kThreads) {
+    s_kr[e][0] = 0xffffffffu;
+    s_kr[e][1] = 0u;
+  }
   __syncthreads();
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   constexpr int kPer = kMaxRank / 32;  // row elements held per lane
@@ -52,8 +57,17 @@ score_simt_kernel(const T* __restrict__ Kc, const float* __restrict__ qlat,
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) scores[off * U + (int64_t)u * nb + t] = acc;
+      if (lane == 0) {
+        scores[off * U + (int64_t)u * nb + t] = acc;
+        atomicMin(&s_kr[u][0], order_key(acc));
+        atomicMax(&s_kr[u][1], order_key(acc));
+      }
     }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < U; e += kThreads) {
+    atomicMin(&krange[2 * ((int64_t)b * U + e)], s_kr[e][0]);
+    atomicMax(&krange[2 * ((int64_t)b * U + e) + 1], s_kr[e][1]);
   }
 }
 
@@ -75,12 +89,14 @@ score_simt_kernel(const T* __restrict__ Kc, const float* __restrict__ qlat,
 // Each CTA owns a contiguous range of tiles (persistent, grid <= #SMs), so
 // Qs is reloaded only at sequence boundaries.
 constexpr int kTcThreads = 192;
+constexpr int kRangeSeqs = 4;  // sequences per CTA whose score ranges are kept in shared memory
 constexpr int kTileM = 128;
 constexpr uint32_t kStageBytes = kTileM * 64 * 2;  // one [128 x 64] bf16 k-block
 
 struct ScoreTcParams {
   const int64_t* seq_off;
   float* scores;
+  uint32_t* krange;
   uint32_t* flags;
   int B, U, npad, r, n_tiles, stages, tmem_cols;
 };
@@ -104,7 +120,16 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
   auto tfull = [&](int a) { return bar0 + 8u * (2 * S + 2 + a); };
   auto tempty = [&](int a) { return bar0 + 8u * (2 * S + 4 + a); };
 
+  // (min, max) score key per unit of the first kRangeSeqs sequences of this
+  // CTA's tile range
+  __shared__ uint32_t s_kr[kRangeSeqs][kMaxUnits][2];
+  __shared__ int s_krb[kRangeSeqs], s_nkr;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int e = threadIdx.x; e < kRangeSeqs * P.U; e += kTcThreads) {
+    s_kr[e / P.U][e % P.U][0] = 0xffffffffu;
+    s_kr[e / P.U][e % P.U][1] = 0u;
+  }
+  if (threadIdx.x == 0) s_nkr = 0;
   const int t_begin = (int)((int64_t)blockIdx.x * P.n_tiles / gridDim.x);
   const int t_end = (int)((int64_t)(blockIdx.x + 1) * P.n_tiles / gridDim.x);
   allow_dependent_launch();
@@ -224,14 +249,24 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
     // the last release of Qs lands before the CTA may exit
     if (ok && nseq > 0) tc::mbar_wait(bempty, (uint32_t)(nseq - 1) & 1u, P.flags);
   } else if (warp >= 2) {
-    // ---------------- epilogue: TMEM -> scores
+    // ---------------- epilogue: TMEM -> scores, and each unit's score range
+    //      (min and max order key, reduced per warp, kept per CTA and
+    //      sequence in shared memory, added to the workspace at the end)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
-    int i = 0;
+    int i = 0, eb = -1, so = -1;  // sequence and its ordinal in this CTA's range
     TileCursor cur;
     cur.start(P.seq_off, P.B, kTileM, t_begin);
     for (int tile = t_begin; tile < t_end; ++tile, ++i, cur.next()) {
+      if (cur.b != eb) {
+        eb = cur.b;
+        ++so;
+        if (so < kRangeSeqs && threadIdx.x == 64) {
+          s_krb[so] = eb;
+          s_nkr = so + 1;
+        }
+      }
       const int acc = i & 1;
       // warp-uniform wait: the TMEM loads below need a converged warp
       const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(tfull(acc), ((uint32_t)i >> 1) & 1u,
@@ -246,11 +281,24 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
         uint32_t v[16];
         tc::tmem_ld16(lane_addr + (uint32_t)(acc * P.npad + c0), v);
         tc::tmem_ld_wait();
-        if (t < nb) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int u = c0 / 2 + j;
-            if (u < P.U) sbase[(int64_t)u * nb] = __uint_as_float(v[2 * j]) + __uint_as_float(v[2 * j + 1]);
+        for (int j = 0; j < 8; ++j) {
+          const int u = c0 / 2 + j;
+          const float sv = __uint_as_float(v[2 * j]) + __uint_as_float(v[2 * j + 1]);
+          const uint32_t key = order_key(sv);
+          const uint32_t kmn = __reduce_min_sync(0xffffffffu, t < nb ? key : 0xffffffffu);
+          const uint32_t kmx = __reduce_max_sync(0xffffffffu, t < nb ? key : 0u);
+          if (u < P.U) {
+            if (t < nb) sbase[(int64_t)u * nb] = sv;
+            if (lane == 0) {
+              if (so < kRangeSeqs) {
+                atomicMin(&s_kr[so][u][0], kmn);
+                atomicMax(&s_kr[so][u][1], kmx);
+              } else {  // more sequences than table rows: straight to the workspace
+                atomicMin(&P.krange[2 * ((int64_t)eb * P.U + u)], kmn);
+                atomicMax(&P.krange[2 * ((int64_t)eb * P.U + u) + 1], kmx);
+              }
+            }
           }
         }
       }
@@ -260,6 +308,11 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
   }
   tc::fence_before_sync();
   __syncthreads();
+  for (int e = threadIdx.x; e < s_nkr * P.U; e += kTcThreads) {
+    const int q = e / P.U, u = e % P.U;
+    atomicMin(&P.krange[2 * ((int64_t)s_krb[q] * P.U + u)], s_kr[q][u][0]);
+    atomicMax(&P.krange[2 * ((int64_t)s_krb[q] * P.U + u) + 1], s_kr[q][u][1]);
+  }
   if (warp == 1) {
     __syncwarp();
     tc::fence_after_sync();
@@ -305,6 +358,7 @@ cudaError_t launch_score_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream
   ScoreTcParams P;
   P.seq_off = a.seq_off;
   P.scores = a.scores;
+  P.krange = a.krange;
   P.flags = a.flags;
   P.B = p.B;
   P.U = p.U;
@@ -332,7 +386,7 @@ cudaError_t launch_score(const DecodePlan& p, const DecodeArgs& a, cudaStream_t 
     if (e != cudaSuccess) return e;
     e = launch_k(k, dim3(p.n_score_tiles), dim3(kThreads), smem, s, true,
                  (const __nv_bfloat16*)a.Kc, (const float*)a.qlat, (const int64_t*)a.seq_off,
-                 a.scores, p.B, p.U, p.r, p.score_tile);
+                 a.scores, a.krange, p.B, p.U, p.r, p.score_tile);
     if (e != cudaSuccess) return e;
   } else {
     static int done[kMaxDevices] = {};
@@ -340,8 +394,8 @@ cudaError_t launch_score(const DecodePlan& p, const DecodeArgs& a, cudaStream_t 
     cudaError_t e = ensure_smem(k, smem, done);
     if (e != cudaSuccess) return e;
     e = launch_k(k, dim3(p.n_score_tiles), dim3(kThreads), smem, s, true, (const float*)a.Kc,
-                 (const float*)a.qlat, (const int64_t*)a.seq_off, a.scores, p.B, p.U, p.r,
-                 p.score_tile);
+                 (const float*)a.qlat, (const int64_t*)a.seq_off, a.scores, a.krange, p.B, p.U,
+                 p.r, p.score_tile);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();

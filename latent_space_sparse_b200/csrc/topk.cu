@@ -7,23 +7,24 @@
 //
 // Design: C CTAs (a thread-block cluster when C > 1) own one unit.  Each CTA
 // loads a contiguous slice of the unit's scores into shared memory once, as
-// 32-bit keys whose unsigned order is the float order, and the unit's score
-// range [min, max] is found.  Each CTA histograms its slice into 2048 bins of
-// equal width over that range (the bin is a monotone function of the score,
-// and scores spread over many bins, so the shared-memory atomics barely
-// contend); the C histograms are summed through distributed shared memory and
-// every CTA finds, with a block-wide scan, the bin that holds the k_b-th
-// largest score.  The pairs (key, index) of that bin are few for any smooth
-// score distribution: they are gathered from the cluster, and the one whose
-// rank (score descending, index ascending) is the number still needed gives
-// the exact threshold T.  When that bin holds more than kCand pairs (heavily
-// repeated or extreme scores), a radix select on rel = key - kmin with 11-bit
-// digits, starting at the top bit of the key range (at most three passes),
-// finds T instead.  The final compaction gives every warp a contiguous
-// segment of the slice: one counting pass, one prefix over warps (and cluster
-// ranks), one writing pass with warp ballots.  Output order is the index order of the
-// keys > T followed by the lowest-index keys == T, so the result is
-// deterministic.  No full sort, no global-memory scratch.
+// 32-bit keys whose unsigned order is the float order; the unit's score range
+// [min, max] comes from the scoring kernel.  Each CTA histograms its slice
+// into 512 bins of equal width over that range (the bin is a monotone
+// function of the score, and scores spread over many bins, so the
+// shared-memory atomics barely contend); the C histograms are summed through
+// distributed shared memory and every CTA finds, with a block-wide scan, the
+// bin that holds the k_b-th largest score.  A second pass counts, per warp
+// segment, the keys above that bin and lists the (key, index) pairs inside
+// it, which are few for any smooth score distribution: the lists of the
+// cluster are merged, and the pair whose rank (score descending, index
+// ascending) is the number still needed is the exact threshold.  The counts
+// and the kept candidates give every warp its output offset, and a third pass
+// writes the kept indices of each warp's segment in index order, so the
+// result is deterministic.  When the boundary bin holds more than kCand pairs
+// (heavily repeated or extreme scores), a radix select on rel = key - kmin
+// with 11-bit digits, starting at the top bit of the key range (at most three
+// passes), finds the threshold instead, followed by a counting and a writing
+// pass.  No full sort, no global-memory scratch.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -38,28 +39,22 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kBatch = 32;  // keys a thread loads before converting them
 constexpr int kMaxCluster = 8;  // largest cluster of CTAs per unit
 
-// Unsigned key with the same order as the float; -0 and +0 map to one key.
-__device__ __forceinline__ uint32_t order_key(float f) {
-  uint32_t u = __float_as_uint(f);
-  if (u == 0x80000000u) u = 0u;
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
 // Float whose order_key is `key` (-0 comes back as +0).
 __device__ __forceinline__ float key_float(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
-constexpr int kBins = 2048;  // 11-bit digits
+constexpr int kBins = 2048;  // 11-bit digits of the radix fallback
 constexpr int kDigit = 11;
-constexpr int kCand = 1024;  // most candidates the boundary bin may hold for the fast path
+constexpr int kLinBins = 512;  // bins of the linear pass
+constexpr int kCand = 1024;    // most candidates the boundary bin may hold for the fast path
 
-// Bin of a key in the linear partition of [fmin, fmax] into kBins bins: a
+// Bin of a key in the linear partition of [fmin, fmax] into kLinBins bins: a
 // composition of monotone roundings, so a larger score never lands in a lower
 // bin and equal scores share a bin.
 __device__ __forceinline__ int linear_bin(uint32_t key, float fmin, float scale) {
   const float x = (key_float(key) - fmin) * scale;
-  return min(kBins - 1, (int)x);
+  return min(kLinBins - 1, (int)x);
 }
 
 // Block-wide search for the digit that holds the target rank: `cnt` holds the
@@ -68,8 +63,8 @@ __device__ __forceinline__ int linear_bin(uint32_t key, float fmin, float scale)
 __device__ __forceinline__ void find_digit(const uint32_t* cnt, uint32_t target, int nbins,
                                            uint32_t* wsum, uint32_t* s_digit, uint32_t* s_above) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int b0 = kBins - 1 - 2 * tid, b1 = b0 - 1;
-  const uint32_t c0 = b0 < nbins ? cnt[b0] : 0u, c1 = b1 < nbins ? cnt[b1] : 0u;
+  const int b0 = nbins - 1 - 2 * tid, b1 = b0 - 1;  // nbins <= 2 * kThreads
+  const uint32_t c0 = b0 >= 0 ? cnt[b0] : 0u, c1 = b1 >= 0 ? cnt[b1] : 0u;
   const uint32_t mine = c0 + c1;
   uint32_t incl = mine;
 #pragma unroll
@@ -103,7 +98,7 @@ __device__ __forceinline__ void find_digit(const uint32_t* cnt, uint32_t target,
 template <bool kCluster>
 __global__ void __launch_bounds__(kThreads)
 topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_off,
-            int32_t* __restrict__ idx_out, int U, int k) {
+            const uint32_t* __restrict__ krange, int32_t* __restrict__ idx_out, int U, int k) {
   cg::cluster_group cluster = cg::this_cluster();
   const int C = kCluster ? (int)cluster.num_blocks() : 1;
   const int rank = kCluster ? (int)cluster.block_rank() : 0;
@@ -111,31 +106,57 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
   const int b = unit / U, u = unit % U;
 
   extern __shared__ uint32_t keys[];
-  __shared__ uint32_t hist[2][kBins];
-  __shared__ uint32_t total[kBins];
+  __shared__ uint32_t hist[2][kBins];  // [0]: histogram, [1]: candidate list (both read by the cluster)
+  __shared__ uint32_t total[kBins];    // cluster histogram, then the merged candidate list
   __shared__ uint32_t wsum[64];
-  __shared__ uint32_t mm[2];      // this CTA's (min key, max key), read by the cluster
-  __shared__ uint32_t counts[2];  // this CTA's (#keys > T, #keys == T), read by the cluster
+  __shared__ uint32_t counts[2];       // fallback: this CTA's (#keys > T, #keys == T)
   __shared__ uint32_t wcnt[kWarps][2];
   __shared__ uint32_t wbase[kWarps][2];
-  __shared__ uint32_t s_digit, s_above, s_base_gt, s_base_eq, s_ncand;
+  __shared__ uint32_t s_kc[kMaxCluster], s_gtq[kMaxCluster], s_nq[kMaxCluster];
+  __shared__ uint32_t s_cbase[kMaxCluster + 1];
+  __shared__ uint32_t s_digit, s_above, s_base_gt, s_base_eq, s_ncand, s_gtc, s_T, s_Tidx;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // shared memory of cluster rank q (this CTA's own when not a cluster)
   auto remote = [&](uint32_t* ptr, int q) -> uint32_t* {
     return kCluster ? cluster.map_shared_rank(ptr, q) : ptr;
   };
+  auto cluster_sync = [&]() {
+    if (kCluster) cluster.sync(); else __syncthreads();
+  };
+  for (int i = tid; i < kLinBins; i += kThreads) hist[0][i] = 0u;
+  if (tid < kWarps) wcnt[tid][1] = 0u;  // kept candidates per warp segment
+  if (tid < kMaxCluster) s_kc[tid] = 0u;
+  if (tid == 0) s_ncand = 0u;
   allow_dependent_launch();
   const int64_t off = seq_off[b];
   const int64_t nb = seq_off[b + 1] - off;
   const int64_t kb = nb < k ? nb : k;
   const float* s = scores + off * U + (int64_t)u * nb;
-  grid_dependency_wait();  // the scores come from the previous kernel
   const int64_t lo = nb * rank / C, hi = nb * (rank + 1) / C;
   const int n_loc = (int)(hi - lo);
+  const int seg = (n_loc + kWarps - 1) / kWarps;  // warp w owns keys [w*seg, (w+1)*seg)
+  const int s0 = warp * seg, s1 = min(s0 + seg, n_loc);
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int32_t* out = idx_out + ((int64_t)b * U + u) * k;
+  grid_dependency_wait();  // the scores and their range come from the previous kernel
+  if (kb == nb) {
+    // keep every token, in index order
+    for (int i = tid; i < n_loc; i += kThreads) out[lo + i] = (int32_t)(lo + i);
+    if (rank == 0)
+      for (int64_t j = kb + tid; j < k; j += kThreads) out[j] = -1;
+    return;
+  }
+  // the unit's key range, reduced by the scoring kernel
+  uint32_t kmin = krange[2 * ((int64_t)b * U + u)], kmax = krange[2 * ((int64_t)b * U + u) + 1];
+  const float fmin = key_float(kmin), fmax = key_float(kmax);
+  const float frange = fmax - fmin;
+  const float scale = (float)kLinBins / frange;
+  const bool lin = isfinite(frange) && frange > 0.f && isfinite(scale);
+  const int n_iter = (n_loc + kThreads - 1) / kThreads;
+  __syncthreads();  // the zeroed histogram and counters
 
-  // ---- keys of the slice (loads of a batch issued before their stores) and their range
-  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  // ---- pass 1: keys of the slice into shared memory, histogram of their bins
   for (int base = 0; base < n_loc; base += kThreads * kBatch) {
     float v[kBatch];
 #pragma unroll
@@ -149,153 +170,145 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
       if (i < n_loc) {
         const uint32_t key = order_key(v[j]);
         keys[i] = key;
-        kmin = min(kmin, key);
-        kmax = max(kmax, key);
+        if (lin) atomicAdd(&hist[0][linear_bin(key, fmin, scale)], 1u);
       }
     }
   }
+  bool fast = lin;
+  int bstar = 0;
+  uint32_t need = 0u, n_cand = 0u;
+  if (fast) {
+    cluster_sync();
+    const uint32_t* cnt = hist[0];
+    if (kCluster) {
+      for (int i = tid; i < kLinBins; i += kThreads) {
+        uint32_t t = 0u;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+        for (int q = 0; q < kMaxCluster; ++q)
+          if (q < C) t += remote(hist[0], q)[i];
+        total[i] = t;
+      }
+      cnt = total;
+      __syncthreads();
+    }
+    find_digit(cnt, (uint32_t)kb, kLinBins, wsum, &s_digit, &s_above);
+    __syncthreads();
+    bstar = (int)s_digit;
+    need = (uint32_t)kb - s_above;  // 1 <= need <= cnt[bstar]
+    n_cand = cnt[bstar];
+    fast = n_cand <= (uint32_t)kCand;
   }
-  if (lane == 0) {
-    wcnt[warp][0] = kmin;
-    wcnt[warp][1] = kmax;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t a = wcnt[lane][0], z = wcnt[lane][1];
+  if (fast) {
+    // ---- pass 2: classify.  Keys above the boundary bin become ~0, keys below
+    //      it 0 (both on the right side of any finite threshold key); the
+    //      boundary bin's (key, index) pairs go to this CTA's candidate list.
+    uint32_t* loc = hist[1];  // [kCand] keys, then [kCand] indices
+    uint32_t ngt = 0u;
+    for (int c0 = s0; c0 < s1; c0 += 32) {
+      const int i = c0 + lane;
+      const bool valid = i < s1;
+      const uint32_t key = valid ? keys[i] : 0u;
+      const int bin = linear_bin(key, fmin, scale);
+      const bool gt = valid && bin > bstar, cand = valid && bin == bstar;
+      ngt += __popc(__ballot_sync(0xffffffffu, gt));
+      if (cand) {
+        const uint32_t pos = atomicAdd(&s_ncand, 1u);
+        loc[pos] = key;
+        loc[kCand + pos] = (uint32_t)(lo + i);
+      }
+      if (valid) keys[i] = gt ? 0xffffffffu : (cand ? key : 0u);
+    }
+    if (lane == 0) wcnt[warp][0] = ngt;
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t x = wcnt[lane][0];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      a = min(a, __shfl_xor_sync(0xffffffffu, a, o));
-      z = max(z, __shfl_xor_sync(0xffffffffu, z, o));
+      for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+      if (lane == 0) s_gtc = x;
     }
-    if (lane == 0) {
-      mm[0] = a;
-      mm[1] = z;
+    cluster_sync();
+    // ---- the cluster's candidates, merged in rank order into `total`, and
+    //      every rank's count of keys above the boundary bin
+    if (tid < C) {
+      s_nq[tid] = *remote(&s_ncand, tid);
+      s_gtq[tid] = *remote(&s_gtc, tid);
     }
-  }
-  if (kCluster) {
-    cluster.sync();
+    __syncthreads();
     if (tid == 0) {
-      uint32_t a = 0xffffffffu, z = 0u;
-#pragma unroll
-      for (int q = 0; q < kMaxCluster; ++q) {
-        if (q < C) {
-          const uint32_t* r = remote(mm, q);
-          a = min(a, r[0]);
-          z = max(z, r[1]);
-        }
+      uint32_t cb = 0u;
+      for (int q = 0; q < C; ++q) {
+        s_cbase[q] = cb;
+        cb += s_nq[q];
       }
-      wsum[0] = a;
-      wsum[1] = z;
+      s_cbase[C] = cb;
     }
-  } else if (tid == 0) {
-    wsum[0] = mm[0];
-    wsum[1] = mm[1];
+    __syncthreads();
+    for (uint32_t e = tid; e < n_cand; e += kThreads) {
+      int q = 0;
+      while (q + 1 < C && e >= s_cbase[q + 1]) ++q;
+      const uint32_t* rl = remote(loc, q);
+      const uint32_t j = e - s_cbase[q];
+      total[e] = rl[j];
+      total[kCand + e] = rl[kCand + j];
+    }
+    __syncthreads();
+    // ---- the need-th best pair (score descending, index ascending) is the
+    //      threshold; a candidate is kept when it is not worse
+    for (uint32_t t = tid; t < n_cand; t += kThreads) {
+      const uint32_t kt = total[t], it_ = total[kCand + t];
+      uint32_t better = 0u;
+      for (uint32_t j = 0; j < n_cand; ++j) {
+        const uint32_t kj = total[j], ij = total[kCand + j];
+        better += (kj > kt) || (kj == kt && ij < it_);
+      }
+      if (better == need - 1u) {
+        s_T = kt;
+        s_Tidx = it_;
+      }
+      if (better < need) {
+        int q = 0;
+        while (q + 1 < C && t >= s_cbase[q + 1]) ++q;
+        atomicAdd(&s_kc[q], 1u);
+        if (q == rank) atomicAdd(&wcnt[(it_ - (uint32_t)lo) / (uint32_t)seg][1], 1u);
+      }
+    }
+    __syncthreads();
+    // ---- output offsets: ranks before this one, then warps before this one
+    if (warp == 0) {
+      uint32_t before = 0u;
+      for (int q = 0; q < rank; ++q) before += s_gtq[q] + s_kc[q];
+      const uint32_t mine = wcnt[lane][0] + wcnt[lane][1];
+      uint32_t x = mine;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += t;
+      }
+      wbase[lane][0] = before + x - mine;
+    }
+    cluster_sync();  // every CTA is done with the others' shared memory
+    // ---- pass 3: write the kept indices of this warp's segment in order
+    const uint32_t T = s_T, Tidx = s_Tidx;
+    uint32_t run = wbase[warp][0];
+    for (int c0 = s0; c0 < s1; c0 += 32) {
+      const int i = c0 + lane;
+      const bool valid = i < s1;
+      const uint32_t key = valid ? keys[i] : 0u;
+      const bool keep = valid && (key > T || (key == T && (uint32_t)(lo + i) <= Tidx));
+      const uint32_t bk = __ballot_sync(0xffffffffu, keep);
+      if (keep) out[run + __popc(bk & lt_mask)] = (int32_t)(lo + i);
+      run += __popc(bk);
+    }
+    if (rank == 0)
+      for (int64_t j = kb + tid; j < k; j += kThreads) out[j] = -1;
+    return;
   }
-  __syncthreads();
-  kmin = wsum[0];
-  kmax = wsum[1];
-  __syncthreads();
-
-  // ---- radix select on rel = key - kmin, 11-bit digits from the top bit of the range:
-  //      T = kmin + prefix is the kb-th largest key; `remaining` ends as the number
-  //      of keys equal to T that are kept
+  // ======== fallback: radix select over the keys' bits
+  if (lin && kCluster) cluster.sync();  // the others are done reading this histogram
   uint64_t prefix = 0u;
   uint32_t remaining = (uint32_t)kb;
   uint32_t T = 0u;
-  const int n_iter = (n_loc + kThreads - 1) / kThreads;
-  bool resolved = false;
-  if (kb == nb) {
-    remaining = 0u;  // keep everything: every finite score has key > 0
-    resolved = true;
-  } else {
-    // ---- linear pass: bins of equal width over [min score, max score]
-    const float fmin = key_float(kmin), fmax = key_float(kmax);
-    const float frange = fmax - fmin;
-    const float scale = (float)kBins / frange;
-    if (isfinite(frange) && frange > 0.f && isfinite(scale)) {
-      uint32_t* h = hist[0];
-      for (int i = tid; i < kBins; i += kThreads) h[i] = 0u;
-      __syncthreads();
-      for (int it = 0; it < n_iter; ++it) {
-        const int i = it * kThreads + tid;
-        if (i < n_loc) atomicAdd(&h[linear_bin(keys[i], fmin, scale)], 1u);
-      }
-      const uint32_t* cnt = h;
-      if (kCluster) {
-        cluster.sync();
-        for (int i = tid; i < kBins; i += kThreads) {
-          uint32_t t = 0u;
-#pragma unroll
-          for (int q = 0; q < kMaxCluster; ++q)
-            if (q < C) t += remote(h, q)[i];
-          total[i] = t;
-        }
-        cnt = total;
-      }
-      __syncthreads();
-      find_digit(cnt, (uint32_t)kb, kBins, wsum, &s_digit, &s_above);
-      __syncthreads();
-      const int bstar = (int)s_digit;
-      const uint32_t need = (uint32_t)kb - s_above;  // 1 <= need <= cnt[bstar]
-      const uint32_t n_cand = cnt[bstar];
-      if (n_cand <= (uint32_t)kCand) {
-        // ---- the boundary bin's (key, index) pairs: a short list per CTA ...
-        uint32_t* loc = hist[1];  // [kCand] keys, then [kCand] indices
-        if (tid == 0) s_ncand = 0u;
-        __syncthreads();
-        for (int it = 0; it < n_iter; ++it) {
-          const int i = it * kThreads + tid;
-          if (i < n_loc && linear_bin(keys[i], fmin, scale) == bstar) {
-            const uint32_t pos = atomicAdd(&s_ncand, 1u);
-            loc[pos] = keys[i];
-            loc[kCand + pos] = (uint32_t)(lo + i);
-          }
-        }
-        if (kCluster) cluster.sync(); else __syncthreads();
-        // ... merged in rank order into `total`: [n_cand] keys, then [n_cand] indices
-        uint32_t base = 0u;
-#pragma unroll
-        for (int q = 0; q < kMaxCluster; ++q) {
-          if (q < C) {
-            uint32_t* rl = remote(loc, q);
-            const uint32_t nq = *remote(&s_ncand, q);
-            for (uint32_t j = tid; j < nq; j += kThreads) {
-              total[base + j] = rl[j];
-              total[kCand + base + j] = rl[kCand + j];
-            }
-            base += nq;
-          }
-        }
-        __syncthreads();
-        // ---- the need-th best pair (score descending, index ascending) is the threshold
-        for (uint32_t t = tid; t < n_cand; t += kThreads) {
-          const uint32_t kt = total[t], it_ = total[kCand + t];
-          uint32_t better = 0u, eq_le = 0u;
-          for (uint32_t j = 0; j < n_cand; ++j) {
-            const uint32_t kj = total[j], ij = total[kCand + j];
-            better += (kj > kt) || (kj == kt && ij < it_);
-            eq_le += (kj == kt) && (ij <= it_);
-          }
-          if (better == need - 1u) {
-            s_digit = kt;     // T
-            s_above = eq_le;  // keys equal to T that are kept
-          }
-        }
-        __syncthreads();
-        T = s_digit;
-        remaining = s_above;
-        resolved = true;
-      } else if (kCluster) {
-        cluster.sync();  // the other CTAs have read this pass's histogram before it is reused
-      }
-    }
-  }
-  if (!resolved) {
-    // ---- fallback: radix select over the keys' bits
+  {
     const uint32_t range = kmax - kmin;
     int hi_bit = range == 0u ? 0 : 32 - __clz(range);  // bits of rel still to resolve: [0, hi_bit)
     int pass = 0;
@@ -339,8 +352,6 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
   const uint32_t n_gt_total = (uint32_t)kb - need_eq;
 
   // ---- compaction: warp w owns keys [w*seg, min((w+1)*seg, n_loc))
-  const int seg = (n_loc + kWarps - 1) / kWarps;
-  const int s0 = warp * seg, s1 = min(s0 + seg, n_loc);
   uint32_t cgt = 0u, ceq = 0u;
   for (int i = s0 + lane; i < s1; i += 32) {
     const uint32_t key = keys[i];
@@ -397,9 +408,7 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
   }
   __syncthreads();
 
-  int32_t* out = idx_out + ((int64_t)b * U + u) * k;
   uint32_t run_gt = s_base_gt + wbase[warp][0], run_eq = s_base_eq + wbase[warp][1];
-  const uint32_t lt_mask = (1u << lane) - 1u;
   for (int c0 = s0; c0 < s1; c0 += 32) {
     const int i = c0 + lane;
     const bool valid = i < s1;
@@ -430,7 +439,8 @@ cudaError_t launch_topk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s
     cudaError_t e = ensure_smem(topk_kernel<false>, smem, done);
     if (e != cudaSuccess) return e;
     return launch_k(topk_kernel<false>, dim3(p.B * p.U), dim3(kThreads), smem, s, true,
-                    (const float*)a.scores, (const int64_t*)a.seq_off, a.idx, p.U, p.k);
+                    (const float*)a.scores, (const int64_t*)a.seq_off, (const uint32_t*)a.krange, a.idx,
+                    p.U, p.k);
   }
   static int done[kMaxDevices] = {};
   cudaError_t e = ensure_smem(topk_kernel<true>, smem, done);
@@ -449,8 +459,8 @@ cudaError_t launch_topk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, topk_kernel<true>, (const float*)a.scores, a.seq_off, a.idx,
-                            p.U, p.k);
+  return cudaLaunchKernelEx(&cfg, topk_kernel<true>, (const float*)a.scores, a.seq_off,
+                            (const uint32_t*)a.krange, a.idx, p.U, p.k);
 }
 
 }  // namespace salsc
