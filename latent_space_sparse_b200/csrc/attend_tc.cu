@@ -153,8 +153,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
   float* const s_qr = (float*)(s_theta + HALF);              // [G][D/2] rotated (q_i, q_i+d/2)
   float* const s_pd = s_qr + G * D;                          // [2][G][128] half-pair dots
   float* const s_lg = s_pd + 2 * G * kTile;                  // [G][128] logits -> weights
-  float* const s_stat = s_lg + G * kTile;                    // [G][2] (m, l)
-  int* const s_tok = (int*)(s_stat + 2 * G);                 // [2][128] token per row
+  float* const s_stat = s_lg + G * kTile;                    // [2][G][2] tile's (m, l)
+  int* const s_tok = (int*)(s_stat + 4 * G);                 // [2][128] token per row
   float* const s_run = (float*)(s_tok + 2 * kTile);          // [G][2] segment's running (m, l)
   float* const s_ab = s_run + 2 * G;                         // [G][2] rescale factors
   uint64_t* const s_bars = (uint64_t*)(((uintptr_t)(s_ab + 2 * G) + 7) & ~(uintptr_t)7);
@@ -250,6 +250,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       tc::mbar_wait(bar(B_VFULL + bi), ((uint32_t)last_v >> 1) & 1u, P.flags);
   } else if (warp == kMmaWarp) {
     // ======================= MMA issuer (lane 0) =======================
+    // An event loop: the reconstruction of tile nk (after its key rows have
+    // landed and its TMEM buffer is free, with Pk_u reloaded at unit
+    // boundaries) and the value MMA of tile np (after its weights and value
+    // rows are ready) are each issued as soon as their own inputs are, so
+    // neither waits behind the other.  At most two reconstructions run ahead
+    // of the value MMAs (two tile buffers, two K_sel buffers in TMEM).
     if (lane == 0) {
       const uint32_t idesc_k = tc::idesc_bf16_f32(kTile, D);
       const uint32_t idesc_v = tc::idesc_bf16_f32_amn(128, kPRows);
@@ -257,72 +263,86 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
       int cur_b = -1, cur_u = -1;
       uint32_t pk_phase = 0;
-      bool ok = true;
-      auto issue_pv = [=](int j) -> bool {
-        const int bj = j & 1;
-        const uint32_t ph = ((uint32_t)j >> 1) & 1u;
-        if (!tc::mbar_wait(bar(B_PREADY + bj), ph, P.flags)) return false;
-        if (!tc::mbar_wait(bar(B_VFULL + bj), ph, P.flags)) return false;
-        if (!tc::mbar_wait(bar(B_TOFREE + bj), ph ^ 1u, P.flags)) return false;
-        tc::fence_after_sync();
-        const uint32_t v0 = tc::smem_u32((bj ? s_buf1 : s_buf0)), p0 = tc::smem_u32((bj ? s_pbuf1 : s_pbuf0));
-        for (int ch = 0; ch < n_chunks; ++ch) {
-          const uint32_t d_tmem = tmem_base + o_col0 + (uint32_t)bj * o_cols + (uint32_t)ch * 16;
+      int pk_step = 0;  // 1: waiting to reload Pk, 2: Pk load in flight
+      int nk = 0, np = 0;
+      uint64_t idle_since = 0;
+      const uint32_t pkb = tc::smem_u32(s_pk);
+      while (np < n) {
+        bool progress = false;
+        if (nk < n && nk <= np + 2) {
+          if (pk_step == 0 && (cur.b != cur_b || cur.u != cur_u)) pk_step = 1;
+          // Pk_u of a new unit, once the previous reconstruction is done with Pk
+          if (pk_step == 1 &&
+              (nk == 0 ||
+               tc::mbar_test_wait(bar(B_KDONE + ((nk - 1) & 1)), ((uint32_t)(nk - 1) >> 1) & 1u))) {
+            tc::mbar_expect_tx(bar(B_PK), pk_bytes);
+            for (int kb = 0; kb < KB; ++kb)
+              tc::tma_load_2d(pkb + (uint32_t)kb * D * 128, &tmap_pk, kb * 64, cur.u * D, bar(B_PK));
+            pk_step = 2;
+            progress = true;
+          }
+          if (pk_step == 2 && tc::mbar_test_wait(bar(B_PK), pk_phase)) {
+            pk_phase ^= 1u;
+            cur_b = cur.b;
+            cur_u = cur.u;
+            pk_step = 0;
+            progress = true;
+          }
+          const int bk = nk & 1;
+          if (pk_step == 0 && tc::mbar_test_wait(bar(B_KFULL + bk), ((uint32_t)nk >> 1) & 1u) &&
+              tc::mbar_test_wait(bar(B_TKFREE + bk), (((uint32_t)nk >> 1) & 1u) ^ 1u)) {
+            tc::fence_after_sync();
+            const uint32_t kb0 = tc::smem_u32(bk ? s_buf1 : s_buf0);
+            const uint32_t d_tmem = tmem_base + (uint32_t)bk * D;
+            for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
-          for (int ks = 0; ks < kTile / 16; ++ks) {
-            // A = Vc_tile^T: latent columns ch*128.. (MN), tokens ks*16.. (K)
-            const uint64_t ad = tc::sdesc_mnmajor_sw128(
-                v0 + (uint32_t)ch * 2 * 16384 + (uint32_t)(ks * 2) * 1024, 16384, 1024);
-            // B = p rows (hi/lo per head), tokens ks*16..: K-major k-block ks/4
-            const uint64_t bd =
-                tc::sdesc_kmajor_sw128(p0 + (uint32_t)(ks >> 2) * 2048 + (uint32_t)(ks & 3) * 32);
-            tc::mma_bf16(d_tmem, ad, bd, idesc_v, ks != 0);
+              for (int k = 0; k < 4; ++k)
+                tc::mma_bf16(d_tmem, tc::sdesc_kmajor_sw128(kb0 + kb * 16384 + 32 * k),
+                             tc::sdesc_kmajor_sw128(pkb + kb * D * 128 + 32 * k), idesc_k,
+                             (kb | k) != 0);
+            tc::mma_commit(bar(B_KDONE + bk));
+            ++nk;
+            cur.next();
+            progress = true;
           }
         }
-        tc::mma_commit(bar(B_PDONE + bj));
-        return true;
-      };
-      for (int i = 0; i < n && ok; ++i, cur.next()) {
-        const int bi = i & 1;
-        const uint32_t ph = ((uint32_t)i >> 1) & 1u;
-        if (cur.b != cur_b || cur.u != cur_u) {
-          // Pk_u of the new unit; the previous reconstruction must be done with Pk
-          if (i > 0 &&
-              !tc::mbar_wait(bar(B_KDONE + ((i - 1) & 1)), ((uint32_t)(i - 1) >> 1) & 1u,
-                             P.flags)) {
-            ok = false;
+        const int bp = np & 1;
+        if (np < nk && tc::mbar_test_wait(bar(B_PREADY + bp), ((uint32_t)np >> 1) & 1u) &&
+            tc::mbar_test_wait(bar(B_VFULL + bp), ((uint32_t)np >> 1) & 1u) &&
+            tc::mbar_test_wait(bar(B_TOFREE + bp), (((uint32_t)np >> 1) & 1u) ^ 1u)) {
+          tc::fence_after_sync();
+          const uint32_t p0 = tc::smem_u32(bp ? s_pbuf1 : s_pbuf0);
+          const uint32_t vb0 = tc::smem_u32(bp ? s_buf1 : s_buf0);
+          for (int ch = 0; ch < n_chunks; ++ch) {
+            const uint32_t d_tmem = tmem_base + o_col0 + (uint32_t)bp * o_cols + (uint32_t)ch * 16;
+#pragma unroll
+            for (int ks = 0; ks < kTile / 16; ++ks) {
+              // A = Vc_tile^T: latent columns ch*128.. (MN), tokens ks*16.. (K)
+              const uint64_t ad = tc::sdesc_mnmajor_sw128(
+                  vb0 + (uint32_t)ch * 2 * 16384 + (uint32_t)(ks * 2) * 1024, 16384, 1024);
+              // B = p rows (hi/lo per head), tokens ks*16..: K-major k-block ks/4
+              const uint64_t bd =
+                  tc::sdesc_kmajor_sw128(p0 + (uint32_t)(ks >> 2) * 2048 + (uint32_t)(ks & 3) * 32);
+              tc::mma_bf16(d_tmem, ad, bd, idesc_v, ks != 0);
+            }
+          }
+          tc::mma_commit(bar(B_PDONE + bp));
+          ++np;
+          progress = true;
+        }
+        if (progress) {
+          idle_since = 0;
+        } else {
+          const uint64_t now = tc::globaltimer_ns();
+          if (idle_since == 0) {
+            idle_since = now;
+          } else if (now - idle_since > tc::kWaitLimitNs) {
+            atomicOr(P.flags, FLAG_WAIT_TIMEOUT);
             break;
           }
-          tc::mbar_expect_tx(bar(B_PK), pk_bytes);
-          for (int kb = 0; kb < KB; ++kb)
-            tc::tma_load_2d(tc::smem_u32(s_pk + (size_t)kb * D * 128), &tmap_pk, kb * 64,
-                            cur.u * D, bar(B_PK));
-          if (!tc::mbar_wait(bar(B_PK), pk_phase, P.flags)) {
-            ok = false;
-            break;
-          }
-          pk_phase ^= 1u;
-          cur_b = cur.b;
-          cur_u = cur.u;
+          __nanosleep(32);
         }
-        if (!tc::mbar_wait(bar(B_KFULL + bi), ph, P.flags) ||
-            !tc::mbar_wait(bar(B_TKFREE + bi), ph ^ 1u, P.flags)) {
-          ok = false;
-          break;
-        }
-        tc::fence_after_sync();
-        const uint32_t a0 = tc::smem_u32((bi ? s_buf1 : s_buf0)), b0 = tc::smem_u32(s_pk);
-        const uint32_t d_tmem = tmem_base + (uint32_t)bi * D;
-        for (int kb = 0; kb < KB; ++kb)
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc::mma_bf16(d_tmem, tc::sdesc_kmajor_sw128(a0 + kb * 16384 + 32 * k),
-                         tc::sdesc_kmajor_sw128(b0 + kb * D * 128 + 32 * k), idesc_k,
-                         (kb | k) != 0);
-        tc::mma_commit(bar(B_KDONE + bi));
-        if (i > 0 && !issue_pv(i - 1)) ok = false;
       }
-      if (ok && n > 0) issue_pv(n - 1);
     }
   } else {
     // ======================= epilogue (warps 0-7) =======================
@@ -339,6 +359,80 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       s_run[2 * tid] = -INFINITY;
       s_run[2 * tid + 1] = 0.f;
     }
+    // Fold tile j (the cursor fc is at it) into its unit segment's running
+    // (m, l, acc) and publish the segment at its end.  Tile j is folded after
+    // the weights of tile j+1 are computed, so that the value MMA of tile j
+    // runs meanwhile.
+    UnitTileCursor fc = cur;
+    auto fold = [&](int j) {
+      const int bj = j & 1;
+      const uint32_t phj = ((uint32_t)j >> 1) & 1u;
+      // heads' scale factors
+      if (tid < G) {
+        const float mt = s_stat[bj * 2 * G + 2 * tid], lt = s_stat[bj * 2 * G + 2 * tid + 1];
+        const float mr = s_run[2 * tid], lr = s_run[2 * tid + 1];
+        const float mx = fmaxf(mr, mt);
+        float al = 0.f, be = 0.f;
+        if (mx != -INFINITY) {
+          al = mr == -INFINITY ? 0.f : expf(mr - mx);
+          be = mt == -INFINITY ? 0.f : expf(mt - mx);
+        }
+        s_ab[2 * tid] = al;
+        s_ab[2 * tid + 1] = be;
+        s_run[2 * tid] = mx;
+        s_run[2 * tid + 1] = lr * al + lt * be;
+      }
+      // the tile's acc from TMEM: warp (quarter, half) holds latent column
+      // c = half*128 + quarter*32 + lane
+      const bool ok2 = __all_sync(0xffffffffu, tc::mbar_wait(bar(B_PDONE + bj), phj, P.flags));
+      tc::fence_after_sync();
+      uint32_t v[16];
+      if (ok2 && half < n_chunks) {
+        tc::tmem_ld16(tmem_base + ((uint32_t)(quarter * 32) << 16) + o_col0 +
+                          (uint32_t)bj * o_cols + (uint32_t)half * 16,
+                      v);
+        tc::tmem_ld_wait();
+      }
+      tc::fence_before_sync();
+      tc::named_sync(kEpiBar, kEpiThreads);
+      if (tid == 0) tc::mbar_arrive(bar(B_TOFREE + bj));
+      if (ok2 && half < n_chunks) {
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+          acc_run[g] = acc_run[g] * s_ab[2 * g] +
+                       (__uint_as_float(v[2 * g]) + __uint_as_float(v[2 * g + 1])) * s_ab[2 * g + 1];
+      }
+      // end of this CTA's segment of the unit: publish it
+      UnitTileCursor nx = fc;
+      nx.next();
+      const bool seg_end = j + 1 == n || nx.b != fc.b || nx.u != fc.u;
+      ++seg_tiles;
+      if (seg_end) {
+        const int s0 = fc.slot + 1 - seg_tiles;  // first slot of the segment
+        const int c = half * 128 + quarter * 32 + lane;
+        const int64_t row0 = ((int64_t)fc.b * P.Hq + fc.u * G) * P.n_slots + s0;
+        if (half < n_chunks && c < P.r) {
+#pragma unroll
+          for (int g = 0; g < G; ++g)
+            P.part[(row0 + (int64_t)g * P.n_slots) * part_row(P.r) + kPartAcc + c] = acc_run[g];
+        }
+        if (tid < G) {
+          float* pp = P.part + (row0 + (int64_t)tid * P.n_slots) * part_row(P.r);
+          pp[0] = s_run[2 * tid];
+          pp[1] = s_run[2 * tid + 1];
+        }
+        // a new segment starts with the next tile
+        seg_tiles = 0;
+#pragma unroll
+        for (int g = 0; g < G; ++g) acc_run[g] = 0.f;
+        if (tid < G) {
+          s_run[2 * tid] = -INFINITY;
+          s_run[2 * tid + 1] = 0.f;
+        }
+      }
+      tc::named_sync(kEpiBar, kEpiThreads);
+      fc = nx;
+    };
     for (int i = 0; i < n; ++i, cur.next()) {
       const int bi = i & 1;
       const uint32_t ph = ((uint32_t)i >> 1) & 1u;
@@ -431,8 +525,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
         if (lane == 0) {
-          s_stat[2 * g] = mx;
-          s_stat[2 * g + 1] = sum;
+          s_stat[bi * 2 * G + 2 * g] = mx;
+          s_stat[bi * 2 * G + 2 * g + 1] = sum;
         }
       }
       tc::named_sync(kEpiBar, kEpiThreads);
@@ -456,71 +550,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       tc::fence_proxy_async_smem();
       tc::named_sync(kEpiBar, kEpiThreads);
       if (tid == 0) tc::mbar_arrive(bar(B_PREADY + bi));
-      // ---- fold this tile into the unit segment's running (m, l, acc): heads' scale factors
-      if (tid < G) {
-        const float mt = s_stat[2 * tid], lt = s_stat[2 * tid + 1];
-        const float mr = s_run[2 * tid], lr = s_run[2 * tid + 1];
-        const float mx = fmaxf(mr, mt);
-        float al = 0.f, be = 0.f;
-        if (mx != -INFINITY) {
-          al = mr == -INFINITY ? 0.f : expf(mr - mx);
-          be = mt == -INFINITY ? 0.f : expf(mt - mx);
-        }
-        s_ab[2 * tid] = al;
-        s_ab[2 * tid + 1] = be;
-        s_run[2 * tid] = mx;
-        s_run[2 * tid + 1] = lr * al + lt * be;
-      }
-      // ---- this tile's acc from TMEM: warp (quarter, half) holds latent column
-      //      c = half*128 + quarter*32 + lane
-      const bool ok2 = __all_sync(0xffffffffu, tc::mbar_wait(bar(B_PDONE + bi), ph, P.flags));
-      tc::fence_after_sync();
-      uint32_t v[16];
-      if (ok2 && half < n_chunks) {
-        tc::tmem_ld16(tmem_base + ((uint32_t)(quarter * 32) << 16) + o_col0 +
-                          (uint32_t)bi * o_cols + (uint32_t)half * 16,
-                      v);
-        tc::tmem_ld_wait();
-      }
-      tc::fence_before_sync();
-      tc::named_sync(kEpiBar, kEpiThreads);
-      if (tid == 0) tc::mbar_arrive(bar(B_TOFREE + bi));
-      if (ok2 && half < n_chunks) {
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-          acc_run[g] = acc_run[g] * s_ab[2 * g] +
-                       (__uint_as_float(v[2 * g]) + __uint_as_float(v[2 * g + 1])) * s_ab[2 * g + 1];
-      }
-      // ---- end of this CTA's segment of the unit: publish it
-      UnitTileCursor nx = cur;
-      nx.next();
-      const bool seg_end = i + 1 == n || nx.b != cur.b || nx.u != cur.u;
-      ++seg_tiles;
-      if (seg_end) {
-        const int s0 = cur.slot + 1 - seg_tiles;  // first slot of the segment
-        const int c = half * 128 + quarter * 32 + lane;
-        const int64_t row0 = ((int64_t)cur.b * P.Hq + cur.u * G) * P.n_slots + s0;
-        if (half < n_chunks && c < P.r) {
-#pragma unroll
-          for (int g = 0; g < G; ++g)
-            P.part[(row0 + (int64_t)g * P.n_slots) * part_row(P.r) + kPartAcc + c] = acc_run[g];
-        }
-        if (tid < G) {
-          float* pp = P.part + (row0 + (int64_t)tid * P.n_slots) * part_row(P.r);
-          pp[0] = s_run[2 * tid];
-          pp[1] = s_run[2 * tid + 1];
-        }
-        // a new segment starts with the next tile
-        seg_tiles = 0;
-#pragma unroll
-        for (int g = 0; g < G; ++g) acc_run[g] = 0.f;
-        if (tid < G) {
-          s_run[2 * tid] = -INFINITY;
-          s_run[2 * tid + 1] = 0.f;
-        }
-        tc::named_sync(kEpiBar, kEpiThreads);
-      }
+      if (i > 0) fold(i - 1);
     }
+    if (n > 0) fold(n - 1);
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -547,7 +579,7 @@ template <int G, int D>
 size_t smem_bytes(int r) {
   const int KB = r / 64;
   return 1024 + (size_t)KB * D * 128 + 2 * (size_t)KB * 16384 + 2 * 4096 + 8 * (D / 2) * 2 +
-         4 * (G * D + 2 * G * kTile + G * kTile + 2 * G + 2 * kTile + 4 * G) + 8 +
+         4 * (G * D + 2 * G * kTile + G * kTile + 4 * G + 2 * kTile + 4 * G) + 8 +
          8 * B_COUNT + 16;
 }
 
