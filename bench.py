@@ -45,7 +45,9 @@ UNIT = "us/layer-step"
 # DRAM bytes (read + write) of one launch, from an ncu capture of the named
 # kernel on the named workload (the summary under profiles/ gives the command).
 # An entry is removed whenever its kernel changes after the capture.
-PROFILED_TRAFFIC: dict[tuple[str, str], float] = {}
+PROFILED_TRAFFIC: dict[tuple[str, str], float] = {
+    ("mistral_7b_gqa32x8_d128_r256_n32768_b4_k2048_bf16", "attend"): 54.446848e6 + 0.374272e6,
+}
 DEFAULT_WORKLOAD = workloads.MISTRAL_32K_B4.name
 THROTTLE_BITS = {
     0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -66,6 +68,10 @@ def parse_args():
                     help="skip the oracle timing on the host cores")
     ap.add_argument("--no-compress", action="store_true",
                     help="skip the prefill compression GEMM timing")
+    ap.add_argument("--compress-only", action="store_true",
+                    help="time only the prefill compression GEMM and print its JSON object")
+    ap.add_argument("--compress-rows", type=int, default=0,
+                    help="rows of K and V for the compression GEMM (default: 16 x 4096)")
     return ap.parse_args()
 
 
@@ -87,13 +93,13 @@ def measured_bf16_peak():
     return 1590.0, "fallback"
 
 
-def bench_compress(salsc, dev, reps: int = 20, warmup: int = 3):
+def bench_compress(salsc, dev, reps: int = 20, warmup: int = 3, rows: int = 0):
     """The prefill compression GEMM of the LLaMA2-7B-shaped batch (16 x 4096
     rows of K and V, hidden 4096, r 512), both halves in one salsc_compress
     call, timed alone with CUDA events; torch.matmul (cuBLAS) on the same
     operands is timed beside it as a library reference point."""
     w = workloads.LLAMA2_4K_B16
-    n, hid, r = w.compress_rows, w.hidden, w.rank
+    n, hid, r = rows or w.compress_rows, w.hidden, w.rank
     g = torch.Generator(device=dev)
     g.manual_seed(w.seed)
     K = torch.randn(n, hid, device=dev, generator=g).to(torch.bfloat16)
@@ -315,6 +321,11 @@ def main():
         return
 
     from latent_space_sparse_b200 import salsc
+    if args.compress_only:
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        print(json.dumps(bench_compress(salsc, torch.device("cuda"), rows=args.compress_rows)),
+              flush=True)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -465,7 +476,7 @@ def main():
                        "and out copied back every step; host waits for each step"},
     }
     if not args.no_compress:
-        line["compress"] = bench_compress(salsc, dev)
+        line["compress"] = bench_compress(salsc, dev, rows=args.compress_rows)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         line["cpu_baseline"] = cpu_baseline(w, oracle.default_threads())
