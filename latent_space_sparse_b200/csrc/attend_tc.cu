@@ -1,6 +1,6 @@
 // attend_tc.cu -- selective reconstruction, RoPE, softmax and the latent
 // value sum over the kept tokens, on tcgen05 (bf16 storage, d in {64, 128},
-// r <= 256, G in {1, 2, 4, 8}).
+// r <= 256, or r <= 512 in two latent halves, G in {1, 2, 4, 8}).
 //
 // SALS technical framework, stages 3-4, with RoPE applied after
 // reconstruction (abstract).  Work unit: a tile of 128 kept tokens of one
@@ -127,9 +127,14 @@ __device__ __forceinline__ int row_token(const AttendTcParams& P, const UnitTile
 
 // barrier indices
 enum { B_PK = 0, B_KFULL = 1, B_VFULL = 3, B_KDONE = 5, B_PDONE = 7, B_PREADY = 9,
-       B_TKFREE = 11, B_TOFREE = 13, B_COUNT = 15 };
+       B_TKFREE = 11, B_TOFREE = 13, B_PKDONE = 15, B_COUNT = 16 };
 
-template <int G, int D>
+// W = 1: the latent width r <= 256 fits one tile buffer; two buffers hold two
+// tiles, and tiles are pipelined.  W = 2 (256 < r <= 512): the two buffers hold
+// the two latent halves of one tile, Pk_u is loaded half by half (the
+// reconstruction accumulates over the halves), and tiles run one after the
+// other.
+template <int G, int D, int W>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
                  const __grid_constant__ CUtensorMap tmap_kc,
@@ -138,7 +143,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
   constexpr int QPAIRS = HALF / 2;  // RoPE pairs per epilogue thread
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  const int KB = P.r / 64;
+  const int KB = P.r / 64 / W;              // k-blocks of 64 latent columns per buffer
   const int n_chunks = (P.r + 127) / 128;  // M = 128 slices of the latent width
   const uint32_t pk_bytes = (uint32_t)KB * D * 128;
   const uint32_t buf_bytes = (uint32_t)KB * 16384;
@@ -191,7 +196,132 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
   tc::fence_after_sync();
   const uint32_t tmem_base = *s_tmem_slot;
 
-  if (warp >= kLoadWarp0) {
+  if (W == 2 && warp >= kLoadWarp0) {
+    // ======================= gather warps, two latent halves =================
+    // Group h (4 warps) fills buffer h with latent half h of every tile: the
+    // key rows, then, once the reconstruction is done, the value rows.
+    const int h = (warp - kLoadWarp0) / kGatherWarps;
+    const int gt = tid - (kLoadWarp0 + h * kGatherWarps) * 32;  // 0..127
+    const uint32_t gbar = 2 + h;
+    int* tk = s_tok + h * kTile;
+    const uint32_t buf_s = tc::smem_u32(h ? s_buf1 : s_buf0);
+    const uint32_t tile_bytes = (uint32_t)kTile * KB * 128;
+    const int g4 = gt % 32;
+    UnitTileCursor cur;
+    cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
+    grid_dependency_wait();  // the kept indices come from the previous kernel
+    int t_next = n > 0 ? row_token(P, cur, gt) : -1;
+    int last_v = -1;
+    bool ok = true;
+    for (int i = 0; i < n && ok; ++i) {
+      const int64_t off = cur.off;
+      // the buffer is free once the value MMA of the previous tile is done
+      if (i >= 1) ok = tc::mbar_wait(bar(B_PDONE + ((i - 1) & 1)), ((uint32_t)(i - 1) >> 1) & 1u, P.flags);
+      tk[gt] = t_next;
+      if (gt == 0) tc::mbar_expect_tx(bar(B_KFULL + h), tile_bytes);
+      tc::named_sync(gbar, kGatherThreads);
+      int rows[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int t = tk[4 * g4 + j];
+        rows[j] = (int)(off + (t < 0 ? 0 : t));  // no token: weight 0, any valid row
+      }
+      for (int kb = gt / 32; kb < KB; kb += kGatherThreads / 32)
+        tc::tma_gather4(buf_s + kb * 16384u + (uint32_t)(g4 >> 1) * 1024u + (uint32_t)(g4 & 1) * 512u,
+                        &tmap_kc, (h * KB + kb) * 64, rows[0], rows[1], rows[2], rows[3],
+                        bar(B_KFULL + h));
+      cur.next();
+      t_next = i + 1 < n ? row_token(P, cur, gt) : -1;
+      if (!tc::mbar_wait(bar(B_KDONE + (i & 1)), ((uint32_t)i >> 1) & 1u, P.flags)) break;
+      if (gt == 0) tc::mbar_expect_tx(bar(B_VFULL + h), tile_bytes);
+      tc::named_sync(gbar, kGatherThreads);
+      for (int kb = gt / 32; kb < KB; kb += kGatherThreads / 32)
+        tc::tma_gather4(buf_s + kb * 16384u + (uint32_t)(g4 >> 1) * 1024u + (uint32_t)(g4 & 1) * 512u,
+                        &tmap_vc, (h * KB + kb) * 64, rows[0], rows[1], rows[2], rows[3],
+                        bar(B_VFULL + h));
+      last_v = i;
+    }
+    if (gt == 0 && last_v >= 0) tc::mbar_wait(bar(B_VFULL + h), (uint32_t)last_v & 1u, P.flags);
+  } else if (W == 2 && warp == kMmaWarp) {
+    // ======================= MMA issuer, two latent halves (lane 0) ==========
+    // Per tile: Pk_u half 0 -> reconstruction over half 0 -> Pk_u half 1 ->
+    // reconstruction over half 1 (accumulating) -> value MMA over the four
+    // 128-column chunks of the latent width.  Half 0 of the next tile's Pk_u
+    // is loaded while the epilogue works on this tile.
+    if (lane == 0) {
+      const uint32_t idesc_k = tc::idesc_bf16_f32(kTile, D);
+      const uint32_t idesc_v = tc::idesc_bf16_f32_amn(128, kPRows);
+      const uint32_t pkb = tc::smem_u32(s_pk);
+      UnitTileCursor cur;
+      cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
+      uint32_t pk_phase = 0, pkd_phase = 0;
+      auto load_pk = [&](int u, int hh) {
+        tc::mbar_expect_tx(bar(B_PK), pk_bytes);
+        for (int kb = 0; kb < KB; ++kb)
+          tc::tma_load_2d(pkb + (uint32_t)kb * D * 128, &tmap_pk, (hh * KB + kb) * 64, u * D, bar(B_PK));
+      };
+      auto kmma = [&](uint32_t a0, uint32_t d_tmem, bool acc0) {
+        for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc::mma_bf16(d_tmem, tc::sdesc_kmajor_sw128(a0 + kb * 16384 + 32 * k),
+                         tc::sdesc_kmajor_sw128(pkb + kb * D * 128 + 32 * k), idesc_k,
+                         (acc0 || kb || k) ? 1u : 0u);
+      };
+      bool ok = true;
+      if (n > 0) load_pk(cur.u, 0);
+      for (int i = 0; i < n && ok; ++i, cur.next()) {
+        const int bi = i & 1;
+        const uint32_t ph = ((uint32_t)i >> 1) & 1u;
+        const uint32_t d_tmem = tmem_base + (uint32_t)bi * D;
+        ok = tc::mbar_wait(bar(B_PK), pk_phase, P.flags) &&
+             tc::mbar_wait(bar(B_KFULL + 0), (uint32_t)i & 1u, P.flags) &&
+             tc::mbar_wait(bar(B_TKFREE + bi), ph ^ 1u, P.flags);
+        if (!ok) break;
+        pk_phase ^= 1u;
+        tc::fence_after_sync();
+        kmma(tc::smem_u32(s_buf0), d_tmem, false);
+        tc::mma_commit(bar(B_PKDONE));
+        if (!(ok = tc::mbar_wait(bar(B_PKDONE), pkd_phase, P.flags))) break;
+        pkd_phase ^= 1u;
+        load_pk(cur.u, 1);
+        ok = tc::mbar_wait(bar(B_PK), pk_phase, P.flags) &&
+             tc::mbar_wait(bar(B_KFULL + 1), (uint32_t)i & 1u, P.flags);
+        if (!ok) break;
+        pk_phase ^= 1u;
+        tc::fence_after_sync();
+        kmma(tc::smem_u32(s_buf1), d_tmem, true);
+        tc::mma_commit(bar(B_KDONE + bi));
+        if (i + 1 < n) {
+          // half 0 of the next tile's Pk_u, once this reconstruction is done with Pk
+          if (!(ok = tc::mbar_wait(bar(B_KDONE + bi), ph, P.flags))) break;
+          UnitTileCursor nx = cur;
+          nx.next();
+          load_pk(nx.u, 0);
+        }
+        // value MMA: acc^T[r x 2G] = Vc_tile^T . p, chunk ch from buffer ch / 2
+        ok = tc::mbar_wait(bar(B_PREADY + bi), ph, P.flags) &&
+             tc::mbar_wait(bar(B_VFULL + 0), (uint32_t)i & 1u, P.flags) &&
+             tc::mbar_wait(bar(B_VFULL + 1), (uint32_t)i & 1u, P.flags) &&
+             tc::mbar_wait(bar(B_TOFREE + bi), ph ^ 1u, P.flags);
+        if (!ok) break;
+        tc::fence_after_sync();
+        const uint32_t p0 = tc::smem_u32(bi ? s_pbuf1 : s_pbuf0);
+        for (int ch = 0; ch < n_chunks; ++ch) {
+          const uint32_t d_acc = tmem_base + o_col0 + (uint32_t)bi * o_cols + (uint32_t)ch * 16;
+          const uint32_t v0 = tc::smem_u32((ch >> 1) ? s_buf1 : s_buf0) + (uint32_t)(ch & 1) * 2 * 16384;
+#pragma unroll
+          for (int ks = 0; ks < kTile / 16; ++ks) {
+            const uint64_t ad = tc::sdesc_mnmajor_sw128(v0 + (uint32_t)(ks * 2) * 1024, 16384, 1024);
+            const uint64_t bd =
+                tc::sdesc_kmajor_sw128(p0 + (uint32_t)(ks >> 2) * 2048 + (uint32_t)(ks & 3) * 32);
+            tc::mma_bf16(d_acc, ad, bd, idesc_v, ks != 0);
+          }
+        }
+        tc::mma_commit(bar(B_PDONE + bi));
+      }
+    }
+  } else if (warp >= kLoadWarp0) {
     // ======================= gather warps =======================
     // Group bi (4 warps, 128 threads) fills buffer bi with tiles bi, bi+2, ...:
     // first the latent key rows Kc_b[idx], then, once the reconstruction is
@@ -351,9 +481,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     UnitTileCursor cur;
     cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
     int cur_b = -1, cur_u = -1;
-    float acc_run[G];  // this thread's latent column of the segment's running sum
+    // this thread's latent columns c = ch*128 + quarter*32 + lane, chunks
+    // ch = half, half + 2: the segment's running sum
+    float acc_run[W][G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) acc_run[g] = 0.f;
+    for (int w = 0; w < W; ++w)
+#pragma unroll
+      for (int g = 0; g < G; ++g) acc_run[w][g] = 0.f;
     int seg_tiles = 0;
     if (tid < G) {
       s_run[2 * tid] = -INFINITY;
@@ -386,21 +520,26 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       // c = half*128 + quarter*32 + lane
       const bool ok2 = __all_sync(0xffffffffu, tc::mbar_wait(bar(B_PDONE + bj), phj, P.flags));
       tc::fence_after_sync();
-      uint32_t v[16];
-      if (ok2 && half < n_chunks) {
-        tc::tmem_ld16(tmem_base + ((uint32_t)(quarter * 32) << 16) + o_col0 +
-                          (uint32_t)bj * o_cols + (uint32_t)half * 16,
-                      v);
-        tc::tmem_ld_wait();
-      }
+      uint32_t v[W][16];
+#pragma unroll
+      for (int w = 0; w < W; ++w)
+        if (ok2 && half + 2 * w < n_chunks)
+          tc::tmem_ld16(tmem_base + ((uint32_t)(quarter * 32) << 16) + o_col0 +
+                            (uint32_t)bj * o_cols + (uint32_t)(half + 2 * w) * 16,
+                        v[w]);
+      tc::tmem_ld_wait();
       tc::fence_before_sync();
       tc::named_sync(kEpiBar, kEpiThreads);
       if (tid == 0) tc::mbar_arrive(bar(B_TOFREE + bj));
-      if (ok2 && half < n_chunks) {
 #pragma unroll
-        for (int g = 0; g < G; ++g)
-          acc_run[g] = acc_run[g] * s_ab[2 * g] +
-                       (__uint_as_float(v[2 * g]) + __uint_as_float(v[2 * g + 1])) * s_ab[2 * g + 1];
+      for (int w = 0; w < W; ++w) {
+        if (ok2 && half + 2 * w < n_chunks) {
+#pragma unroll
+          for (int g = 0; g < G; ++g)
+            acc_run[w][g] = acc_run[w][g] * s_ab[2 * g] +
+                            (__uint_as_float(v[w][2 * g]) + __uint_as_float(v[w][2 * g + 1])) *
+                                s_ab[2 * g + 1];
+        }
       }
       // end of this CTA's segment of the unit: publish it
       UnitTileCursor nx = fc;
@@ -409,12 +548,15 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       ++seg_tiles;
       if (seg_end) {
         const int s0 = fc.slot + 1 - seg_tiles;  // first slot of the segment
-        const int c = half * 128 + quarter * 32 + lane;
         const int64_t row0 = ((int64_t)fc.b * P.Hq + fc.u * G) * P.n_slots + s0;
-        if (half < n_chunks && c < P.r) {
 #pragma unroll
-          for (int g = 0; g < G; ++g)
-            P.part[(row0 + (int64_t)g * P.n_slots) * part_row(P.r) + kPartAcc + c] = acc_run[g];
+        for (int w = 0; w < W; ++w) {
+          const int c = (half + 2 * w) * 128 + quarter * 32 + lane;
+          if (half + 2 * w < n_chunks && c < P.r) {
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+              P.part[(row0 + (int64_t)g * P.n_slots) * part_row(P.r) + kPartAcc + c] = acc_run[w][g];
+          }
         }
         if (tid < G) {
           float* pp = P.part + (row0 + (int64_t)tid * P.n_slots) * part_row(P.r);
@@ -424,7 +566,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
         // a new segment starts with the next tile
         seg_tiles = 0;
 #pragma unroll
-        for (int g = 0; g < G; ++g) acc_run[g] = 0.f;
+        for (int w = 0; w < W; ++w)
+#pragma unroll
+          for (int g = 0; g < G; ++g) acc_run[w][g] = 0.f;
         if (tid < G) {
           s_run[2 * tid] = -INFINITY;
           s_run[2 * tid + 1] = 0.f;
@@ -459,8 +603,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       tc::fence_after_sync();
       // this row's token: written by the gather warp before it released the
       // Kc barrier of this tile, which is acquired here (its phase is complete)
-      tc::mbar_wait(bar(B_KFULL + bi), ph, P.flags);
-      const int t = s_tok[bi * kTile + m];
+      const int t = W == 1 ? (tc::mbar_wait(bar(B_KFULL + bi), ph, P.flags), s_tok[bi * kTile + m])
+                           : (tc::mbar_wait(bar(B_KFULL), (uint32_t)i & 1u, P.flags), s_tok[m]);
       float dot[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) dot[g] = 0.f;
@@ -575,24 +719,24 @@ int num_sms_att() {
   return cached[dev];
 }
 
-template <int G, int D>
+template <int G, int D, int W>
 size_t smem_bytes(int r) {
-  const int KB = r / 64;
+  const int KB = r / 64 / W;
   return 1024 + (size_t)KB * D * 128 + 2 * (size_t)KB * 16384 + 2 * 4096 + 8 * (D / 2) * 2 +
          4 * (G * D + 2 * G * kTile + G * kTile + 4 * G + 2 * kTile + 4 * G) + 8 +
          8 * B_COUNT + 16;
 }
 
-template <int G, int D>
+template <int G, int D, int W>
 cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
-  const size_t smem = smem_bytes<G, D>(p.r);
+  const size_t smem = smem_bytes<G, D, W>(p.r);
   CUtensorMap tpk, tkc, tvc;
   if (!make_tmap_bf16_2d(&tpk, a.Pk, (uint64_t)p.U * D, (uint64_t)p.r, D, 64) ||
       !make_tmap_bf16_2d(&tkc, a.Kc, (uint64_t)p.N, (uint64_t)p.r, 1, 64) ||
       !make_tmap_bf16_2d(&tvc, a.Vc, (uint64_t)p.N, (uint64_t)p.r, 1, 64))
     return cudaErrorInvalidValue;
   static int done[kMaxDevices] = {};
-  cudaError_t e = ensure_smem(attend_tc_kernel<G, D>, smem, done);
+  cudaError_t e = ensure_smem(attend_tc_kernel<G, D, W>, smem, done);
   if (e != cudaSuccess) return e;
   AttendTcParams P;
   P.q = (const __nv_bfloat16*)a.q;
@@ -612,8 +756,28 @@ cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s)
   P.n_tiles = p.att_tiles;
   P.scale = p.scale;
   P.base = p.rope_base;
-  return launch_k(attend_tc_kernel<G, D>, dim3(attend_tc_grid(p)), dim3(kThreads), smem, s, true,
-                  tpk, tkc, tvc, P);
+  return launch_k(attend_tc_kernel<G, D, W>, dim3(attend_tc_grid(p)), dim3(kThreads), smem, s,
+                  true, tpk, tkc, tvc, P);
+}
+
+template <int W>
+cudaError_t launch_w(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
+  if (p.d == 128) {
+    switch (p.G) {
+      case 1: return launch_g_d<1, 128, W>(p, a, s);
+      case 2: return launch_g_d<2, 128, W>(p, a, s);
+      case 4: return launch_g_d<4, 128, W>(p, a, s);
+      case 8: return launch_g_d<8, 128, W>(p, a, s);
+    }
+  } else {
+    switch (p.G) {
+      case 1: return launch_g_d<1, 64, W>(p, a, s);
+      case 2: return launch_g_d<2, 64, W>(p, a, s);
+      case 4: return launch_g_d<4, 64, W>(p, a, s);
+      case 8: return launch_g_d<8, 64, W>(p, a, s);
+    }
+  }
+  return cudaErrorInvalidConfiguration;
 }
 
 }  // namespace
@@ -624,28 +788,15 @@ int attend_tc_grid(const DecodePlan& p) {
 
 bool attend_tc_supported(const DecodePlan& p) {
   const int64_t k_eff = p.k < p.n_max ? p.k : p.n_max;
-  return p.dtype == SALSC_BF16 && p.r % 64 == 0 && p.r <= 256 && (p.d == 64 || p.d == 128) &&
+  // r <= 256: one tile per buffer; 256 < r <= 512 with r % 128 == 0: two latent halves
+  const bool width_ok = (p.r % 64 == 0 && p.r <= 256) || (p.r % 128 == 0 && p.r <= 512);
+  return p.dtype == SALSC_BF16 && width_ok && (p.d == 64 || p.d == 128) &&
          (p.G == 1 || p.G == 2 || p.G == 4 || p.G == 8) && p.N <= INT32_MAX &&
          (k_eff + kTile - 1) / kTile <= kTile;  // the merge takes <= 128 slots per unit
 }
 
 cudaError_t launch_attend_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
-  if (p.d == 128) {
-    switch (p.G) {
-      case 1: return launch_g_d<1, 128>(p, a, s);
-      case 2: return launch_g_d<2, 128>(p, a, s);
-      case 4: return launch_g_d<4, 128>(p, a, s);
-      case 8: return launch_g_d<8, 128>(p, a, s);
-    }
-  } else {
-    switch (p.G) {
-      case 1: return launch_g_d<1, 64>(p, a, s);
-      case 2: return launch_g_d<2, 64>(p, a, s);
-      case 4: return launch_g_d<4, 64>(p, a, s);
-      case 8: return launch_g_d<8, 64>(p, a, s);
-    }
-  }
-  return cudaErrorInvalidConfiguration;
+  return p.r <= 256 ? launch_w<1>(p, a, s) : launch_w<2>(p, a, s);
 }
 
 }  // namespace salsc
