@@ -299,7 +299,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
           nx.next();
           load_pk(nx.u, 0);
         }
-        // value MMA: acc^T[r x 2G] = Vc_tile^T . p, chunk ch from buffer ch / 2
+        // value MMA: acc^T[r x 2G] = Vc_tile^T . p.  The two buffers are adjacent,
+        // so latent k-block j of the tile is at s_buf0 + j * 16 KiB and chunk ch
+        // (k-blocks 2ch, 2ch+1) may straddle them.
         ok = tc::mbar_wait(bar(B_PREADY + bi), ph, P.flags) &&
              tc::mbar_wait(bar(B_VFULL + 0), (uint32_t)i & 1u, P.flags) &&
              tc::mbar_wait(bar(B_VFULL + 1), (uint32_t)i & 1u, P.flags) &&
@@ -309,7 +311,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
         const uint32_t p0 = tc::smem_u32(bi ? s_pbuf1 : s_pbuf0);
         for (int ch = 0; ch < n_chunks; ++ch) {
           const uint32_t d_acc = tmem_base + o_col0 + (uint32_t)bi * o_cols + (uint32_t)ch * 16;
-          const uint32_t v0 = tc::smem_u32((ch >> 1) ? s_buf1 : s_buf0) + (uint32_t)(ch & 1) * 2 * 16384;
+          const uint32_t v0 = tc::smem_u32(s_buf0) + (uint32_t)ch * 2 * 16384;
 #pragma unroll
           for (int ks = 0; ks < kTile / 16; ++ks) {
             const uint64_t ad = tc::sdesc_mnmajor_sw128(v0 + (uint32_t)(ks * 2) * 1024, 16384, 1024);

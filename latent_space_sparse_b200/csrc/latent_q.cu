@@ -14,39 +14,38 @@
 namespace salsc {
 namespace {
 
-constexpr int kCols = 16;                  // latent columns per CTA
-constexpr int kSlices = 32;                // row slices of Pk_u per CTA
-constexpr int kThreads = kCols * kSlices;  // thread (slice, column): 512
-constexpr int kWarps = kThreads / 32;
-constexpr int kBatchChunk = 8;             // sequences per pass
-constexpr int kRowsMax = kMaxHeadDim / kSlices;
+constexpr int kThreads = 512;
+constexpr int kBatchChunk = 8;  // sequences per pass
 
 // CTA (u, column block): q_lat[b, u, c] = sum_i qsum[b, i] * Pk[u*d + i, c] for
-// 16 columns c.  Thread (slice, column) owns d/32 rows of one column of Pk_u;
-// Pk is a weight, not an output of the previous kernel, so those loads are
-// issued before the dependency wait (the kernel is launched with programmatic
-// dependent launch).  After the wait the group sums of the queries are formed
-// in shared memory (one query element per thread), each thread adds up its
-// rows for every sequence, and the 32 slices are summed: lanes l and l+16 of a
-// warp by a shuffle, then the 16 warps through shared memory.  Many short
-// threads rather than a few long ones: with one CTA per SM the latency of
-// each instruction is hidden only by other warps.
-template <typename T>
+// COLS columns c.  Thread (slice, column) owns d/SLICES rows of one column of
+// Pk_u; Pk is a weight, not an output of the previous kernel, so those loads
+// are issued before the dependency wait (the kernel is launched with
+// programmatic dependent launch).  After the wait the group sums of the
+// queries are formed in shared memory (one query element per thread), each
+// thread adds up its rows for every sequence, and the slices are summed
+// through shared memory.  Many short threads rather than a few long ones:
+// with one CTA per SM the latency of each instruction is hidden only by
+// other warps.  COLS = 16 spreads a small Pk (GQA) over enough CTAs; COLS = 64
+// keeps a large one (MHA, r = 512) to a few hundred CTAs.
+template <typename T, int COLS>
 __global__ void __launch_bounds__(kThreads)
 latent_q_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __restrict__ qlat,
                 __nv_bfloat16* __restrict__ qsplit, uint32_t* __restrict__ krange, int B, int Hq,
                 int U, int G, int d, int r, int npad) {
+  constexpr int SLICES = kThreads / COLS;
+  constexpr int kRowsMax = (kMaxHeadDim + SLICES - 1) / SLICES;
   __shared__ float qsum[kBatchChunk][kMaxHeadDim];
-  __shared__ float red[kWarps][kBatchChunk][kCols];
+  __shared__ float red[SLICES][kBatchChunk][COLS];
   const int u = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
-  const int col = tid % kCols, slice = tid / kCols;
-  const int c = blockIdx.y * kCols + col;
-  const int rows = d / kSlices, i0 = slice * rows;
+  const int tid = threadIdx.x;
+  const int col = tid % COLS, slice = tid / COLS;
+  const int c = blockIdx.y * COLS + col;
+  const int rows = (d + SLICES - 1) / SLICES, i0 = slice * rows;
   float pk[kRowsMax];
 #pragma unroll
   for (int j = 0; j < kRowsMax; ++j)
-    pk[j] = (j < rows && c < r) ? to_f32(Pk[((size_t)u * d + i0 + j) * r + c]) : 0.f;
+    pk[j] = (j < rows && i0 + j < d && c < r) ? to_f32(Pk[((size_t)u * d + i0 + j) * r + c]) : 0.f;
   allow_dependent_launch();
   grid_dependency_wait();  // q and the workspace belong to the previous kernel until now
   // empty key range of every unit, narrowed by the scoring kernel's atomics
@@ -75,26 +74,21 @@ latent_q_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __rest
                              ((v[j][4] + v[j][5]) + (v[j][6] + v[j][7]));
     }
     __syncthreads();
-    float acc[kBatchChunk];
 #pragma unroll
     for (int bb = 0; bb < kBatchChunk; ++bb) {
-      acc[bb] = 0.f;
+      float acc = 0.f;
 #pragma unroll
       for (int j = 0; j < kRowsMax; ++j)
-        if (j < rows && bb < nb) acc[bb] = fmaf(qsum[bb][i0 + j], pk[j], acc[bb]);
-      acc[bb] += __shfl_xor_sync(0xffffffffu, acc[bb], 16);  // the warp's two slices
-    }
-    if (lane < kCols) {
-#pragma unroll
-      for (int bb = 0; bb < kBatchChunk; ++bb) red[warp][bb][lane] = acc[bb];
+        if (j < rows && i0 + j < d && bb < nb) acc = fmaf(qsum[bb][i0 + j], pk[j], acc);
+      red[slice][bb][col] = acc;
     }
     __syncthreads();
-    if (tid < nb * kCols) {
-      const int bb = tid / kCols, cl = tid % kCols;
-      const int cc = blockIdx.y * kCols + cl;
+    if (tid < nb * COLS) {
+      const int bb = tid / COLS, cl = tid % COLS;
+      const int cc = blockIdx.y * COLS + cl;
       float sum = 0.f;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) sum += red[w][bb][cl];
+      for (int sl = 0; sl < SLICES; ++sl) sum += red[sl][bb][cl];
       if (cc < r) {
         const int b = b0 + bb;
         qlat[((size_t)b * U + u) * r + cc] = sum;
@@ -112,17 +106,25 @@ latent_q_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __rest
   }
 }
 
+template <typename T, int COLS>
+cudaError_t launch_cols(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
+  dim3 grid(p.U, (p.r + COLS - 1) / COLS);
+  return launch_k(latent_q_kernel<T, COLS>, grid, dim3(kThreads), 0, s, true, (const T*)a.q,
+                  (const T*)a.Pk, a.qlat, a.qsplit, a.krange, p.B, p.Hq, p.U, p.G, p.d, p.r,
+                  p.npad);
+}
+
+template <typename T>
+cudaError_t launch_t(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
+  // 16 columns per CTA unless that makes more than 512 CTAs
+  return (int64_t)p.U * ((p.r + 15) / 16) > 512 ? launch_cols<T, 64>(p, a, s)
+                                                  : launch_cols<T, 16>(p, a, s);
+}
+
 }  // namespace
 
 cudaError_t launch_latent_q(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
-  dim3 grid(p.U, (p.r + kCols - 1) / kCols);
-  if (p.dtype == SALSC_BF16)
-    return launch_k(latent_q_kernel<__nv_bfloat16>, grid, dim3(kThreads), 0, s, true,
-                    (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.Pk, a.qlat, a.qsplit,
-                    a.krange, p.B, p.Hq, p.U, p.G, p.d, p.r, p.npad);
-  return launch_k(latent_q_kernel<float>, grid, dim3(kThreads), 0, s, true, (const float*)a.q,
-                  (const float*)a.Pk, a.qlat, a.qsplit, a.krange, p.B, p.Hq, p.U, p.G, p.d, p.r,
-                  p.npad);
+  return p.dtype == SALSC_BF16 ? launch_t<__nv_bfloat16>(p, a, s) : launch_t<float>(p, a, s);
 }
 
 }  // namespace salsc

@@ -139,6 +139,21 @@ def test_head_dim_64_gqa_bf16():
     check(w, synth.decode_inputs(w))
 
 
+def test_wide_rank_384_gqa():
+    # 256 < r <= 512: the attention takes the latent width in two halves of
+    # three 64-column blocks each
+    w = W.Workload(name="gqa_r384", batch=2, n_q_heads=8, n_kv_heads=4, head_dim=128, rank=384,
+                   top_k=200, seq_lens=(700, 300), dtype="bf16", rope_base=10000.0, low_rank=64,
+                   seed=97)
+    check(w, synth.decode_inputs(w))
+
+
+def test_wide_rank_512_mha_many_tiles():
+    # r = 512 with several tiles per unit and per CTA (tiles run one after another)
+    w = W.LLAMA2_4K_B1
+    check(w, synth.decode_inputs(w, seq_lens=(4096,)), top_k=1000)
+
+
 def test_small_rank_f32():
     w = W.Workload(name="f32_r16", batch=3, n_q_heads=6, n_kv_heads=3, head_dim=64, rank=16,
                    top_k=9, seq_lens=(50, 17, 200), dtype="f32", rope_base=500000.0, low_rank=4,
