@@ -136,6 +136,11 @@ salsc_status salsc_decode_prepare(const salsc_decode_desc* desc, void* ws, size_
  *   ws       workspace of at least salsc_decode_workspace_size bytes,
  *            prepared once with salsc_decode_prepare; 256-byte aligned
  * No allocation, no host synchronisation: safe to capture in a CUDA graph.
+ * Stream order: the kernels are launched with programmatic dependent launch.
+ * Until the work enqueued before the step has finished, the step reads only
+ * Pk; after that its later kernels may start early and read the other inputs
+ * (Kc, Vc, Pv, q, the sequence offsets), so no input may change until the
+ * step has completed.
  * Errors: INVALID_ARG (desc or null pointer), UNSUPPORTED (shape without a
  * kernel), WORKSPACE, CUDA.
  */
@@ -203,6 +208,29 @@ salsc_status salsc_decode_step_static_ws(const salsc_decode_desc* desc, const vo
                                          const void* Kc, const void* Vc, const void* Pk,
                                          const void* Pv, void* out, int32_t* idx_out,
                                          salsc_stream stream);
+
+/*
+ * Decode-time append (SALS technical framework, stage 1 applied to the token
+ * being decoded): for every sequence b < batch,
+ *   Kc[rows_dev[b]] = K_new[b] . Pk   and   Vc[rows_dev[b]] = V_new[b] . Pv
+ * with fp32 accumulation and one rounding to the storage dtype.  Together with
+ * the decode step this keeps the latent cache up to date token by token.
+ *
+ *   K_new, V_new [batch][hidden]  the new token's key (before RoPE) and value
+ *                                 rows; either may be NULL to skip that half
+ *   Pk, Pv       [hidden][rank]   projections (the ones given to compress)
+ *   Kc, Vc       [*][rank]        latent caches, written at the given rows only
+ *   rows_dev     [batch] int64    device array: destination row of sequence b
+ *                                 (the caller's packing, e.g. seq_offsets[b]+n_b
+ *                                 with spare capacity); rows must be distinct
+ *                                 and inside Kc/Vc (not checked)
+ * Allocates nothing, stream-ordered, graph-capturable.
+ * Errors: INVALID_ARG (dtype, negative batch, null required pointer),
+ * UNSUPPORTED (hidden > 8192), CUDA.
+ */
+salsc_status salsc_append(const void* K_new, const void* V_new, const void* Pk, const void* Pv,
+                          void* Kc, void* Vc, const int64_t* rows_dev, int32_t batch,
+                          int32_t hidden, int32_t rank, salsc_dtype dtype, salsc_stream stream);
 
 /*
  * Device-side anomaly flags recorded in a workspace since salsc_decode_prepare

@@ -188,6 +188,24 @@ salsc_status salsc_decode_read_flags(void* ws, size_t ws_bytes, uint32_t* flags_
   return SALSC_OK;
 }
 
+salsc_status salsc_append(const void* K_new, const void* V_new, const void* Pk, const void* Pv,
+                          void* Kc, void* Vc, const int64_t* rows_dev, int32_t batch,
+                          int32_t hidden, int32_t rank, salsc_dtype dtype, salsc_stream stream) {
+  if (dtype != SALSC_F32 && dtype != SALSC_BF16) return SALSC_ERR_INVALID_ARG;
+  if (batch < 0 || hidden < 1 || rank < 1 || !rows_dev) return SALSC_ERR_INVALID_ARG;
+  if (!K_new && !V_new) return SALSC_ERR_INVALID_ARG;
+  if (K_new && (!Pk || !Kc)) return SALSC_ERR_INVALID_ARG;
+  if (V_new && (!Pv || !Vc)) return SALSC_ERR_INVALID_ARG;
+  if (hidden > 8 * 1024) return SALSC_ERR_UNSUPPORTED;
+  if (batch == 0) return SALSC_OK;
+  const void* X[2] = {K_new ? K_new : V_new, V_new};
+  const void* Pm[2] = {K_new ? Pk : Pv, Pv};
+  void* Y[2] = {K_new ? Kc : Vc, Vc};
+  cudaError_t e = salsc::launch_append(X, Pm, Y, (K_new && V_new) ? 2 : 1, rows_dev, batch, hidden,
+                                       rank, dtype, (cudaStream_t)stream);
+  return e == cudaSuccess ? SALSC_OK : cuda_fail(e);
+}
+
 }  // extern "C"
 
 namespace {

@@ -76,7 +76,9 @@ combine_kernel(const CombineParams P) {
                   bar_pv);
   }
   allow_dependent_launch();
-  grid_dependency_wait();  // the partials come from the attention kernel
+  // The used slots follow from the sequence lengths and the tile partition
+  // alone (inputs of the step, not outputs of the attention kernel), so they
+  // are found before the dependency wait.
   if (warp == 0) {
     // slots of unit (b, u) and, with the tile partition, the unit's first tile:
     // every lane reads one sequence's offsets, a warp scan sums the tiles
@@ -117,6 +119,7 @@ combine_kernel(const CombineParams P) {
       s_L[lane] = 0.f;
     }
   }
+  grid_dependency_wait();  // the partials come from the attention kernel
   __syncthreads();
   const int nseg = s_nseg;
   // this thread's latent columns tid, tid + 256 for every head

@@ -85,6 +85,10 @@ cudaError_t launch_attend_tc(const DecodePlan& p, const DecodeArgs& a, cudaStrea
 cudaError_t launch_compress(const void* X, const void* P, void* Y, int64_t n, int hid, int r,
                             salsc_dtype dt, cudaStream_t s);
 bool compress_tc_supported(int hid, int r, salsc_dtype dt);
+// Decode-time append: Y[i][rows[b]] = X[i][b] . Pm[i] for the n_mats (1 or 2) matrices.
+cudaError_t launch_append(const void* const X[2], const void* const Pm[2], void* const Y[2],
+                          int n_mats, const int64_t* rows, int B, int hid, int r, salsc_dtype dt,
+                          cudaStream_t s);
 // Tensor-core compression of n_mats (1 or 2) matrices X[i] . Pm[i] -> Y[i] in one launch.
 cudaError_t launch_compress_tc(const void* const X[2], const void* const Pm[2], void* const Y[2],
                                int n_mats, int64_t n, int hid, int r, cudaStream_t s);

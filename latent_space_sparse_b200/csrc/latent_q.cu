@@ -46,8 +46,11 @@ latent_q_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __rest
 #pragma unroll
   for (int j = 0; j < kRowsMax; ++j)
     pk[j] = (j < rows && i0 + j < d && c < r) ? to_f32(Pk[((size_t)u * d + i0 + j) * r + c]) : 0.f;
-  allow_dependent_launch();
   grid_dependency_wait();  // q and the workspace belong to the previous kernel until now
+  // Only now may the step's later kernels start: they read step inputs (Kc,
+  // the sequence offsets) before their own dependency waits, and everything
+  // the stream did before this step is complete once the wait above returns.
+  allow_dependent_launch();
   // empty key range of every unit, narrowed by the scoring kernel's atomics
   if (blockIdx.y == 0)
     for (int b = tid; b < B; b += kThreads) {

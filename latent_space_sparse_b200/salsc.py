@@ -23,7 +23,7 @@ WS_ALIGN = 256
 
 EXPORTS = (
     "salsc_compress", "salsc_decode_workspace_size", "salsc_decode_prepare", "salsc_decode_step",
-    "salsc_decode_step_timed", "salsc_decode_step_static_ws", "salsc_decode_launch_count", "salsc_decode_read_flags", "salsc_status_string", "salsc_last_cuda_error", "salsc_version",
+    "salsc_decode_step_timed", "salsc_decode_step_static_ws", "salsc_decode_launch_count", "salsc_append", "salsc_decode_read_flags", "salsc_status_string", "salsc_last_cuda_error", "salsc_version",
 )
 
 
@@ -73,6 +73,8 @@ def _lib():
         lib.salsc_decode_prepare.argtypes = [dp, vp, sz, vp]
         lib.salsc_decode_step.restype = ctypes.c_int
         lib.salsc_decode_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.salsc_append.restype = ctypes.c_int
+        lib.salsc_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, ctypes.c_int, vp]
         lib.salsc_decode_launch_count.restype = ctypes.c_int32
         lib.salsc_decode_launch_count.argtypes = [dp]
         lib.salsc_decode_step_timed.restype = ctypes.c_int
@@ -135,6 +137,19 @@ def salsc_compress(K, V, Pk, Pv, Kc, Vc, stream=None):
     st = _lib().salsc_compress(_ptr(K), _ptr(V), _ptr(Pk), _ptr(Pv), _ptr(Kc), _ptr(Vc), n, hid, r,
                                _dtype_code(x.dtype), _stream(stream))
     _check(st, "salsc_compress")
+
+
+def salsc_append(K_new, V_new, Pk, Pv, Kc, Vc, rows, stream=None):
+    """Kc[rows[b]] = K_new[b] . Pk and Vc[rows[b]] = V_new[b] . Pv (rows: int64
+    device tensor); K_new or V_new may be None."""
+    x = K_new if K_new is not None else V_new
+    batch, hid = x.shape
+    r = (Pk if K_new is not None else Pv).shape[1]
+    if rows.dtype != torch.int64 or not rows.is_cuda:
+        raise ValueError("rows must be an int64 device tensor")
+    st = _lib().salsc_append(_ptr(K_new), _ptr(V_new), _ptr(Pk), _ptr(Pv), _ptr(Kc), _ptr(Vc),
+                             _ptr(rows), batch, hid, r, _dtype_code(x.dtype), _stream(stream))
+    _check(st, "salsc_append")
 
 
 def make_desc(batch, n_q_heads, n_kv_heads, head_dim, rank, top_k, seq_offsets_host,

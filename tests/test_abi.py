@@ -110,6 +110,28 @@ def test_prepare_rejects_short_workspace():
     assert st == salsc.SALSC_ERR_WORKSPACE
 
 
+def test_append_validation_before_launch():
+    lib = salsc.load()
+    vp = ctypes.c_void_p
+    ok = dict(K=vp(1 << 20), V=vp(1 << 21), Pk=vp(1 << 22), Pv=vp(1 << 23), Kc=vp(1 << 24),
+              Vc=vp(1 << 25), rows=vp(1 << 26))
+
+    def call(batch=2, hidden=1024, rank=256, dtype=1, **kw):
+        a = dict(ok)
+        a.update(kw)
+        return lib.salsc_append(a["K"], a["V"], a["Pk"], a["Pv"], a["Kc"], a["Vc"], a["rows"],
+                                batch, hidden, rank, dtype, None)
+
+    assert call(K=None, V=None) == salsc.SALSC_ERR_INVALID_ARG
+    assert call(rows=None) == salsc.SALSC_ERR_INVALID_ARG
+    assert call(Pk=None) == salsc.SALSC_ERR_INVALID_ARG
+    assert call(V=vp(1 << 21), Vc=None) == salsc.SALSC_ERR_INVALID_ARG
+    assert call(batch=-1) == salsc.SALSC_ERR_INVALID_ARG
+    assert call(dtype=7) == salsc.SALSC_ERR_INVALID_ARG
+    assert call(hidden=16384) == salsc.SALSC_ERR_UNSUPPORTED
+    assert call(batch=0) == salsc.SALSC_OK  # nothing to do, nothing launched
+
+
 def test_compress_validation_before_launch():
     lib = salsc.load()
     vp = ctypes.c_void_p

@@ -251,3 +251,43 @@ def test_compress_tensor_core_one_half_only():
     torch.cuda.synchronize()
     ref = oracle.compress(x["K"], x["Pk"])
     assert max_rel_err(Kc.float().cpu().numpy(), ref) <= TOL["bf16"]
+
+
+# ------------------------------------------------------------ decode-time append
+
+@pytest.mark.parametrize("wname,dt", [("LLAMA2_4K_B16", "bf16"), ("MISTRAL_32K_B4", "bf16"),
+                                      ("TINY_F32", "f32")])
+def test_append_new_rows_match_the_oracle(wname, dt):
+    w = getattr(W, wname)
+    B = max(3, w.batch)
+    x = synth.compress_inputs(w, rows=B, seed=w.seed + 5)
+    K, V, Pk, Pv = (x[n].to(DEV) for n in ("K", "V", "Pk", "Pv"))
+    tdt = synth.torch_dtype(dt)
+    n_rows = 50 + 7 * B
+    Kc = torch.full((n_rows, w.rank), 3.0, dtype=tdt, device=DEV)
+    Vc = torch.full_like(Kc, -2.0)
+    # destination rows: distinct, not in order
+    rows_np = np.random.default_rng(1).choice(n_rows, B, replace=False).astype(np.int64)
+    rows = torch.from_numpy(rows_np).to(DEV)
+    salsc.salsc_append(K, V, Pk, Pv, Kc, Vc, rows)
+    torch.cuda.synchronize()
+    for got, X, P, fill in ((Kc, x["K"], x["Pk"], 3.0), (Vc, x["V"], x["Pv"], -2.0)):
+        g = got.float().cpu().numpy()
+        ref = oracle.compress(X, P)
+        assert max_rel_err(g[rows_np], ref) <= TOL[dt]
+        others = np.setdiff1d(np.arange(n_rows), rows_np)
+        assert (g[others] == fill).all()  # nothing else written
+
+
+def test_append_one_half_and_batch_above_one_pass():
+    w = W.MISTRAL_32K_B4
+    B = 37  # more sequences than one pass of the kernel takes
+    x = synth.compress_inputs(w, rows=B, seed=3)
+    V, Pv = x["V"].to(DEV), x["Pv"].to(DEV)
+    Vc = torch.zeros(B + 5, w.rank, dtype=torch.bfloat16, device=DEV)
+    rows = torch.arange(5, B + 5, dtype=torch.int64, device=DEV)
+    salsc.salsc_append(None, V, None, Pv, None, Vc, rows)
+    torch.cuda.synchronize()
+    ref = oracle.compress(x["V"], x["Pv"])
+    assert max_rel_err(Vc[5:].float().cpu().numpy(), ref) <= TOL["bf16"]
+    assert (Vc[:5] == 0).all()
