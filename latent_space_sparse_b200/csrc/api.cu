@@ -24,7 +24,9 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 constexpr int kScoreTile = 128;
-constexpr int kTopkSliceTarget = 8192;  // keys per top-k CTA before the cluster grows
+constexpr int kTopkTargetCtas = 148;    // top-k CTAs aimed at (one per SM)
+constexpr int kTopkMinSlice = 4096;     // keys per CTA at which the cluster stops growing
+constexpr int kTopkMaxSlice = 40960;    // keys per CTA in shared memory (160 KiB)
 constexpr int kTopkMaxCluster = 8;
 constexpr int kAttendTargetCtas = 2 * 148;
 
@@ -70,11 +72,18 @@ salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
   p.n_max = n_max;
   p.score_tile = kScoreTile;
   p.n_score_tiles = n_tiles;
+  // Top-k: C CTAs per unit, about one CTA per SM in all (up to 8 per unit, and
+  // enough for a slice of the scores to fit shared memory); many small units
+  // take 256-thread CTAs, several resident per SM.
   int c = 1;
-  while (c < kTopkMaxCluster && (n_max + c - 1) / c > kTopkSliceTarget) c *= 2;
+  while (c < kTopkMaxCluster && (int64_t)p.B * p.U * c * 2 <= kTopkTargetCtas &&
+         (n_max + c - 1) / c > kTopkMinSlice)
+    c *= 2;
+  while (c < kTopkMaxCluster && (n_max + c - 1) / c > kTopkMaxSlice) c *= 2;
   p.topk_cluster = c;
   p.topk_slice = (int)((n_max + c - 1) / c);
-  if ((size_t)p.topk_slice * 4 > 200u * 1024u) return SALSC_ERR_UNSUPPORTED;  // slice in smem
+  if (p.topk_slice > kTopkMaxSlice) return SALSC_ERR_UNSUPPORTED;  // slice in smem
+  p.topk_threads = (int64_t)p.B * p.U * c > kTopkTargetCtas ? 256 : 1024;
   const int64_t k_eff = D->top_k < n_max ? D->top_k : n_max;
   p.attend_tc = salsc::attend_tc_supported(p);
   if (p.attend_tc) {

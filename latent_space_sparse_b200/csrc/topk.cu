@@ -34,8 +34,6 @@ namespace cg = cooperative_groups;
 namespace salsc {
 namespace {
 
-constexpr int kThreads = 1024;
-constexpr int kWarps = kThreads / 32;
 constexpr int kBatch = 32;  // keys a thread loads before converting them
 constexpr int kMaxCluster = 8;  // largest cluster of CTAs per unit
 
@@ -59,13 +57,21 @@ __device__ __forceinline__ int linear_bin(uint32_t key, float fmin, float scale)
 
 // Block-wide search for the digit that holds the target rank: `cnt` holds the
 // histogram (ascending bins); bins are scanned from the top.  Thread t looks
-// at bins 2047-2t and 2046-2t.  Returns through s_digit / s_above.
+// at the `per` bins nbins-1-t*per .. nbins-(t+1)*per (per = nbins / THREADS,
+// at least 1).  Returns through s_digit / s_above.
+template <int THREADS>
 __device__ __forceinline__ void find_digit(const uint32_t* cnt, uint32_t target, int nbins,
                                            uint32_t* wsum, uint32_t* s_digit, uint32_t* s_above) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int b0 = nbins - 1 - 2 * tid, b1 = b0 - 1;  // nbins <= 2 * kThreads
-  const uint32_t c0 = b0 >= 0 ? cnt[b0] : 0u, c1 = b1 >= 0 ? cnt[b1] : 0u;
-  const uint32_t mine = c0 + c1;
+  const int per = nbins / THREADS > 1 ? nbins / THREADS : 1;  // nbins / THREADS <= 8
+  const int top = nbins - 1 - tid * per;
+  uint32_t c[8];
+  uint32_t mine = 0u;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    c[j] = (j < per && top - j >= 0) ? cnt[top - j] : 0u;
+    mine += c[j];
+  }
   uint32_t incl = mine;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -75,7 +81,7 @@ __device__ __forceinline__ void find_digit(const uint32_t* cnt, uint32_t target,
   if (lane == 31) wsum[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    const uint32_t v = wsum[lane];
+    const uint32_t v = lane < THREADS / 32 ? wsum[lane] : 0u;
     uint32_t x = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -85,20 +91,22 @@ __device__ __forceinline__ void find_digit(const uint32_t* cnt, uint32_t target,
     wsum[32 + lane] = x - v;  // exclusive prefix of the warps above
   }
   __syncthreads();
-  const uint32_t above0 = wsum[32 + warp] + incl - mine;  // keys in bins above b0
-  if (above0 < target && target <= above0 + c0) {
-    *s_digit = (uint32_t)b0;
-    *s_above = above0;
-  } else if (above0 + c0 < target && target <= above0 + c0 + c1) {
-    *s_digit = (uint32_t)b1;
-    *s_above = above0 + c0;
+  uint32_t above = wsum[32 + warp] + incl - mine;  // keys in bins above this thread's
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j < per && above < target && target <= above + c[j]) {
+      *s_digit = (uint32_t)(top - j);
+      *s_above = above;
+    }
+    above += c[j];
   }
 }
 
-template <bool kCluster>
+template <bool kCluster, int kThreads>
 __global__ void __launch_bounds__(kThreads)
 topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_off,
             const uint32_t* __restrict__ krange, int32_t* __restrict__ idx_out, int U, int k) {
+  constexpr int kWarps = kThreads / 32;
   cg::cluster_group cluster = cg::this_cluster();
   const int C = kCluster ? (int)cluster.num_blocks() : 1;
   const int rank = kCluster ? (int)cluster.block_rank() : 0;
@@ -191,7 +199,7 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
       cnt = total;
       __syncthreads();
     }
-    find_digit(cnt, (uint32_t)kb, kLinBins, wsum, &s_digit, &s_above);
+    find_digit<kThreads>(cnt, (uint32_t)kb, kLinBins, wsum, &s_digit, &s_above);
     __syncthreads();
     bstar = (int)s_digit;
     need = (uint32_t)kb - s_above;  // 1 <= need <= cnt[bstar]
@@ -221,7 +229,7 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
     if (lane == 0) wcnt[warp][0] = ngt;
     __syncthreads();
     if (warp == 0) {
-      uint32_t x = wcnt[lane][0];
+      uint32_t x = lane < kWarps ? wcnt[lane][0] : 0u;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
       if (lane == 0) s_gtc = x;
@@ -277,14 +285,14 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
     if (warp == 0) {
       uint32_t before = 0u;
       for (int q = 0; q < rank; ++q) before += s_gtq[q] + s_kc[q];
-      const uint32_t mine = wcnt[lane][0] + wcnt[lane][1];
+      const uint32_t mine = lane < kWarps ? wcnt[lane][0] + wcnt[lane][1] : 0u;
       uint32_t x = mine;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const uint32_t t = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += t;
       }
-      wbase[lane][0] = before + x - mine;
+      if (lane < kWarps) wbase[lane][0] = before + x - mine;
     }
     cluster_sync();  // every CTA is done with the others' shared memory
     // ---- pass 3: write the kept indices of this warp's segment in order
@@ -339,7 +347,7 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
         cnt = total;
       }
       __syncthreads();
-      find_digit(cnt, remaining, 1 << width, wsum, &s_digit, &s_above);
+      find_digit<kThreads>(cnt, remaining, 1 << width, wsum, &s_digit, &s_above);
       __syncthreads();
       prefix |= (uint64_t)s_digit << lo_bit;
       remaining -= s_above;
@@ -369,7 +377,7 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
   }
   __syncthreads();
   if (warp == 0) {
-    const uint32_t g = wcnt[lane][0], e = wcnt[lane][1];
+    const uint32_t g = lane < kWarps ? wcnt[lane][0] : 0u, e = lane < kWarps ? wcnt[lane][1] : 0u;
     uint32_t ig = g, ie = e;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -380,8 +388,10 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
         ie += te;
       }
     }
-    wbase[lane][0] = ig - g;
-    wbase[lane][1] = ie - e;
+    if (lane < kWarps) {
+      wbase[lane][0] = ig - g;
+      wbase[lane][1] = ie - e;
+    }
     if (lane == 31) {
       counts[0] = ig;
       counts[1] = ie;
@@ -430,20 +440,11 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
   if (kCluster) cluster.sync();  // no CTA leaves while another may still read its counts
 }
 
-}  // namespace
-
-cudaError_t launch_topk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
+template <bool kCluster, int kThreads>
+cudaError_t launch_tk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
   const size_t smem = sizeof(uint32_t) * (size_t)p.topk_slice;
-  if (p.topk_cluster == 1) {
-    static int done[kMaxDevices] = {};
-    cudaError_t e = ensure_smem(topk_kernel<false>, smem, done);
-    if (e != cudaSuccess) return e;
-    return launch_k(topk_kernel<false>, dim3(p.B * p.U), dim3(kThreads), smem, s, true,
-                    (const float*)a.scores, (const int64_t*)a.seq_off, (const uint32_t*)a.krange, a.idx,
-                    p.U, p.k);
-  }
   static int done[kMaxDevices] = {};
-  cudaError_t e = ensure_smem(topk_kernel<true>, smem, done);
+  cudaError_t e = ensure_smem(topk_kernel<kCluster, kThreads>, smem, done);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(p.B * p.U * p.topk_cluster));
@@ -451,16 +452,26 @@ cudaError_t launch_topk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)p.topk_cluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)p.topk_cluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, topk_kernel<true>, (const float*)a.scores, a.seq_off,
-                            (const uint32_t*)a.krange, a.idx, p.U, p.k);
+  cfg.numAttrs = kCluster ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, topk_kernel<kCluster, kThreads>, (const float*)a.scores,
+                            (const int64_t*)a.seq_off, (const uint32_t*)a.krange, a.idx, p.U, p.k);
+}
+
+}  // namespace
+
+cudaError_t launch_topk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
+  // 1024 threads when the CTAs fit one per SM, else 256 (small units: many
+  // CTAs resident per SM)
+  const bool small = p.topk_threads == 256;
+  if (p.topk_cluster == 1) return small ? launch_tk<false, 256>(p, a, s) : launch_tk<false, 1024>(p, a, s);
+  return small ? launch_tk<true, 256>(p, a, s) : launch_tk<true, 1024>(p, a, s);
 }
 
 }  // namespace salsc
