@@ -99,6 +99,30 @@ struct ScoreTcParams {
   uint32_t* krange;
   uint32_t* flags;
   int B, U, npad, r, n_tiles, stages, tmem_cols;
+  int ng, ncol;  // unit groups, and the 2 * units-per-group query rows of one group
+};
+
+// Walks the work items of a CTA: item w is tile w % n_tiles of unit group
+// w / n_tiles (groups outermost, so the CTAs that read the same tile for
+// different groups run at about the same time and share it through L2).
+struct ItemCursor {
+  TileCursor tc_;
+  int n_tiles, tile, g;
+  __device__ void start(const int64_t* so, int B, int n_tiles_, int w) {
+    n_tiles = n_tiles_;
+    g = w / n_tiles;
+    tile = w % n_tiles;
+    tc_.start(so, B, kTileM, tile);
+  }
+  __device__ void next(const int64_t* so, int B) {
+    if (++tile == n_tiles) {
+      tile = 0;
+      ++g;
+      tc_.start(so, B, kTileM, 0);
+    } else {
+      tc_.next();
+    }
+  }
 };
 
 __global__ void __launch_bounds__(kTcThreads)
@@ -108,7 +132,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int KB = P.r / 64;
   const int S = P.stages;
-  const uint32_t b_kblock_bytes = (uint32_t)P.npad * 128u;
+  const uint32_t b_kblock_bytes = (uint32_t)P.ncol * 128u;
+  const int n_items = P.n_tiles * P.ng;
   uint8_t* a_ring = smem;
   uint8_t* b_buf = a_ring + (size_t)S * kStageBytes;
   uint64_t* bars = (uint64_t*)(b_buf + (size_t)KB * b_kblock_bytes);
@@ -130,8 +155,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
     s_kr[e / P.U][e % P.U][1] = 0u;
   }
   if (threadIdx.x == 0) s_nkr = 0;
-  const int t_begin = (int)((int64_t)blockIdx.x * P.n_tiles / gridDim.x);
-  const int t_end = (int)((int64_t)(blockIdx.x + 1) * P.n_tiles / gridDim.x);
+  const int t_begin = (int)((int64_t)blockIdx.x * n_items / gridDim.x);
+  const int t_end = (int)((int64_t)(blockIdx.x + 1) * n_items / gridDim.x);
   allow_dependent_launch();
 
   if (threadIdx.x == 0) {
@@ -158,14 +183,16 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
     uint32_t it = 0, bpar = 0;
-    int cur_b = -1;
+    int cur_bg = -1;
     bool ok = true;
-    TileCursor cur;
-    cur.start(P.seq_off, P.B, kTileM, t_begin);
-    for (int tile = t_begin; tile < t_end && ok; ++tile, cur.next()) {
+    ItemCursor ic;
+    ic.start(P.seq_off, P.B, P.n_tiles, t_begin);
+    for (int tile = t_begin; tile < t_end && ok; ++tile, ic.next(P.seq_off, P.B)) {
+      const TileCursor& cur = ic.tc_;
       const int b = cur.b;
-      if (b != cur_b) {
-        if (cur_b >= 0) {
+      const int bg = b * P.ng + ic.g;
+      if (bg != cur_bg) {
+        if (cur_bg >= 0) {
           ok = tc::mbar_wait(bempty, bpar, P.flags);
           bpar ^= 1u;
           if (!ok) break;
@@ -184,8 +211,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
         tc::mbar_expect_tx(bfull, (uint32_t)KB * b_kblock_bytes);
         for (int kb = 0; kb < KB; ++kb)
           tc::tma_load_2d(tc::smem_u32(b_buf + (size_t)kb * b_kblock_bytes), &tmap_q, kb * 64,
-                          b * P.npad, bfull);
-        cur_b = b;
+                          b * P.npad + ic.g * P.ncol, bfull);
+        cur_bg = bg;
       }
       const int row0 = (int)(cur.off + cur.t0);
       for (int kb = 0; kb < KB; ++kb, ++it) {
@@ -206,24 +233,25 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
       tc::mbar_wait(full((int)(j % (uint32_t)S)), (j / (uint32_t)S) & 1u, P.flags);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
-    const uint32_t idesc = tc::idesc_bf16_f32(kTileM, P.npad);
+    const uint32_t idesc = tc::idesc_bf16_f32(kTileM, P.ncol);
     uint32_t it = 0, bpar = 0;
-    int cur_b = -1, nseq = 0, i = 0;
+    int cur_bg = -1, nseq = 0, i = 0;
     bool ok = true;
-    TileCursor cur;
-    cur.start(P.seq_off, P.B, kTileM, t_begin);
-    for (int tile = t_begin; tile < t_end && ok; ++tile, ++i, cur.next()) {
-      const int b = cur.b;
-      if (b != cur_b) {
+    ItemCursor ic;
+    ic.start(P.seq_off, P.B, P.n_tiles, t_begin);
+    for (int tile = t_begin; tile < t_end && ok; ++tile, ++i, ic.next(P.seq_off, P.B)) {
+      const TileCursor& cur = ic.tc_;
+      const int bg = cur.b * P.ng + ic.g;
+      if (bg != cur_bg) {
         if (!tc::mbar_wait(bfull, bpar, P.flags)) break;
         bpar ^= 1u;
-        cur_b = b;
+        cur_bg = bg;
         ++nseq;
       }
       const int acc = i & 1;
       if (!tc::mbar_wait(tempty(acc), (((uint32_t)i >> 1) & 1u) ^ 1u, P.flags)) break;
       tc::fence_after_sync();
-      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * P.npad);
+      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * P.ncol);
       for (int kb = 0; kb < KB; ++kb, ++it) {
         const int s = (int)(it % (uint32_t)S);
         const uint32_t ph = (it / (uint32_t)S) & 1u;
@@ -242,7 +270,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
       }
       if (!ok) break;
       tc::mma_commit(tfull(acc));
-      // last tile of this sequence in the CTA's range: the sequence's Qs is then free
+      // last item of this (sequence, group) in the CTA's range: its Qs is then free
       const bool last_of_seq = tile + 1 == t_end || cur.t0 + kTileM >= cur.nb;
       if (last_of_seq) tc::mma_commit(bempty);
     }
@@ -256,9 +284,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
     int i = 0, eb = -1, so = -1;  // sequence and its ordinal in this CTA's range
-    TileCursor cur;
-    cur.start(P.seq_off, P.B, kTileM, t_begin);
-    for (int tile = t_begin; tile < t_end; ++tile, ++i, cur.next()) {
+    ItemCursor ic;
+    ic.start(P.seq_off, P.B, P.n_tiles, t_begin);
+    for (int tile = t_begin; tile < t_end; ++tile, ++i, ic.next(P.seq_off, P.B)) {
+      const TileCursor& cur = ic.tc_;
       if (cur.b != eb) {
         eb = cur.b;
         ++so;
@@ -277,13 +306,14 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
       const int64_t nb = cur.nb;
       const int64_t t = cur.t0 + row;
       float* sbase = P.scores + off * P.U + t;
-      for (int c0 = 0; c0 < 2 * P.U; c0 += 16) {
+      const int u0 = ic.g * (P.ncol / 2);  // first unit of the group
+      for (int c0 = 0; c0 < P.ncol; c0 += 16) {
         uint32_t v[16];
-        tc::tmem_ld16(lane_addr + (uint32_t)(acc * P.npad + c0), v);
+        tc::tmem_ld16(lane_addr + (uint32_t)(acc * P.ncol + c0), v);
         tc::tmem_ld_wait();
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const int u = c0 / 2 + j;
+          const int u = u0 + c0 / 2 + j;
           const float sv = __uint_as_float(v[2 * j]) + __uint_as_float(v[2 * j + 1]);
           const uint32_t key = order_key(sv);
           const uint32_t kmn = __reduce_min_sync(0xffffffffu, t < nb ? key : 0xffffffffu);
@@ -334,11 +364,22 @@ int num_sms() {
 
 cudaError_t launch_score_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
   const int KB = p.r / 64;
-  const size_t b_bytes = (size_t)KB * p.npad * 128;
-  // Small query blocks (GQA): two CTAs per SM with a 4-deep ring each; large
-  // ones (MHA, 64 KiB of Qs) one CTA per SM with an 8-deep ring.
+  // Unit groups: the units' query rows are split into ng groups of ncol rows
+  // (ncol a multiple of 16) when there are too few tiles to give every SM two
+  // work items, or when one group's query block is too large for two CTAs per
+  // SM.  Each group re-reads the latent rows of its tiles (from L2 after the
+  // first group).
+  int ng = 1;
+  auto qbytes = [&](int g) { return (size_t)KB * (2 * p.U / g) * 128; };
+  while ((2 * p.U) % (16 * ng * 2) == 0 &&
+         ((int64_t)p.n_score_tiles * ng < 2 * num_sms() || qbytes(ng) > 45 * 1024))
+    ng *= 2;
+  const int ncol = (2 * p.U) % 16 == 0 ? 2 * p.U / ng : p.npad;
+  const size_t b_bytes = (size_t)KB * ncol * 128;
+  // Small query blocks: two CTAs per SM with a 4-deep ring each; large ones one
+  // CTA per SM with a deeper ring.
   int stages, ctas_per_sm;
-  if (b_bytes <= 16384) {
+  if (b_bytes <= 45 * 1024) {
     stages = 4;
     ctas_per_sm = 2;
   } else {
@@ -350,7 +391,7 @@ cudaError_t launch_score_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream
   const size_t smem = 1024 + (size_t)stages * kStageBytes + b_bytes + (2 * stages + 6) * 8 + 16;
   CUtensorMap tk, tq;
   if (!make_tmap_bf16_2d(&tk, a.Kc, (uint64_t)p.N, (uint64_t)p.r, kTileM, 64) ||
-      !make_tmap_bf16_2d(&tq, a.qsplit, (uint64_t)p.B * p.npad, (uint64_t)p.r, p.npad, 64))
+      !make_tmap_bf16_2d(&tq, a.qsplit, (uint64_t)p.B * p.npad, (uint64_t)p.r, ncol, 64))
     return cudaErrorInvalidValue;
   static int done[kMaxDevices] = {};
   cudaError_t e = ensure_smem(score_tc_kernel, smem, done);
@@ -366,11 +407,14 @@ cudaError_t launch_score_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream
   P.r = p.r;
   P.n_tiles = p.n_score_tiles;
   P.stages = stages;
+  P.ng = ng;
+  P.ncol = ncol;
   int cols = 32;
-  while (cols < 2 * p.npad) cols *= 2;
+  while (cols < 2 * ncol) cols *= 2;
   P.tmem_cols = cols;
   const int max_ctas = num_sms() * ctas_per_sm;
-  const int grid = p.n_score_tiles < max_ctas ? p.n_score_tiles : max_ctas;
+  const int64_t items = (int64_t)p.n_score_tiles * ng;
+  const int grid = items < max_ctas ? (int)items : max_ctas;
   return launch_k(score_tc_kernel, dim3(grid), dim3(kTcThreads), smem, s, true, tk, tq, P);
 }
 
