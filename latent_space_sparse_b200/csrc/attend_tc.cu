@@ -5,17 +5,19 @@
 // SALS technical framework, stages 3-4, with RoPE applied after
 // reconstruction (abstract).  Work unit: a tile of 128 kept tokens of one
 // selection unit (b, u):
-//   1. TMA gather4 brings the 128 latent key rows Kc_b[idx] into shared memory
-//      (128-byte swizzled, K-major);
+//   1. a gather warp copies the 128 latent key rows Kc_b[idx] into shared
+//      memory (cp.async, 16 bytes a lane, into the 128-byte swizzled K-major
+//      layout);
 //   2. tcgen05: K_sel[128 x d] = Kc_tile . Pk_u^T into TMEM (fp32; Pk_u comes
 //      by TMA once per unit and stays in shared memory);
-//   3. the same rows of Vc are gathered (TMA gather4) into the buffer the
-//      MMA has finished with;
-//   4. eight epilogue warps (one thread per token row and half of the RoPE
-//      pairs) read K_sel from TMEM, rotate pair (i, i+d/2) by the angle
+//   3. the same rows of Vc are copied into the buffer the MMA has finished
+//      with;
+//   4. sixteen epilogue warps (one thread per token row and a quarter of the
+//      RoPE pairs) read K_sel from TMEM, rotate pair (i, i+d/2) by the angle
 //      t * base^(-2i/d) and dot it with every rotated query head of the unit;
-//      the tile's softmax (max m, normaliser l) follows, and the weights p are
-//      written to shared memory as bf16 hi + lo parts;
+//      the tile's softmax (max m, normaliser l) follows, one thread per
+//      (head, token), and the weights p are written to shared memory as bf16
+//      hi + lo parts;
 //   5. tcgen05: acc^T[r x 2G] = Vc_tile^T . [p_hi p_lo] into TMEM (Vc_tile read
 //      as an MN-major operand, so the latent value rows need no transpose);
 //   6. the epilogue reads acc[c] = D[c][2g] + D[c][2g+1] and writes the
@@ -27,9 +29,12 @@
 //      so the combine kernel finds the used slots from the tile partition
 //      alone; it merges the few segments of a unit and applies the deferred
 //      Pv_u^T.
-// Warp roles (544 threads): warps 0-7 epilogue, warp 8 TMEM owner and MMA
-// issuer, warps 9-12 and 13-16 row gathers (one group of four per tile
-// buffer; latent key and value rows by TMA gather4).  Each CTA walks a contiguous range of tiles;
+// Warp roles (608 threads): warps 0-15 epilogue, warp 16 TMEM owner and MMA
+// issuer, warps 17 and 18 row gathers (one per tile buffer).  The epilogue is
+// the busiest role (RoPE needs a sine and a cosine per pair and token), so it
+// has four warps per scheduler; 19 warps keep 96 registers per thread (at
+// most five warps share a scheduler's registers).  Each CTA walks a contiguous
+// range of tiles;
 // the two tile buffers alternate (Kc(i) -> Vc(i) -> Kc(i+2)), so the
 // reconstruction of tile i+1 runs during the epilogue of tile i.
 //
@@ -41,13 +46,14 @@
 namespace salsc {
 namespace {
 
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;
 constexpr int kEpiThreads = kEpiWarps * 32;
-constexpr int kMmaWarp = 8;
-constexpr int kLoadWarp0 = 9;  // warps 9-12 fill buffer 0 (even tiles), 13-16 buffer 1
+constexpr int kEpiParts = kEpiWarps / 4;  // threads per token row
+constexpr int kMmaWarp = 16;
+constexpr int kLoadWarp0 = 17;  // warps 17-20 fill buffer 0 (even tiles), 21-24 buffer 1
 constexpr int kGatherWarps = 4;
 constexpr int kGatherThreads = kGatherWarps * 32;
-constexpr int kThreads = (kLoadWarp0 + 2 * kGatherWarps) * 32;  // 544
+constexpr int kThreads = (kLoadWarp0 + 2 * kGatherWarps) * 32;  // 800
 constexpr int kTile = 128;
 constexpr int kPRows = 16;  // rows of the p operand (2G <= 16)
 constexpr uint32_t kEpiBar = 1;
@@ -125,6 +131,31 @@ __device__ __forceinline__ int row_token(const AttendTcParams& P, const UnitTile
   return t;
 }
 
+constexpr int kGatherRows = kTile / kGatherThreads;  // token rows per gather thread
+
+// Gather thread gt's share of one tile's latent rows: items e = gt + 128j
+// over 32 row groups x KB k-blocks; item e copies rows tk[4g .. 4g+3]
+// (g = e % 32), latent columns (kb0 + kb)*64 .. +63 (kb = e / 32), by TMA
+// gather4 into k-block kb of the buffer (128-byte swizzled [128 x 64] blocks,
+// rows 4g .. 4g+3 at byte (g/2)*1024 + (g%2)*512).  A row without a token
+// (-1) copies row `off`, which gets weight 0.
+__device__ __forceinline__ void gather_rows(const int* tk, int64_t off, uint32_t buf_s,
+                                            const CUtensorMap* tmap, int kb0, int KB, int gt,
+                                            uint32_t mbar) {
+  for (int e = gt; e < 32 * KB; e += kGatherThreads) {
+    const int g4 = e & 31, kb = e >> 5;
+    int rows[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int t = tk[4 * g4 + j];
+      rows[j] = (int)(off + (t < 0 ? 0 : t));
+    }
+    tc::tma_gather4(buf_s + (uint32_t)kb * 16384u + (uint32_t)(g4 >> 1) * 1024u +
+                        (uint32_t)(g4 & 1) * 512u,
+                    tmap, (kb0 + kb) * 64, rows[0], rows[1], rows[2], rows[3], mbar);
+  }
+}
+
 // barrier indices
 enum { B_PK = 0, B_KFULL = 1, B_VFULL = 3, B_KDONE = 5, B_PDONE = 7, B_PREADY = 9,
        B_TKFREE = 11, B_TOFREE = 13, B_PKDONE = 15, B_COUNT = 16 };
@@ -140,7 +171,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
                  const __grid_constant__ CUtensorMap tmap_kc,
                  const __grid_constant__ CUtensorMap tmap_vc, const AttendTcParams P) {
   constexpr int HALF = D / 2;
-  constexpr int QPAIRS = HALF / 2;  // RoPE pairs per epilogue thread
+  constexpr int QP = HALF / kEpiParts;                     // RoPE pairs per epilogue thread
+  constexpr int kPasses = (G * kTile + kEpiThreads - 1) / kEpiThreads;  // softmax items per thread
+  constexpr int kSlots = (2 * W * G + 3) / 4;  // (chunk, head) accumulators per epilogue thread
+  static_assert(QP % 8 == 0, "TMEM loads of 8 columns");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int KB = P.r / 64 / W;              // k-blocks of 64 latent columns per buffer
@@ -155,11 +189,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
   uint8_t* const s_pbuf1 = s_pbuf0 + 4096;
   uint64_t* const s_fturn = (uint64_t*)(s_pbuf1 + 4096);    // [D/2] fixed-point turns
   double* const s_theta = (double*)(s_fturn + HALF);         // [D/2]
-  float* const s_qr = (float*)(s_theta + HALF);              // [G][D/2] rotated (q_i, q_i+d/2)
-  float* const s_pd = s_qr + G * D;                          // [2][G][128] half-pair dots
-  float* const s_lg = s_pd + 2 * G * kTile;                  // [G][128] logits -> weights
-  float* const s_stat = s_lg + G * kTile;                    // [2][G][2] tile's (m, l)
-  int* const s_tok = (int*)(s_stat + 4 * G);                 // [2][128] token per row
+  float* const s_qr = (float*)(s_theta + HALF);              // [D/2][G] rotated (q_i, q_i+d/2)
+  float* const s_pd = s_qr + G * D;                          // [parts][G][128] partial dots
+  float* const s_wmax = s_pd + kEpiParts * G * kTile;        // [2][G][4] per-warp maxima
+  float* const s_wsum = s_wmax + 8 * G;                      // [2][G][4] per-warp sums
+  int* const s_tok = (int*)(s_wsum + 8 * G);                 // [2][128] token per row
   float* const s_run = (float*)(s_tok + 2 * kTile);          // [G][2] segment's running (m, l)
   float* const s_ab = s_run + 2 * G;                         // [G][2] rescale factors
   uint64_t* const s_bars = (uint64_t*)(((uintptr_t)(s_ab + 2 * G) + 7) & ~(uintptr_t)7);
@@ -198,57 +232,50 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
 
   if (W == 2 && warp >= kLoadWarp0) {
     // ======================= gather warps, two latent halves =================
-    // Group h (4 warps) fills buffer h with latent half h of every tile: the
-    // key rows, then, once the reconstruction is done, the value rows.
+    // Warp h fills buffer h with latent half h of every tile: the key rows,
+    // then, once the reconstruction is done, the value rows (copy_rows).  Lane
+    // gt looks up the tokens of rows gt + 32j.
     const int h = (warp - kLoadWarp0) / kGatherWarps;
     const int gt = tid - (kLoadWarp0 + h * kGatherWarps) * 32;  // 0..127
     const uint32_t gbar = 2 + h;
     int* tk = s_tok + h * kTile;
     const uint32_t buf_s = tc::smem_u32(h ? s_buf1 : s_buf0);
     const uint32_t tile_bytes = (uint32_t)kTile * KB * 128;
-    const int g4 = gt % 32;
     UnitTileCursor cur;
     cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
     grid_dependency_wait();  // the kept indices come from the previous kernel
-    int t_next = n > 0 ? row_token(P, cur, gt) : -1;
-    int last_v = -1;
+    int t_next[kGatherRows];
+#pragma unroll
+    for (int j = 0; j < kGatherRows; ++j)
+      t_next[j] = n > 0 ? row_token(P, cur, gt + j * kGatherThreads) : -1;
     bool ok = true;
     for (int i = 0; i < n && ok; ++i) {
       const int64_t off = cur.off;
       // the buffer is free once the value MMA of the previous tile is done
       if (i >= 1) ok = tc::mbar_wait(bar(B_PDONE + ((i - 1) & 1)), ((uint32_t)(i - 1) >> 1) & 1u, P.flags);
-      tk[gt] = t_next;
+#pragma unroll
+      for (int j = 0; j < kGatherRows; ++j) tk[gt + j * kGatherThreads] = t_next[j];
       if (gt == 0) tc::mbar_expect_tx(bar(B_KFULL + h), tile_bytes);
       tc::named_sync(gbar, kGatherThreads);
-      int rows[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int t = tk[4 * g4 + j];
-        rows[j] = (int)(off + (t < 0 ? 0 : t));  // no token: weight 0, any valid row
-      }
-      for (int kb = gt / 32; kb < KB; kb += kGatherThreads / 32)
-        tc::tma_gather4(buf_s + kb * 16384u + (uint32_t)(g4 >> 1) * 1024u + (uint32_t)(g4 & 1) * 512u,
-                        &tmap_kc, (h * KB + kb) * 64, rows[0], rows[1], rows[2], rows[3],
-                        bar(B_KFULL + h));
+      gather_rows(tk, off, buf_s, &tmap_kc, h * KB, KB, gt, bar(B_KFULL + h));
       cur.next();
-      t_next = i + 1 < n ? row_token(P, cur, gt) : -1;
+#pragma unroll
+      for (int j = 0; j < kGatherRows; ++j)
+        t_next[j] = i + 1 < n ? row_token(P, cur, gt + j * kGatherThreads) : -1;
       if (!tc::mbar_wait(bar(B_KDONE + (i & 1)), ((uint32_t)i >> 1) & 1u, P.flags)) break;
       if (gt == 0) tc::mbar_expect_tx(bar(B_VFULL + h), tile_bytes);
       tc::named_sync(gbar, kGatherThreads);
-      for (int kb = gt / 32; kb < KB; kb += kGatherThreads / 32)
-        tc::tma_gather4(buf_s + kb * 16384u + (uint32_t)(g4 >> 1) * 1024u + (uint32_t)(g4 & 1) * 512u,
-                        &tmap_vc, (h * KB + kb) * 64, rows[0], rows[1], rows[2], rows[3],
-                        bar(B_VFULL + h));
-      last_v = i;
+      gather_rows(tk, off, buf_s, &tmap_vc, h * KB, KB, gt, bar(B_VFULL + h));
     }
-    if (gt == 0 && last_v >= 0) tc::mbar_wait(bar(B_VFULL + h), (uint32_t)last_v & 1u, P.flags);
   } else if (W == 2 && warp == kMmaWarp) {
-    // ======================= MMA issuer, two latent halves (lane 0) ==========
+    // ======================= MMA issuer, two latent halves ===================
     // Per tile: Pk_u half 0 -> reconstruction over half 0 -> Pk_u half 1 ->
     // reconstruction over half 1 (accumulating) -> value MMA over the four
     // 128-column chunks of the latent width.  Half 0 of the next tile's Pk_u
-    // is loaded while the epilogue works on this tile.
-    if (lane == 0) {
+    // is loaded while the epilogue works on this tile.  The whole warp runs
+    // the sequence (warp-uniform state and descriptors); one elected lane
+    // issues each group of loads, MMAs and its commit.
+    {
       const uint32_t idesc_k = tc::idesc_bf16_f32(kTile, D);
       const uint32_t idesc_v = tc::idesc_bf16_f32_amn(128, kPRows);
       const uint32_t pkb = tc::smem_u32(s_pk);
@@ -256,17 +283,29 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
       uint32_t pk_phase = 0, pkd_phase = 0;
       auto load_pk = [&](int u, int hh) {
-        tc::mbar_expect_tx(bar(B_PK), pk_bytes);
-        for (int kb = 0; kb < KB; ++kb)
-          tc::tma_load_2d(pkb + (uint32_t)kb * D * 128, &tmap_pk, (hh * KB + kb) * 64, u * D, bar(B_PK));
+        if (tc::elect_one()) {
+          tc::mbar_expect_tx(bar(B_PK), pk_bytes);
+          for (int kb = 0; kb < KB; ++kb)
+            tc::tma_load_2d(pkb + (uint32_t)kb * D * 128, &tmap_pk, (hh * KB + kb) * 64, u * D,
+                            bar(B_PK));
+        }
+        __syncwarp();
       };
-      auto kmma = [&](uint32_t a0, uint32_t d_tmem, bool acc0) {
-        for (int kb = 0; kb < KB; ++kb)
+      // reconstruction over one latent half, then a commit to `done`
+      auto kmma = [&](uint32_t a0, uint32_t d_tmem, bool acc0, uint32_t done) {
+        if (tc::elect_one()) {
+          for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc::mma_bf16(d_tmem, tc::sdesc_kmajor_sw128(a0 + kb * 16384 + 32 * k),
-                         tc::sdesc_kmajor_sw128(pkb + kb * D * 128 + 32 * k), idesc_k,
-                         (acc0 || kb || k) ? 1u : 0u);
+            for (int k = 0; k < 4; ++k)
+              tc::mma_bf16(d_tmem, tc::sdesc_kmajor_sw128(a0 + kb * 16384 + 32 * k),
+                           tc::sdesc_kmajor_sw128(pkb + kb * D * 128 + 32 * k), idesc_k,
+                           (acc0 || kb || k) ? 1u : 0u);
+          tc::mma_commit(done);
+        }
+        __syncwarp();
+      };
+      auto wait = [&](uint32_t b, uint32_t parity) {
+        return __all_sync(0xffffffffu, tc::mbar_wait(b, parity, P.flags));
       };
       bool ok = true;
       if (n > 0) load_pk(cur.u, 0);
@@ -274,27 +313,23 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
         const int bi = i & 1;
         const uint32_t ph = ((uint32_t)i >> 1) & 1u;
         const uint32_t d_tmem = tmem_base + (uint32_t)bi * D;
-        ok = tc::mbar_wait(bar(B_PK), pk_phase, P.flags) &&
-             tc::mbar_wait(bar(B_KFULL + 0), (uint32_t)i & 1u, P.flags) &&
-             tc::mbar_wait(bar(B_TKFREE + bi), ph ^ 1u, P.flags);
+        ok = wait(bar(B_PK), pk_phase) && wait(bar(B_KFULL + 0), (uint32_t)i & 1u) &&
+             wait(bar(B_TKFREE + bi), ph ^ 1u);
         if (!ok) break;
         pk_phase ^= 1u;
         tc::fence_after_sync();
-        kmma(tc::smem_u32(s_buf0), d_tmem, false);
-        tc::mma_commit(bar(B_PKDONE));
-        if (!(ok = tc::mbar_wait(bar(B_PKDONE), pkd_phase, P.flags))) break;
+        kmma(tc::smem_u32(s_buf0), d_tmem, false, bar(B_PKDONE));
+        if (!(ok = wait(bar(B_PKDONE), pkd_phase))) break;
         pkd_phase ^= 1u;
         load_pk(cur.u, 1);
-        ok = tc::mbar_wait(bar(B_PK), pk_phase, P.flags) &&
-             tc::mbar_wait(bar(B_KFULL + 1), (uint32_t)i & 1u, P.flags);
+        ok = wait(bar(B_PK), pk_phase) && wait(bar(B_KFULL + 1), (uint32_t)i & 1u);
         if (!ok) break;
         pk_phase ^= 1u;
         tc::fence_after_sync();
-        kmma(tc::smem_u32(s_buf1), d_tmem, true);
-        tc::mma_commit(bar(B_KDONE + bi));
+        kmma(tc::smem_u32(s_buf1), d_tmem, true, bar(B_KDONE + bi));
         if (i + 1 < n) {
           // half 0 of the next tile's Pk_u, once this reconstruction is done with Pk
-          if (!(ok = tc::mbar_wait(bar(B_KDONE + bi), ph, P.flags))) break;
+          if (!(ok = wait(bar(B_KDONE + bi), ph))) break;
           UnitTileCursor nx = cur;
           nx.next();
           load_pk(nx.u, 0);
@@ -302,47 +337,49 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
         // value MMA: acc^T[r x 2G] = Vc_tile^T . p.  The two buffers are adjacent,
         // so latent k-block j of the tile is at s_buf0 + j * 16 KiB and chunk ch
         // (k-blocks 2ch, 2ch+1) may straddle them.
-        ok = tc::mbar_wait(bar(B_PREADY + bi), ph, P.flags) &&
-             tc::mbar_wait(bar(B_VFULL + 0), (uint32_t)i & 1u, P.flags) &&
-             tc::mbar_wait(bar(B_VFULL + 1), (uint32_t)i & 1u, P.flags) &&
-             tc::mbar_wait(bar(B_TOFREE + bi), ph ^ 1u, P.flags);
+        ok = wait(bar(B_PREADY + bi), ph) && wait(bar(B_VFULL + 0), (uint32_t)i & 1u) &&
+             wait(bar(B_VFULL + 1), (uint32_t)i & 1u) && wait(bar(B_TOFREE + bi), ph ^ 1u);
         if (!ok) break;
         tc::fence_after_sync();
         const uint32_t p0 = tc::smem_u32(bi ? s_pbuf1 : s_pbuf0);
-        for (int ch = 0; ch < n_chunks; ++ch) {
-          const uint32_t d_acc = tmem_base + o_col0 + (uint32_t)bi * o_cols + (uint32_t)ch * 16;
-          const uint32_t v0 = tc::smem_u32(s_buf0) + (uint32_t)ch * 2 * 16384;
+        if (tc::elect_one()) {
+          for (int ch = 0; ch < n_chunks; ++ch) {
+            const uint32_t d_acc = tmem_base + o_col0 + (uint32_t)bi * o_cols + (uint32_t)ch * 16;
+            const uint32_t v0 = tc::smem_u32(s_buf0) + (uint32_t)ch * 2 * 16384;
 #pragma unroll
-          for (int ks = 0; ks < kTile / 16; ++ks) {
-            const uint64_t ad = tc::sdesc_mnmajor_sw128(v0 + (uint32_t)(ks * 2) * 1024, 16384, 1024);
-            const uint64_t bd =
-                tc::sdesc_kmajor_sw128(p0 + (uint32_t)(ks >> 2) * 2048 + (uint32_t)(ks & 3) * 32);
-            tc::mma_bf16(d_acc, ad, bd, idesc_v, ks != 0);
+            for (int ks = 0; ks < kTile / 16; ++ks) {
+              const uint64_t ad =
+                  tc::sdesc_mnmajor_sw128(v0 + (uint32_t)(ks * 2) * 1024, 16384, 1024);
+              const uint64_t bd = tc::sdesc_kmajor_sw128(p0 + (uint32_t)(ks >> 2) * 2048 +
+                                                         (uint32_t)(ks & 3) * 32);
+              tc::mma_bf16(d_acc, ad, bd, idesc_v, ks != 0);
+            }
           }
+          tc::mma_commit(bar(B_PDONE + bi));
         }
-        tc::mma_commit(bar(B_PDONE + bi));
+        __syncwarp();
       }
     }
   } else if (warp >= kLoadWarp0) {
     // ======================= gather warps =======================
-    // Group bi (4 warps, 128 threads) fills buffer bi with tiles bi, bi+2, ...:
-    // first the latent key rows Kc_b[idx], then, once the reconstruction is
-    // done with them, the same rows of Vc, both by TMA gather4 (thread t: row
-    // group t % 32, k-block t / 32).  The next tile's token of row t is loaded
-    // while the current tile is in flight.
+    // Warp bi fills buffer bi with tiles bi, bi+2, ...: first the latent key
+    // rows Kc_b[idx], then, once the reconstruction is done with them, the
+    // same rows of Vc (copy_rows).  Lane gt looks up the tokens of rows
+    // gt + 32j; the next tile's are loaded while the current tile is in flight.
     const int bi = (warp - kLoadWarp0) / kGatherWarps;
     const int gt = tid - (kLoadWarp0 + bi * kGatherWarps) * 32;  // 0..127
-    const uint32_t gbar = 2 + bi;                                 // named barrier of the group
+    const uint32_t gbar = 2 + bi;  // named barrier of the group
     int* tk = s_tok + bi * kTile;
     const uint32_t buf_s = tc::smem_u32(bi ? s_buf1 : s_buf0);
     const uint32_t tile_bytes = (uint32_t)kTile * P.r * 2;
-    const int g4 = gt % 32;
     UnitTileCursor cur;
     cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
     if (bi == 1) cur.next();
     grid_dependency_wait();  // the kept indices come from the previous kernel
-    int t_next = bi < n ? row_token(P, cur, gt) : -1;
-    int last_v = -1;  // last tile whose value rows were requested
+    int t_next[kGatherRows];
+#pragma unroll
+    for (int j = 0; j < kGatherRows; ++j)
+      t_next[j] = bi < n ? row_token(P, cur, gt + j * kGatherThreads) : -1;
     bool ok = true;
     for (int i = bi; i < n && ok; i += 2) {
       const uint32_t ph = ((uint32_t)i >> 1) & 1u;
@@ -351,44 +388,35 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       if (i >= 2) {
         ok = tc::mbar_wait(bar(B_PDONE + bi), ph ^ 1u, P.flags);
       }
-      tk[gt] = t_next;
+#pragma unroll
+      for (int j = 0; j < kGatherRows; ++j) tk[gt + j * kGatherThreads] = t_next[j];
       if (gt == 0) tc::mbar_expect_tx(bar(B_KFULL + bi), tile_bytes);
       tc::named_sync(gbar, kGatherThreads);
-      int rows[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int t = tk[4 * g4 + j];
-        rows[j] = (int)(off + (t < 0 ? 0 : t));  // no token: weight 0, any valid row
-      }
-      for (int kb = gt / 32; kb < KB; kb += kGatherThreads / 32)
-        tc::tma_gather4(buf_s + kb * 16384u + (uint32_t)(g4 >> 1) * 1024u + (uint32_t)(g4 & 1) * 512u,
-                        &tmap_kc, kb * 64, rows[0], rows[1], rows[2], rows[3], bar(B_KFULL + bi));
+      gather_rows(tk, off, buf_s, &tmap_kc, 0, KB, gt, bar(B_KFULL + bi));
       // next tile of this group: its tokens arrive during this tile
       cur.next();
       cur.next();
-      t_next = i + 2 < n ? row_token(P, cur, gt) : -1;
+#pragma unroll
+      for (int j = 0; j < kGatherRows; ++j)
+        t_next[j] = i + 2 < n ? row_token(P, cur, gt + j * kGatherThreads) : -1;
       // the reconstruction is done with the key rows: bring the value rows
       if (!tc::mbar_wait(bar(B_KDONE + bi), ph, P.flags)) break;
       if (gt == 0) tc::mbar_expect_tx(bar(B_VFULL + bi), tile_bytes);
       tc::named_sync(gbar, kGatherThreads);
-      for (int kb = gt / 32; kb < KB; kb += kGatherThreads / 32)
-        tc::tma_gather4(buf_s + kb * 16384u + (uint32_t)(g4 >> 1) * 1024u + (uint32_t)(g4 & 1) * 512u,
-                        &tmap_vc, kb * 64, rows[0], rows[1], rows[2], rows[3], bar(B_VFULL + bi));
-      last_v = i;
+      gather_rows(tk, off, buf_s, &tmap_vc, 0, KB, gt, bar(B_VFULL + bi));
     }
-    // this group's copies have all landed before the CTA may exit (a no-op
-    // unless a wait above gave up)
-    if (gt == 0 && last_v >= 0)
-      tc::mbar_wait(bar(B_VFULL + bi), ((uint32_t)last_v >> 1) & 1u, P.flags);
   } else if (warp == kMmaWarp) {
-    // ======================= MMA issuer (lane 0) =======================
+    // ======================= MMA issuer =======================
     // An event loop: the reconstruction of tile nk (after its key rows have
     // landed and its TMEM buffer is free, with Pk_u reloaded at unit
     // boundaries) and the value MMA of tile np (after its weights and value
     // rows are ready) are each issued as soon as their own inputs are, so
     // neither waits behind the other.  At most two reconstructions run ahead
-    // of the value MMAs (two tile buffers, two K_sel buffers in TMEM).
-    if (lane == 0) {
+    // of the value MMAs (two tile buffers, two K_sel buffers in TMEM).  The
+    // whole warp runs the loop, so its state and the descriptors are
+    // warp-uniform; one elected lane issues each group of loads, MMAs and its
+    // commit.
+    {
       const uint32_t idesc_k = tc::idesc_bf16_f32(kTile, D);
       const uint32_t idesc_v = tc::idesc_bf16_f32_amn(128, kPRows);
       UnitTileCursor cur;
@@ -399,21 +427,27 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       int nk = 0, np = 0;
       uint64_t idle_since = 0;
       const uint32_t pkb = tc::smem_u32(s_pk);
+      auto ready = [](uint32_t b, uint32_t parity) {
+        return __all_sync(0xffffffffu, tc::mbar_test_wait(b, parity));
+      };
       while (np < n) {
         bool progress = false;
         if (nk < n && nk <= np + 2) {
           if (pk_step == 0 && (cur.b != cur_b || cur.u != cur_u)) pk_step = 1;
           // Pk_u of a new unit, once the previous reconstruction is done with Pk
           if (pk_step == 1 &&
-              (nk == 0 ||
-               tc::mbar_test_wait(bar(B_KDONE + ((nk - 1) & 1)), ((uint32_t)(nk - 1) >> 1) & 1u))) {
-            tc::mbar_expect_tx(bar(B_PK), pk_bytes);
-            for (int kb = 0; kb < KB; ++kb)
-              tc::tma_load_2d(pkb + (uint32_t)kb * D * 128, &tmap_pk, kb * 64, cur.u * D, bar(B_PK));
+              (nk == 0 || ready(bar(B_KDONE + ((nk - 1) & 1)), ((uint32_t)(nk - 1) >> 1) & 1u))) {
+            if (tc::elect_one()) {
+              tc::mbar_expect_tx(bar(B_PK), pk_bytes);
+              for (int kb = 0; kb < KB; ++kb)
+                tc::tma_load_2d(pkb + (uint32_t)kb * D * 128, &tmap_pk, kb * 64, cur.u * D,
+                                bar(B_PK));
+            }
+            __syncwarp();
             pk_step = 2;
             progress = true;
           }
-          if (pk_step == 2 && tc::mbar_test_wait(bar(B_PK), pk_phase)) {
+          if (pk_step == 2 && ready(bar(B_PK), pk_phase)) {
             pk_phase ^= 1u;
             cur_b = cur.b;
             cur_u = cur.u;
@@ -421,55 +455,61 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
             progress = true;
           }
           const int bk = nk & 1;
-          if (pk_step == 0 && tc::mbar_test_wait(bar(B_KFULL + bk), ((uint32_t)nk >> 1) & 1u) &&
-              tc::mbar_test_wait(bar(B_TKFREE + bk), (((uint32_t)nk >> 1) & 1u) ^ 1u)) {
+          if (pk_step == 0 && ready(bar(B_KFULL + bk), ((uint32_t)nk >> 1) & 1u) &&
+              ready(bar(B_TKFREE + bk), (((uint32_t)nk >> 1) & 1u) ^ 1u)) {
             tc::fence_after_sync();
             const uint32_t kb0 = tc::smem_u32(bk ? s_buf1 : s_buf0);
             const uint32_t d_tmem = tmem_base + (uint32_t)bk * D;
-            for (int kb = 0; kb < KB; ++kb)
+            if (tc::elect_one()) {
+              for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
-              for (int k = 0; k < 4; ++k)
-                tc::mma_bf16(d_tmem, tc::sdesc_kmajor_sw128(kb0 + kb * 16384 + 32 * k),
-                             tc::sdesc_kmajor_sw128(pkb + kb * D * 128 + 32 * k), idesc_k,
-                             (kb | k) != 0);
-            tc::mma_commit(bar(B_KDONE + bk));
+                for (int k = 0; k < 4; ++k)
+                  tc::mma_bf16(d_tmem, tc::sdesc_kmajor_sw128(kb0 + kb * 16384 + 32 * k),
+                               tc::sdesc_kmajor_sw128(pkb + kb * D * 128 + 32 * k), idesc_k,
+                               (kb | k) != 0);
+              tc::mma_commit(bar(B_KDONE + bk));
+            }
+            __syncwarp();
             ++nk;
             cur.next();
             progress = true;
           }
         }
         const int bp = np & 1;
-        if (np < nk && tc::mbar_test_wait(bar(B_PREADY + bp), ((uint32_t)np >> 1) & 1u) &&
-            tc::mbar_test_wait(bar(B_VFULL + bp), ((uint32_t)np >> 1) & 1u) &&
-            tc::mbar_test_wait(bar(B_TOFREE + bp), (((uint32_t)np >> 1) & 1u) ^ 1u)) {
+        if (np < nk && ready(bar(B_PREADY + bp), ((uint32_t)np >> 1) & 1u) &&
+            ready(bar(B_VFULL + bp), ((uint32_t)np >> 1) & 1u) &&
+            ready(bar(B_TOFREE + bp), (((uint32_t)np >> 1) & 1u) ^ 1u)) {
           tc::fence_after_sync();
           const uint32_t p0 = tc::smem_u32(bp ? s_pbuf1 : s_pbuf0);
           const uint32_t vb0 = tc::smem_u32(bp ? s_buf1 : s_buf0);
-          for (int ch = 0; ch < n_chunks; ++ch) {
-            const uint32_t d_tmem = tmem_base + o_col0 + (uint32_t)bp * o_cols + (uint32_t)ch * 16;
+          if (tc::elect_one()) {
+            for (int ch = 0; ch < n_chunks; ++ch) {
+              const uint32_t d_tmem = tmem_base + o_col0 + (uint32_t)bp * o_cols + (uint32_t)ch * 16;
 #pragma unroll
-            for (int ks = 0; ks < kTile / 16; ++ks) {
-              // A = Vc_tile^T: latent columns ch*128.. (MN), tokens ks*16.. (K)
-              const uint64_t ad = tc::sdesc_mnmajor_sw128(
-                  vb0 + (uint32_t)ch * 2 * 16384 + (uint32_t)(ks * 2) * 1024, 16384, 1024);
-              // B = p rows (hi/lo per head), tokens ks*16..: K-major k-block ks/4
-              const uint64_t bd =
-                  tc::sdesc_kmajor_sw128(p0 + (uint32_t)(ks >> 2) * 2048 + (uint32_t)(ks & 3) * 32);
-              tc::mma_bf16(d_tmem, ad, bd, idesc_v, ks != 0);
+              for (int ks = 0; ks < kTile / 16; ++ks) {
+                // A = Vc_tile^T: latent columns ch*128.. (MN), tokens ks*16.. (K)
+                const uint64_t ad = tc::sdesc_mnmajor_sw128(
+                    vb0 + (uint32_t)ch * 2 * 16384 + (uint32_t)(ks * 2) * 1024, 16384, 1024);
+                // B = p rows (hi/lo per head), tokens ks*16..: K-major k-block ks/4
+                const uint64_t bd = tc::sdesc_kmajor_sw128(p0 + (uint32_t)(ks >> 2) * 2048 +
+                                                           (uint32_t)(ks & 3) * 32);
+                tc::mma_bf16(d_tmem, ad, bd, idesc_v, ks != 0);
+              }
             }
+            tc::mma_commit(bar(B_PDONE + bp));
           }
-          tc::mma_commit(bar(B_PDONE + bp));
+          __syncwarp();
           ++np;
           progress = true;
         }
         if (progress) {
           idle_since = 0;
         } else {
-          const uint64_t now = tc::globaltimer_ns();
+          const uint64_t now = __shfl_sync(0xffffffffu, tc::globaltimer_ns(), 0);
           if (idle_since == 0) {
             idle_since = now;
           } else if (now - idle_since > tc::kWaitLimitNs) {
-            atomicOr(P.flags, FLAG_WAIT_TIMEOUT);
+            if (lane == 0) atomicOr(P.flags, FLAG_WAIT_TIMEOUT);
             break;
           }
           __nanosleep(32);
@@ -477,19 +517,22 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       }
     }
   } else {
-    // ======================= epilogue (warps 0-7) =======================
-    const int quarter = warp & 3, half = warp >> 2;
+    // ======================= epilogue (warps 0-15) =======================
+    // Warp w reads TMEM lanes 32*(w%4).. (its token rows) and takes the RoPE
+    // pairs [part*QP, (part+1)*QP) of them, part = w/4; the parts' partial
+    // logits meet in shared memory, where thread e takes head e/128 and token
+    // e%128 for the tile's softmax.
+    const int quarter = warp & 3, part = warp >> 2;
     const int m = quarter * 32 + lane;  // token row = TMEM lane
     UnitTileCursor cur;
     cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
     int cur_b = -1, cur_u = -1;
-    // this thread's latent columns c = ch*128 + quarter*32 + lane, chunks
-    // ch = half, half + 2: the segment's running sum
-    float acc_run[W][G];
+    // the segment's running sums: slot s = part + 4j (j < kSlots) holds latent
+    // column (s / G)*128 + quarter*32 + lane of head s % G
+    const int n_used = n_chunks * G;
+    float acc_run[kSlots];
 #pragma unroll
-    for (int w = 0; w < W; ++w)
-#pragma unroll
-      for (int g = 0; g < G; ++g) acc_run[w][g] = 0.f;
+    for (int j = 0; j < kSlots; ++j) acc_run[j] = 0.f;
     int seg_tiles = 0;
     if (tid < G) {
       s_run[2 * tid] = -INFINITY;
@@ -503,9 +546,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     auto fold = [&](int j) {
       const int bj = j & 1;
       const uint32_t phj = ((uint32_t)j >> 1) & 1u;
+      // the tile's (m, l) per head from the per-warp maxima and sums, and the
       // heads' scale factors
       if (tid < G) {
-        const float mt = s_stat[bj * 2 * G + 2 * tid], lt = s_stat[bj * 2 * G + 2 * tid + 1];
+        const float* wm = s_wmax + (bj * G + tid) * 4;
+        const float* ws = s_wsum + (bj * G + tid) * 4;
+        const float mt = fmaxf(fmaxf(wm[0], wm[1]), fmaxf(wm[2], wm[3]));
+        const float lt = (ws[0] + ws[1]) + (ws[2] + ws[3]);
         const float mr = s_run[2 * tid], lr = s_run[2 * tid + 1];
         const float mx = fmaxf(mr, mt);
         float al = 0.f, be = 0.f;
@@ -518,29 +565,29 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
         s_run[2 * tid] = mx;
         s_run[2 * tid + 1] = lr * al + lt * be;
       }
-      // the tile's acc from TMEM: warp (quarter, half) holds latent column
-      // c = half*128 + quarter*32 + lane
+      // the tile's acc from TMEM: columns (hi, lo) of head g in chunk c
       const bool ok2 = __all_sync(0xffffffffu, tc::mbar_wait(bar(B_PDONE + bj), phj, P.flags));
       tc::fence_after_sync();
-      uint32_t v[W][16];
+      uint32_t v[kSlots][2];
 #pragma unroll
-      for (int w = 0; w < W; ++w)
-        if (ok2 && half + 2 * w < n_chunks)
-          tc::tmem_ld16(tmem_base + ((uint32_t)(quarter * 32) << 16) + o_col0 +
-                            (uint32_t)bj * o_cols + (uint32_t)(half + 2 * w) * 16,
-                        v[w]);
+      for (int jj = 0; jj < kSlots; ++jj) {
+        const int sl = part + 4 * jj;
+        if (ok2 && sl < n_used)
+          tc::tmem_ld2(tmem_base + ((uint32_t)(quarter * 32) << 16) + o_col0 + (uint32_t)bj * o_cols +
+                           (uint32_t)(sl / G) * 16 + 2u * (uint32_t)(sl % G),
+                       v[jj]);
+      }
       tc::tmem_ld_wait();
       tc::fence_before_sync();
       tc::named_sync(kEpiBar, kEpiThreads);
       if (tid == 0) tc::mbar_arrive(bar(B_TOFREE + bj));
 #pragma unroll
-      for (int w = 0; w < W; ++w) {
-        if (ok2 && half + 2 * w < n_chunks) {
-#pragma unroll
-          for (int g = 0; g < G; ++g)
-            acc_run[w][g] = acc_run[w][g] * s_ab[2 * g] +
-                            (__uint_as_float(v[w][2 * g]) + __uint_as_float(v[w][2 * g + 1])) *
-                                s_ab[2 * g + 1];
+      for (int jj = 0; jj < kSlots; ++jj) {
+        const int sl = part + 4 * jj;
+        if (ok2 && sl < n_used) {
+          const int g = sl % G;
+          acc_run[jj] = acc_run[jj] * s_ab[2 * g] +
+                        (__uint_as_float(v[jj][0]) + __uint_as_float(v[jj][1])) * s_ab[2 * g + 1];
         }
       }
       // end of this CTA's segment of the unit: publish it
@@ -552,38 +599,32 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
         const int s0 = fc.slot + 1 - seg_tiles;  // first slot of the segment
         const int64_t row0 = ((int64_t)fc.b * P.Hq + fc.u * G) * P.n_slots + s0;
 #pragma unroll
-        for (int w = 0; w < W; ++w) {
-          const int c = (half + 2 * w) * 128 + quarter * 32 + lane;
-          if (half + 2 * w < n_chunks && c < P.r) {
-#pragma unroll
-            for (int g = 0; g < G; ++g)
-              P.part[(row0 + (int64_t)g * P.n_slots) * part_row(P.r) + kPartAcc + c] = acc_run[w][g];
-          }
+        for (int jj = 0; jj < kSlots; ++jj) {
+          const int sl = part + 4 * jj;
+          const int c = (sl / G) * 128 + quarter * 32 + lane;
+          if (sl < n_used && c < P.r)
+            P.part[(row0 + (int64_t)(sl % G) * P.n_slots) * part_row(P.r) + kPartAcc + c] =
+                acc_run[jj];
+          acc_run[jj] = 0.f;
         }
         if (tid < G) {
           float* pp = P.part + (row0 + (int64_t)tid * P.n_slots) * part_row(P.r);
           pp[0] = s_run[2 * tid];
           pp[1] = s_run[2 * tid + 1];
-        }
-        // a new segment starts with the next tile
-        seg_tiles = 0;
-#pragma unroll
-        for (int w = 0; w < W; ++w)
-#pragma unroll
-          for (int g = 0; g < G; ++g) acc_run[w][g] = 0.f;
-        if (tid < G) {
           s_run[2 * tid] = -INFINITY;
           s_run[2 * tid + 1] = 0.f;
         }
+        // a new segment starts with the next tile
+        seg_tiles = 0;
       }
-      tc::named_sync(kEpiBar, kEpiThreads);
       fc = nx;
     };
     for (int i = 0; i < n; ++i, cur.next()) {
       const int bi = i & 1;
       const uint32_t ph = ((uint32_t)i >> 1) & 1u;
       if (cur.b != cur_b || cur.u != cur_u) {
-        // rotated queries of the unit's heads (angles reduced in fp64)
+        // rotated queries of the unit's heads (angles reduced in fp64), as
+        // pairs (q_i, q_i+d/2) in the order [pair][head]
         const double qpos = P.q_pos ? (double)P.q_pos[cur.b] : (double)cur.nb;
         for (int e = tid; e < G * HALF; e += kEpiThreads) {
           const int g = e / HALF, ii = e % HALF;
@@ -593,13 +634,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
           float s, c;
           sincosf((float)fma(-nt, kTwoPi, a), &s, &c);
           const float x0 = __bfloat162float(qh[ii]), x1 = __bfloat162float(qh[ii + HALF]);
-          *(float2*)(s_qr + g * D + 2 * ii) = make_float2(x0 * c - x1 * s, x1 * c + x0 * s);
+          *(float2*)(s_qr + 2 * (ii * G + g)) = make_float2(x0 * c - x1 * s, x1 * c + x0 * s);
         }
         cur_b = cur.b;
         cur_u = cur.u;
         tc::named_sync(kEpiBar, kEpiThreads);
       }
-      // ---- K_sel row m, pairs [half*QPAIRS, (half+1)*QPAIRS)
+      // ---- K_sel row m, pairs [part*QP, (part+1)*QP)
       const bool ok =
           __all_sync(0xffffffffu, tc::mbar_wait(bar(B_KDONE + bi), ph, P.flags));
       tc::fence_after_sync();
@@ -612,17 +653,17 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       for (int g = 0; g < G; ++g) dot[g] = 0.f;
       if (ok) {
         const uint32_t row_addr =
-            tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)bi * D;
+            tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)bi * D + (uint32_t)(part * QP);
         const uint32_t tu = (uint32_t)(t < 0 ? 0 : t);
 #pragma unroll 1
-        for (int i0 = half * QPAIRS; i0 < (half + 1) * QPAIRS; i0 += 8) {
+        for (int c8 = 0; c8 < QP; c8 += 8) {
           uint32_t v0[8], v1[8];
-          tc::tmem_ld8(row_addr + i0, v0);
-          tc::tmem_ld8(row_addr + HALF + i0, v1);
+          tc::tmem_ld8(row_addr + c8, v0);
+          tc::tmem_ld8(row_addr + HALF + c8, v1);
           tc::tmem_ld_wait();
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj) {
-            const int ii = i0 + jj;
+            const int ii = part * QP + c8 + jj;
             const uint64_t F = s_fturn[ii];
             const uint32_t turn = __umulhi(tu, (uint32_t)F) + tu * (uint32_t)(F >> 32);
             float s, c;
@@ -630,66 +671,72 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
             const float x0 = __uint_as_float(v0[jj]), x1 = __uint_as_float(v1[jj]);
             const float k0 = x0 * c - x1 * s;
             const float k1 = x1 * c + x0 * s;
+            const float* qp = s_qr + 2 * ii * G;
+            if constexpr (G % 2 == 0) {
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-              const float2 qv = *(const float2*)(s_qr + g * D + 2 * ii);
-              dot[g] = fmaf(qv.x, k0, fmaf(qv.y, k1, dot[g]));
+              for (int g = 0; g < G; g += 2) {
+                const float4 qv = *(const float4*)(qp + 2 * g);
+                dot[g] = fmaf(qv.x, k0, fmaf(qv.y, k1, dot[g]));
+                dot[g + 1] = fmaf(qv.z, k0, fmaf(qv.w, k1, dot[g + 1]));
+              }
+            } else {
+              const float2 qv = *(const float2*)qp;
+              dot[0] = fmaf(qv.x, k0, fmaf(qv.y, k1, dot[0]));
             }
           }
         }
       }
+      // a row without a token gets logit -inf through part 0's partial dot
 #pragma unroll
-      for (int g = 0; g < G; ++g) s_pd[(half * G + g) * kTile + m] = dot[g];
+      for (int g = 0; g < G; ++g)
+        s_pd[(part * G + g) * kTile + m] = (part == 0 && t < 0) ? -INFINITY : dot[g];
       tc::fence_before_sync();
       tc::named_sync(kEpiBar, kEpiThreads);
       if (tid == 0) tc::mbar_arrive(bar(B_TKFREE + bi));  // K_sel[bi] may be overwritten
-      if (tid < kTile) {  // half 0: m == tid
+      // ---- logits and the tile's softmax: thread e takes head e / 128 and
+      // token e % 128, so warp w covers 32 tokens of one head
+      float lg[kPasses];
 #pragma unroll
-        for (int g = 0; g < G; ++g)
-          s_lg[g * kTile + tid] =
-              t >= 0 ? (s_pd[g * kTile + tid] + s_pd[(G + g) * kTile + tid]) * P.scale : -INFINITY;
-      }
-      tc::named_sync(kEpiBar, kEpiThreads);
-      // ---- softmax inside the tile: warp w takes head w
-      if (warp < G) {
-        const int g = warp;
-        float v[4], mx = -INFINITY;
+      for (int ps = 0; ps < kPasses; ++ps) {
+        const int e = tid + ps * kEpiThreads;
+        const int g = e >> 7, mm = e & (kTile - 1);
+        float l = -INFINITY;
+        if (e < G * kTile) {
+          float sum = 0.f;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          v[q] = s_lg[g * kTile + lane + 32 * q];
-          mx = fmaxf(mx, v[q]);
+          for (int pt = 0; pt < kEpiParts; ++pt) sum += s_pd[(pt * G + g) * kTile + mm];
+          l = sum * P.scale;
         }
+        lg[ps] = l;
+        float mx = l;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        float sum = 0.f;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float p = v[q] == -INFINITY ? 0.f : expf(v[q] - mx);
-          s_lg[g * kTile + lane + 32 * q] = p;
-          sum += p;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if (lane == 0) {
-          s_stat[bi * 2 * G + 2 * g] = mx;
-          s_stat[bi * 2 * G + 2 * g + 1] = sum;
-        }
+        if (lane == 0 && e < G * kTile) s_wmax[(bi * G + g) * 4 + (mm >> 5)] = mx;
       }
       tc::named_sync(kEpiBar, kEpiThreads);
-      // ---- p as bf16 hi/lo rows 2g, 2g+1 of the value MMA's B operand
-      if (tid < kTile) {
-        const int mm = tid;
-        uint8_t* pb = (bi ? s_pbuf1 : s_pbuf0) + (mm >> 6) * 2048;
-        const int col = mm & 63, chunk = col >> 3, within = col & 7;
+      // ---- weights p = exp(l - m) as bf16 hi/lo rows 2g, 2g+1 of the value
+      // MMA's B operand (K-major, 128-byte swizzle)
+      uint8_t* const pb = bi ? s_pbuf1 : s_pbuf0;
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float p = s_lg[g * kTile + mm];
+      for (int ps = 0; ps < kPasses; ++ps) {
+        const int e = tid + ps * kEpiThreads;
+        const int g = e >> 7, mm = e & (kTile - 1);
+        if (e < G * kTile) {
+          const float* wm = s_wmax + (bi * G + g) * 4;
+          const float mt = fmaxf(fmaxf(wm[0], wm[1]), fmaxf(wm[2], wm[3]));
+          const float p = lg[ps] == -INFINITY ? 0.f : expf(lg[ps] - mt);
+          float sum = p;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+          if (lane == 0) s_wsum[(bi * G + g) * 4 + (mm >> 5)] = sum;
           const __nv_bfloat16 hi = __float2bfloat16_rn(p);
           const __nv_bfloat16 lo = __float2bfloat16_rn(p - __bfloat162float(hi));
+          uint8_t* const pk = pb + (mm >> 6) * 2048;
+          const int col = mm & 63, chunk = col >> 3, within = col & 7;
           const int r0 = 2 * g, r1 = 2 * g + 1;
-          *(__nv_bfloat16*)(pb + (r0 >> 3) * 1024 + (r0 & 7) * 128 + ((chunk ^ (r0 & 7)) << 4) +
+          *(__nv_bfloat16*)(pk + (r0 >> 3) * 1024 + (r0 & 7) * 128 + ((chunk ^ (r0 & 7)) << 4) +
                             within * 2) = hi;
-          *(__nv_bfloat16*)(pb + (r1 >> 3) * 1024 + (r1 & 7) * 128 + ((chunk ^ (r1 & 7)) << 4) +
+          *(__nv_bfloat16*)(pk + (r1 >> 3) * 1024 + (r1 & 7) * 128 + ((chunk ^ (r1 & 7)) << 4) +
                             within * 2) = lo;
         }
       }
@@ -698,7 +745,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       if (tid == 0) tc::mbar_arrive(bar(B_PREADY + bi));
       if (i > 0) fold(i - 1);
     }
-    if (n > 0) fold(n - 1);
+    if (n > 0) {
+      // the previous fold's readers of the scale factors are done
+      tc::named_sync(kEpiBar, kEpiThreads);
+      fold(n - 1);
+    }
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -725,7 +776,7 @@ template <int G, int D, int W>
 size_t smem_bytes(int r) {
   const int KB = r / 64 / W;
   return 1024 + (size_t)KB * D * 128 + 2 * (size_t)KB * 16384 + 2 * 4096 + 8 * (D / 2) * 2 +
-         4 * (G * D + 2 * G * kTile + G * kTile + 4 * G + 2 * kTile + 4 * G) + 8 +
+         4 * (G * D + kEpiParts * G * kTile + 16 * G + 2 * kTile + 4 * G) + 8 +
          8 * B_COUNT + 16;
 }
 
