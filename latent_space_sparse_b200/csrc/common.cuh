@@ -7,7 +7,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
 #include <utility>
+#include <vector>
 
 #include "salsc.h"
 
@@ -109,6 +111,25 @@ cudaError_t ensure_smem(K* kernel, size_t bytes, int (&done)[kMaxDevices]) {
   return e;
 }
 
+// Every decode kernel asks for the largest shared-memory carveout, so that an
+// SM still running one kernel's CTAs can take the next kernel's CTAs (launched
+// early by programmatic dependent launch) without first draining to change its
+// L1 / shared-memory split.  Set once per kernel and device.
+inline cudaError_t prefer_max_shared(const void* fn) {
+  static std::mutex mu;
+  static std::vector<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto& d : done)
+    if (d.first == fn && d.second == dev) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess) done.emplace_back(fn, dev);
+  return e;
+}
+
 // Launch `kernel` on `s`; with `pdl` the launch may begin while the previous
 // kernel on the stream is still running (programmatic dependent launch): the
 // kernel must execute grid_dependency_wait() before it reads anything the
@@ -116,6 +137,8 @@ cudaError_t ensure_smem(K* kernel, size_t bytes, int (&done)[kMaxDevices]) {
 template <typename... KArgs, typename... Args>
 cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                      bool pdl, Args&&... args) {
+  const cudaError_t e = prefer_max_shared((const void*)kernel);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;

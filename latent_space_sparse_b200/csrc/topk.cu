@@ -9,22 +9,25 @@
 // loads a contiguous slice of the unit's scores into shared memory once, as
 // 32-bit keys whose unsigned order is the float order; the unit's score range
 // [min, max] comes from the scoring kernel.  Each CTA histograms its slice
-// into 512 bins of equal width over that range (the bin is a monotone
+// into 2048 bins of equal width over that range (the bin is a monotone
 // function of the score, and scores spread over many bins, so the
-// shared-memory atomics barely contend); the C histograms are summed through
-// distributed shared memory and every CTA finds, with a block-wide scan, the
-// bin that holds the k_b-th largest score.  A second pass counts, per warp
-// segment, the keys above that bin and lists the (key, index) pairs inside
-// it, which are few for any smooth score distribution: the lists of the
-// cluster are merged, and the pair whose rank (score descending, index
-// ascending) is the number still needed is the exact threshold.  The counts
-// and the kept candidates give every warp its output offset, and a third pass
-// writes the kept indices of each warp's segment in index order, so the
-// result is deterministic.  When the boundary bin holds more than kCand pairs
-// (heavily repeated or extreme scores), a radix select on rel = key - kmin
-// with 11-bit digits, starting at the top bit of the key range (at most three
-// passes), finds the threshold instead, followed by a counting and a writing
-// pass.  No full sort, no global-memory scratch.
+// shared-memory atomics barely contend) and adds it into every CTA's copy of
+// the cluster histogram through distributed shared memory; every CTA then
+// finds, with a block-wide scan, the bin that holds the k_b-th largest score.
+// A second pass packs, per warp segment, the indices of the keys above that
+// bin (all kept) and stores the (key, index) pairs inside it, which are few
+// for any smooth score distribution, into every CTA's candidate list; each
+// CTA ranks its own pairs (score descending, index ascending) against the
+// whole list, and the pairs ranked below the number still needed are kept.
+// The output holds the indices above the boundary bin first (in index order)
+// and then the kept pairs in rank order, so the result is deterministic.
+// Data crosses between the CTAs only as stores into the others' shared memory
+// before a cluster barrier (no remote load waits for a reply).  When the
+// boundary bin holds more pairs than one rank's part of the list (heavily
+// repeated or extreme scores), a radix select on rel = key - kmin with 11-bit
+// digits, starting at the top bit of the key range (at most three passes),
+// finds the threshold instead, followed by a counting and a writing pass.  No
+// full sort, no global-memory scratch.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -34,8 +37,34 @@ namespace cg = cooperative_groups;
 namespace salsc {
 namespace {
 
-constexpr int kBatch = 32;  // keys a thread loads before converting them
+constexpr int kBatch = 8;  // keys a thread loads before converting them (the loop is unrolled: short code)
 constexpr int kMaxCluster = 8;  // largest cluster of CTAs per unit
+
+// Shared-memory address of `p` in cluster CTA `rank`, for the stores below.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(r)
+               : "r"((uint32_t)__cvta_generic_to_shared(p)), "r"(rank));
+  return r;
+}
+// Store and atomic add into the shared memory of another CTA of the cluster:
+// no reply is awaited, and the next cluster barrier makes them visible.
+__device__ __forceinline__ void st_cluster(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_add_cluster(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Split cluster barrier: arrive (releasing this thread's shared-memory reads
+// and writes) and, later, wait for every thread of the cluster to arrive.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 
 // Float whose order_key is `key` (-0 comes back as +0).
 __device__ __forceinline__ float key_float(uint32_t key) {
@@ -44,7 +73,7 @@ __device__ __forceinline__ float key_float(uint32_t key) {
 
 constexpr int kBins = 2048;  // 11-bit digits of the radix fallback
 constexpr int kDigit = 11;
-constexpr int kLinBins = 512;  // bins of the linear pass
+constexpr int kLinBins = 2048;  // bins of the linear pass
 constexpr int kCand = 1024;    // most candidates the boundary bin may hold for the fast path
 
 // Bin of a key in the linear partition of [fmin, fmax] into kLinBins bins: a
@@ -55,13 +84,15 @@ __device__ __forceinline__ int linear_bin(uint32_t key, float fmin, float scale)
   return min(kLinBins - 1, (int)x);
 }
 
-// Block-wide search for the digit that holds the target rank: `cnt` holds the
-// histogram (ascending bins); bins are scanned from the top.  Thread t looks
-// at the `per` bins nbins-1-t*per .. nbins-(t+1)*per (per = nbins / THREADS,
-// at least 1).  Returns through s_digit / s_above.
-template <int THREADS>
-__device__ __forceinline__ void find_digit(const uint32_t* cnt, uint32_t target, int nbins,
-                                           uint32_t* wsum, uint32_t* s_digit, uint32_t* s_above) {
+// Block-wide search for the digit that holds the target rank: cnt(i) is the
+// count of bin i (ascending bins); bins are scanned from the top.  Thread t
+// looks at the `per` bins nbins-1-t*per .. nbins-(t+1)*per (per = nbins /
+// THREADS, at least 1).  Returns through s_digit / s_above / s_count (the
+// digit's own count).
+template <int THREADS, typename Cnt>
+__device__ __forceinline__ void find_digit(Cnt cnt, uint32_t target, int nbins, uint32_t* wsum,
+                                           uint32_t* s_digit, uint32_t* s_above,
+                                           uint32_t* s_count) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int per = nbins / THREADS > 1 ? nbins / THREADS : 1;  // nbins / THREADS <= 8
   const int top = nbins - 1 - tid * per;
@@ -69,7 +100,7 @@ __device__ __forceinline__ void find_digit(const uint32_t* cnt, uint32_t target,
   uint32_t mine = 0u;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    c[j] = (j < per && top - j >= 0) ? cnt[top - j] : 0u;
+    c[j] = (j < per && top - j >= 0) ? cnt(top - j) : 0u;
     mine += c[j];
   }
   uint32_t incl = mine;
@@ -97,6 +128,7 @@ __device__ __forceinline__ void find_digit(const uint32_t* cnt, uint32_t target,
     if (j < per && above < target && target <= above + c[j]) {
       *s_digit = (uint32_t)(top - j);
       *s_above = above;
+      *s_count = c[j];
     }
     above += c[j];
   }
@@ -114,15 +146,14 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
   const int b = unit / U, u = unit % U;
 
   extern __shared__ uint32_t keys[];
-  __shared__ uint32_t hist[2][kBins];  // [0]: histogram, [1]: candidate list (both read by the cluster)
-  __shared__ uint32_t total[kBins];    // cluster histogram, then the merged candidate list
+  __shared__ uint32_t hist[2][kBins];  // [0]: this CTA's histogram, [1]: the cluster's candidates
+  __shared__ uint32_t total[kBins];    // the cluster histogram
   __shared__ uint32_t wsum[64];
   __shared__ uint32_t counts[2];       // fallback: this CTA's (#keys > T, #keys == T)
   __shared__ uint32_t wcnt[kWarps][2];
   __shared__ uint32_t wbase[kWarps][2];
-  __shared__ uint32_t s_kc[kMaxCluster], s_gtq[kMaxCluster], s_nq[kMaxCluster];
-  __shared__ uint32_t s_cbase[kMaxCluster + 1];
-  __shared__ uint32_t s_digit, s_above, s_base_gt, s_base_eq, s_ncand, s_gtc, s_T, s_Tidx;
+  __shared__ uint32_t s_nq[kMaxCluster], s_gq[kMaxCluster];  // per rank: candidates, keys above
+  __shared__ uint32_t s_digit, s_above, s_count, s_base_gt, s_base_eq, s_ncand, s_ngt;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // shared memory of cluster rank q (this CTA's own when not a cluster)
@@ -132,9 +163,10 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
   auto cluster_sync = [&]() {
     if (kCluster) cluster.sync(); else __syncthreads();
   };
-  for (int i = tid; i < kLinBins; i += kThreads) hist[0][i] = 0u;
-  if (tid < kWarps) wcnt[tid][1] = 0u;  // kept candidates per warp segment
-  if (tid < kMaxCluster) s_kc[tid] = 0u;
+  for (int i = tid; i < kLinBins; i += kThreads) {
+    hist[0][i] = 0u;
+    total[i] = 0u;
+  }
   if (tid == 0) s_ncand = 0u;
   allow_dependent_launch();
   const int64_t off = seq_off[b];
@@ -147,6 +179,9 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
   const int s0 = warp * seg, s1 = min(s0 + seg, n_loc);
   const uint32_t lt_mask = (1u << lane) - 1u;
   int32_t* out = idx_out + ((int64_t)b * U + u) * k;
+  // From here on the other CTAs of the cluster may add into this CTA's zeroed
+  // cluster histogram (they wait for this arrival before they do).
+  if (kCluster && kb != nb) cluster_arrive();
   grid_dependency_wait();  // the scores and their range come from the previous kernel
   if (kb == nb) {
     // keep every token, in index order
@@ -182,35 +217,40 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
       }
     }
   }
+  if (kCluster) cluster_wait();  // every CTA's cluster histogram is zeroed
   bool fast = lin;
   int bstar = 0;
   uint32_t need = 0u, n_cand = 0u;
   if (fast) {
-    cluster_sync();
-    const uint32_t* cnt = hist[0];
-    if (kCluster) {
-      for (int i = tid; i < kLinBins; i += kThreads) {
-        uint32_t t = 0u;
-#pragma unroll
-        for (int q = 0; q < kMaxCluster; ++q)
-          if (q < C) t += remote(hist[0], q)[i];
-        total[i] = t;
+    // this CTA's histogram is added into every CTA's cluster histogram (pushed,
+    // not read back: a remote load waits for its reply)
+    __syncthreads();
+    for (int i = tid; i < kLinBins; i += kThreads) {
+      const uint32_t c = hist[0][i];
+      if (!kCluster) {
+        total[i] = c;
+      } else if (c != 0u) {
+        for (int q = 0; q < C; ++q) red_add_cluster(cluster_addr(&total[i], q), c);
       }
-      cnt = total;
-      __syncthreads();
     }
-    find_digit<kThreads>(cnt, (uint32_t)kb, kLinBins, wsum, &s_digit, &s_above);
+    cluster_sync();
+    find_digit<kThreads>([&](int i) { return total[i]; }, (uint32_t)kb, kLinBins, wsum, &s_digit,
+                         &s_above, &s_count);
     __syncthreads();
     bstar = (int)s_digit;
-    need = (uint32_t)kb - s_above;  // 1 <= need <= cnt[bstar]
-    n_cand = cnt[bstar];
-    fast = n_cand <= (uint32_t)kCand;
+    need = (uint32_t)kb - s_above;  // 1 <= need <= count of bin bstar
+    n_cand = s_count;
+    fast = n_cand <= (uint32_t)(kCand / C);  // every rank's candidates fit its part of the list
   }
   if (fast) {
-    // ---- pass 2: classify.  Keys above the boundary bin become ~0, keys below
-    //      it 0 (both on the right side of any finite threshold key); the
-    //      boundary bin's (key, index) pairs go to this CTA's candidate list.
-    uint32_t* loc = hist[1];  // [kCand] keys, then [kCand] indices
+    // ---- pass 2: classify.  The indices of the keys above the boundary bin
+    //      (all kept) are packed, in index order, at the start of the warp's
+    //      segment of `keys` (a write never passes the key being read); the
+    //      boundary bin's (key, index) pairs are stored into every CTA's
+    //      candidate list, in this rank's part of it.
+    const uint32_t cap = (uint32_t)(kCand / C);
+    uint32_t* ckey = hist[1];          // [kCand] keys, rank q's at [q*cap, (q+1)*cap)
+    uint32_t* cidx = hist[1] + kCand;  // their token indices
     uint32_t ngt = 0u;
     for (int c0 = s0; c0 < s1; c0 += 32) {
       const int i = c0 + lane;
@@ -218,74 +258,47 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
       const uint32_t key = valid ? keys[i] : 0u;
       const int bin = linear_bin(key, fmin, scale);
       const bool gt = valid && bin > bstar, cand = valid && bin == bstar;
-      ngt += __popc(__ballot_sync(0xffffffffu, gt));
+      const uint32_t bg = __ballot_sync(0xffffffffu, gt);
       if (cand) {
-        const uint32_t pos = atomicAdd(&s_ncand, 1u);
-        loc[pos] = key;
-        loc[kCand + pos] = (uint32_t)(lo + i);
+        const uint32_t slot = (uint32_t)rank * cap + atomicAdd(&s_ncand, 1u);
+        if (!kCluster) {
+          ckey[slot] = key;
+          cidx[slot] = (uint32_t)(lo + i);
+        } else {
+          for (int q = 0; q < C; ++q) {
+            st_cluster(cluster_addr(&ckey[slot], q), key);
+            st_cluster(cluster_addr(&cidx[slot], q), (uint32_t)(lo + i));
+          }
+        }
       }
-      if (valid) keys[i] = gt ? 0xffffffffu : (cand ? key : 0u);
+      if (gt) keys[s0 + ngt + __popc(bg & lt_mask)] = (uint32_t)(lo + i);
+      ngt += __popc(bg);
     }
     if (lane == 0) wcnt[warp][0] = ngt;
     __syncthreads();
+    // this rank's counts into every CTA
     if (warp == 0) {
       uint32_t x = lane < kWarps ? wcnt[lane][0] : 0u;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-      if (lane == 0) s_gtc = x;
-    }
-    cluster_sync();
-    // ---- the cluster's candidates, merged in rank order into `total`, and
-    //      every rank's count of keys above the boundary bin
-    if (tid < C) {
-      s_nq[tid] = *remote(&s_ncand, tid);
-      s_gtq[tid] = *remote(&s_gtc, tid);
-    }
-    __syncthreads();
-    if (tid == 0) {
-      uint32_t cb = 0u;
-      for (int q = 0; q < C; ++q) {
-        s_cbase[q] = cb;
-        cb += s_nq[q];
-      }
-      s_cbase[C] = cb;
-    }
-    __syncthreads();
-    for (uint32_t e = tid; e < n_cand; e += kThreads) {
-      int q = 0;
-      while (q + 1 < C && e >= s_cbase[q + 1]) ++q;
-      const uint32_t* rl = remote(loc, q);
-      const uint32_t j = e - s_cbase[q];
-      total[e] = rl[j];
-      total[kCand + e] = rl[kCand + j];
-    }
-    __syncthreads();
-    // ---- the need-th best pair (score descending, index ascending) is the
-    //      threshold; a candidate is kept when it is not worse
-    for (uint32_t t = tid; t < n_cand; t += kThreads) {
-      const uint32_t kt = total[t], it_ = total[kCand + t];
-      uint32_t better = 0u;
-      for (uint32_t j = 0; j < n_cand; ++j) {
-        const uint32_t kj = total[j], ij = total[kCand + j];
-        better += (kj > kt) || (kj == kt && ij < it_);
-      }
-      if (better == need - 1u) {
-        s_T = kt;
-        s_Tidx = it_;
-      }
-      if (better < need) {
-        int q = 0;
-        while (q + 1 < C && t >= s_cbase[q + 1]) ++q;
-        atomicAdd(&s_kc[q], 1u);
-        if (q == rank) atomicAdd(&wcnt[(it_ - (uint32_t)lo) / (uint32_t)seg][1], 1u);
+      if (lane < C) {
+        if (!kCluster) {
+          s_nq[0] = s_ncand;
+          s_gq[0] = x;
+        } else {
+          st_cluster(cluster_addr(&s_nq[rank], lane), s_ncand);
+          st_cluster(cluster_addr(&s_gq[rank], lane), x);
+        }
       }
     }
-    __syncthreads();
-    // ---- output offsets: ranks before this one, then warps before this one
+    cluster_sync();  // every CTA's candidates and counts have arrived
+    // ---- output offsets: the keys above the boundary bin first (ranks, then
+    //      warps, in index order), then the kept candidates best first
     if (warp == 0) {
-      uint32_t before = 0u;
-      for (int q = 0; q < rank; ++q) before += s_gtq[q] + s_kc[q];
-      const uint32_t mine = lane < kWarps ? wcnt[lane][0] + wcnt[lane][1] : 0u;
+      const uint32_t gq = lane < C ? s_gq[lane] : 0u;
+      const uint32_t ngt_all = __reduce_add_sync(0xffffffffu, gq);
+      const uint32_t before = __reduce_add_sync(0xffffffffu, lane < rank ? gq : 0u);
+      const uint32_t mine = lane < kWarps ? wcnt[lane][0] : 0u;
       uint32_t x = mine;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -293,22 +306,37 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
         if (lane >= o) x += t;
       }
       if (lane < kWarps) wbase[lane][0] = before + x - mine;
+      if (lane == 0) s_ngt = ngt_all;
     }
-    cluster_sync();  // every CTA is done with the others' shared memory
-    // ---- pass 3: write the kept indices of this warp's segment in order
-    const uint32_t T = s_T, Tidx = s_Tidx;
-    uint32_t run = wbase[warp][0];
-    for (int c0 = s0; c0 < s1; c0 += 32) {
-      const int i = c0 + lane;
-      const bool valid = i < s1;
-      const uint32_t key = valid ? keys[i] : 0u;
-      const bool keep = valid && (key > T || (key == T && (uint32_t)(lo + i) <= Tidx));
-      const uint32_t bk = __ballot_sync(0xffffffffu, keep);
-      if (keep) out[run + __popc(bk & lt_mask)] = (int32_t)(lo + i);
-      run += __popc(bk);
+    __syncthreads();
+    // ---- each of this CTA's candidates is ranked (score descending, index
+    //      ascending) against the whole cluster's; it is kept when fewer than
+    //      `need` pairs beat it, and that count is its place.  One warp per
+    //      candidate.
+    {
+      const uint32_t ngt_all = s_ngt, n_own = s_nq[rank];
+      for (uint32_t t = warp; t < n_own; t += kWarps) {
+        const uint32_t kt = ckey[rank * cap + t], it_ = cidx[rank * cap + t];
+        uint32_t better = 0u;
+        for (int q = 0; q < C; ++q) {
+          const uint32_t nq = s_nq[q];
+          for (uint32_t j = lane; j < nq; j += 32) {
+            const uint32_t kj = ckey[q * cap + j], ij = cidx[q * cap + j];
+            better += (kj > kt) || (kj == kt && ij < it_);
+          }
+        }
+        better = __reduce_add_sync(0xffffffffu, better);
+        if (lane == 0 && better < need) out[ngt_all + better] = (int32_t)it_;
+      }
+    }
+    // ---- pass 3: the packed indices of this warp's keys above the boundary bin
+    {
+      const uint32_t n_w = wcnt[warp][0], base = wbase[warp][0];
+      for (uint32_t j = lane; j < n_w; j += 32) out[base + j] = (int32_t)keys[s0 + j];
     }
     if (rank == 0)
       for (int64_t j = kb + tid; j < k; j += kThreads) out[j] = -1;
+    // nothing reads or writes this CTA's shared memory from other CTAs any more
     return;
   }
   // ======== fallback: radix select over the keys' bits
@@ -347,7 +375,8 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
         cnt = total;
       }
       __syncthreads();
-      find_digit<kThreads>(cnt, remaining, 1 << width, wsum, &s_digit, &s_above);
+      find_digit<kThreads>([&](int i) { return cnt[i]; }, remaining, 1 << width, wsum, &s_digit,
+                           &s_above, &s_count);
       __syncthreads();
       prefix |= (uint64_t)s_digit << lo_bit;
       remaining -= s_above;
@@ -445,6 +474,8 @@ cudaError_t launch_tk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) 
   const size_t smem = sizeof(uint32_t) * (size_t)p.topk_slice;
   static int done[kMaxDevices] = {};
   cudaError_t e = ensure_smem(topk_kernel<kCluster, kThreads>, smem, done);
+  if (e != cudaSuccess) return e;
+  e = prefer_max_shared((const void*)topk_kernel<kCluster, kThreads>);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(p.B * p.U * p.topk_cluster));
