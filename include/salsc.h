@@ -149,25 +149,30 @@ salsc_status salsc_decode_step(const salsc_decode_desc* desc, const void* q, con
                                int32_t* idx_out, void* ws, size_t ws_bytes, salsc_stream stream);
 
 /*
- * Number of kernels one decode layer-step launches, in order: latent query,
- * latent scoring, top-k, attention over the kept tokens, split merge (with
- * the deferred value projection).
+ * Stages of one decode layer-step, in order: latent query, latent scoring,
+ * top-k, attention over the kept tokens, split merge (with the deferred value
+ * projection).  Each stage is one kernel, except that for some shapes the
+ * attention kernel merges its own partials (one thread-block cluster per
+ * selection unit) and the merge stage launches nothing.
  */
 #define SALSC_DECODE_KERNELS 5
 
 /*
- * Number of kernels salsc_decode_step launches for this descriptor
- * (SALSC_DECODE_KERNELS for every supported shape), or -1 when the
- * descriptor is invalid or unsupported.
+ * Number of kernels salsc_decode_step launches for this descriptor:
+ * SALSC_DECODE_KERNELS, or one fewer when the attention kernel merges its own
+ * partials (the descriptor's units, each given a cluster of up to 8 CTAs,
+ * occupy at least as many SMs as an even split of the attention tiles, with
+ * the latent width r <= 256); -1 when the descriptor is invalid or
+ * unsupported.
  */
 int32_t salsc_decode_launch_count(const salsc_decode_desc* desc);
 
 /*
  * salsc_decode_step with timing marks: the same work, plus
- * cudaEventRecord(events[i], stream) just before kernel i and
+ * cudaEventRecord(events[i], stream) just before stage i and
  * events[SALSC_DECODE_KERNELS] after the last, so that
- * cudaEventElapsedTime(events[i], events[i+1]) is kernel i's time on the
- * stream.  events: SALSC_DECODE_KERNELS + 1 cudaEvent_t handles created by
+ * cudaEventElapsedTime(events[i], events[i+1]) is stage i's time on the
+ * stream (about zero for a merge stage that launches nothing).  events: SALSC_DECODE_KERNELS + 1 cudaEvent_t handles created by
  * the caller (cast to void*); n_events must equal that count.
  * Errors: as salsc_decode_step; INVALID_ARG for a missing or short event list.
  */

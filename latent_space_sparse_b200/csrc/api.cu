@@ -111,6 +111,7 @@ salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
     p.chunk = chunk;
     p.att_tiles = 0;
   }
+  p.att_cluster = p.attend_tc ? salsc::attend_merge_cluster(p) : 0;
   if (!salsc::combine_supported(p)) return SALSC_ERR_UNSUPPORTED;
   p.scale = D->softmax_scale != 0.0f ? D->softmax_scale : (float)(1.0 / sqrt((double)p.d));
   p.rope_base = D->rope_base;
@@ -166,7 +167,7 @@ const char* salsc_version(void) { return "salsc 0.1 (sm_100a)"; }
 int32_t salsc_decode_launch_count(const salsc_decode_desc* desc) {
   salsc::DecodePlan p;
   if (make_plan(desc, &p) != SALSC_OK) return -1;
-  return SALSC_DECODE_KERNELS;
+  return p.att_cluster > 0 ? SALSC_DECODE_KERNELS - 1 : SALSC_DECODE_KERNELS;
 }
 
 size_t salsc_decode_workspace_size(const salsc_decode_desc* desc) {

@@ -68,7 +68,10 @@ struct AttendTcParams {
   const int32_t* q_pos;
   float* part;
   uint32_t* flags;
+  const __nv_bfloat16* Pv;  // merged in the kernel: the value projection
+  __nv_bfloat16* out;
   int B, Hq, U, r, k, n_slots, n_tiles;
+  int cluster;  // merged in the kernel: CTAs per unit (one thread-block cluster)
   float scale;
   double base;
 };
@@ -158,14 +161,14 @@ __device__ __forceinline__ void gather_rows(const int* tk, int64_t off, uint32_t
 
 // barrier indices
 enum { B_PK = 0, B_KFULL = 1, B_VFULL = 3, B_KDONE = 5, B_PDONE = 7, B_PREADY = 9,
-       B_TKFREE = 11, B_TOFREE = 13, B_PKDONE = 15, B_COUNT = 16 };
+       B_TKFREE = 11, B_TOFREE = 13, B_PKDONE = 15, B_PV = 16, B_COUNT = 17 };
 
 // W = 1: the latent width r <= 256 fits one tile buffer; two buffers hold two
 // tiles, and tiles are pipelined.  W = 2 (256 < r <= 512): the two buffers hold
 // the two latent halves of one tile, Pk_u is loaded half by half (the
 // reconstruction accumulates over the halves), and tiles run one after the
 // other.
-template <int G, int D, int W>
+template <int G, int D, int W, bool kMerge>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
                  const __grid_constant__ CUtensorMap tmap_kc,
@@ -203,9 +206,26 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   allow_dependent_launch();
-  const int t_begin = (int)((int64_t)blockIdx.x * P.n_tiles / gridDim.x);
-  const int t_end = (int)((int64_t)(blockIdx.x + 1) * P.n_tiles / gridDim.x);
-  const int n = t_end - t_begin;
+  // Tile range: a contiguous share of all tiles, or (kMerge) the rank's share
+  // of its unit's tiles, the unit being (blockIdx.x / cluster).
+  int t_begin, n, m_unit = 0, m_rank = 0;
+  if constexpr (kMerge) {
+    m_rank = (int)(blockIdx.x % (unsigned)P.cluster);
+    m_unit = (int)(blockIdx.x / (unsigned)P.cluster);
+    const int mb = m_unit / P.U;
+    int before = 0, tu = 0;
+    for (int bb = 0; bb <= mb; ++bb) {
+      const int64_t nbb = P.seq_off[bb + 1] - P.seq_off[bb];
+      const int t = (int)(((nbb < P.k ? nbb : (int64_t)P.k) + kTile - 1) / kTile);
+      if (bb < mb) before += P.U * t; else tu = t;
+    }
+    const int lo = tu * m_rank / P.cluster, hi = tu * (m_rank + 1) / P.cluster;
+    t_begin = before + (m_unit % P.U) * tu + lo;
+    n = hi - lo;
+  } else {
+    t_begin = (int)((int64_t)blockIdx.x * P.n_tiles / gridDim.x);
+    n = (int)((int64_t)(blockIdx.x + 1) * P.n_tiles / gridDim.x) - t_begin;
+  }
   // TMEM columns: K_sel [2][D], then acc [2][n_chunks * 16]
   const uint32_t o_col0 = 2 * D;
   const uint32_t o_cols = (uint32_t)n_chunks * 16;
@@ -233,8 +253,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
   if (W == 2 && warp >= kLoadWarp0) {
     // ======================= gather warps, two latent halves =================
     // Warp h fills buffer h with latent half h of every tile: the key rows,
-    // then, once the reconstruction is done, the value rows (copy_rows).  Lane
-    // gt looks up the tokens of rows gt + 32j.
+    // then, once the reconstruction is done, the value rows (gather_rows).
+    // Thread gt looks up the token of row gt.
     const int h = (warp - kLoadWarp0) / kGatherWarps;
     const int gt = tid - (kLoadWarp0 + h * kGatherWarps) * 32;  // 0..127
     const uint32_t gbar = 2 + h;
@@ -364,8 +384,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     // ======================= gather warps =======================
     // Warp bi fills buffer bi with tiles bi, bi+2, ...: first the latent key
     // rows Kc_b[idx], then, once the reconstruction is done with them, the
-    // same rows of Vc (copy_rows).  Lane gt looks up the tokens of rows
-    // gt + 32j; the next tile's are loaded while the current tile is in flight.
+    // same rows of Vc (gather_rows).  Thread gt looks up the token of row gt;
+    // the next tile's is loaded while the current tile is in flight.
     const int bi = (warp - kLoadWarp0) / kGatherWarps;
     const int gt = tid - (kLoadWarp0 + bi * kGatherWarps) * 32;  // 0..127
     const uint32_t gbar = 2 + bi;  // named barrier of the group
@@ -515,6 +535,22 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
           __nanosleep(32);
         }
       }
+      if constexpr (kMerge) {
+        // this rank's rows of Pv_u for the value projection, into the Pk
+        // buffer once the last reconstruction is done with it
+        const bool okp =
+            n == 0 || __all_sync(0xffffffffu, tc::mbar_wait(bar(B_KDONE + ((n - 1) & 1)),
+                                                            ((uint32_t)(n - 1) >> 1) & 1u, P.flags));
+        if (okp && tc::elect_one()) {
+          const int dq = D / P.cluster;
+          const uint32_t bytes = (uint32_t)dq * (uint32_t)P.r * 2u;
+          tc::mbar_expect_tx(bar(B_PV), bytes);
+          tc::bulk_load(tc::smem_u32(s_pk),
+                        P.Pv + ((int64_t)(m_unit % P.U) * D + (int64_t)m_rank * dq) * P.r, bytes,
+                        bar(B_PV));
+        }
+        __syncwarp();
+      }
     }
   } else {
     // ======================= epilogue (warps 0-15) =======================
@@ -595,7 +631,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       nx.next();
       const bool seg_end = j + 1 == n || nx.b != fc.b || nx.u != fc.u;
       ++seg_tiles;
-      if (seg_end) {
+      if (!kMerge && seg_end) {
         const int s0 = fc.slot + 1 - seg_tiles;  // first slot of the segment
         const int64_t row0 = ((int64_t)fc.b * P.Hq + fc.u * G) * P.n_slots + s0;
 #pragma unroll
@@ -750,6 +786,89 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       tc::named_sync(kEpiBar, kEpiThreads);
       fold(n - 1);
     }
+    if constexpr (kMerge) {
+      // this CTA's partial of the unit, (m, l) and acc[r] per head, staged in
+      // the first tile buffer (every MMA and copy into it has completed) for
+      // the cluster's merge
+      float* const st = (float*)s_buf0;
+#pragma unroll
+      for (int jj = 0; jj < kSlots; ++jj) {
+        const int sl = part + 4 * jj;
+        const int c = (sl / G) * 128 + quarter * 32 + lane;
+        if (sl < n_used && c < P.r) st[2 * G + (sl % G) * P.r + c] = acc_run[jj];
+      }
+      if (tid < G) {
+        st[2 * tid] = s_run[2 * tid];
+        st[2 * tid + 1] = s_run[2 * tid + 1];
+      }
+    }
+  }
+  if constexpr (kMerge) {
+    // ---- the unit's partials, merged across the cluster (the same online-
+    //      softmax combination as the merge kernel, over ranks in order), and
+    //      the deferred value projection: rank q writes output dims
+    //      q*d/C .. (q+1)*d/C - 1 of the unit's heads, out = acc . Pv_u^T
+    cluster_arrive();
+    cluster_wait();  // every CTA's partial is staged
+    constexpr int kMaxCl = 8;
+    const int C = P.cluster;
+    float* const accm = (float*)s_buf1;  // merged acc [G][r]
+    if (warp < kEpiWarps) {
+      uint32_t rs[kMaxCl];  // each rank's staged partial
+#pragma unroll
+      for (int q = 0; q < kMaxCl; ++q) rs[q] = q < C ? cluster_addr(s_buf0, q) : 0u;
+      for (int e = tid; e < G * P.r; e += kEpiThreads) {
+        const int g = e / P.r, c = e % P.r;
+        float mq[kMaxCl], lq[kMaxCl], aq[kMaxCl];
+#pragma unroll
+        for (int q = 0; q < kMaxCl; ++q) {
+          if (q < C) {
+            mq[q] = ld_cluster_f32(rs[q] + 4u * (uint32_t)(2 * g));
+            lq[q] = ld_cluster_f32(rs[q] + 4u * (uint32_t)(2 * g + 1));
+            aq[q] = ld_cluster_f32(rs[q] + 4u * (uint32_t)(2 * G + g * P.r + c));
+          }
+        }
+        float M = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < kMaxCl; ++q)
+          if (q < C) M = fmaxf(M, mq[q]);
+        float L = 0.f, a = 0.f;
+#pragma unroll
+        for (int q = 0; q < kMaxCl; ++q) {
+          if (q < C && mq[q] != -INFINITY) {
+            const float w = expf(mq[q] - M);
+            L += w * lq[q];
+            a += w * aq[q];
+          }
+        }
+        accm[e] = L > 0.f ? a / L : 0.f;
+      }
+    }
+    cluster_arrive();  // done with the other CTAs' shared memory
+    if (warp < kEpiWarps) {
+      tc::named_sync(kEpiBar, kEpiThreads);  // the merged acc is complete
+      const bool okv = __all_sync(0xffffffffu, tc::mbar_wait(bar(B_PV), 0u, P.flags));
+      const int dq = D / C;
+      const int u = m_unit % P.U, mb = m_unit / P.U;
+      // four threads per output (G x dq outputs, dq a multiple of 8)
+      for (int e = tid; e < G * dq * 4; e += kEpiThreads) {
+        const int o = e >> 2, sub = e & 3;
+        const int g = o / dq, dd = o % dq;
+        const __nv_bfloat162* pvr = (const __nv_bfloat162*)(s_pk + (size_t)dd * P.r * 2);
+        const float* ar = accm + g * P.r;
+        float acc = 0.f;
+        if (okv)
+          for (int c = 2 * sub; c < P.r; c += 8) {
+            const float2 pv = __bfloat1622float2(pvr[c >> 1]);
+            acc = fmaf(ar[c], pv.x, fmaf(ar[c + 1], pv.y, acc));
+          }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        if (sub == 0)
+          P.out[((int64_t)mb * P.Hq + u * G + g) * D + m_rank * dq + dd] = __float2bfloat16_rn(acc);
+      }
+    }
+    cluster_wait();
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -780,7 +899,7 @@ size_t smem_bytes(int r) {
          8 * B_COUNT + 16;
 }
 
-template <int G, int D, int W>
+template <int G, int D, int W, bool kMerge>
 cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
   const size_t smem = smem_bytes<G, D, W>(p.r);
   CUtensorMap tpk, tkc, tvc;
@@ -789,7 +908,7 @@ cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s)
       !make_tmap_bf16_2d(&tvc, a.Vc, (uint64_t)p.N, (uint64_t)p.r, 1, 64))
     return cudaErrorInvalidValue;
   static int done[kMaxDevices] = {};
-  cudaError_t e = ensure_smem(attend_tc_kernel<G, D, W>, smem, done);
+  cudaError_t e = ensure_smem(attend_tc_kernel<G, D, W, kMerge>, smem, done);
   if (e != cudaSuccess) return e;
   AttendTcParams P;
   P.q = (const __nv_bfloat16*)a.q;
@@ -800,6 +919,8 @@ cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s)
   P.q_pos = a.q_pos;
   P.part = a.part;
   P.flags = a.flags;
+  P.Pv = (const __nv_bfloat16*)a.Pv;
+  P.out = (__nv_bfloat16*)a.out;
   P.B = p.B;
   P.Hq = p.Hq;
   P.U = p.U;
@@ -807,27 +928,49 @@ cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s)
   P.k = p.k;
   P.n_slots = p.splits;
   P.n_tiles = p.att_tiles;
+  P.cluster = kMerge ? p.att_cluster : 1;
   P.scale = p.scale;
   P.base = p.rope_base;
-  return launch_k(attend_tc_kernel<G, D, W>, dim3(attend_tc_grid(p)), dim3(kThreads), smem, s,
-                  true, tpk, tkc, tvc, P);
+  if constexpr (!kMerge) {
+    return launch_k(attend_tc_kernel<G, D, W, false>, dim3(attend_tc_grid(p)), dim3(kThreads),
+                    smem, s, true, tpk, tkc, tvc, P);
+  } else {
+    // one cluster of att_cluster CTAs per unit
+    e = prefer_max_shared((const void*)attend_tc_kernel<G, D, W, true>);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.B * p.U * p.att_cluster));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)p.att_cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, attend_tc_kernel<G, D, W, true>, tpk, tkc, tvc, P);
+  }
 }
 
-template <int W>
+template <int W, bool kMerge>
 cudaError_t launch_w(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
   if (p.d == 128) {
     switch (p.G) {
-      case 1: return launch_g_d<1, 128, W>(p, a, s);
-      case 2: return launch_g_d<2, 128, W>(p, a, s);
-      case 4: return launch_g_d<4, 128, W>(p, a, s);
-      case 8: return launch_g_d<8, 128, W>(p, a, s);
+      case 1: return launch_g_d<1, 128, W, kMerge>(p, a, s);
+      case 2: return launch_g_d<2, 128, W, kMerge>(p, a, s);
+      case 4: return launch_g_d<4, 128, W, kMerge>(p, a, s);
+      case 8: return launch_g_d<8, 128, W, kMerge>(p, a, s);
     }
   } else {
     switch (p.G) {
-      case 1: return launch_g_d<1, 64, W>(p, a, s);
-      case 2: return launch_g_d<2, 64, W>(p, a, s);
-      case 4: return launch_g_d<4, 64, W>(p, a, s);
-      case 8: return launch_g_d<8, 64, W>(p, a, s);
+      case 1: return launch_g_d<1, 64, W, kMerge>(p, a, s);
+      case 2: return launch_g_d<2, 64, W, kMerge>(p, a, s);
+      case 4: return launch_g_d<4, 64, W, kMerge>(p, a, s);
+      case 8: return launch_g_d<8, 64, W, kMerge>(p, a, s);
     }
   }
   return cudaErrorInvalidConfiguration;
@@ -848,8 +991,31 @@ bool attend_tc_supported(const DecodePlan& p) {
          (k_eff + kTile - 1) / kTile <= kTile;  // the merge takes <= 128 slots per unit
 }
 
+int attend_merge_cluster(const DecodePlan& p) {
+  // r <= 256 (one tile buffer per tile), and every unit's cluster resident at
+  // once: the largest power of two C <= 8 with B*U*C <= #SMs (d/C >= 8 output
+  // dims per rank).  The tile phase is bound by the row gathers of all SMs
+  // together, so the clusters are used only when they take at least as many
+  // SMs as the even split of the tiles, and no CTA gets more tiles than there.
+  if (!attend_tc_supported(p) || p.r > 256 || p.att_tiles <= 0) return 0;
+  const int64_t sms = num_sms_att();
+  const int64_t units = (int64_t)p.B * p.U;
+  int c = 0;
+  for (int cc = 1; cc <= 8; cc *= 2)
+    if (units * cc <= sms && p.d / cc >= 8) c = cc;
+  if (c == 0) return 0;
+  const int64_t grid_split = p.att_tiles < sms ? p.att_tiles : sms;
+  const int64_t k_eff = p.k < p.n_max ? p.k : p.n_max;
+  const int64_t tu_max = (k_eff + kTile - 1) / kTile;
+  if (units * c < grid_split ||
+      (tu_max + c - 1) / c > (p.att_tiles + grid_split - 1) / grid_split)
+    return 0;
+  return c;
+}
+
 cudaError_t launch_attend_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
-  return p.r <= 256 ? launch_w<1>(p, a, s) : launch_w<2>(p, a, s);
+  if (p.r > 256) return launch_w<2, false>(p, a, s);
+  return p.att_cluster > 0 ? launch_w<1, true>(p, a, s) : launch_w<1, false>(p, a, s);
 }
 
 }  // namespace salsc

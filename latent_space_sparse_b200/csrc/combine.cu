@@ -264,6 +264,7 @@ bool combine_supported(const DecodePlan& p) {
 }
 
 cudaError_t launch_combine(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
+  if (p.att_cluster > 0) return cudaSuccess;  // the attention kernel merged the partials
   if (!combine_supported(p)) return cudaErrorInvalidConfiguration;
   CombineParams P;
   P.part = a.part;

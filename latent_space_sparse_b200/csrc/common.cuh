@@ -47,6 +47,8 @@ struct DecodePlan {
   int chunk;            // kept tokens per slot
   bool attend_tc;       // tensor-core attention path (tiles of 128 kept tokens)
   int att_tiles;        // sum over units of ceil(k_b / 128) (tensor-core path)
+  int att_cluster;      // > 0: the attention kernel merges each unit's partials and projects
+                        // them itself, one cluster of att_cluster CTAs per unit (no merge kernel)
   float scale;
   double rope_base;
   // workspace layout (byte offsets)
@@ -82,6 +84,7 @@ cudaError_t launch_topk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s
 cudaError_t launch_attend(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 bool attend_tc_supported(const DecodePlan& p);
+int attend_merge_cluster(const DecodePlan& p);  // 0: merge kernel; else CTAs per unit
 int attend_tc_grid(const DecodePlan& p);  // CTAs of the tensor-core attention (tile partition)
 bool combine_supported(const DecodePlan& p);
 cudaError_t launch_attend_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
@@ -164,6 +167,39 @@ __device__ __forceinline__ void allow_dependent_launch() {
 }
 
 // ---------------------------------------------------------------- device helpers
+
+// Shared-memory address of `p` in cluster CTA `rank` (thread-block clusters).
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(r)
+               : "r"((uint32_t)__cvta_generic_to_shared(p)), "r"(rank));
+  return r;
+}
+// Store and atomic add into the shared memory of another CTA of the cluster:
+// no reply is awaited, and the next cluster barrier makes them visible.
+__device__ __forceinline__ void st_cluster(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_add_cluster(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+// Load from the shared memory of a CTA of the cluster (waits for the reply).
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// Split cluster barrier: arrive (releasing this thread's shared-memory reads
+// and writes) and, later, wait for every thread of the cluster to arrive.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 
 template <typename T>
 __device__ __forceinline__ float to_f32(T x);

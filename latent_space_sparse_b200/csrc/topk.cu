@@ -40,32 +40,6 @@ namespace {
 constexpr int kBatch = 8;  // keys a thread loads before converting them (the loop is unrolled: short code)
 constexpr int kMaxCluster = 8;  // largest cluster of CTAs per unit
 
-// Shared-memory address of `p` in cluster CTA `rank`, for the stores below.
-__device__ __forceinline__ uint32_t cluster_addr(const void* p, int rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
-               : "=r"(r)
-               : "r"((uint32_t)__cvta_generic_to_shared(p)), "r"(rank));
-  return r;
-}
-// Store and atomic add into the shared memory of another CTA of the cluster:
-// no reply is awaited, and the next cluster barrier makes them visible.
-__device__ __forceinline__ void st_cluster(uint32_t addr, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ void red_add_cluster(uint32_t addr, uint32_t v) {
-  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-
-// Split cluster barrier: arrive (releasing this thread's shared-memory reads
-// and writes) and, later, wait for every thread of the cluster to arrive.
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
 // Float whose order_key is `key` (-0 comes back as +0).
 __device__ __forceinline__ float key_float(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);

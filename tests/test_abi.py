@@ -54,8 +54,14 @@ def test_workspace_size_valid_shapes_grow_with_tokens():
 
 
 def test_launch_count():
-    for kw in (dict(rank=256), dict(rank=512), dict(dtype=torch.float32)):
+    # 8 units of one tile: clusters of 8 CTAs merge inside the attention kernel
+    assert salsc.salsc_decode_launch_count(desc([0, 1000])) == 4
+    # r > 256, the CUDA-core path, and 32 units of 16 tiles (the even split
+    # over all SMs is wider than 32 clusters of 4): a separate merge kernel
+    for kw in (dict(rank=512), dict(dtype=torch.float32)):
         assert salsc.salsc_decode_launch_count(desc([0, 1000], **kw)) == 5
+    offs = [0, 4096, 8192, 12288, 16384]
+    assert salsc.salsc_decode_launch_count(desc(offs, top_k=2048)) == 5
     with pytest.raises(ValueError):
         salsc.salsc_decode_launch_count(desc([0, 10], top_k=0))
 

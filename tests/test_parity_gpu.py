@@ -154,6 +154,43 @@ def test_wide_rank_512_mha_many_tiles():
     check(w, synth.decode_inputs(w, seq_lens=(4096,)), top_k=1000)
 
 
+def launches(w, top_k=None):
+    lens = w.seq_lens
+    dec = salsc.Decoder(len(lens), w.n_q_heads, w.n_kv_heads, w.head_dim, w.rank,
+                        top_k or w.top_k, lens, rope_base=w.rope_base,
+                        dtype=synth.torch_dtype(w.dtype), device=DEV)
+    return salsc.salsc_decode_launch_count(dec.desc)
+
+
+def test_in_kernel_merge_one_tile_per_cta():
+    # one sequence, 32 MHA units of 4 tiles: a cluster of 4 CTAs per unit
+    # merges its partials and projects them inside the attention kernel
+    w = W.Workload(name="mha_merge", batch=1, n_q_heads=32, n_kv_heads=32, head_dim=128,
+                   rank=256, top_k=512, seq_lens=(3000,), dtype="bf16", rope_base=10000.0,
+                   low_rank=32, seed=95)
+    assert launches(w) == len(salsc.DECODE_KERNELS) - 1
+    check(w, synth.decode_inputs(w))
+
+
+def test_in_kernel_merge_ranks_without_tiles():
+    # 2 units of 3 tiles on clusters of 8 CTAs: five ranks hold no tile and
+    # merge an empty partial
+    w = W.Workload(name="gqa_merge", batch=1, n_q_heads=8, n_kv_heads=2, head_dim=128, rank=192,
+                   top_k=300, seq_lens=(900,), dtype="bf16", rope_base=10000.0, low_rank=16,
+                   seed=94)
+    assert launches(w) == len(salsc.DECODE_KERNELS) - 1
+    check(w, synth.decode_inputs(w))
+
+
+def test_separate_merge_kernel_when_the_split_is_wider():
+    # 32 units of 16 tiles: the even split over every SM beats clusters of 4
+    w = W.Workload(name="gqa_split", batch=4, n_q_heads=32, n_kv_heads=8, head_dim=128,
+                   rank=256, top_k=2048, seq_lens=(2500, 2200, 3000, 2049), dtype="bf16",
+                   rope_base=10000.0, low_rank=32, seed=93)
+    assert launches(w) == len(salsc.DECODE_KERNELS)
+    check(w, synth.decode_inputs(w))
+
+
 def test_small_rank_f32():
     w = W.Workload(name="f32_r16", batch=3, n_q_heads=6, n_kv_heads=3, head_dim=64, rank=16,
                    top_k=9, seq_lens=(50, 17, 200), dtype="f32", rope_base=500000.0, low_rank=4,
