@@ -134,7 +134,7 @@ __device__ __forceinline__ int row_token(const AttendTcParams& P, const UnitTile
   return t;
 }
 
-constexpr int kGatherRows = kTile / kGatherThreads;  // token rows per gather thread
+constexpr int kGatherRows = (kTile + kGatherThreads - 1) / kGatherThreads;  // token rows per gather thread
 
 // Gather thread gt's share of one tile's latent rows: items e = gt + 128j
 // over 32 row groups x KB k-blocks; item e copies rows tk[4g .. 4g+3]
@@ -145,7 +145,9 @@ constexpr int kGatherRows = kTile / kGatherThreads;  // token rows per gather th
 __device__ __forceinline__ void gather_rows(const int* tk, int64_t off, uint32_t buf_s,
                                             const CUtensorMap* tmap, int kb0, int KB, int gt,
                                             uint32_t mbar) {
-  for (int e = gt; e < 32 * KB; e += kGatherThreads) {
+  // ops dealt round-robin over the group's warps (a warp issues its ops one
+  // after another)
+  for (int e = (gt % 32) * kGatherWarps + gt / 32; e < 32 * KB; e += kGatherThreads) {
     const int g4 = e & 31, kb = e >> 5;
     int rows[4];
 #pragma unroll
@@ -176,7 +178,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
   constexpr int HALF = D / 2;
   constexpr int QP = HALF / kEpiParts;                     // RoPE pairs per epilogue thread
   constexpr int kPasses = (G * kTile + kEpiThreads - 1) / kEpiThreads;  // softmax items per thread
-  constexpr int kSlots = (2 * W * G + 3) / 4;  // (chunk, head) accumulators per epilogue thread
+  constexpr int kSlots = (2 * W * G + kEpiParts - 1) / kEpiParts;  // (chunk, head) accumulators per epilogue thread
   static_assert(QP % 8 == 0, "TMEM loads of 8 columns");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -267,21 +269,23 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     int t_next[kGatherRows];
 #pragma unroll
     for (int j = 0; j < kGatherRows; ++j)
-      t_next[j] = n > 0 ? row_token(P, cur, gt + j * kGatherThreads) : -1;
+      t_next[j] = n > 0 && gt + j * kGatherThreads < kTile ? row_token(P, cur, gt + j * kGatherThreads) : -1;
     bool ok = true;
     for (int i = 0; i < n && ok; ++i) {
       const int64_t off = cur.off;
       // the buffer is free once the value MMA of the previous tile is done
       if (i >= 1) ok = tc::mbar_wait(bar(B_PDONE + ((i - 1) & 1)), ((uint32_t)(i - 1) >> 1) & 1u, P.flags);
 #pragma unroll
-      for (int j = 0; j < kGatherRows; ++j) tk[gt + j * kGatherThreads] = t_next[j];
+      for (int j = 0; j < kGatherRows; ++j)
+        if (gt + j * kGatherThreads < kTile) tk[gt + j * kGatherThreads] = t_next[j];
       if (gt == 0) tc::mbar_expect_tx(bar(B_KFULL + h), tile_bytes);
       tc::named_sync(gbar, kGatherThreads);
       gather_rows(tk, off, buf_s, &tmap_kc, h * KB, KB, gt, bar(B_KFULL + h));
       cur.next();
 #pragma unroll
       for (int j = 0; j < kGatherRows; ++j)
-        t_next[j] = i + 1 < n ? row_token(P, cur, gt + j * kGatherThreads) : -1;
+        t_next[j] = i + 1 < n && gt + j * kGatherThreads < kTile
+                        ? row_token(P, cur, gt + j * kGatherThreads) : -1;
       if (!tc::mbar_wait(bar(B_KDONE + (i & 1)), ((uint32_t)i >> 1) & 1u, P.flags)) break;
       if (gt == 0) tc::mbar_expect_tx(bar(B_VFULL + h), tile_bytes);
       tc::named_sync(gbar, kGatherThreads);
@@ -399,7 +403,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     int t_next[kGatherRows];
 #pragma unroll
     for (int j = 0; j < kGatherRows; ++j)
-      t_next[j] = bi < n ? row_token(P, cur, gt + j * kGatherThreads) : -1;
+      t_next[j] = bi < n && gt + j * kGatherThreads < kTile ? row_token(P, cur, gt + j * kGatherThreads) : -1;
     bool ok = true;
     for (int i = bi; i < n && ok; i += 2) {
       const uint32_t ph = ((uint32_t)i >> 1) & 1u;
@@ -409,7 +413,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
         ok = tc::mbar_wait(bar(B_PDONE + bi), ph ^ 1u, P.flags);
       }
 #pragma unroll
-      for (int j = 0; j < kGatherRows; ++j) tk[gt + j * kGatherThreads] = t_next[j];
+      for (int j = 0; j < kGatherRows; ++j)
+        if (gt + j * kGatherThreads < kTile) tk[gt + j * kGatherThreads] = t_next[j];
       if (gt == 0) tc::mbar_expect_tx(bar(B_KFULL + bi), tile_bytes);
       tc::named_sync(gbar, kGatherThreads);
       gather_rows(tk, off, buf_s, &tmap_kc, 0, KB, gt, bar(B_KFULL + bi));
@@ -418,7 +423,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       cur.next();
 #pragma unroll
       for (int j = 0; j < kGatherRows; ++j)
-        t_next[j] = i + 2 < n ? row_token(P, cur, gt + j * kGatherThreads) : -1;
+        t_next[j] = i + 2 < n && gt + j * kGatherThreads < kTile
+                        ? row_token(P, cur, gt + j * kGatherThreads) : -1;
       // the reconstruction is done with the key rows: bring the value rows
       if (!tc::mbar_wait(bar(B_KDONE + bi), ph, P.flags)) break;
       if (gt == 0) tc::mbar_expect_tx(bar(B_VFULL + bi), tile_bytes);
@@ -563,7 +569,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     UnitTileCursor cur;
     cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
     int cur_b = -1, cur_u = -1;
-    // the segment's running sums: slot s = part + 4j (j < kSlots) holds latent
+    // the segment's running sums: slot s = part + kEpiParts*j (j < kSlots) holds latent
     // column (s / G)*128 + quarter*32 + lane of head s % G
     const int n_used = n_chunks * G;
     float acc_run[kSlots];
@@ -607,7 +613,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       uint32_t v[kSlots][2];
 #pragma unroll
       for (int jj = 0; jj < kSlots; ++jj) {
-        const int sl = part + 4 * jj;
+        const int sl = part + kEpiParts * jj;
         if (ok2 && sl < n_used)
           tc::tmem_ld2(tmem_base + ((uint32_t)(quarter * 32) << 16) + o_col0 + (uint32_t)bj * o_cols +
                            (uint32_t)(sl / G) * 16 + 2u * (uint32_t)(sl % G),
@@ -619,7 +625,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       if (tid == 0) tc::mbar_arrive(bar(B_TOFREE + bj));
 #pragma unroll
       for (int jj = 0; jj < kSlots; ++jj) {
-        const int sl = part + 4 * jj;
+        const int sl = part + kEpiParts * jj;
         if (ok2 && sl < n_used) {
           const int g = sl % G;
           acc_run[jj] = acc_run[jj] * s_ab[2 * g] +
@@ -636,7 +642,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
         const int64_t row0 = ((int64_t)fc.b * P.Hq + fc.u * G) * P.n_slots + s0;
 #pragma unroll
         for (int jj = 0; jj < kSlots; ++jj) {
-          const int sl = part + 4 * jj;
+          const int sl = part + kEpiParts * jj;
           const int c = (sl / G) * 128 + quarter * 32 + lane;
           if (sl < n_used && c < P.r)
             P.part[(row0 + (int64_t)(sl % G) * P.n_slots) * part_row(P.r) + kPartAcc + c] =
@@ -793,7 +799,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       float* const st = (float*)s_buf0;
 #pragma unroll
       for (int jj = 0; jj < kSlots; ++jj) {
-        const int sl = part + 4 * jj;
+        const int sl = part + kEpiParts * jj;
         const int c = (sl / G) * 128 + quarter * 32 + lane;
         if (sl < n_used && c < P.r) st[2 * G + (sl % G) * P.r + c] = acc_run[jj];
       }
