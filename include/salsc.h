@@ -149,6 +149,25 @@ salsc_status salsc_decode_step(const salsc_decode_desc* desc, const void* q, con
                                int32_t* idx_out, void* ws, size_t ws_bytes, salsc_stream stream);
 
 /*
+ * salsc_append followed by salsc_decode_step in one call: the new token's key
+ * and value rows (K_new, V_new [batch][Hkv*d], either may be NULL) are
+ * projected and written to Kc/Vc at rows_dev[b] (as salsc_append), then the
+ * step runs over the updated caches; its first kernel starts its weight loads
+ * while the rows are written.  The descriptor's sequence lengths and q_pos
+ * are taken as given: with the new token already in the cache (row
+ * seq_offsets[b] + n_b - 1) the usual decode query position is n_b - 1, to be
+ * passed in q_pos_dev.  Arguments otherwise as salsc_append and
+ * salsc_decode_step; every argument is checked before anything is enqueued.
+ * Errors: as salsc_decode_step, INVALID_ARG (both rows NULL, rows_dev NULL),
+ * UNSUPPORTED (Hkv*d > 8192).
+ */
+salsc_status salsc_decode_step_append(const salsc_decode_desc* desc, const void* K_new,
+                                      const void* V_new, const int64_t* rows_dev, const void* q,
+                                      void* Kc, void* Vc, const void* Pk, const void* Pv,
+                                      void* out, int32_t* idx_out, void* ws, size_t ws_bytes,
+                                      salsc_stream stream);
+
+/*
  * Stages of one decode layer-step, in order: latent query, latent scoring,
  * top-k, attention over the kept tokens, split merge (with the deferred value
  * projection).  Each stage is one kernel, except that for some shapes the

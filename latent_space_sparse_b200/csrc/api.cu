@@ -220,13 +220,26 @@ salsc_status salsc_append(const void* K_new, const void* V_new, const void* Pk, 
 
 namespace {
 
+// The new token's rows, appended to the latent caches before the step reads
+// them (salsc_decode_step_append).
+struct AppendArgs {
+  const void* K_new;
+  const void* V_new;
+  const int64_t* rows;
+};
+
 salsc_status decode_step_impl(const salsc_decode_desc* desc, const void* q, const void* Kc,
                               const void* Vc, const void* Pk, const void* Pv, void* out,
                               int32_t* idx_out, void* ws, size_t ws_bytes, salsc_stream stream,
-                              void* const* events, int32_t n_events) {
+                              void* const* events, int32_t n_events,
+                              const AppendArgs* app = nullptr) {
   salsc::DecodePlan p;
   salsc_status st = make_plan(desc, &p);
   if (st != SALSC_OK) return st;
+  if (app) {
+    if ((!app->K_new && !app->V_new) || !app->rows) return SALSC_ERR_INVALID_ARG;
+    if (p.U * p.d > 8 * 1024) return SALSC_ERR_UNSUPPORTED;
+  }
   if (!desc->seq_offsets_dev || !q || !Kc || !Vc || !Pk || !Pv || !out)
     return SALSC_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(Pk) || !aligned16(Pv) ||
@@ -264,6 +277,16 @@ salsc_status decode_step_impl(const salsc_decode_desc* desc, const void* q, cons
                                               salsc::launch_combine};
   // the tensor-core attention merges its own tiles (no separate merge kernel)
   cudaError_t e;
+  if (app) {
+    // the new rows first, in stream order (the step's kernels then wait for
+    // them like for any earlier work); Kc and Vc are written, hence non-const
+    const void* X[2] = {app->K_new ? app->K_new : app->V_new, app->V_new};
+    const void* Pm[2] = {app->K_new ? Pk : Pv, Pv};
+    void* Y[2] = {app->K_new ? (void*)Kc : (void*)Vc, (void*)Vc};
+    if ((e = salsc::launch_append(X, Pm, Y, (app->K_new && app->V_new) ? 2 : 1, app->rows, p.B,
+                                  p.U * p.d, p.r, p.dtype, s)) != cudaSuccess)
+      return cuda_fail(e);
+  }
   // Inside stream capture an event record must be an external node to
   // record at replay time.
   unsigned rec_flags = cudaEventRecordDefault;
@@ -292,6 +315,16 @@ salsc_status salsc_decode_step(const salsc_decode_desc* desc, const void* q, con
                                const void* Vc, const void* Pk, const void* Pv, void* out,
                                int32_t* idx_out, void* ws, size_t ws_bytes, salsc_stream stream) {
   return decode_step_impl(desc, q, Kc, Vc, Pk, Pv, out, idx_out, ws, ws_bytes, stream, nullptr, 0);
+}
+
+salsc_status salsc_decode_step_append(const salsc_decode_desc* desc, const void* K_new,
+                                      const void* V_new, const int64_t* rows_dev, const void* q,
+                                      void* Kc, void* Vc, const void* Pk, const void* Pv,
+                                      void* out, int32_t* idx_out, void* ws, size_t ws_bytes,
+                                      salsc_stream stream) {
+  const AppendArgs app{K_new, V_new, rows_dev};
+  return decode_step_impl(desc, q, Kc, Vc, Pk, Pv, out, idx_out, ws, ws_bytes, stream, nullptr, 0,
+                          &app);
 }
 
 salsc_status salsc_decode_step_timed(const salsc_decode_desc* desc, const void* q, const void* Kc,

@@ -23,7 +23,7 @@ WS_ALIGN = 256
 
 EXPORTS = (
     "salsc_compress", "salsc_decode_workspace_size", "salsc_decode_prepare", "salsc_decode_step",
-    "salsc_decode_step_timed", "salsc_decode_step_static_ws", "salsc_decode_launch_count", "salsc_append", "salsc_decode_read_flags", "salsc_status_string", "salsc_last_cuda_error", "salsc_version",
+    "salsc_decode_step_timed", "salsc_decode_step_static_ws", "salsc_decode_launch_count", "salsc_append", "salsc_decode_step_append", "salsc_decode_read_flags", "salsc_status_string", "salsc_last_cuda_error", "salsc_version",
 )
 
 
@@ -73,6 +73,9 @@ def _lib():
         lib.salsc_decode_prepare.argtypes = [dp, vp, sz, vp]
         lib.salsc_decode_step.restype = ctypes.c_int
         lib.salsc_decode_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.salsc_decode_step_append.restype = ctypes.c_int
+        lib.salsc_decode_step_append.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                                 vp]
         lib.salsc_append.restype = ctypes.c_int
         lib.salsc_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, ctypes.c_int, vp]
         lib.salsc_decode_launch_count.restype = ctypes.c_int32
@@ -182,6 +185,18 @@ def salsc_decode_step(desc: DecodeDesc, q, Kc, Vc, Pk, Pv, out, idx_out, ws, str
                                   _ptr(Pv), _ptr(out), _ptr(idx_out), _ptr(ws),
                                   ws.numel() * ws.element_size(), _stream(stream))
     _check(st, "salsc_decode_step")
+
+
+def salsc_decode_step_append(desc: DecodeDesc, K_new, V_new, rows, q, Kc, Vc, Pk, Pv, out, idx_out,
+                             ws, stream=None):
+    """salsc_append then salsc_decode_step in one call (rows: int64 device tensor)."""
+    if rows is None or rows.dtype != torch.int64 or not rows.is_cuda:
+        raise ValueError("rows must be an int64 device tensor")
+    st = _lib().salsc_decode_step_append(ctypes.byref(desc), _ptr(K_new), _ptr(V_new), _ptr(rows),
+                                         _ptr(q), _ptr(Kc), _ptr(Vc), _ptr(Pk), _ptr(Pv), _ptr(out),
+                                         _ptr(idx_out), _ptr(ws), ws.numel() * ws.element_size(),
+                                         _stream(stream))
+    _check(st, "salsc_decode_step_append")
 
 
 DECODE_KERNELS = ("latent_q", "score", "topk", "attend", "combine")

@@ -138,6 +138,29 @@ def test_append_validation_before_launch():
     assert call(batch=0) == salsc.SALSC_OK  # nothing to do, nothing launched
 
 
+def test_step_append_validation_before_launch():
+    lib = salsc.load()
+    vp = ctypes.c_void_p
+
+    class Dev:  # a device address that is never dereferenced
+        def data_ptr(self):
+            return 1 << 27
+
+    def call(n_kv_heads=8, **kw):
+        host = torch.tensor([0, 100, 250], dtype=torch.int64)
+        d = salsc.make_desc(2, n_kv_heads * 4 if n_kv_heads <= 8 else n_kv_heads, n_kv_heads, 128,
+                            256, 64, host, Dev(), None, 10000.0, 0.0, torch.bfloat16)
+        a = dict(K=vp(1 << 20), V=vp(1 << 21), rows=vp(1 << 26))
+        a.update(kw)
+        buf = [vp(1 << (28 + i)) for i in range(7)]
+        return lib.salsc_decode_step_append(ctypes.byref(d), a["K"], a["V"], a["rows"], *buf[:6],
+                                            None, buf[6], 1 << 30, None)
+
+    assert call(rows=None) == salsc.SALSC_ERR_INVALID_ARG
+    assert call(K=None, V=None) == salsc.SALSC_ERR_INVALID_ARG
+    assert call(n_kv_heads=128) == salsc.SALSC_ERR_UNSUPPORTED  # Hkv*d = 16384 > 8192
+
+
 def test_compress_validation_before_launch():
     lib = salsc.load()
     vp = ctypes.c_void_p

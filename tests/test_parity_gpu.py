@@ -316,6 +316,49 @@ def test_append_new_rows_match_the_oracle(wname, dt):
         assert (g[others] == fill).all()  # nothing else written
 
 
+def test_step_append_equals_append_then_step():
+    # the new token's rows written at each sequence's last row, then the step
+    # over the updated caches with the query at that token's position
+    w = W.Workload(name="gqa_app", batch=2, n_q_heads=8, n_kv_heads=2, head_dim=128, rank=128,
+                   top_k=64, seq_lens=(300, 201), dtype="bf16", rope_base=10000.0, low_rank=16,
+                   seed=92)
+    x = synth.decode_inputs(w)
+    offs = x["seq_offsets"].numpy()
+    lens = np.diff(offs)
+    new = synth.compress_inputs(w, rows=w.batch, seed=w.seed + 1)
+    K_new = new["K"][:, : w.n_kv_heads * w.head_dim].contiguous().to(DEV)
+    V_new = new["V"][:, : w.n_kv_heads * w.head_dim].contiguous().to(DEV)
+    rows = torch.from_numpy(offs[1:] - 1).to(DEV)
+    q_pos = torch.from_numpy((lens - 1).astype(np.int32))
+    t = {n: x[n].to(DEV) for n in ("q", "Pk", "Pv")}
+    dec = salsc.Decoder(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.rank, w.top_k, lens,
+                        rope_base=w.rope_base, dtype=torch.bfloat16, device=DEV, q_pos=q_pos)
+    res = []
+    for fused in (False, True):
+        Kc, Vc = x["Kc"].to(DEV), x["Vc"].to(DEV)
+        out = torch.empty_like(t["q"])
+        idx = torch.empty((w.batch, w.n_kv_heads, w.top_k), dtype=torch.int32, device=DEV)
+        if fused:
+            salsc.salsc_decode_step_append(dec.desc, K_new, V_new, rows, t["q"], Kc, Vc, t["Pk"],
+                                           t["Pv"], out, idx, dec.ws)
+        else:
+            salsc.salsc_append(K_new, V_new, t["Pk"], t["Pv"], Kc, Vc, rows)
+            dec.step(t["q"], Kc, Vc, t["Pk"], t["Pv"], out=out, idx_out=idx)
+        torch.cuda.synchronize()
+        res.append((Kc.cpu(), Vc.cpu(), out.cpu(), idx.cpu()))
+    assert dec.flags() == 0
+    for a_, b_ in zip(res[0], res[1]):
+        assert torch.equal(a_, b_)
+    # the oracle on the updated caches
+    Kc, Vc, out, idx = res[1]
+    x2 = dict(x, Kc=Kc, Vc=Vc)
+    p = problem_of(w, offs, q_pos.numpy())
+    ora = oracle.decode(p, x2["q"], x2["Kc"], x2["Vc"], x2["Pk"], x2["Pv"])
+    check_topk(p, idx.numpy(), ora)
+    given = oracle.attend_given_idx(p, x2["q"], x2["Kc"], x2["Vc"], x2["Pk"], x2["Pv"], idx.numpy())
+    assert max_rel_err(out.float().numpy(), given["out"]) <= TOL["bf16"]
+
+
 def test_append_one_half_and_batch_above_one_pass():
     w = W.MISTRAL_32K_B4
     B = 37  # more sequences than one pass of the kernel takes
