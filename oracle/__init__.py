@@ -48,6 +48,8 @@ class _Desc(ctypes.Structure):
         ("rope_base", ctypes.c_double),
         ("softmax_scale", ctypes.c_double),
         ("n_threads", ctypes.c_int32),
+        ("select_mode", ctypes.c_int32),
+        ("select_threshold", ctypes.c_double),
     ]
 
 
@@ -139,6 +141,7 @@ class Problem:
     rope_base: float = 10000.0
     softmax_scale: float = 0.0
     q_pos: np.ndarray | None = None  # int32 [B] or None
+    select_threshold: float | None = None  # None: top-k; else keep the top-k scores >= it
 
 
 def _desc(p: Problem, n_threads: int | None, keep: list) -> _Desc:
@@ -151,7 +154,9 @@ def _desc(p: Problem, n_threads: int | None, keep: list) -> _Desc:
     return _Desc(p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim, p.rank, p.top_k,
                  offs.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
                  qp.ctypes.data_as(_I32) if qp is not None else None,
-                 float(p.rope_base), float(p.softmax_scale), int(n_threads or default_threads()))
+                 float(p.rope_base), float(p.softmax_scale), int(n_threads or default_threads()),
+                 0 if p.select_threshold is None else 1,
+                 0.0 if p.select_threshold is None else float(p.select_threshold))
 
 
 def decode(p: Problem, q, Kc, Vc, Pk, Pv, n_threads: int | None = None) -> dict:

@@ -25,6 +25,10 @@
  *     sum of the raw latent scores of its G query heads;
  *   - top-k keeps k_b = min(k, n_b) tokens; ties go to the lower index;
  *     unused slots hold -1;
+ *   - threshold selection (select_mode 1, the alternative to Top-K the
+ *     page's key designs name): of those k_b tokens, the ones whose unit
+ *     score is below the threshold are dropped (a threshold alone is the
+ *     case k >= n_b); a head with no token left outputs zeros;
  *   - RoPE is the rotate-half pairing (i, i + d/2), theta_i = base^(-2i/d),
  *     cached token t sits at position t, the query at q_pos[b] (default n_b);
  *   - softmax scale 1/sqrt(head_dim) unless given.
@@ -56,6 +60,8 @@ typedef struct {
   double rope_base;
   double softmax_scale;       /* 0 -> 1/sqrt(head_dim) */
   int32_t n_threads;          /* <= 0 -> 1 */
+  int32_t select_mode;        /* 0: top-k; 1: top-k, then unit score >= select_threshold */
+  double select_threshold;
 } oracle_desc;
 
 /* ---------------------------------------------------------------------- */
@@ -240,12 +246,16 @@ static int decode_unit(decode_ctx* C, int32_t b, int32_t u) {
       double* dst = C->scores_out + off * U + (int64_t)u * nb;
       memcpy(dst, s_u, sizeof(double) * (size_t)nb);
     }
-    /* Top-k by exhaustive sort. */
+    /* Top-k by exhaustive sort; with a threshold, the sorted prefix whose
+     * scores reach it. */
     for (int64_t t = 0; t < nb; ++t) order[t] = (scored_token){s_u[t], t};
     qsort(order, (size_t)nb, sizeof(scored_token), cmp_scored);
-    for (int64_t j = 0; j < kb; ++j) sel[n_sel++] = order[j].t;
+    for (int64_t j = 0; j < kb; ++j) {
+      if (D->select_mode == 1 && !(order[j].s >= D->select_threshold)) break;
+      sel[n_sel++] = order[j].t;
+    }
     int32_t* io = C->idx_out + ((int64_t)b * U + u) * k;
-    for (int64_t j = 0; j < k; ++j) io[j] = j < kb ? (int32_t)order[j].t : -1;
+    for (int64_t j = 0; j < k; ++j) io[j] = j < n_sel ? (int32_t)sel[j] : -1;
     free(s_u);
     free(qlat);
     free(order);
@@ -332,7 +342,7 @@ static void* decode_worker(void* arg) {
 static int check_desc(const oracle_desc* D) {
   if (!D || !D->seq_offsets) return ORACLE_ERR_ARG;
   if (D->batch < 1 || D->n_q_heads < 1 || D->n_kv_heads < 1 || D->head_dim < 2 ||
-      D->rank < 1 || D->top_k < 1)
+      D->rank < 1 || D->top_k < 1 || D->select_mode < 0 || D->select_mode > 1)
     return ORACLE_ERR_ARG;
   if (D->head_dim % 2 || D->n_q_heads % D->n_kv_heads) return ORACLE_ERR_ARG;
   if (D->seq_offsets[0] != 0) return ORACLE_ERR_ARG;

@@ -33,6 +33,7 @@ MUTANTS = {
     "sequence_offset": ("const double* Kc_b = C->Kc + off * r;", "const double* Kc_b = C->Kc;"),
     "compress_transposed": ("acc += x[h] * j->P[(int64_t)h * j->r + c];", "acc += x[h] * j->P[(int64_t)c * j->hid + h];"),
     "bf16_ties_away": ("double y = ldexp(nearbyint(ldexp(m, 8)), e - 8);", "double y = ldexp(round(ldexp(m, 8)), e - 8);"),
+    "threshold_strict": ("!(order[j].s >= D->select_threshold)", "!(order[j].s > D->select_threshold)"),
     "bf16_width": ("double y = ldexp(nearbyint(ldexp(m, 8)), e - 8);", "double y = ldexp(nearbyint(ldexp(m, 9)), e - 9);"),
 }
 

@@ -268,6 +268,63 @@ def test_topk_equals_exhaustive_sort_with_ties(oracle_lib):
             assert (res["idx"][b, u, kb:] == -1).all()
 
 
+def threshold_problem(oracle, p, tau):
+    return oracle.Problem(p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim, p.rank, p.top_k,
+                          p.seq_offsets, p.rope_base, p.softmax_scale, p.q_pos, tau)
+
+
+def test_threshold_selection_equals_filtered_exhaustive_sort(oracle_lib):
+    """Threshold selection (score >= tau among the top-k) against numpy on exact
+    small-integer scores, with tau equal to a score that several tokens share."""
+    rng = np.random.default_rng(21)
+    B, Hq, Hkv, d, r = 2, 4, 2, 4, 3
+    hid, lens = 8, [40, 33]
+    q = rng.integers(-2, 3, (B, Hq, d)).astype(np.float64)
+    Kc = rng.integers(-2, 3, (73, r)).astype(np.float64)
+    Vc = rng.standard_normal((73, r))
+    Pk = rng.integers(-1, 2, (hid, r)).astype(np.float64)
+    Pv = rng.standard_normal((hid, r))
+    ref = naive_scores(q, Kc, Pk, problem(oracle_lib, B, Hq, Hkv, d, r, 1, lens).seq_offsets, Hkv)
+    checked = 0
+    for k in (5, 17, 40):
+        p = problem(oracle_lib, B, Hq, Hkv, d, r, k, lens)
+        for (b, u), sc in ref.items():
+            nb = lens[b]
+            order = np.lexsort((np.arange(nb), -sc))
+            kb = min(k, nb)
+            for tau in (sc[order[kb // 2]], sc[order[0]] + 0.5, -1e300):
+                res = oracle_lib.decode(threshold_problem(oracle_lib, p, tau), q, Kc, Vc, Pk, Pv)
+                keep = [t for t in order[:kb] if sc[t] >= tau]
+                np.testing.assert_array_equal(res["idx"][b, u, :len(keep)], keep)
+                assert (res["idx"][b, u, len(keep):] == -1).all()
+                checked += 1
+    assert checked == 3 * 3 * 4
+
+
+def test_threshold_extremes(oracle_lib):
+    """tau = -inf is top-k; tau above every score keeps nothing and outputs zeros;
+    the output equals the attention over the kept set."""
+    rng = np.random.default_rng(22)
+    Hq, Hkv, d, r = 4, 2, 8, 8
+    lens = [30, 17]
+    q = rng.standard_normal((2, Hq, d))
+    Kc, Vc = rng.standard_normal((47, r)), rng.standard_normal((47, r))
+    Pk, Pv = random_orthogonal(rng, 16, r), random_orthogonal(rng, 16, r)
+    p = problem(oracle_lib, 2, Hq, Hkv, d, r, 20, lens)
+    base = oracle_lib.decode(p, q, Kc, Vc, Pk, Pv)
+    low = oracle_lib.decode(threshold_problem(oracle_lib, p, -math.inf), q, Kc, Vc, Pk, Pv)
+    np.testing.assert_array_equal(low["idx"], base["idx"])
+    np.testing.assert_array_equal(low["out"], base["out"])
+    high = oracle_lib.decode(threshold_problem(oracle_lib, p, 1e300), q, Kc, Vc, Pk, Pv)
+    assert (high["idx"] == -1).all()
+    assert (high["out"] == 0).all()
+    mid_tau = float(np.median(base["scores"]))
+    mid = oracle_lib.decode(threshold_problem(oracle_lib, p, mid_tau), q, Kc, Vc, Pk, Pv)
+    assert (mid["idx"] >= 0).sum() < (base["idx"] >= 0).sum()
+    given = oracle_lib.attend_given_idx(p, q, Kc, Vc, Pk, Pv, mid["idx"])
+    np.testing.assert_allclose(mid["out"], given["out"], atol=1e-13)
+
+
 def test_softmax_weights_sum_to_one(oracle_lib):
     rng = np.random.default_rng(12)
     B, Hq, Hkv, d, r = 2, 4, 4, 16, 16
