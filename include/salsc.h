@@ -96,6 +96,11 @@ typedef struct {
   double rope_base;                /* RoPE base (10000, 500000, ...) > 1 */
   float softmax_scale;             /* 0 -> 1/sqrt(head_dim) */
   salsc_dtype dtype;               /* storage type of q, Kc, Vc, Pk, Pv and out */
+  int32_t select_mode;             /* 0: top-k; 1: threshold selection: of the top-k tokens,
+                                      those whose unit score is below select_threshold are
+                                      dropped (slots left over hold -1; a head with no token
+                                      left outputs zeros) */
+  float select_threshold;          /* the threshold of select_mode 1 (not NaN) */
 } salsc_decode_desc;
 
 /*

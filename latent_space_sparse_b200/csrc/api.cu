@@ -84,6 +84,18 @@ salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
   p.topk_slice = (int)((n_max + c - 1) / c);
   if (p.topk_slice > kTopkMaxSlice) return SALSC_ERR_UNSUPPORTED;  // slice in smem
   p.topk_threads = (int64_t)p.B * p.U * c > kTopkTargetCtas ? 256 : 1024;
+  // threshold selection: keys (order-preserving bit patterns of the fp32
+  // scores) below the threshold's are dropped; 0 keeps every key
+  if (D->select_mode != 0 && D->select_mode != 1) return SALSC_ERR_INVALID_ARG;
+  p.topk_kthr = 0u;
+  if (D->select_mode == 1) {
+    if (isnan(D->select_threshold)) return SALSC_ERR_INVALID_ARG;
+    float f = D->select_threshold;
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if (u == 0x80000000u) u = 0u;  // -0 is +0
+    p.topk_kthr = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  }
   const int64_t k_eff = D->top_k < n_max ? D->top_k : n_max;
   p.attend_tc = salsc::attend_tc_supported(p);
   if (p.attend_tc) {

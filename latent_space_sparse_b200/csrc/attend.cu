@@ -94,7 +94,7 @@ attend_simt_kernel(const T* __restrict__ q, const T* __restrict__ Kc, const T* _
       int t = -1;
       if (jt + tid < j1) {
         t = uidx[jt + tid];
-        if (t < 0 || t >= nb) {
+        if (t < -1 || t >= nb) {  // -1: no token (a slot threshold selection left empty)
           atomicOr(flags, FLAG_BAD_INDEX);
           t = -1;
         }

@@ -119,14 +119,15 @@ struct UnitTileCursor {
 
 
 // Token of row `row` of the cursor's tile, or -1 past the unit's k_b kept
-// tokens; an index outside [0, n_b) raises FLAG_BAD_INDEX and reads as -1.
+// tokens or on -1 (a slot threshold selection left empty); any other index
+// outside [0, n_b) raises FLAG_BAD_INDEX and reads as -1.
 __device__ __forceinline__ int row_token(const AttendTcParams& P, const UnitTileCursor& c,
                                          int row) {
   const int64_t jj = (int64_t)c.slot * kTile + row;
   int t = -1;
   if (jj < c.kb) {
     t = P.idx[((int64_t)c.b * P.U + c.u) * P.k + jj];
-    if (t < 0 || t >= c.nb) {
+    if (t < -1 || t >= c.nb) {  // -1: no token (a slot threshold selection left empty)
       atomicOr(P.flags, FLAG_BAD_INDEX);
       t = -1;
     }

@@ -43,6 +43,7 @@ struct DecodePlan {
   int topk_cluster;     // CTAs per selection unit in the top-k kernel
   int topk_slice;       // max keys per top-k CTA
   int topk_threads;     // threads per top-k CTA (1024, or 256 for many small units)
+  uint32_t topk_kthr;   // threshold selection: order key of the threshold (0: plain top-k)
   int splits;           // partial-result slots per head (attention CTAs or tiles per unit)
   int chunk;            // kept tokens per slot
   bool attend_tc;       // tensor-core attention path (tiles of 128 kept tokens)

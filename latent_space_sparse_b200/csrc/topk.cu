@@ -111,7 +111,8 @@ __device__ __forceinline__ void find_digit(Cnt cnt, uint32_t target, int nbins, 
 template <bool kCluster, int kThreads>
 __global__ void __launch_bounds__(kThreads)
 topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_off,
-            const uint32_t* __restrict__ krange, int32_t* __restrict__ idx_out, int U, int k) {
+            const uint32_t* __restrict__ krange, int32_t* __restrict__ idx_out, int U, int k,
+            uint32_t kthr) {
   constexpr int kWarps = kThreads / 32;
   cg::cluster_group cluster = cg::this_cluster();
   const int C = kCluster ? (int)cluster.num_blocks() : 1;
@@ -153,11 +154,15 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
   const int s0 = warp * seg, s1 = min(s0 + seg, n_loc);
   const uint32_t lt_mask = (1u << lane) - 1u;
   int32_t* out = idx_out + ((int64_t)b * U + u) * k;
+  // Threshold selection (kthr > 0): keys below kthr are not kept, so the
+  // kept tokens are not all k_b; every slot starts at -1 and the kept ones are
+  // written over it after a cluster barrier.
+  const bool keep_all = kb == nb && kthr == 0u;
   // From here on the other CTAs of the cluster may add into this CTA's zeroed
   // cluster histogram (they wait for this arrival before they do).
-  if (kCluster && kb != nb) cluster_arrive();
+  if (kCluster && !keep_all) cluster_arrive();
   grid_dependency_wait();  // the scores and their range come from the previous kernel
-  if (kb == nb) {
+  if (keep_all) {
     // keep every token, in index order
     for (int i = tid; i < n_loc; i += kThreads) out[lo + i] = (int32_t)(lo + i);
     if (rank == 0)
@@ -190,6 +195,10 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
         if (lin) atomicAdd(&hist[0][linear_bin(key, fmin, scale)], 1u);
       }
     }
+  }
+  if (kthr != 0u) {
+    const int64_t j0 = (int64_t)k * rank / C, j1 = (int64_t)k * (rank + 1) / C;
+    for (int64_t j = j0 + tid; j < j1; j += kThreads) out[j] = -1;
   }
   if (kCluster) cluster_wait();  // every CTA's cluster histogram is zeroed
   bool fast = lin;
@@ -231,7 +240,7 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
       const bool valid = i < s1;
       const uint32_t key = valid ? keys[i] : 0u;
       const int bin = linear_bin(key, fmin, scale);
-      const bool gt = valid && bin > bstar, cand = valid && bin == bstar;
+      const bool gt = valid && bin > bstar && key >= kthr, cand = valid && bin == bstar;
       const uint32_t bg = __ballot_sync(0xffffffffu, gt);
       if (cand) {
         const uint32_t slot = (uint32_t)rank * cap + atomicAdd(&s_ncand, 1u);
@@ -300,7 +309,7 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
           }
         }
         better = __reduce_add_sync(0xffffffffu, better);
-        if (lane == 0 && better < need) out[ngt_all + better] = (int32_t)it_;
+        if (lane == 0 && better < need && kt >= kthr) out[ngt_all + better] = (int32_t)it_;
       }
     }
     // ---- pass 3: the packed indices of this warp's keys above the boundary bin
@@ -366,8 +375,8 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
   uint32_t cgt = 0u, ceq = 0u;
   for (int i = s0 + lane; i < s1; i += 32) {
     const uint32_t key = keys[i];
-    cgt += key > T;
-    ceq += key == T;
+    cgt += key > T && key >= kthr;
+    ceq += key == T && key >= kthr;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -426,8 +435,8 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
     const int i = c0 + lane;
     const bool valid = i < s1;
     const uint32_t key = valid ? keys[i] : 0u;
-    const bool g = valid && key > T;
-    const bool e = valid && key == T && need_eq > 0u;
+    const bool g = valid && key > T && key >= kthr;
+    const bool e = valid && key == T && key >= kthr && need_eq > 0u;
     const uint32_t bg = __ballot_sync(0xffffffffu, g);
     const uint32_t be = __ballot_sync(0xffffffffu, e);
     if (g) out[run_gt + __popc(bg & lt_mask)] = (int32_t)(lo + i);
@@ -466,7 +475,8 @@ cudaError_t launch_tk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) 
   cfg.attrs = attr;
   cfg.numAttrs = kCluster ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, topk_kernel<kCluster, kThreads>, (const float*)a.scores,
-                            (const int64_t*)a.seq_off, (const uint32_t*)a.krange, a.idx, p.U, p.k);
+                            (const int64_t*)a.seq_off, (const uint32_t*)a.krange, a.idx, p.U, p.k,
+                            p.topk_kthr);
 }
 
 }  // namespace

@@ -50,6 +50,8 @@ class DecodeDesc(ctypes.Structure):
         ("rope_base", ctypes.c_double),
         ("softmax_scale", ctypes.c_float),
         ("dtype", ctypes.c_int),
+        ("select_mode", ctypes.c_int32),
+        ("select_threshold", ctypes.c_float),
     ]
 
 
@@ -157,9 +159,10 @@ def salsc_append(K_new, V_new, Pk, Pv, Kc, Vc, rows, stream=None):
 
 def make_desc(batch, n_q_heads, n_kv_heads, head_dim, rank, top_k, seq_offsets_host,
               seq_offsets_dev=None, q_pos_dev=None, rope_base=10000.0, softmax_scale=0.0,
-              dtype=torch.bfloat16):
+              dtype=torch.bfloat16, select_threshold=None):
     """Build a DecodeDesc; ``seq_offsets_host`` must be a contiguous CPU int64 tensor kept alive
-    by the caller (the descriptor points into it)."""
+    by the caller (the descriptor points into it).  ``select_threshold``: None for top-k, else
+    threshold selection (of the top-k tokens, those with a unit score below it are dropped)."""
     assert seq_offsets_host.dtype == torch.int64 and not seq_offsets_host.is_cuda
     assert seq_offsets_host.is_contiguous()
     return DecodeDesc(
@@ -167,7 +170,9 @@ def make_desc(batch, n_q_heads, n_kv_heads, head_dim, rank, top_k, seq_offsets_h
         ctypes.cast(seq_offsets_host.data_ptr(), ctypes.POINTER(ctypes.c_int64)),
         None if seq_offsets_dev is None else seq_offsets_dev.data_ptr(),
         None if q_pos_dev is None else q_pos_dev.data_ptr(),
-        float(rope_base), float(softmax_scale), _dtype_code(dtype))
+        float(rope_base), float(softmax_scale), _dtype_code(dtype),
+        0 if select_threshold is None else 1,
+        0.0 if select_threshold is None else float(select_threshold))
 
 
 def salsc_decode_workspace_size(desc: DecodeDesc) -> int:
@@ -261,7 +266,7 @@ class Decoder:
 
     def __init__(self, batch, n_q_heads, n_kv_heads, head_dim, rank, top_k, seq_lens,
                  rope_base=10000.0, softmax_scale=0.0, dtype=torch.bfloat16, device="cuda",
-                 q_pos=None):
+                 q_pos=None, select_threshold=None):
         lens = [int(x) for x in seq_lens]
         offs = [0]
         for n in lens:
@@ -274,7 +279,7 @@ class Decoder:
         self.dtype = dtype
         self.desc = make_desc(batch, n_q_heads, n_kv_heads, head_dim, rank, top_k,
                               self.seq_offsets_host, self.seq_offsets_dev, self.q_pos, rope_base,
-                              softmax_scale, dtype)
+                              softmax_scale, dtype, select_threshold)
         nbytes = salsc_decode_workspace_size(self.desc)
         if nbytes == 0:
             raise SalscError(SALSC_ERR_INVALID_ARG, "salsc_decode_workspace_size")

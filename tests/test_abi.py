@@ -138,6 +138,18 @@ def test_append_validation_before_launch():
     assert call(batch=0) == salsc.SALSC_OK  # nothing to do, nothing launched
 
 
+def test_select_mode_validation():
+    d = desc([0, 1000])
+    assert salsc.salsc_decode_workspace_size(d) > 0
+    d.select_mode = 2
+    assert salsc.salsc_decode_workspace_size(d) == 0  # invalid descriptor
+    d.select_mode = 1
+    d.select_threshold = float("nan")
+    assert salsc.salsc_decode_workspace_size(d) == 0
+    d.select_threshold = -1e30
+    assert salsc.salsc_decode_workspace_size(d) > 0
+
+
 def test_step_append_validation_before_launch():
     lib = salsc.load()
     vp = ctypes.c_void_p

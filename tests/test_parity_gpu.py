@@ -22,13 +22,14 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def gpu_decode(w, x, top_k=None, q_pos=None):
+def gpu_decode(w, x, top_k=None, q_pos=None, threshold=None):
     offs = x["seq_offsets"].numpy()
     lens = np.diff(offs)
     k = top_k or w.top_k
     dec = salsc.Decoder(len(lens), w.n_q_heads, w.n_kv_heads, w.head_dim, w.rank, k, lens,
                         rope_base=w.rope_base, dtype=synth.torch_dtype(w.dtype), device=DEV,
-                        q_pos=None if q_pos is None else torch.as_tensor(q_pos))
+                        q_pos=None if q_pos is None else torch.as_tensor(q_pos),
+                        select_threshold=threshold)
     t = {n: x[n].to(DEV) for n in ("q", "Kc", "Vc", "Pk", "Pv")}
     idx = torch.full((len(lens), w.n_kv_heads, k), -7, dtype=torch.int32, device=DEV)
     out = dec.step(t["q"], t["Kc"], t["Vc"], t["Pk"], t["Pv"], idx_out=idx)
@@ -189,6 +190,72 @@ def test_separate_merge_kernel_when_the_split_is_wider():
                    rope_base=10000.0, low_rank=32, seed=93)
     assert launches(w) == len(salsc.DECODE_KERNELS)
     check(w, synth.decode_inputs(w))
+
+
+def check_threshold(w, x, tau, top_k=None):
+    """Threshold selection: the kept set is the oracle's up to tokens whose score lies within
+    the tie band of the k-th score or of the threshold; the output matches the oracle over
+    the GPU's kept set."""
+    out, idx = gpu_decode(w, x, top_k, threshold=tau)
+    p = problem_of(w, x["seq_offsets"].numpy(), None, top_k)
+    p.select_threshold = tau
+    ora = oracle.decode(p, x["q"], x["Kc"], x["Vc"], x["Pk"], x["Pv"])
+    k = p.top_k
+    n_kept = 0
+    for b in range(p.batch):
+        for u in range(p.n_kv_heads):
+            s = oracle.unit_scores(p, ora["scores"], b, u)
+            g = idx[b, u]
+            gk = g[g >= 0]
+            n_kept += gk.size
+            assert (g[gk.size:] == -1).all(), "kept slots are not a prefix"
+            assert len(np.unique(gk)) == gk.size
+            o = ora["idx"][b, u]
+            o = o[o >= 0]
+            lim = 1e-4 * np.abs(s).max()
+            for t in np.setxor1d(gk, o):
+                near_tau = abs(s[t] - tau) <= lim
+                kth = np.sort(s)[::-1][min(k, s.size) - 1]
+                assert near_tau or abs(s[t] - kth) <= lim, (b, u, t, s[t], tau)
+            assert all(s[t] >= tau - lim for t in gk)
+    given = oracle.attend_given_idx(p, x["q"], x["Kc"], x["Vc"], x["Pk"], x["Pv"], idx)
+    assert max_rel_err(out, given["out"]) <= TOL[w.dtype] or np.abs(given["out"]).max() == 0
+    if np.abs(given["out"]).max() == 0:
+        assert np.abs(out).max() == 0
+    return n_kept, ora
+
+
+@pytest.mark.parametrize("wname,frac", [("MISTRAL_32K_B4", 0.5), ("MISTRAL_32K_B4", 0.97),
+                                        ("TINY_F32", 0.6)])
+def test_threshold_selection(wname, frac):
+    # tau at a quantile of the top-k scores: part of the top-k set is dropped
+    w = getattr(W, wname)
+    x = synth.decode_inputs(w, seq_lens=(3000, 1500)) if w.dtype == "bf16" else synth.decode_inputs(w)
+    k = 256 if w.dtype == "bf16" else w.top_k
+    p = problem_of(w, x["seq_offsets"].numpy(), None, k)
+    ora = oracle.decode(p, x["q"], x["Kc"], x["Vc"], x["Pk"], x["Pv"])
+    kept = [oracle.unit_scores(p, ora["scores"], b, u)[t] for b in range(p.batch)
+            for u in range(p.n_kv_heads) for t in ora["idx"][b, u] if t >= 0]
+    tau = float(np.quantile(kept, frac))
+    n_kept, ora = check_threshold(w, x, tau, top_k=k)
+    assert 0 < n_kept < (ora["idx"] >= 0).size
+
+
+def test_threshold_above_every_score_keeps_nothing():
+    w = W.MISTRAL_32K_B4
+    x = synth.decode_inputs(w, seq_lens=(700, 300))
+    out, idx = gpu_decode(w, x, top_k=128, threshold=1e30)
+    assert (idx == -1).all()
+    assert np.abs(out).max() == 0
+
+
+def test_threshold_minus_infinity_is_top_k():
+    w = W.MISTRAL_32K_B4
+    x = synth.decode_inputs(w, seq_lens=(900, 450))
+    out0, idx0 = gpu_decode(w, x, top_k=200)
+    out1, idx1 = gpu_decode(w, x, top_k=200, threshold=-np.inf)
+    np.testing.assert_array_equal(np.sort(idx0, axis=-1), np.sort(idx1, axis=-1))
+    np.testing.assert_array_equal(out0, out1)
 
 
 def test_small_rank_f32():
