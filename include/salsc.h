@@ -262,6 +262,36 @@ salsc_status salsc_append(const void* K_new, const void* V_new, const void* Pk, 
                           int32_t hidden, int32_t rank, salsc_dtype dtype, salsc_stream stream);
 
 /*
+ * Learned projection (SALS page, key designs: a low-rank projection from the
+ * SVD / PCA of the keys): P [hidden][rank] with orthonormal columns spanning
+ * the dominant rank-dimensional right-singular subspace of a calibration
+ * matrix X [n][hidden] (keys for Pk, values for Pv; pre-RoPE keys).  The decode
+ * path uses P only through P P^T, so any orthonormal basis of the subspace is
+ * equivalent; this one is the result of subspace iteration on the Gram matrix
+ * C = X^T X from the random start omega:
+ *     V_0 = orth(omega),  V_{i+1} = orth(C V_i) for i < iters,  P = V_iters
+ * (orth: Cholesky-QR twice; all arithmetic fp64).  The subspace error falls
+ * as (sigma_{rank+1} / sigma_rank)^(2 iters) of X's singular values.
+ *
+ *   X       [n][hidden]      calibration rows, dtype; n >= rank
+ *   omega   [hidden][rank]   fp32 device array: the random start (e.g.
+ *                            standard normal entries, drawn by the caller)
+ *   P_out   [hidden][rank]   output, dtype
+ *   ws      >= salsc_fit_workspace_size(hidden, rank) bytes of device memory,
+ *           256-byte aligned (about 8*hidden^2 bytes); word 0 holds flags,
+ *           read with salsc_decode_read_flags: bit 2 set when a Cholesky pivot
+ *           was not positive (rank-deficient X or omega; P is then unreliable)
+ * Requirements: 1 <= rank <= min(hidden, 1024), iters >= 0.  Stream-ordered,
+ * allocates nothing.  Errors: INVALID_ARG (shapes, null pointers, dtype),
+ * UNSUPPORTED (rank > 1024), WORKSPACE, CUDA.
+ */
+size_t salsc_fit_workspace_size(int32_t hidden, int32_t rank);
+salsc_status salsc_fit_projection(const void* X, int64_t n, int32_t hidden, int32_t rank,
+                                  const float* omega, int32_t iters, void* P_out,
+                                  salsc_dtype dtype, void* ws, size_t ws_bytes,
+                                  salsc_stream stream);
+
+/*
  * Device-side anomaly flags recorded in a workspace since salsc_decode_prepare
  * (bit 0: a selected index fell outside its sequence; bit 1: a pipeline wait
  * gave up after its iteration limit).  Copies one word to *flags_host and

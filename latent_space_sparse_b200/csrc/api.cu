@@ -24,6 +24,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 constexpr int kScoreTile = 128;
+constexpr int kFitMaxRank = 1024;  // learned projections: columns (one-CTA factorisations)
 constexpr int kTopkTargetCtas = 148;    // top-k CTAs aimed at (one per SM)
 constexpr int kTopkMinSlice = 4096;     // keys per CTA at which the cluster stops growing
 constexpr int kTopkMaxSlice = 40960;    // keys per CTA in shared memory (160 KiB)
@@ -197,6 +198,28 @@ salsc_status salsc_decode_prepare(const salsc_decode_desc* desc, void* ws, size_
   cudaError_t e = cudaMemsetAsync((char*)ws + p.off_flags, 0, 16, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e);
   return SALSC_OK;
+}
+
+size_t salsc_fit_workspace_size(int32_t hidden, int32_t rank) {
+  if (hidden < 1 || rank < 1 || rank > hidden || rank > kFitMaxRank) return 0;
+  return salsc::fit_workspace_size(hidden, rank);
+}
+
+salsc_status salsc_fit_projection(const void* X, int64_t n, int32_t hidden, int32_t rank,
+                                  const float* omega, int32_t iters, void* P_out,
+                                  salsc_dtype dtype, void* ws, size_t ws_bytes,
+                                  salsc_stream stream) {
+  if (dtype != SALSC_F32 && dtype != SALSC_BF16) return SALSC_ERR_INVALID_ARG;
+  if (!X || !omega || !P_out || hidden < 1 || rank < 1 || rank > hidden || n < rank ||
+      n > INT32_MAX || iters < 0)
+    return SALSC_ERR_INVALID_ARG;
+  if (rank > kFitMaxRank) return SALSC_ERR_UNSUPPORTED;
+  if (!ws || ((uintptr_t)ws % salsc::kWsAlign) != 0 ||
+      ws_bytes < salsc::fit_workspace_size(hidden, rank))
+    return SALSC_ERR_WORKSPACE;
+  const cudaError_t e = salsc::fit_projection(X, n, hidden, rank, omega, iters, P_out, dtype, ws,
+                                              (cudaStream_t)stream);
+  return e == cudaSuccess ? SALSC_OK : cuda_fail(e);
 }
 
 salsc_status salsc_decode_read_flags(void* ws, size_t ws_bytes, uint32_t* flags_host,

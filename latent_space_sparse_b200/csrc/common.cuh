@@ -86,6 +86,9 @@ cudaError_t launch_attend(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
 cudaError_t launch_combine(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 bool attend_tc_supported(const DecodePlan& p);
 int attend_merge_cluster(const DecodePlan& p);  // 0: merge kernel; else CTAs per unit
+size_t fit_workspace_size(int64_t hidden, int64_t rank);
+cudaError_t fit_projection(const void* X, int64_t n, int hidden, int rank, const float* omega,
+                           int iters, void* P_out, salsc_dtype dt, void* ws, cudaStream_t s);
 int attend_tc_grid(const DecodePlan& p);  // CTAs of the tensor-core attention (tile partition)
 bool combine_supported(const DecodePlan& p);
 cudaError_t launch_attend_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);

@@ -23,7 +23,8 @@ WS_ALIGN = 256
 
 EXPORTS = (
     "salsc_compress", "salsc_decode_workspace_size", "salsc_decode_prepare", "salsc_decode_step",
-    "salsc_decode_step_timed", "salsc_decode_step_static_ws", "salsc_decode_launch_count", "salsc_append", "salsc_decode_step_append", "salsc_decode_read_flags", "salsc_status_string", "salsc_last_cuda_error", "salsc_version",
+    "salsc_decode_step_timed", "salsc_decode_step_static_ws", "salsc_decode_launch_count", "salsc_append", "salsc_decode_step_append", "salsc_fit_workspace_size",
+    "salsc_fit_projection", "salsc_decode_read_flags", "salsc_status_string", "salsc_last_cuda_error", "salsc_version",
 )
 
 
@@ -78,6 +79,10 @@ def _lib():
         lib.salsc_decode_step_append.restype = ctypes.c_int
         lib.salsc_decode_step_append.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                                  vp]
+        lib.salsc_fit_workspace_size.restype = sz
+        lib.salsc_fit_workspace_size.argtypes = [i32, i32]
+        lib.salsc_fit_projection.restype = ctypes.c_int
+        lib.salsc_fit_projection.argtypes = [vp, i64, i32, i32, vp, i32, vp, ctypes.c_int, vp, sz, vp]
         lib.salsc_append.restype = ctypes.c_int
         lib.salsc_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, ctypes.c_int, vp]
         lib.salsc_decode_launch_count.restype = ctypes.c_int32
@@ -155,6 +160,27 @@ def salsc_append(K_new, V_new, Pk, Pv, Kc, Vc, rows, stream=None):
     st = _lib().salsc_append(_ptr(K_new), _ptr(V_new), _ptr(Pk), _ptr(Pv), _ptr(Kc), _ptr(Vc),
                              _ptr(rows), batch, hid, r, _dtype_code(x.dtype), _stream(stream))
     _check(st, "salsc_append")
+
+
+FLAG_FIT_NOT_SPD = 4
+
+
+def salsc_fit_projection(X, rank, omega, iters, out=None, stream=None):
+    """Orthonormal basis [hidden][rank] of the dominant right-singular subspace of X [n][hidden]
+    (subspace iteration from omega, fp32 [hidden][rank]); returns (P, flags)."""
+    n, hidden = X.shape
+    if omega.dtype != torch.float32 or tuple(omega.shape) != (hidden, rank):
+        raise ValueError("omega must be float32 [hidden][rank]")
+    nbytes = int(_lib().salsc_fit_workspace_size(hidden, rank))
+    if nbytes == 0:
+        raise ValueError("salsc_fit_workspace_size: unsupported shape")
+    ws = alloc_workspace(nbytes, X.device)
+    P = torch.empty((hidden, rank), dtype=X.dtype, device=X.device) if out is None else out
+    st = _lib().salsc_fit_projection(_ptr(X), n, hidden, rank, _ptr(omega), iters, _ptr(P),
+                                     _dtype_code(X.dtype), _ptr(ws), ws.numel() * ws.element_size(),
+                                     _stream(stream))
+    _check(st, "salsc_fit_projection")
+    return P, salsc_decode_read_flags(ws, stream)
 
 
 def make_desc(batch, n_q_heads, n_kv_heads, head_dim, rank, top_k, seq_offsets_host,

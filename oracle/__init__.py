@@ -182,6 +182,16 @@ def decode(p: Problem, q, Kc, Vc, Pk, Pv, n_threads: int | None = None) -> dict:
     return {"idx": idx, "scores": scores, "probs": probs, "out": out}
 
 
+def fit_subspace(X, rank: int) -> np.ndarray:
+    """Learned projection (SALS page, key designs: a low-rank projection from the SVD of the
+    keys): the top-``rank`` right singular vectors of X [n][hidden] as columns, [hidden][rank],
+    fp64.  Any orthonormal basis of the same subspace is an equivalent projection (the decode
+    path uses P only through P P^T), so results are compared as projectors."""
+    x = _f64(X)
+    _, _, vt = np.linalg.svd(x, full_matrices=False)
+    return np.ascontiguousarray(vt[:rank].T)
+
+
 def unit_scores(p: Problem, scores: np.ndarray, b: int, u: int) -> np.ndarray:
     """View of the packed score vector of unit (b, u)."""
     off = int(p.seq_offsets[b])

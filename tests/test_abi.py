@@ -138,6 +138,29 @@ def test_append_validation_before_launch():
     assert call(batch=0) == salsc.SALSC_OK  # nothing to do, nothing launched
 
 
+def test_fit_validation_before_launch():
+    lib = salsc.load()
+    vp = ctypes.c_void_p
+    assert lib.salsc_fit_workspace_size(512, 64) >= 8 * 512 * 512
+    assert lib.salsc_fit_workspace_size(64, 65) == 0     # rank > hidden
+    assert lib.salsc_fit_workspace_size(4096, 2048) == 0  # rank > 1024
+    ws = vp(1 << 24)
+
+    def call(X=vp(1 << 20), n=1000, hidden=512, rank=64, omega=vp(1 << 21), iters=4,
+             P=vp(1 << 22), dtype=1, ws=ws, ws_bytes=1 << 30):
+        return lib.salsc_fit_projection(X, n, hidden, rank, omega, iters, P, dtype, ws, ws_bytes,
+                                        None)
+
+    assert call(X=None) == salsc.SALSC_ERR_INVALID_ARG
+    assert call(omega=None) == salsc.SALSC_ERR_INVALID_ARG
+    assert call(n=10) == salsc.SALSC_ERR_INVALID_ARG      # n < rank
+    assert call(iters=-1) == salsc.SALSC_ERR_INVALID_ARG
+    assert call(dtype=9) == salsc.SALSC_ERR_INVALID_ARG
+    assert call(rank=2048, hidden=4096, n=5000) == salsc.SALSC_ERR_UNSUPPORTED
+    assert call(ws=vp((1 << 24) + 8)) == salsc.SALSC_ERR_WORKSPACE  # misaligned
+    assert call(ws_bytes=1000) == salsc.SALSC_ERR_WORKSPACE
+
+
 def test_select_mode_validation():
     d = desc([0, 1000])
     assert salsc.salsc_decode_workspace_size(d) > 0

@@ -325,6 +325,28 @@ def test_threshold_extremes(oracle_lib):
     np.testing.assert_allclose(mid["out"], given["out"], atol=1e-13)
 
 
+def spectrum_matrix(rng, n, h, sig):
+    """X = U diag(sig) V^T with known orthonormal U [n x h'] and orthogonal V [h x h]."""
+    k = len(sig)
+    U = random_orthogonal(rng, n, k)
+    V = random_orthogonal(rng, h)
+    return (U * sig) @ V[:, :k].T, V
+
+
+def test_fit_subspace_recovers_a_known_dominant_subspace(oracle_lib):
+    rng = np.random.default_rng(31)
+    n, h, r = 300, 40, 6
+    sig = np.concatenate([np.linspace(10.0, 5.0, r), np.linspace(1.0, 0.1, h - r)])
+    X, V = spectrum_matrix(rng, n, h, sig)
+    P = oracle_lib.fit_subspace(X, r)
+    assert P.shape == (h, r)
+    np.testing.assert_allclose(P.T @ P, np.eye(r), atol=1e-12)
+    np.testing.assert_allclose(P @ P.T, V[:, :r] @ V[:, :r].T, atol=1e-10)
+    # scaling and row order leave the subspace alone
+    Q = oracle_lib.fit_subspace(3.5 * X[rng.permutation(n)], r)
+    np.testing.assert_allclose(Q @ Q.T, P @ P.T, atol=1e-10)
+
+
 def test_softmax_weights_sum_to_one(oracle_lib):
     rng = np.random.default_rng(12)
     B, Hq, Hkv, d, r = 2, 4, 4, 16, 16

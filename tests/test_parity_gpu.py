@@ -258,6 +258,29 @@ def test_threshold_minus_infinity_is_top_k():
     np.testing.assert_array_equal(out0, out1)
 
 
+@pytest.mark.parametrize("dt,n,h,r", [("f32", 2048, 512, 64), ("bf16", 3000, 1024, 256),
+                                       ("f32", 257, 96, 96)])
+def test_fit_projection_spans_the_dominant_subspace(dt, n, h, r):
+    # a matrix with a known spectrum and a gap after the r-th singular value;
+    # the oracle takes the same stored (rounded) matrix
+    rng = np.random.default_rng(n + h + r)
+    k = min(n, h)
+    sig = np.concatenate([np.geomspace(20.0, 6.0, r), np.geomspace(2.0, 0.05, k - r)])[:k]
+    U, _ = np.linalg.qr(rng.standard_normal((n, k)))
+    V, _ = np.linalg.qr(rng.standard_normal((h, h)))
+    X = (U * sig) @ V[:, :k].T
+    Xt = torch.from_numpy(X).to(synth.torch_dtype(dt))
+    omega = torch.from_numpy(rng.standard_normal((h, r)).astype(np.float32))
+    P, flags = salsc.salsc_fit_projection(Xt.to(DEV), r, omega.to(DEV), iters=12)
+    torch.cuda.synchronize()
+    assert flags == 0
+    Pg = P.double().cpu().numpy()
+    ref = oracle.fit_subspace(Xt, r)
+    tol = TOL[dt]
+    assert np.abs(Pg.T @ Pg - np.eye(r)).max() <= tol
+    assert np.abs(Pg @ Pg.T - ref @ ref.T).max() <= tol
+
+
 def test_small_rank_f32():
     w = W.Workload(name="f32_r16", batch=3, n_q_heads=6, n_kv_heads=3, head_dim=64, rank=16,
                    top_k=9, seq_lens=(50, 17, 200), dtype="f32", rope_base=500000.0, low_rank=4,
