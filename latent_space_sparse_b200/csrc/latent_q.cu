@@ -14,8 +14,15 @@
 namespace salsc {
 namespace {
 
-constexpr int kThreads = 512;
 constexpr int kBatchChunk = 8;  // sequences per pass
+
+// Threads and register cap per column width.  COLS = 16 (at most a few hundred
+// CTAs, e.g. 128 for 8 units of r = 256): 768 threads of at most 48 registers,
+// 36K registers a CTA, so that two CTAs never share an SM (73K > 64K) and the
+// scoring kernel's CTAs, launched early two per SM (21K), fit beside each one
+// instead of waiting for the SM to drain.  COLS = 64 (many units and a wide
+// latent space): 512 threads.
+template <int COLS> constexpr int lq_threads() { return COLS == 16 ? 768 : 512; }
 
 // CTA (u, column block): q_lat[b, u, c] = sum_i qsum[b, i] * Pk[u*d + i, c] for
 // COLS columns c.  Thread (slice, column) owns d/SLICES rows of one column of
@@ -29,10 +36,12 @@ constexpr int kBatchChunk = 8;  // sequences per pass
 // other warps.  COLS = 16 spreads a small Pk (GQA) over enough CTAs; COLS = 64
 // keeps a large one (MHA, r = 512) to a few hundred CTAs.
 template <typename T, int COLS>
-__global__ void __launch_bounds__(kThreads)
-latent_q_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __restrict__ qlat,
-                __nv_bfloat16* __restrict__ qsplit, uint32_t* __restrict__ krange, int B, int Hq,
-                int U, int G, int d, int r, int npad) {
+__device__ __forceinline__ void latent_q_body(const T* __restrict__ q, const T* __restrict__ Pk,
+                                              float* __restrict__ qlat,
+                                              __nv_bfloat16* __restrict__ qsplit,
+                                              uint32_t* __restrict__ krange, int B, int Hq, int U,
+                                              int G, int d, int r, int npad) {
+  constexpr int kThreads = lq_threads<COLS>();
   constexpr int SLICES = kThreads / COLS;
   constexpr int kRowsMax = (kMaxHeadDim + SLICES - 1) / SLICES;
   __shared__ float qsum[kBatchChunk][kMaxHeadDim];
@@ -57,7 +66,7 @@ latent_q_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __rest
       krange[2 * ((size_t)b * U + u)] = 0xffffffffu;
       krange[2 * ((size_t)b * U + u) + 1] = 0u;
     }
-  constexpr int kElems = kBatchChunk * kMaxHeadDim / kThreads;  // query sums per thread: 2
+  constexpr int kElems = (kBatchChunk * kMaxHeadDim + kThreads - 1) / kThreads;  // query sums per thread
   for (int b0 = 0; b0 < B; b0 += kBatchChunk) {
     const int nb = min(kBatchChunk, B - b0);
     float v[kElems][8];
@@ -109,10 +118,27 @@ latent_q_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __rest
   }
 }
 
+template <typename T>
+__global__ void __maxnreg__(48)
+latent_q16_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __restrict__ qlat,
+                  __nv_bfloat16* __restrict__ qsplit, uint32_t* __restrict__ krange, int B, int Hq,
+                  int U, int G, int d, int r, int npad) {
+  latent_q_body<T, 16>(q, Pk, qlat, qsplit, krange, B, Hq, U, G, d, r, npad);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(lq_threads<64>())
+latent_q64_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __restrict__ qlat,
+                  __nv_bfloat16* __restrict__ qsplit, uint32_t* __restrict__ krange, int B, int Hq,
+                  int U, int G, int d, int r, int npad) {
+  latent_q_body<T, 64>(q, Pk, qlat, qsplit, krange, B, Hq, U, G, d, r, npad);
+}
+
 template <typename T, int COLS>
 cudaError_t launch_cols(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
   dim3 grid(p.U, (p.r + COLS - 1) / COLS);
-  return launch_k(latent_q_kernel<T, COLS>, grid, dim3(kThreads), 0, s, true, (const T*)a.q,
+  auto kernel = COLS == 16 ? latent_q16_kernel<T> : latent_q64_kernel<T>;
+  return launch_k(kernel, grid, dim3(lq_threads<COLS>()), 0, s, true, (const T*)a.q,
                   (const T*)a.Pk, a.qlat, a.qsplit, a.krange, p.B, p.Hq, p.U, p.G, p.d, p.r,
                   p.npad);
 }
