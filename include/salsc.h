@@ -292,6 +292,78 @@ salsc_status salsc_fit_projection(const void* X, int64_t n, int32_t hidden, int3
                                   salsc_stream stream);
 
 /*
+ * Token-sharded decode: the tokens of every sequence split over N GPUs, shard
+ * s holding a contiguous slice (its own Kc/Vc rows; q, Pk, Pv replicated).
+ * Selection stays exact: a token among a unit's k best overall has fewer than
+ * k better tokens in its slice, so it is in that slice's local top-k (SALS
+ * technical framework, stages 2-4; the pages run one GPU, the exchange is this
+ * library's).  One layer-step on every shard, with the caller's all-gathers
+ * (e.g. NCCL) between the calls:
+ *   1. salsc_shard_candidates   local scoring + top-k -> (score, global index)
+ *   2. all-gather the candidates of the N shards
+ *   3. salsc_shard_select       the same global top-k on every shard; this
+ *                               shard's tokens as local indices
+ *   4. salsc_shard_attend       attention over them -> one partial row per head
+ *   5. all-gather the partial rows
+ *   6. salsc_shard_merge        merge the N rows of every head, apply Pv
+ * The result equals salsc_decode_step on the whole sequences (up to rounding
+ * order); ties in score go to the lower global token index.  The shard's
+ * descriptor describes its slices (seq_offsets: local lengths).
+ *
+ * salsc_shard_candidates: stages 2 and top-k on this shard's slices.
+ *   shard_off_dev [B] int64   global index of the slice's first token
+ *   cand_score    [B][U][k]   fp32 score of each locally kept token (-inf in
+ *                             empty slots)
+ *   cand_idx      [B][U][k]   int32 global token index (-1 in empty slots)
+ *   ws            workspace of salsc_decode_workspace_size(desc), prepared
+ * Requires select_mode 0 (top-k); UNSUPPORTED otherwise.
+ *
+ * salsc_shard_select: per unit, the k best of the N*k gathered candidates
+ * (score descending, lower global index first among equal scores; empty
+ * candidates never selected), by an exact radix select.
+ *   cand_score_all [N][B][U][k], cand_idx_all [N][B][U][k]  the gathered
+ *                  candidates, shard-major (an all-gather's layout)
+ *   local_offsets_dev [B+1] int64  this shard's slice offsets (its descriptor's
+ *                  seq_offsets_dev); shard_off_dev [B] as above
+ *   idx_local [B][U][k] int32  this shard's selected tokens as slice-local
+ *                  indices, in candidate order, then -1
+ * Requires N*k <= 16384, U <= 256 (UNSUPPORTED otherwise).
+ *
+ * salsc_shard_attend: stages 3-4 over idx_local, without the projection.
+ *   desc->q_pos_dev is required (the query's global position); RoPE of a kept
+ *   token uses shard_off_dev[b] + its local index.
+ *   part_out [B][Hq][r+4] fp32, 16-byte aligned: per head (m, l, 0, 0,
+ *   acc[r]): the maximum logit over this shard's kept tokens (-inf if none),
+ *   the softmax normaliser relative to it, and the unnormalised latent value
+ *   sum sum_t e^{l_t - m} Vc[t].
+ *
+ * salsc_shard_merge: out[b][h] = (sum_s w_s acc_s / sum_s w_s l_s) . Pv_u^T
+ * with w_s = e^{m_s - max_s m_s}, over the N gathered rows part_all
+ * [N][B][Hq][r+4] (16-byte aligned).  ws: any prepared decode workspace
+ * (word 0 records wait timeouts).
+ *
+ * All four are stream-ordered and allocate nothing.  Errors: INVALID_ARG
+ * (null or misaligned pointers, shapes, missing q_pos), UNSUPPORTED,
+ * WORKSPACE, CUDA.
+ */
+salsc_status salsc_shard_candidates(const salsc_decode_desc* desc, const void* q, const void* Kc,
+                                    const void* Pk, const int64_t* shard_off_dev,
+                                    float* cand_score, int32_t* cand_idx, void* ws,
+                                    size_t ws_bytes, salsc_stream stream);
+salsc_status salsc_shard_select(const float* cand_score_all, const int32_t* cand_idx_all,
+                                int32_t n_shards, int32_t batch, int32_t n_units, int32_t top_k,
+                                const int64_t* local_offsets_dev, const int64_t* shard_off_dev,
+                                int32_t* idx_local, salsc_stream stream);
+salsc_status salsc_shard_attend(const salsc_decode_desc* desc, const void* q, const void* Kc,
+                                const void* Vc, const void* Pk, const int32_t* idx_local,
+                                const int64_t* shard_off_dev, float* part_out, void* ws,
+                                size_t ws_bytes, salsc_stream stream);
+salsc_status salsc_shard_merge(const float* part_all, int32_t n_shards, int32_t batch,
+                               int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                               int32_t rank, salsc_dtype dtype, const void* Pv, void* out,
+                               void* ws, size_t ws_bytes, salsc_stream stream);
+
+/*
  * Device-side anomaly flags recorded in a workspace since salsc_decode_prepare
  * (bit 0: a selected index fell outside its sequence; bit 1: a pipeline wait
  * gave up after its iteration limit).  Copies one word to *flags_host and

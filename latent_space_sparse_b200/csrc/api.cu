@@ -263,6 +263,30 @@ struct AppendArgs {
   const int64_t* rows;
 };
 
+// Pointers of one call: the caller's arrays and the workspace's regions.
+salsc::DecodeArgs make_args(const salsc::DecodePlan& p, const salsc_decode_desc* desc,
+                            const void* q, const void* Kc, const void* Vc, const void* Pk,
+                            const void* Pv, void* out, int32_t* idx_out, void* ws) {
+  char* w = (char*)ws;
+  salsc::DecodeArgs a;
+  a.q = q;
+  a.Kc = Kc;
+  a.Vc = Vc;
+  a.Pk = Pk;
+  a.Pv = Pv;
+  a.out = out;
+  a.idx = idx_out ? idx_out : (int32_t*)(w + p.off_idx);
+  a.seq_off = desc->seq_offsets_dev;
+  a.q_pos = desc->q_pos_dev;
+  a.flags = (uint32_t*)(w + p.off_flags);
+  a.qlat = (float*)(w + p.off_qlat);
+  a.qsplit = (__nv_bfloat16*)(w + p.off_qsplit);
+  a.scores = (float*)(w + p.off_scores);
+  a.krange = (uint32_t*)(w + p.off_krange);
+  a.part = (float*)(w + p.off_part);
+  return a;
+}
+
 salsc_status decode_step_impl(const salsc_decode_desc* desc, const void* q, const void* Kc,
                               const void* Vc, const void* Pk, const void* Pv, void* out,
                               int32_t* idx_out, void* ws, size_t ws_bytes, salsc_stream stream,
@@ -287,23 +311,7 @@ salsc_status decode_step_impl(const salsc_decode_desc* desc, const void* q, cons
   }
   if ((st = check_ws(p, ws, ws_bytes)) != SALSC_OK) return st;
 
-  char* w = (char*)ws;
-  salsc::DecodeArgs a;
-  a.q = q;
-  a.Kc = Kc;
-  a.Vc = Vc;
-  a.Pk = Pk;
-  a.Pv = Pv;
-  a.out = out;
-  a.idx = idx_out ? idx_out : (int32_t*)(w + p.off_idx);
-  a.seq_off = desc->seq_offsets_dev;
-  a.q_pos = desc->q_pos_dev;
-  a.flags = (uint32_t*)(w + p.off_flags);
-  a.qlat = (float*)(w + p.off_qlat);
-  a.qsplit = (__nv_bfloat16*)(w + p.off_qsplit);
-  a.scores = (float*)(w + p.off_scores);
-  a.krange = (uint32_t*)(w + p.off_krange);
-  a.part = (float*)(w + p.off_part);
+  salsc::DecodeArgs a = make_args(p, desc, q, Kc, Vc, Pk, Pv, out, idx_out, ws);
 
   cudaStream_t s = (cudaStream_t)stream;
   typedef cudaError_t (*launcher)(const salsc::DecodePlan&, const salsc::DecodeArgs&, cudaStream_t);
@@ -399,6 +407,103 @@ salsc_status salsc_compress(const void* K, const void* V, const void* Pk, const 
   if (V && (e = salsc::launch_compress(V, Pv, Vc, n_tokens, hidden, rank, dtype, s)) != cudaSuccess)
     return cuda_fail(e);
   return SALSC_OK;
+}
+
+salsc_status salsc_shard_candidates(const salsc_decode_desc* desc, const void* q, const void* Kc,
+                                    const void* Pk, const int64_t* shard_off_dev,
+                                    float* cand_score, int32_t* cand_idx, void* ws,
+                                    size_t ws_bytes, salsc_stream stream) {
+  salsc::DecodePlan p;
+  salsc_status st = make_plan(desc, &p);
+  if (st != SALSC_OK) return st;
+  if (desc->select_mode != 0) return SALSC_ERR_UNSUPPORTED;
+  if (!desc->seq_offsets_dev || !q || !Kc || !Pk || !shard_off_dev || !cand_score || !cand_idx)
+    return SALSC_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(Kc) || !aligned16(Pk) || ((uintptr_t)cand_score & 3u) ||
+      ((uintptr_t)cand_idx & 3u) || ((uintptr_t)shard_off_dev & 7u))
+    return SALSC_ERR_INVALID_ARG;
+  if ((st = check_ws(p, ws, ws_bytes)) != SALSC_OK) return st;
+  const salsc::DecodeArgs a = make_args(p, desc, q, Kc, nullptr, Pk, nullptr, nullptr, nullptr, ws);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e;
+  if ((e = salsc::launch_latent_q(p, a, s)) != cudaSuccess ||
+      (e = salsc::launch_score(p, a, s)) != cudaSuccess ||
+      (e = salsc::launch_topk(p, a, s)) != cudaSuccess ||
+      (e = salsc::launch_shard_gather(p, a, shard_off_dev, cand_score, cand_idx, s)) !=
+          cudaSuccess)
+    return cuda_fail(e);
+  return SALSC_OK;
+}
+
+salsc_status salsc_shard_select(const float* cand_score_all, const int32_t* cand_idx_all,
+                                int32_t n_shards, int32_t batch, int32_t n_units, int32_t top_k,
+                                const int64_t* local_offsets_dev, const int64_t* shard_off_dev,
+                                int32_t* idx_local, salsc_stream stream) {
+  if (!cand_score_all || !cand_idx_all || !local_offsets_dev || !shard_off_dev || !idx_local)
+    return SALSC_ERR_INVALID_ARG;
+  if (n_shards < 1 || batch < 1 || n_units < 1 || top_k < 1) return SALSC_ERR_INVALID_ARG;
+  if (n_units > salsc::kMaxUnits || (int64_t)n_shards * top_k > salsc::kMaxShardCandidates)
+    return SALSC_ERR_UNSUPPORTED;
+  const cudaError_t e =
+      salsc::launch_shard_select(cand_score_all, cand_idx_all, n_shards, batch, n_units, top_k,
+                                 local_offsets_dev, shard_off_dev, idx_local, (cudaStream_t)stream);
+  return e == cudaSuccess ? SALSC_OK : cuda_fail(e);
+}
+
+salsc_status salsc_shard_attend(const salsc_decode_desc* desc, const void* q, const void* Kc,
+                                const void* Vc, const void* Pk, const int32_t* idx_local,
+                                const int64_t* shard_off_dev, float* part_out, void* ws,
+                                size_t ws_bytes, salsc_stream stream) {
+  salsc::DecodePlan p;
+  salsc_status st = make_plan(desc, &p);
+  if (st != SALSC_OK) return st;
+  // the shards' partials are merged after the exchange, so the attention
+  // kernel does not merge (nor project) them itself
+  p.att_cluster = 0;
+  if (!desc->seq_offsets_dev || !desc->q_pos_dev || !q || !Kc || !Vc || !Pk || !idx_local ||
+      !shard_off_dev || !part_out)
+    return SALSC_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(Pk) ||
+      ((uintptr_t)idx_local & 3u) || ((uintptr_t)part_out & 15u) || ((uintptr_t)shard_off_dev & 7u))
+    return SALSC_ERR_INVALID_ARG;
+  if ((st = check_ws(p, ws, ws_bytes)) != SALSC_OK) return st;
+  salsc::DecodeArgs a =
+      make_args(p, desc, q, Kc, Vc, Pk, nullptr, nullptr, const_cast<int32_t*>(idx_local), ws);
+  a.pos_off = shard_off_dev;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e;
+  if ((e = salsc::launch_attend(p, a, s)) != cudaSuccess ||
+      (e = salsc::launch_combine_partial(p, a, part_out, s)) != cudaSuccess)
+    return cuda_fail(e);
+  return SALSC_OK;
+}
+
+salsc_status salsc_shard_merge(const float* part_all, int32_t n_shards, int32_t batch,
+                               int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                               int32_t rank, salsc_dtype dtype, const void* Pv, void* out,
+                               void* ws, size_t ws_bytes, salsc_stream stream) {
+  if (dtype != SALSC_F32 && dtype != SALSC_BF16) return SALSC_ERR_INVALID_ARG;
+  if (!part_all || !Pv || !out || n_shards < 1 || batch < 1 || n_kv_heads < 1 || rank < 1 ||
+      n_q_heads < n_kv_heads || n_q_heads % n_kv_heads != 0)
+    return SALSC_ERR_INVALID_ARG;
+  if (((uintptr_t)part_all & 15u) || !aligned16(Pv) || !aligned16(out)) return SALSC_ERR_INVALID_ARG;
+  if (!ws || ((uintptr_t)ws % salsc::kWsAlign) != 0 || ws_bytes < 16) return SALSC_ERR_WORKSPACE;
+  salsc::DecodePlan p{};
+  p.B = batch;
+  p.Hq = n_q_heads;
+  p.U = n_kv_heads;
+  p.G = n_q_heads / n_kv_heads;
+  p.d = head_dim;
+  p.r = rank;
+  p.dtype = dtype;
+  p.splits = n_shards;
+  if ((head_dim != 64 && head_dim != 128) || rank > salsc::kMaxRank || p.G > 8 ||
+      n_kv_heads > salsc::kMaxUnits || rank > n_kv_heads * head_dim ||
+      !salsc::combine_supported(p))
+    return SALSC_ERR_UNSUPPORTED;
+  const cudaError_t e = salsc::launch_shard_merge(p, part_all, n_shards, Pv, out, (uint32_t*)ws,
+                                                  (cudaStream_t)stream);
+  return e == cudaSuccess ? SALSC_OK : cuda_fail(e);
 }
 
 }  // extern "C"

@@ -35,7 +35,8 @@ __global__ void __launch_bounds__(kThreads)
 attend_simt_kernel(const T* __restrict__ q, const T* __restrict__ Kc, const T* __restrict__ Vc,
                    const T* __restrict__ Pk, const int32_t* __restrict__ idx,
                    const int64_t* __restrict__ seq_off, const int32_t* __restrict__ q_pos,
-                   float* __restrict__ part, uint32_t* __restrict__ flags, int Hq, int U, int G,
+                   const int64_t* __restrict__ pos_off, float* __restrict__ part,
+                   uint32_t* __restrict__ flags, int Hq, int U, int G,
                    int d, int r, int k, int chunk, int splits, float scale, double base) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int split = blockIdx.x;
@@ -61,6 +62,7 @@ attend_simt_kernel(const T* __restrict__ q, const T* __restrict__ Kc, const T* _
   const int64_t nb = seq_off[b + 1] - off;
   const int64_t kb = nb < k ? nb : k;
   const double qpos = q_pos ? (double)q_pos[b] : (double)nb;
+  const double pos0 = pos_off ? (double)pos_off[b] : 0.0;  // position of the sequence's token 0
   allow_dependent_launch();
   grid_dependency_wait();  // the kept indices come from the previous kernel
 
@@ -139,7 +141,7 @@ attend_simt_kernel(const T* __restrict__ q, const T* __restrict__ Kc, const T* _
       const int t = tok[j];
       if (t < 0) continue;
       float c, s;
-      rope_cs((double)t, theta[i], c, s);
+      rope_cs((double)t + pos0, theta[i], c, s);
       float* kr = ks + j * kMaxHeadDim;
       const float x0 = kr[i], x1 = kr[i + half];
       kr[i] = x0 * c - x1 * s;
@@ -229,7 +231,7 @@ cudaError_t launch_attend(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
     e = launch_k(kern, grid, dim3(kThreads), smem, s, true, (const __nv_bfloat16*)a.q,
                  (const __nv_bfloat16*)a.Kc, (const __nv_bfloat16*)a.Vc,
                  (const __nv_bfloat16*)a.Pk, (const int32_t*)a.idx, (const int64_t*)a.seq_off,
-                 (const int32_t*)a.q_pos, a.part, a.flags, p.Hq, p.U, p.G, p.d, p.r, p.k, p.chunk,
+                 (const int32_t*)a.q_pos, a.pos_off, a.part, a.flags, p.Hq, p.U, p.G, p.d, p.r, p.k, p.chunk,
                  p.splits, p.scale, p.rope_base);
     if (e != cudaSuccess) return e;
   } else {
@@ -240,7 +242,7 @@ cudaError_t launch_attend(const DecodePlan& p, const DecodeArgs& a, cudaStream_t
     if (e != cudaSuccess) return e;
     e = launch_k(kern, grid, dim3(kThreads), smem, s, true, (const float*)a.q,
                  (const float*)a.Kc, (const float*)a.Vc, (const float*)a.Pk, (const int32_t*)a.idx,
-                 (const int64_t*)a.seq_off, (const int32_t*)a.q_pos, a.part, a.flags, p.Hq, p.U,
+                 (const int64_t*)a.seq_off, (const int32_t*)a.q_pos, a.pos_off, a.part, a.flags, p.Hq, p.U,
                  p.G, p.d, p.r, p.k, p.chunk, p.splits, p.scale, p.rope_base);
     if (e != cudaSuccess) return e;
   }

@@ -66,6 +66,7 @@ struct AttendTcParams {
   const int32_t* idx;
   const int64_t* seq_off;
   const int32_t* q_pos;
+  const int64_t* pos_off;  // [B] or null: added to a kept token's index for RoPE
   float* part;
   uint32_t* flags;
   const __nv_bfloat16* Pv;  // merged in the kernel: the value projection
@@ -570,6 +571,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     UnitTileCursor cur;
     cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
     int cur_b = -1, cur_u = -1;
+    uint32_t pos_b = 0;  // position of the sequence's token 0 (token-sharded caches)
     // the segment's running sums: slot s = part + kEpiParts*j (j < kSlots) holds latent
     // column (s / G)*128 + quarter*32 + lane of head s % G
     const int n_used = n_chunks * G;
@@ -669,6 +671,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
         // rotated queries of the unit's heads (angles reduced in fp64), as
         // pairs (q_i, q_i+d/2) in the order [pair][head]
         const double qpos = P.q_pos ? (double)P.q_pos[cur.b] : (double)cur.nb;
+        pos_b = P.pos_off ? (uint32_t)P.pos_off[cur.b] : 0u;
         for (int e = tid; e < G * HALF; e += kEpiThreads) {
           const int g = e / HALF, ii = e % HALF;
           const __nv_bfloat16* qh = P.q + ((int64_t)cur.b * P.Hq + cur.u * G + g) * D;
@@ -697,7 +700,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       if (ok) {
         const uint32_t row_addr =
             tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)bi * D + (uint32_t)(part * QP);
-        const uint32_t tu = (uint32_t)(t < 0 ? 0 : t);
+        const uint32_t tu = (uint32_t)(t < 0 ? 0 : t) + pos_b;
 #pragma unroll 1
         for (int c8 = 0; c8 < QP; c8 += 8) {
           uint32_t v0[8], v1[8];
@@ -924,6 +927,7 @@ cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s)
   P.idx = a.idx;
   P.seq_off = a.seq_off;
   P.q_pos = a.q_pos;
+  P.pos_off = a.pos_off;
   P.part = a.part;
   P.flags = a.flags;
   P.Pv = (const __nv_bfloat16*)a.Pv;

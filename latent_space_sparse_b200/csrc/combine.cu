@@ -22,6 +22,11 @@
 // starts there or the unit starts there, which follows from the tile
 // partition; with the CUDA-core attention every slot of the unit is used.
 // The sums run over slots in slot order, so the result is deterministic.
+//
+// Two more uses for token-sharded decode: with part_out set, the kernel stops
+// after the merge and writes the merged (M, L, acc) of every head as one
+// partial row (one CTA per unit, no projection); with the row strides set to
+// (1, B*Hq), it merges one such row per shard (every slot used) and projects.
 #include "tc.cuh"
 
 namespace salsc {
@@ -32,7 +37,7 @@ constexpr int kRows = 16;                      // output rows per CTA
 constexpr int kTpr = kThreads / kRows;         // threads per output row
 constexpr int kColsPer = kMaxRank / kThreads;  // latent columns per thread (r <= 512)
 constexpr uint32_t kRowBuf = 32u * 1024u;      // bytes of partial rows per batch
-constexpr int kMaxSegs = 128;
+constexpr int kMaxSegs = kMaxShardCandidates / 64 > 128 ? kMaxShardCandidates / 64 : 128;
 
 struct CombineParams {
   const float* part;
@@ -42,6 +47,9 @@ struct CombineParams {
   uint32_t* flags;
   int B, Hq, U, d, r, k, n_slots, chunk;
   int seg_grid, seg_tiles;  // tensor-core tile partition (seg_grid = 0: every slot used)
+  int64_t bh_stride, slot_stride;  // partial row of (b, h, slot): (b*Hq + h)*bh_stride + slot*slot_stride
+  float* part_out;  // non-null: write the merged partial row of every head, no projection
+  int fixed_slots;  // > 0: every unit has this many slots (no tile count from the lengths)
 };
 
 template <typename T, int G>
@@ -59,7 +67,7 @@ combine_kernel(const CombineParams P) {
   __shared__ __align__(8) uint64_t s_bar[2];
   const uint32_t bar_pv = tc::smem_u32(&s_bar[0]), bar_rows = tc::smem_u32(&s_bar[1]);
 
-  const int n_slices = P.d / kRows;
+  const int n_slices = P.part_out ? 1 : P.d / kRows;
   const int slice = blockIdx.x % n_slices;
   const int bu = blockIdx.x / n_slices;
   const int b = bu / P.U, u = bu % P.U;
@@ -70,10 +78,12 @@ combine_kernel(const CombineParams P) {
     tc::mbar_init(bar_rows, 1);
     tc::mbar_fence_init();
     // the 16 rows of Pv_u: a weight, copied before the dependency wait
-    tc::mbar_expect_tx(bar_pv, pv_bytes);
-    tc::bulk_load(tc::smem_u32(pv_s),
-                  (const T*)P.Pv + ((int64_t)u * P.d + (int64_t)slice * kRows) * P.r, pv_bytes,
-                  bar_pv);
+    if (!P.part_out) {
+      tc::mbar_expect_tx(bar_pv, pv_bytes);
+      tc::bulk_load(tc::smem_u32(pv_s),
+                    (const T*)P.Pv + ((int64_t)u * P.d + (int64_t)slice * kRows) * P.r, pv_bytes,
+                    bar_pv);
+    }
   }
   allow_dependent_launch();
   // The used slots follow from the sequence lengths and the tile partition
@@ -83,8 +93,8 @@ combine_kernel(const CombineParams P) {
     // slots of unit (b, u) and, with the tile partition, the unit's first tile:
     // every lane reads one sequence's offsets, a warp scan sums the tiles
     int64_t before = 0;  // tiles of the sequences before b
-    int tb = 0;
-    for (int b0 = 0; b0 <= b; b0 += 32) {
+    int tb = P.fixed_slots;
+    for (int b0 = 0; b0 <= b && P.fixed_slots == 0; b0 += 32) {
       const int bb = b0 + lane;
       int64_t t = 0;
       if (bb <= b && bb < P.B) {
@@ -98,7 +108,7 @@ combine_kernel(const CombineParams P) {
       for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
       before += x;
     }
-    tb = __reduce_max_sync(0xffffffffu, tb);  // set by the lane of sequence b only
+    if (P.fixed_slots == 0) tb = __reduce_max_sync(0xffffffffu, tb);  // set by the lane of sequence b only
     const int64_t unit_tile0 = before * P.U + (int64_t)u * tb;
     int cnt = 0;
     for (int s0 = 0; s0 < tb; s0 += 32) {
@@ -130,7 +140,7 @@ combine_kernel(const CombineParams P) {
     for (int j = 0; j < kColsPer; ++j) acc[g][j] = 0.f;
   int bs = (int)(kRowBuf / (uint32_t)(rowf * 4)) / G;  // slots per batch
   if (bs * G > 32) bs = 32 / G;  // one row copy per lane of warp 0
-  const float* part_u = P.part + ((int64_t)b * P.Hq + (int64_t)u * G) * P.n_slots * rowf;
+  const float* part_u = P.part + ((int64_t)b * P.Hq + (int64_t)u * G) * P.bh_stride * rowf;
   uint32_t phase = 0;
   bool ok = true;
   for (int q0 = 0; q0 < nseg; q0 += bs, phase ^= 1u) {
@@ -142,7 +152,7 @@ combine_kernel(const CombineParams P) {
       if (lane < G * nq) {
         const int g = lane / nq, j = lane % nq;
         tc::bulk_load(tc::smem_u32(rows_s + (size_t)lane * rowf),
-                      part_u + ((int64_t)g * P.n_slots + s_seg[q0 + j]) * rowf,
+                      part_u + ((int64_t)g * P.bh_stride + s_seg[q0 + j] * P.slot_stride) * rowf,
                       (uint32_t)(rowf * 4), bar_rows);
       }
       ok = tc::mbar_wait(bar_rows, phase, P.flags) && ok;
@@ -185,6 +195,25 @@ combine_kernel(const CombineParams P) {
       }
     }
     __syncthreads();  // the row buffer is refilled by the next batch
+  }
+  if (P.part_out) {
+    // the merged partial of every head: (M, L) and the unnormalised sum
+    float* po = P.part_out + ((int64_t)b * P.Hq + (int64_t)u * G) * rowf;
+#pragma unroll
+    for (int j = 0; j < kColsPer; ++j) {
+      const int c = tid + j * kThreads;
+      if (c < P.r) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) po[(int64_t)g * rowf + kPartAcc + c] = acc[g][j];
+      }
+    }
+    if (tid < G) {
+      po[(int64_t)tid * rowf] = s_M[tid];
+      po[(int64_t)tid * rowf + 1] = s_L[tid];
+      po[(int64_t)tid * rowf + 2] = 0.f;
+      po[(int64_t)tid * rowf + 3] = 0.f;
+    }
+    return;
   }
 #pragma unroll
   for (int j = 0; j < kColsPer; ++j) {
@@ -239,7 +268,7 @@ cudaError_t launch_tg(const CombineParams& P, const DecodePlan& p, cudaStream_t 
   const size_t smem = combine_smem(p);
   cudaError_t e = ensure_smem(combine_kernel<T, G>, smem, done);
   if (e != cudaSuccess) return e;
-  const dim3 grid((unsigned)(p.B * p.U * (p.d / kRows)));
+  const dim3 grid((unsigned)(p.B * p.U * (P.part_out ? 1 : p.d / kRows)));
   return launch_k(combine_kernel<T, G>, grid, dim3(kThreads), smem, s, true, P);
 }
 
@@ -263,9 +292,9 @@ bool combine_supported(const DecodePlan& p) {
          (uint32_t)(p.G * part_row(p.r) * 4) <= kRowBuf && p.splits <= kMaxSegs;
 }
 
-cudaError_t launch_combine(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
-  if (p.att_cluster > 0) return cudaSuccess;  // the attention kernel merged the partials
-  if (!combine_supported(p)) return cudaErrorInvalidConfiguration;
+namespace {
+
+CombineParams base_params(const DecodePlan& p, const DecodeArgs& a) {
   CombineParams P;
   P.part = a.part;
   P.Pv = a.Pv;
@@ -282,7 +311,49 @@ cudaError_t launch_combine(const DecodePlan& p, const DecodeArgs& a, cudaStream_
   P.chunk = p.chunk;
   P.seg_grid = p.attend_tc ? attend_tc_grid(p) : 0;
   P.seg_tiles = p.att_tiles;
+  P.bh_stride = p.splits;
+  P.slot_stride = 1;
+  P.part_out = nullptr;
+  P.fixed_slots = 0;
+  return P;
+}
+
+cudaError_t launch_params(const CombineParams& P, const DecodePlan& p, cudaStream_t s) {
   return p.dtype == SALSC_BF16 ? launch_t<__nv_bfloat16>(P, p, s) : launch_t<float>(P, p, s);
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
+  if (p.att_cluster > 0) return cudaSuccess;  // the attention kernel merged the partials
+  if (!combine_supported(p)) return cudaErrorInvalidConfiguration;
+  return launch_params(base_params(p, a), p, s);
+}
+
+cudaError_t launch_combine_partial(const DecodePlan& p, const DecodeArgs& a, float* part_out,
+                                   cudaStream_t s) {
+  if (p.att_cluster > 0 || !combine_supported(p)) return cudaErrorInvalidConfiguration;
+  CombineParams P = base_params(p, a);
+  P.part_out = part_out;
+  return launch_params(P, p, s);
+}
+
+cudaError_t launch_shard_merge(const DecodePlan& p, const float* part_all, int n_shards,
+                               const void* Pv, void* out, uint32_t* flags, cudaStream_t s) {
+  if (n_shards < 1 || n_shards > kMaxSegs) return cudaErrorInvalidValue;
+  DecodeArgs a{};
+  a.part = (float*)part_all;
+  a.Pv = Pv;
+  a.out = out;
+  a.flags = flags;
+  CombineParams P = base_params(p, a);
+  // slot s of head (b, h) is shard s's merged row: part_all[s][b][h]
+  P.n_slots = n_shards;
+  P.seg_grid = 0;  // every slot used
+  P.fixed_slots = n_shards;
+  P.bh_stride = 1;
+  P.slot_stride = (int64_t)p.B * p.Hq;
+  return launch_params(P, p, s);
 }
 
 }  // namespace salsc

@@ -31,6 +31,7 @@ __host__ __device__ constexpr int part_row(int r) { return r + kPartAcc; }
 constexpr int kMaxHeadDim = 128;
 constexpr int kMaxUnits = 256;  // KV heads per layer
 constexpr size_t kWsAlign = 256;
+constexpr int kMaxShardCandidates = 16384;  // token-sharded selection: shards x k per unit
 
 // Host-side plan of one decode layer-step, derived from the descriptor only.
 struct DecodePlan {
@@ -73,6 +74,7 @@ struct DecodeArgs {
   float* scores;               // packed per (b,u)
   uint32_t* krange;            // [B][U][2] (min, max) order key of each unit's scores
   float* part;                 // [B][Hq][splits][part_row(r)]
+  const int64_t* pos_off = nullptr;  // [B] or null: added to a kept token's index for RoPE
 };
 
 // Record a CUDA error for salsc_last_cuda_error() and return SALSC_ERR_CUDA.
@@ -84,6 +86,18 @@ cudaError_t launch_score(const DecodePlan& p, const DecodeArgs& a, cudaStream_t 
 cudaError_t launch_topk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_attend(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
+// Token-sharded decode (shard.cu, combine.cu): the local selection as
+// candidates (score, global index); the global selection of this shard's
+// tokens; the merged partial row of every head; the merge of the shards' rows.
+cudaError_t launch_shard_gather(const DecodePlan& p, const DecodeArgs& a, const int64_t* shard_off,
+                                float* cand_score, int32_t* cand_idx, cudaStream_t s);
+cudaError_t launch_shard_select(const float* cand_score, const int32_t* cand_idx, int N, int B,
+                                int U, int k, const int64_t* local_off, const int64_t* shard_off,
+                                int32_t* idx_local, cudaStream_t s);
+cudaError_t launch_combine_partial(const DecodePlan& p, const DecodeArgs& a, float* part_out,
+                                   cudaStream_t s);
+cudaError_t launch_shard_merge(const DecodePlan& p, const float* part_all, int n_shards,
+                               const void* Pv, void* out, uint32_t* flags, cudaStream_t s);
 bool attend_tc_supported(const DecodePlan& p);
 int attend_merge_cluster(const DecodePlan& p);  // 0: merge kernel; else CTAs per unit
 size_t fit_workspace_size(int64_t hidden, int64_t rank);

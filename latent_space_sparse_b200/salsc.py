@@ -24,7 +24,9 @@ WS_ALIGN = 256
 EXPORTS = (
     "salsc_compress", "salsc_decode_workspace_size", "salsc_decode_prepare", "salsc_decode_step",
     "salsc_decode_step_timed", "salsc_decode_step_static_ws", "salsc_decode_launch_count", "salsc_append", "salsc_decode_step_append", "salsc_fit_workspace_size",
-    "salsc_fit_projection", "salsc_decode_read_flags", "salsc_status_string", "salsc_last_cuda_error", "salsc_version",
+    "salsc_fit_projection", "salsc_shard_candidates", "salsc_shard_select", "salsc_shard_attend",
+    "salsc_shard_merge", "salsc_decode_read_flags", "salsc_status_string", "salsc_last_cuda_error",
+    "salsc_version",
 )
 
 
@@ -83,6 +85,15 @@ def _lib():
         lib.salsc_fit_workspace_size.argtypes = [i32, i32]
         lib.salsc_fit_projection.restype = ctypes.c_int
         lib.salsc_fit_projection.argtypes = [vp, i64, i32, i32, vp, i32, vp, ctypes.c_int, vp, sz, vp]
+        lib.salsc_shard_candidates.restype = ctypes.c_int
+        lib.salsc_shard_candidates.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.salsc_shard_select.restype = ctypes.c_int
+        lib.salsc_shard_select.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp]
+        lib.salsc_shard_attend.restype = ctypes.c_int
+        lib.salsc_shard_attend.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.salsc_shard_merge.restype = ctypes.c_int
+        lib.salsc_shard_merge.argtypes = [vp, i32, i32, i32, i32, i32, i32, ctypes.c_int, vp, vp,
+                                          vp, sz, vp]
         lib.salsc_append.restype = ctypes.c_int
         lib.salsc_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, ctypes.c_int, vp]
         lib.salsc_decode_launch_count.restype = ctypes.c_int32
@@ -228,6 +239,45 @@ def salsc_decode_step_append(desc: DecodeDesc, K_new, V_new, rows, q, Kc, Vc, Pk
                                          _ptr(idx_out), _ptr(ws), ws.numel() * ws.element_size(),
                                          _stream(stream))
     _check(st, "salsc_decode_step_append")
+
+
+def salsc_shard_candidates(desc: DecodeDesc, q, Kc, Pk, shard_off, cand_score, cand_idx, ws,
+                           stream=None):
+    """Token-sharded step 1: this shard's top-k per unit as (score, global index) candidates."""
+    st = _lib().salsc_shard_candidates(ctypes.byref(desc), _ptr(q), _ptr(Kc), _ptr(Pk),
+                                       _ptr(shard_off), _ptr(cand_score), _ptr(cand_idx), _ptr(ws),
+                                       ws.numel() * ws.element_size(), _stream(stream))
+    _check(st, "salsc_shard_candidates")
+
+
+def salsc_shard_select(cand_score_all, cand_idx_all, local_offsets, shard_off, idx_local,
+                       stream=None):
+    """Token-sharded step 3: the global top-k of the gathered candidates [N][B][U][k]; this
+    shard's tokens as slice-local indices in idx_local [B][U][k] (-1 elsewhere)."""
+    n, b, u, k = cand_score_all.shape
+    st = _lib().salsc_shard_select(_ptr(cand_score_all), _ptr(cand_idx_all), n, b, u, k,
+                                   _ptr(local_offsets), _ptr(shard_off), _ptr(idx_local),
+                                   _stream(stream))
+    _check(st, "salsc_shard_select")
+
+
+def salsc_shard_attend(desc: DecodeDesc, q, Kc, Vc, Pk, idx_local, shard_off, part_out, ws,
+                       stream=None):
+    """Token-sharded step 4: attention over idx_local; part_out [B][Hq][r+4] fp32 rows
+    (m, l, 0, 0, acc[r]) per head, before the projection."""
+    st = _lib().salsc_shard_attend(ctypes.byref(desc), _ptr(q), _ptr(Kc), _ptr(Vc), _ptr(Pk),
+                                   _ptr(idx_local), _ptr(shard_off), _ptr(part_out), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _stream(stream))
+    _check(st, "salsc_shard_attend")
+
+
+def salsc_shard_merge(part_all, n_kv_heads, head_dim, Pv, out, ws, stream=None):
+    """Token-sharded step 6: merge the gathered rows part_all [N][B][Hq][r+4] and project."""
+    n, b, hq, rowf = part_all.shape
+    st = _lib().salsc_shard_merge(_ptr(part_all), n, b, hq, n_kv_heads, head_dim, rowf - 4,
+                                  _dtype_code(out.dtype), _ptr(Pv), _ptr(out), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream))
+    _check(st, "salsc_shard_merge")
 
 
 DECODE_KERNELS = ("latent_q", "score", "topk", "attend", "combine")

@@ -210,3 +210,62 @@ def test_compress_validation_before_launch():
     assert lib.salsc_compress(a, None, None, None, c, None, 10, 64, 16, salsc.SALSC_BF16, None) == 1
     # zero rows is a valid no-op (nothing is enqueued)
     assert lib.salsc_compress(a, None, b, None, c, None, 0, 64, 16, salsc.SALSC_BF16, None) == 0
+
+
+def test_shard_validation_before_launch():
+    """Token-sharded entry points: every argument check returns before a launch."""
+    lib = salsc.load()
+    vp = ctypes.c_void_p
+    a, b, c = vp(1 << 20), vp(1 << 21), vp(1 << 22)
+    host = torch.tensor([0, 1000, 1800], dtype=torch.int64)
+
+    class FakeDev:  # a device address that is never dereferenced: every call fails a check
+        def __init__(self, p):
+            self.p = p
+
+        def data_ptr(self):
+            return self.p
+
+    d = salsc.make_desc(2, 32, 8, 128, 256, 64, host, FakeDev(1 << 23), None, 10000.0, 0.0,
+                        torch.bfloat16)
+    need = lib.salsc_decode_workspace_size(ctypes.byref(d))
+    ws = vp(1 << 28)
+
+    def cand(dd=d, q=a, kc=b, pk=c, so=a, cs=b, ci=c, w=ws, n=need):
+        return lib.salsc_shard_candidates(ctypes.byref(dd), q, kc, pk, so, cs, ci, w, n, None)
+
+    assert cand(q=None) == salsc.SALSC_ERR_INVALID_ARG
+    assert cand(so=None) == salsc.SALSC_ERR_INVALID_ARG
+    assert cand(q=vp((1 << 20) + 8)) == salsc.SALSC_ERR_INVALID_ARG  # misaligned
+    assert cand(n=need - 1) == salsc.SALSC_ERR_WORKSPACE
+    dt = salsc.make_desc(2, 32, 8, 128, 256, 64, host, FakeDev(1 << 23), None, 10000.0, 0.0,
+                         torch.bfloat16, 0.5)
+    assert cand(dd=dt) == salsc.SALSC_ERR_UNSUPPORTED  # threshold selection is not sharded
+
+    def sel(cs=a, ci=b, n=2, batch=2, units=8, k=64, lo=c, so=a, out=b):
+        return lib.salsc_shard_select(cs, ci, n, batch, units, k, lo, so, out, None)
+
+    assert sel(cs=None) == salsc.SALSC_ERR_INVALID_ARG
+    assert sel(n=0) == salsc.SALSC_ERR_INVALID_ARG
+    assert sel(n=8, k=4096) == salsc.SALSC_ERR_UNSUPPORTED  # 32768 candidates per unit
+    assert sel(units=300) == salsc.SALSC_ERR_UNSUPPORTED
+
+    def att(dd=d, idx=a, so=b, part=c, w=ws, n=need):
+        return lib.salsc_shard_attend(ctypes.byref(dd), a, b, c, a, idx, so, part, w, n, None)
+
+    assert att() == salsc.SALSC_ERR_INVALID_ARG  # the descriptor has no q_pos
+    dq = salsc.make_desc(2, 32, 8, 128, 256, 64, host, FakeDev(1 << 23), FakeDev(1 << 24),
+                         10000.0, 0.0, torch.bfloat16)
+    assert att(dd=dq, idx=None) == salsc.SALSC_ERR_INVALID_ARG
+    assert att(dd=dq, part=vp((1 << 22) + 4)) == salsc.SALSC_ERR_INVALID_ARG  # part not 16-aligned
+    assert att(dd=dq, n=need - 1) == salsc.SALSC_ERR_WORKSPACE
+
+    def merge(part=a, n=2, batch=2, hq=32, hkv=8, dh=128, r=256, dtype=1, pv=b, out=c, w=ws):
+        return lib.salsc_shard_merge(part, n, batch, hq, hkv, dh, r, dtype, pv, out, w, 16, None)
+
+    assert merge(dtype=7) == salsc.SALSC_ERR_INVALID_ARG
+    assert merge(part=None) == salsc.SALSC_ERR_INVALID_ARG
+    assert merge(hq=30) == salsc.SALSC_ERR_INVALID_ARG  # Hq not a multiple of Hkv
+    assert merge(dh=96) == salsc.SALSC_ERR_UNSUPPORTED
+    assert merge(hq=96, hkv=8) == salsc.SALSC_ERR_UNSUPPORTED  # 12 heads per unit
+    assert merge(w=vp((1 << 28) + 8)) == salsc.SALSC_ERR_WORKSPACE
