@@ -29,12 +29,13 @@
 //      so the combine kernel finds the used slots from the tile partition
 //      alone; it merges the few segments of a unit and applies the deferred
 //      Pv_u^T.
-// Warp roles (608 threads): warps 0-15 epilogue, warp 16 TMEM owner and MMA
-// issuer, warps 17 and 18 row gathers (one per tile buffer).  The epilogue is
-// the busiest role (RoPE needs a sine and a cosine per pair and token), so it
-// has four warps per scheduler; 19 warps keep 96 registers per thread (at
-// most five warps share a scheduler's registers).  Each CTA walks a contiguous
-// range of tiles;
+// Warp roles (800 threads): warps 0-15 epilogue, warp 16 TMEM owner and MMA
+// issuer, warps 17-20 and 21-24 row gathers (four per tile buffer: the issue
+// of TMA gather4 copies bounds the gather chain).  The epilogue is the
+// busiest role (RoPE needs a sine and a cosine per pair and token), so it has
+// four warps per scheduler; 25 warps keep 72 registers per thread (the
+// register file is split per scheduler).  Each CTA walks a contiguous range
+// of tiles;
 // the two tile buffers alternate (Kc(i) -> Vc(i) -> Kc(i+2)), so the
 // reconstruction of tile i+1 runs during the epilogue of tile i.
 //

@@ -169,7 +169,14 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
       for (int64_t j = kb + tid; j < k; j += kThreads) out[j] = -1;
     return;
   }
-  // the unit's key range, reduced by the scoring kernel
+  // the slice's first batch of scores is requested together with the unit's
+  // key range (reduced by the scoring kernel): one round trip, not two
+  float v0[kBatch];
+#pragma unroll
+  for (int j = 0; j < kBatch; ++j) {
+    const int i = j * kThreads + tid;
+    v0[j] = i < n_loc ? s[lo + i] : 0.f;
+  }
   uint32_t kmin = krange[2 * ((int64_t)b * U + u)], kmax = krange[2 * ((int64_t)b * U + u) + 1];
   const float fmin = key_float(kmin), fmax = key_float(kmax);
   const float frange = fmax - fmin;
@@ -184,7 +191,7 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
       const int i = base + j * kThreads + tid;
-      v[j] = i < n_loc ? s[lo + i] : 0.f;
+      v[j] = base == 0 ? v0[j] : (i < n_loc ? s[lo + i] : 0.f);
     }
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
