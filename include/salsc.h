@@ -342,7 +342,13 @@ salsc_status salsc_fit_projection(const void* X, int64_t n, int32_t hidden, int3
  * [N][B][Hq][r+4] (16-byte aligned).  ws: any prepared decode workspace
  * (word 0 records wait timeouts).
  *
- * All four are stream-ordered and allocate nothing.  Errors: INVALID_ARG
+ * All four are stream-ordered and allocate nothing.  Their kernels use
+ * programmatic dependent launch: in salsc_shard_attend and salsc_shard_merge,
+ * Pk, Pv, q and the sequence and slice offsets may be read before the work
+ * enqueued ahead of the call has finished (in salsc_shard_candidates only Pk,
+ * as in salsc_decode_step), so the work before the call must not write them
+ * while it runs; Kc, Vc, the candidates, idx_local and the partial rows are
+ * read only after it.  Errors: INVALID_ARG
  * (null or misaligned pointers, shapes, missing q_pos), UNSUPPORTED,
  * WORKSPACE, CUDA.
  */
