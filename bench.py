@@ -186,6 +186,18 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The largest ``value`` over the ranks of the default process group (a
+    job's time is its slowest rank's); ``value`` itself without one.  Every
+    rank must call it (a collective)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ------------------------------------------------------------------ inputs
 
 def make_layers(w, L, device):
@@ -400,11 +412,7 @@ def main():
             t1.record(stream)
         torch.cuda.synchronize(dev)
     barrier()
-    ms = t0.elapsed_time(t1)
-    if dist is not None:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), dev)
     ms_per_step = ms / args.steps
     us_layer = ms_per_step * 1e3 / L
 
@@ -451,11 +459,7 @@ def main():
             stream.synchronize()  # the host reads the step's result
         e1.record(stream)
     torch.cuda.synchronize(dev)
-    e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        tt = torch.tensor([e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e_ms = float(tt.item())
+    e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     e2e_us = e_ms * 1e3 / (e2e_steps * L)
     qbytes = q_host.numel() * q_host.element_size()
     obytes = out_host.numel() * out_host.element_size()
