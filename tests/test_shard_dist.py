@@ -102,12 +102,16 @@ W_SHARD = W.Workload(name="gqa_shard_f32", batch=2, n_q_heads=4, n_kv_heads=2, h
 Q_POS = np.array([305, 170], dtype=np.int32)
 
 
-def _rank_main(rank, world, port, result_path):
+def _workload(top_k):
+    return W.Workload(**{**W_SHARD.__dict__, "top_k": top_k})
+
+
+def _rank_main(rank, world, port, result_path, top_k):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        w = W_SHARD
+        w = _workload(top_k)
         x = synth.decode_inputs(w)
         local_lens, starts = sharded.split_lengths(w.seq_lens, world)[rank]
         ops = NumpyShardOps(w, local_lens, starts, Q_POS)
@@ -132,15 +136,17 @@ def _free_port():
         return s.getsockname()[1]
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_sharded_decoder_gloo_matches_oracle(world, tmp_path):
+@pytest.mark.parametrize("world,top_k", [(2, 48), (3, 48), (3, 120)])
+def test_sharded_decoder_gloo_matches_oracle(world, top_k, tmp_path):
+    # top_k = 120 over 3 ranks: every slice of the second sequence (57 tokens)
+    # and of the first (100) is shorter than k, so slices keep all their tokens
     path = str(tmp_path / "out.npy")
-    mp.start_processes(_rank_main, args=(world, _free_port(), path), nprocs=world, join=True,
-                       start_method="spawn")
+    mp.start_processes(_rank_main, args=(world, _free_port(), path, top_k), nprocs=world,
+                       join=True, start_method="spawn")
     outs = np.load(path)
     for r in range(1, world):
         np.testing.assert_array_equal(outs[r], outs[0])  # every rank ends with the same output
-    w = W_SHARD
+    w = _workload(top_k)
     x = synth.decode_inputs(w)
     p = problem_of(w, x["seq_offsets"].numpy(), Q_POS)
     ora = oracle.decode(p, x["q"], x["Kc"], x["Vc"], x["Pk"], x["Pv"])
