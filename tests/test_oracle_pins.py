@@ -378,6 +378,27 @@ def test_gqa_unit_score_is_sum_over_group(oracle_lib):
     np.testing.assert_array_equal(gqa["idx"], mha["idx"])
 
 
+def test_units_decompose_into_single_unit_problems(oracle_lib):
+    """Selection units are independent: a decode with U units (G = 2 query heads
+    each) equals U one-unit decodes, unit u taking its heads and its rows
+    u*d .. u*d+d-1 of Pk and Pv (technical framework: every unit selects and
+    attends on its own)."""
+    rng = np.random.default_rng(17)
+    B, Hq, Hkv, d, r, k = 2, 6, 3, 8, 6, 7
+    lens = [21, 13]
+    q = rng.standard_normal((B, Hq, d))
+    Kc, Vc = rng.standard_normal((34, r)), rng.standard_normal((34, r))
+    Pk, Pv = random_orthogonal(rng, Hkv * d, r), random_orthogonal(rng, Hkv * d, r)
+    allu = oracle_lib.decode(problem(oracle_lib, B, Hq, Hkv, d, r, k, lens), q, Kc, Vc, Pk, Pv)
+    G = Hq // Hkv
+    for u in range(Hkv):
+        rows = slice(u * d, (u + 1) * d)
+        one = oracle_lib.decode(problem(oracle_lib, B, G, 1, d, r, k, lens),
+                                q[:, u * G:(u + 1) * G], Kc, Vc, Pk[rows], Pv[rows])
+        np.testing.assert_array_equal(one["idx"][:, 0], allu["idx"][:, u])
+        np.testing.assert_allclose(one["out"], allu["out"][:, u * G:(u + 1) * G], atol=1e-13)
+
+
 def test_ragged_batch_decomposes(oracle_lib):
     rng = np.random.default_rng(14)
     Hq, Hkv, d, r = 4, 2, 8, 6
