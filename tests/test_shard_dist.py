@@ -159,3 +159,23 @@ def test_split_lengths():
     assert [p[1] for p in parts] == [[0, 0], [4, 3], [7, 5]]
     with pytest.raises(ValueError):
         sharded.split_lengths([2], 3)
+
+
+def test_sharded_decoder_checks_its_shapes(tmp_path):
+    # a one-rank gloo group in this process: the checks run before any compute
+    store = dist.FileStore(str(tmp_path / "store"), 1)
+    dist.init_process_group("gloo", store=store, rank=0, world_size=1)
+    try:
+        w = W_SHARD
+        with pytest.raises(ValueError):  # one length per sequence
+            sharded.ShardedDecoder(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.rank,
+                                   w.top_k, (300,), Q_POS, device="cpu", ops=object())
+        sd = sharded.ShardedDecoder(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.rank,
+                                    w.top_k, w.seq_lens, Q_POS, device="cpu", ops=object())
+        assert sd.world == 1 and sd.local_lens == list(w.seq_lens)
+        assert sd.shard_off.tolist() == [0, 0]
+        assert sd.local_offsets.tolist() == [0, 300, 470]
+        assert tuple(sd.cand_score_all.shape) == (1, w.batch, w.n_kv_heads, w.top_k)
+        assert tuple(sd.part_all.shape) == (1, w.batch, w.n_q_heads, w.rank + 4)
+    finally:
+        dist.destroy_process_group()
