@@ -399,6 +399,23 @@ def test_units_decompose_into_single_unit_problems(oracle_lib):
         np.testing.assert_allclose(one["out"], allu["out"][:, u * G:(u + 1) * G], atol=1e-13)
 
 
+def test_heads_permuted_within_a_group(oracle_lib):
+    """A unit's score sums its group's queries, so permuting the heads inside
+    each group keeps every selection and permutes the outputs alike."""
+    rng = np.random.default_rng(18)
+    B, Hq, Hkv, d, r, k = 2, 8, 2, 8, 8, 9
+    lens = [40, 23]
+    q = rng.standard_normal((B, Hq, d))
+    Kc, Vc = rng.standard_normal((63, r)), rng.standard_normal((63, r))
+    Pk, Pv = random_orthogonal(rng, Hkv * d, r), random_orthogonal(rng, Hkv * d, r)
+    p = problem(oracle_lib, B, Hq, Hkv, d, r, k, lens)
+    base = oracle_lib.decode(p, q, Kc, Vc, Pk, Pv)
+    perm = np.concatenate([u * 4 + rng.permutation(4) for u in range(Hkv)])
+    moved = oracle_lib.decode(p, q[:, perm], Kc, Vc, Pk, Pv)
+    np.testing.assert_array_equal(moved["idx"], base["idx"])
+    np.testing.assert_allclose(moved["out"], base["out"][:, perm], atol=1e-13)
+
+
 def test_ragged_batch_decomposes(oracle_lib):
     rng = np.random.default_rng(14)
     Hq, Hkv, d, r = 4, 2, 8, 6
