@@ -84,14 +84,20 @@ class ShardedDecoder:
 
     ``seq_lens`` are the whole sequences' lengths; this rank's slices follow
     from :func:`split_lengths`.  ``q_pos`` (int32 [B]) is the query's global
-    position and is required (a slice does not know where its sequence ends).
+    position; None takes the whole sequence's length, as the single-GPU step
+    does (a slice alone does not know where its sequence ends).
     """
 
-    def __init__(self, batch, n_q_heads, n_kv_heads, head_dim, rank, top_k, seq_lens, q_pos,
+    def __init__(self, batch, n_q_heads, n_kv_heads, head_dim, rank, top_k, seq_lens, q_pos=None,
                  group=None, rope_base=10000.0, softmax_scale=0.0, dtype=torch.bfloat16,
                  device="cuda", ops=None):
         if len(seq_lens) != batch:
             raise ValueError("seq_lens must have one length per sequence")
+        if q_pos is None:
+            q_pos = [int(n) for n in seq_lens]
+        self.q_pos = torch.as_tensor(q_pos, dtype=torch.int32)
+        if self.q_pos.shape != (batch,):
+            raise ValueError("q_pos must have one position per sequence")
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -106,7 +112,7 @@ class ShardedDecoder:
         if ops is None:
             dec = salsc.Decoder(batch, n_q_heads, n_kv_heads, head_dim, rank, top_k, local_lens,
                                 rope_base=rope_base, softmax_scale=softmax_scale, dtype=dtype,
-                                device=device, q_pos=torch.as_tensor(q_pos))
+                                device=device, q_pos=self.q_pos)
             ops = CudaShardOps(dec, self.local_offsets, self.shard_off)
         self.ops = ops
         B, U, k, Hq, W = batch, n_kv_heads, top_k, n_q_heads, self.world

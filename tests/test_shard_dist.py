@@ -177,5 +177,13 @@ def test_sharded_decoder_checks_its_shapes(tmp_path):
         assert sd.local_offsets.tolist() == [0, 300, 470]
         assert tuple(sd.cand_score_all.shape) == (1, w.batch, w.n_kv_heads, w.top_k)
         assert tuple(sd.part_all.shape) == (1, w.batch, w.n_q_heads, w.rank + 4)
+        assert sd.q_pos.tolist() == [305, 170]
+        # the default query position is the whole sequence's length
+        sd0 = sharded.ShardedDecoder(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.rank,
+                                     w.top_k, w.seq_lens, device="cpu", ops=object())
+        assert sd0.q_pos.tolist() == list(w.seq_lens)
+        with pytest.raises(ValueError):
+            sharded.ShardedDecoder(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.rank,
+                                   w.top_k, w.seq_lens, [1, 2, 3], device="cpu", ops=object())
     finally:
         dist.destroy_process_group()
