@@ -21,8 +21,9 @@ from tests.parity import max_rel_err, problem_of
 class NumpyShardOps:
     """The four per-rank steps in fp64 numpy, on this rank's slices."""
 
-    def __init__(self, w, local_lens, starts, q_pos):
+    def __init__(self, w, local_lens, starts, q_pos, tau=None):
         self.w = w
+        self.tau = tau  # threshold selection: local candidates below it are dropped
         self.lens = list(local_lens)
         self.starts = list(starts)
         self.offs = np.concatenate([[0], np.cumsum(local_lens)]).astype(np.int64)
@@ -42,6 +43,8 @@ class NumpyShardOps:
                 ql = q[b, u * G:(u + 1) * G].sum(axis=0) @ Pk[u * d:(u + 1) * d]
                 s = Kc[self._unit(b, u)] @ ql
                 order = np.lexsort((np.arange(s.size), -s))[:min(k, s.size)]
+                if self.tau is not None:
+                    order = order[s[order] >= self.tau]
                 cand_score[b, u, :order.size] = torch.from_numpy(s[order])
                 cand_idx[b, u, :order.size] = torch.from_numpy(order + self.starts[b])
 
@@ -106,7 +109,7 @@ def _workload(top_k):
     return W.Workload(**{**W_SHARD.__dict__, "top_k": top_k})
 
 
-def _rank_main(rank, world, port, result_path, top_k):
+def _rank_main(rank, world, port, result_path, top_k, tau=None):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
@@ -114,7 +117,7 @@ def _rank_main(rank, world, port, result_path, top_k):
         w = _workload(top_k)
         x = synth.decode_inputs(w)
         local_lens, starts = sharded.split_lengths(w.seq_lens, world)[rank]
-        ops = NumpyShardOps(w, local_lens, starts, Q_POS)
+        ops = NumpyShardOps(w, local_lens, starts, Q_POS, tau)
         sd = sharded.ShardedDecoder(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.rank,
                                     w.top_k, w.seq_lens, Q_POS, rope_base=w.rope_base,
                                     dtype=torch.float32, device="cpu", ops=ops)
@@ -187,3 +190,24 @@ def test_sharded_decoder_checks_its_shapes(tmp_path):
                                    w.top_k, w.seq_lens, [1, 2, 3], device="cpu", ops=object())
     finally:
         dist.destroy_process_group()
+
+
+def test_threshold_selection_decomposes_over_slices(tmp_path):
+    """Of the top-k tokens keep those scoring >= tau: each slice's top-k filtered by tau, then
+    the k best of the candidates, gives the oracle's whole-sequence threshold selection (a kept
+    token has fewer than k better tokens anywhere, all of them >= tau)."""
+    world, top_k = 3, 48
+    w = _workload(top_k)
+    x = synth.decode_inputs(w)
+    p = problem_of(w, x["seq_offsets"].numpy(), Q_POS)
+    full = oracle.decode(p, x["q"], x["Kc"], x["Vc"], x["Pk"], x["Pv"])
+    # tau between the 20th and 21st best scores of unit (0, 0): some units keep fewer than k
+    s00 = np.sort(oracle.unit_scores(p, full["scores"], 0, 0))[::-1]
+    tau = float((s00[19] + s00[20]) / 2)
+    path = str(tmp_path / "out.npy")
+    mp.start_processes(_rank_main, args=(world, _free_port(), path, top_k, tau), nprocs=world,
+                       join=True, start_method="spawn")
+    outs = np.load(path)
+    p.select_threshold = tau
+    ora = oracle.decode(p, x["q"], x["Kc"], x["Vc"], x["Pk"], x["Pv"])
+    assert max_rel_err(outs[0], ora["out"]) <= 1e-5
