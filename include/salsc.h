@@ -217,18 +217,21 @@ salsc_status salsc_decode_step_timed(const salsc_decode_desc* desc, const void* 
  * library routine).  The caller still owns q, Kc, Vc, Pk, Pv, out and idx_out.
  *
  *   - Limit: the shape's salsc_decode_workspace_size(desc) must not exceed
- *     SALSC_STATIC_WORKSPACE_BYTES (16 MiB; enough for every workload in the
- *     test-suite, e.g. 4 x 32768 tokens x 8 KV heads).  Larger shapes return
+ *     SALSC_STATIC_WORKSPACE_BYTES (16 MiB; enough for every full-size
+ *     workload of the test-suite, e.g. 4 x 32768 tokens x 8 KV heads or
+ *     245760 ragged tokens x 8 KV heads).  Larger shapes return
  *     SALSC_ERR_WORKSPACE and enqueue nothing.
  *   - Every GPU that loads this part of the library keeps the 16 MiB array
  *     until the process exits.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture.
+ *   - Every call looks up the array's device address (cudaGetSymbolAddress,
+ *     with the caller's device current).  The first call on a device also
+ *     loads the array's module: make that first call before any stream
+ *     capture.
  *   - All calls on a device share the one array and it keeps the last call's
- *     contents; each call clears the part that must start at zero.  Calls
- *     that overlap on the GPU (different streams, or different host threads
- *     without ordering) race on the array: serialise them.
+ *     contents; each call clears the part that must start at zero, after all
+ *     its arguments have been checked (a rejected call enqueues nothing).
+ *     Calls that overlap on the GPU (different streams, or different host
+ *     threads without ordering) race on the array: serialise them.
  *   - The anomaly flags of this variant are not readable by the caller.
  * Errors: as salsc_decode_step; WORKSPACE when the shape needs more scratch.
  */
@@ -237,6 +240,10 @@ salsc_status salsc_decode_step_static_ws(const salsc_decode_desc* desc, const vo
                                          const void* Kc, const void* Vc, const void* Pk,
                                          const void* Pv, void* out, int32_t* idx_out,
                                          salsc_stream stream);
+
+/* SALSC_STATIC_WORKSPACE_BYTES as compiled into the library, so that bindings
+ * need not copy the constant. */
+size_t salsc_static_workspace_bytes(void);
 
 /*
  * Decode-time append (SALS technical framework, stage 1 applied to the token
@@ -316,7 +323,11 @@ salsc_status salsc_fit_projection(const void* X, int64_t n, int32_t hidden, int3
  *                             empty slots)
  *   cand_idx      [B][U][k]   int32 global token index (-1 in empty slots)
  *   ws            workspace of salsc_decode_workspace_size(desc), prepared
- * Requires select_mode 0 (top-k); UNSUPPORTED otherwise.
+ * With select_mode 1 the local top-k keeps only scores >= select_threshold
+ * (dropped slots are empty candidates); the global selection of step 3 then
+ * equals threshold selection on the whole sequences: a kept token is among
+ * the k best overall with a score >= the threshold, so it is a candidate of
+ * its slice, and every candidate clears the threshold.
  *
  * salsc_shard_select: per unit, the k best of the N*k gathered candidates
  * (score descending, lower global index first among equal scores; empty
@@ -377,6 +388,21 @@ salsc_status salsc_shard_merge(const float* part_all, int32_t n_shards, int32_t 
  */
 salsc_status salsc_decode_read_flags(void* ws, size_t ws_bytes, uint32_t* flags_host,
                                      salsc_stream stream);
+
+/*
+ * Check of the device-side failure path (no counterpart in the SALS paper):
+ * one kernel runs the bounded wait that every pipeline wait of the decode
+ * kernels uses, on an mbarrier phase that nothing completes, with a limit of
+ * limit_ns nanoseconds (1 .. 1e9) instead of the kernels' 2 s.  The wait gives
+ * up, sets bit 1 (wait timeout) in the workspace's anomaly word and the kernel
+ * returns; no copy is in flight meanwhile.  Read the word with
+ * salsc_decode_read_flags; clear it with salsc_decode_prepare.
+ *   ws   a decode workspace (or any 256-byte aligned device buffer of at
+ *        least 16 bytes); only its anomaly word is written
+ * Errors: INVALID_ARG (limit out of range), WORKSPACE, CUDA.
+ */
+salsc_status salsc_check_wait_timeout(uint64_t limit_ns, void* ws, size_t ws_bytes,
+                                      salsc_stream stream);
 
 /* Static description of a status code. */
 const char* salsc_status_string(salsc_status status);

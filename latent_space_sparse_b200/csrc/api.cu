@@ -287,11 +287,23 @@ salsc::DecodeArgs make_args(const salsc::DecodePlan& p, const salsc_decode_desc*
   return a;
 }
 
+// The step's pointer arguments: present and aligned.
+salsc_status check_step_pointers(const salsc_decode_desc* desc, const void* q, const void* Kc,
+                                 const void* Vc, const void* Pk, const void* Pv, const void* out,
+                                 const int32_t* idx_out) {
+  if (!desc->seq_offsets_dev || !q || !Kc || !Vc || !Pk || !Pv || !out)
+    return SALSC_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(Pk) || !aligned16(Pv) ||
+      !aligned16(out) || ((uintptr_t)idx_out & 3u))
+    return SALSC_ERR_INVALID_ARG;
+  return SALSC_OK;
+}
+
 salsc_status decode_step_impl(const salsc_decode_desc* desc, const void* q, const void* Kc,
                               const void* Vc, const void* Pk, const void* Pv, void* out,
                               int32_t* idx_out, void* ws, size_t ws_bytes, salsc_stream stream,
                               void* const* events, int32_t n_events,
-                              const AppendArgs* app = nullptr) {
+                              const AppendArgs* app = nullptr, bool clear_flags = false) {
   salsc::DecodePlan p;
   salsc_status st = make_plan(desc, &p);
   if (st != SALSC_OK) return st;
@@ -299,11 +311,7 @@ salsc_status decode_step_impl(const salsc_decode_desc* desc, const void* q, cons
     if ((!app->K_new && !app->V_new) || !app->rows) return SALSC_ERR_INVALID_ARG;
     if (p.U * p.d > 8 * 1024) return SALSC_ERR_UNSUPPORTED;
   }
-  if (!desc->seq_offsets_dev || !q || !Kc || !Vc || !Pk || !Pv || !out)
-    return SALSC_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(Pk) || !aligned16(Pv) ||
-      !aligned16(out) || ((uintptr_t)idx_out & 3u))
-    return SALSC_ERR_INVALID_ARG;
+  if ((st = check_step_pointers(desc, q, Kc, Vc, Pk, Pv, out, idx_out)) != SALSC_OK) return st;
   if (events) {
     if (n_events != SALSC_DECODE_KERNELS + 1) return SALSC_ERR_INVALID_ARG;
     for (int i = 0; i < n_events; ++i)
@@ -314,6 +322,10 @@ salsc_status decode_step_impl(const salsc_decode_desc* desc, const void* q, cons
   salsc::DecodeArgs a = make_args(p, desc, q, Kc, Vc, Pk, Pv, out, idx_out, ws);
 
   cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e0;
+  // every argument has been checked: only now may anything be enqueued
+  if (clear_flags && (e0 = cudaMemsetAsync((char*)ws + p.off_flags, 0, 16, s)) != cudaSuccess)
+    return cuda_fail(e0);
   typedef cudaError_t (*launcher)(const salsc::DecodePlan&, const salsc::DecodeArgs&, cudaStream_t);
   const launcher seq[SALSC_DECODE_KERNELS] = {salsc::launch_latent_q, salsc::launch_score,
                                               salsc::launch_topk, salsc::launch_attend,
@@ -351,6 +363,23 @@ salsc_status decode_step_impl(const salsc_decode_desc* desc, const void* q, cons
 }
 
 }  // namespace
+
+salsc_status salsc::check_decode_step(const salsc_decode_desc* desc, const void* q,
+                                      const void* Kc, const void* Vc, const void* Pk,
+                                      const void* Pv, const void* out, const int32_t* idx_out) {
+  salsc::DecodePlan p;
+  const salsc_status st = make_plan(desc, &p);
+  if (st != SALSC_OK) return st;
+  return check_step_pointers(desc, q, Kc, Vc, Pk, Pv, out, idx_out);
+}
+
+salsc_status salsc::decode_step_clearing_flags(const salsc_decode_desc* desc, const void* q,
+                                               const void* Kc, const void* Vc, const void* Pk,
+                                               const void* Pv, void* out, int32_t* idx_out,
+                                               void* ws, size_t ws_bytes, salsc_stream stream) {
+  return decode_step_impl(desc, q, Kc, Vc, Pk, Pv, out, idx_out, ws, ws_bytes, stream, nullptr, 0,
+                          nullptr, true);
+}
 
 extern "C" {
 
@@ -416,7 +445,6 @@ salsc_status salsc_shard_candidates(const salsc_decode_desc* desc, const void* q
   salsc::DecodePlan p;
   salsc_status st = make_plan(desc, &p);
   if (st != SALSC_OK) return st;
-  if (desc->select_mode != 0) return SALSC_ERR_UNSUPPORTED;
   if (!desc->seq_offsets_dev || !q || !Kc || !Pk || !shard_off_dev || !cand_score || !cand_idx)
     return SALSC_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(Kc) || !aligned16(Pk) || ((uintptr_t)cand_score & 3u) ||

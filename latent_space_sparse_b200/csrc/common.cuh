@@ -80,6 +80,20 @@ struct DecodeArgs {
 // Record a CUDA error for salsc_last_cuda_error() and return SALSC_ERR_CUDA.
 salsc_status record_cuda_error(cudaError_t e);
 
+// The checks salsc_decode_step makes on its descriptor and pointers (all but
+// the workspace); host only, enqueues nothing.
+salsc_status check_decode_step(const salsc_decode_desc* desc, const void* q, const void* Kc,
+                               const void* Vc, const void* Pk, const void* Pv, const void* out,
+                               const int32_t* idx_out);
+
+// salsc_decode_step that first clears the workspace's anomaly word on the
+// stream, after every argument has been checked (a rejected call enqueues
+// nothing).
+salsc_status decode_step_clearing_flags(const salsc_decode_desc* desc, const void* q,
+                                        const void* Kc, const void* Vc, const void* Pk,
+                                        const void* Pv, void* out, int32_t* idx_out, void* ws,
+                                        size_t ws_bytes, salsc_stream stream);
+
 // Launchers (each returns the cudaError_t of its launch).
 cudaError_t launch_latent_q(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_score(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s);

@@ -72,16 +72,20 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 // null) and returns false, so that a broken pipeline ends the kernel instead of
 // hanging the GPU.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t* flags) {
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, uint32_t* flags,
+                                                uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+    if ((i & 255u) == 0u && globaltimer_ns() - t0 > limit_ns) {
       if (flags) atomicOr(flags, FLAG_WAIT_TIMEOUT);
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t* flags) {
+  return mbar_wait_limit(bar, parity, flags, kWaitLimitNs);
 }
 
 // ---------------------------------------------------------------- TMA

@@ -23,9 +23,12 @@ WS_ALIGN = 256
 
 EXPORTS = (
     "salsc_compress", "salsc_decode_workspace_size", "salsc_decode_prepare", "salsc_decode_step",
-    "salsc_decode_step_timed", "salsc_decode_step_static_ws", "salsc_decode_launch_count", "salsc_append", "salsc_decode_step_append", "salsc_fit_workspace_size",
+    "salsc_decode_step_timed", "salsc_decode_step_static_ws", "salsc_static_workspace_bytes",
+    "salsc_decode_launch_count", "salsc_append", "salsc_decode_step_append",
+    "salsc_fit_workspace_size",
     "salsc_fit_projection", "salsc_shard_candidates", "salsc_shard_select", "salsc_shard_attend",
-    "salsc_shard_merge", "salsc_decode_read_flags", "salsc_status_string", "salsc_last_cuda_error",
+    "salsc_shard_merge", "salsc_check_wait_timeout", "salsc_decode_read_flags",
+    "salsc_status_string", "salsc_last_cuda_error",
     "salsc_version",
 )
 
@@ -103,6 +106,10 @@ def _lib():
                                                 ctypes.POINTER(ctypes.c_void_p), i32]
         lib.salsc_decode_step_static_ws.restype = ctypes.c_int
         lib.salsc_decode_step_static_ws.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
+        lib.salsc_static_workspace_bytes.restype = sz
+        lib.salsc_static_workspace_bytes.argtypes = []
+        lib.salsc_check_wait_timeout.restype = ctypes.c_int
+        lib.salsc_check_wait_timeout.argtypes = [ctypes.c_uint64, vp, sz, vp]
         lib.salsc_decode_read_flags.restype = ctypes.c_int
         lib.salsc_decode_read_flags.argtypes = [vp, sz, ctypes.POINTER(ctypes.c_uint32), vp]
         lib.salsc_status_string.restype = ctypes.c_char_p
@@ -306,7 +313,9 @@ def salsc_decode_step_timed(desc: DecodeDesc, q, Kc, Vc, Pk, Pv, out, idx_out, w
     _check(st, "salsc_decode_step_timed")
 
 
-STATIC_WORKSPACE_BYTES = 16 << 20
+def static_workspace_bytes() -> int:
+    """Size of the library's fixed scratch array (salsc_decode_step_static_ws's limit)."""
+    return int(_lib().salsc_static_workspace_bytes())
 
 
 def salsc_decode_step_static_ws(desc: DecodeDesc, q, Kc, Vc, Pk, Pv, out, idx_out, stream=None):
@@ -316,6 +325,14 @@ def salsc_decode_step_static_ws(desc: DecodeDesc, q, Kc, Vc, Pk, Pv, out, idx_ou
                                             _ptr(Pk), _ptr(Pv), _ptr(out), _ptr(idx_out),
                                             _stream(stream))
     _check(st, "salsc_decode_step_static_ws")
+
+
+def salsc_check_wait_timeout(limit_ns: int, ws, stream=None):
+    """Run the decode pipelines' bounded wait on a barrier nothing completes (limit in ns);
+    the wait gives up and sets the timeout bit of ``ws``'s anomaly word."""
+    st = _lib().salsc_check_wait_timeout(int(limit_ns), _ptr(ws), ws.numel() * ws.element_size(),
+                                         _stream(stream))
+    _check(st, "salsc_check_wait_timeout")
 
 
 def salsc_decode_read_flags(ws, stream=None) -> int:

@@ -86,11 +86,15 @@ class ShardedDecoder:
     from :func:`split_lengths`.  ``q_pos`` (int32 [B]) is the query's global
     position; None takes the whole sequence's length, as the single-GPU step
     does (a slice alone does not know where its sequence ends).
+    ``select_threshold``: None for top-k selection, else threshold selection
+    (of the k best tokens of a unit, those scoring below it are dropped); the
+    local selections drop their candidates below it, which gives the same set
+    as on one GPU.
     """
 
     def __init__(self, batch, n_q_heads, n_kv_heads, head_dim, rank, top_k, seq_lens, q_pos=None,
                  group=None, rope_base=10000.0, softmax_scale=0.0, dtype=torch.bfloat16,
-                 device="cuda", ops=None):
+                 device="cuda", ops=None, select_threshold=None):
         if len(seq_lens) != batch:
             raise ValueError("seq_lens must have one length per sequence")
         if q_pos is None:
@@ -112,7 +116,8 @@ class ShardedDecoder:
         if ops is None:
             dec = salsc.Decoder(batch, n_q_heads, n_kv_heads, head_dim, rank, top_k, local_lens,
                                 rope_base=rope_base, softmax_scale=softmax_scale, dtype=dtype,
-                                device=device, q_pos=self.q_pos)
+                                device=device, q_pos=self.q_pos,
+                                select_threshold=select_threshold)
             ops = CudaShardOps(dec, self.local_offsets, self.shard_off)
         self.ops = ops
         B, U, k, Hq, W = batch, n_kv_heads, top_k, n_q_heads, self.world

@@ -240,7 +240,9 @@ def test_shard_validation_before_launch():
     assert cand(n=need - 1) == salsc.SALSC_ERR_WORKSPACE
     dt = salsc.make_desc(2, 32, 8, 128, 256, 64, host, FakeDev(1 << 23), None, 10000.0, 0.0,
                          torch.bfloat16, 0.5)
-    assert cand(dd=dt) == salsc.SALSC_ERR_UNSUPPORTED  # threshold selection is not sharded
+    # threshold selection is sharded too; its arguments are checked the same way
+    assert cand(dd=dt, q=None) == salsc.SALSC_ERR_INVALID_ARG
+    assert cand(dd=dt, n=need - 1) == salsc.SALSC_ERR_WORKSPACE
 
     def sel(cs=a, ci=b, n=2, batch=2, units=8, k=64, lo=c, so=a, out=b):
         return lib.salsc_shard_select(cs, ci, n, batch, units, k, lo, so, out, None)

@@ -75,8 +75,9 @@ def shard_inputs(x, slices):
     return x["Kc"][rows], x["Vc"][rows]
 
 
-def run_shards(w, x, n_shards, q_pos):
-    """The six steps, shard by shard, on this GPU; returns (out, global kept idx)."""
+def run_shards(w, x, n_shards, q_pos, tau=None):
+    """The six steps, shard by shard, on this GPU; returns (out, global kept idx).
+    ``tau``: threshold selection (None: top-k)."""
     offs = x["seq_offsets"].numpy()
     lens = np.diff(offs)
     B, U, k, Hq, r = len(lens), w.n_kv_heads, w.top_k, w.n_q_heads, w.rank
@@ -87,7 +88,7 @@ def run_shards(w, x, n_shards, q_pos):
     shards = []
     for local_lens, starts in parts:
         dec = salsc.Decoder(B, Hq, U, w.head_dim, r, k, local_lens, rope_base=w.rope_base,
-                            dtype=dt, device=DEV, q_pos=qp)
+                            dtype=dt, device=DEV, q_pos=qp, select_threshold=tau)
         Kc, Vc = (t.to(DEV) for t in shard_inputs(x, (local_lens, starts)))
         lo = torch.tensor(np.concatenate([[0], np.cumsum(local_lens)]), dtype=torch.int64,
                           device=DEV)
@@ -158,6 +159,43 @@ def test_sharded_decode_f32_cuda_cores():
     x = synth.decode_inputs(w)
     n = int(x["seq_offsets"][-1])
     check_sharded(w, x, 3, np.array([n + 5], dtype=np.int32))
+
+
+@pytest.mark.parametrize("frac", [0.3, 0.9])
+def test_sharded_threshold_selection_matches_the_oracle(frac):
+    # threshold selection (of the k best tokens, those scoring >= tau) over 2 and 3 shards:
+    # the kept set is the oracle's whole-sequence threshold selection up to tokens whose
+    # score lies within the tie band of the k-th score or of tau; the output matches the
+    # oracle's attention over the kept set
+    w = GQA
+    x = synth.decode_inputs(w)
+    q_pos = np.array([1500, 1100], dtype=np.int32)
+    p = problem_of(w, x["seq_offsets"].numpy(), q_pos)
+    ora = oracle.decode(p, x["q"], x["Kc"], x["Vc"], x["Pk"], x["Pv"])
+    kept = [oracle.unit_scores(p, ora["scores"], b, u)[t] for b in range(p.batch)
+            for u in range(p.n_kv_heads) for t in ora["idx"][b, u] if t >= 0]
+    tau = float(np.quantile(kept, frac))
+    p.select_threshold = tau
+    ora = oracle.decode(p, x["q"], x["Kc"], x["Vc"], x["Pk"], x["Pv"])
+    for n_shards in (2, 3):
+        out, gidx = run_shards(w, x, n_shards, q_pos, tau)
+        n_kept = 0
+        for b in range(p.batch):
+            for u in range(p.n_kv_heads):
+                s = oracle.unit_scores(p, ora["scores"], b, u)
+                g = gidx[b, u][gidx[b, u] >= 0]
+                n_kept += g.size
+                assert len(np.unique(g)) == g.size
+                o = ora["idx"][b, u]
+                o = o[o >= 0]
+                lim = 1e-4 * np.abs(s).max()
+                kth = np.sort(s)[::-1][min(p.top_k, s.size) - 1]
+                for t in np.setxor1d(g, o):
+                    assert abs(s[t] - tau) <= lim or abs(s[t] - kth) <= lim, (b, u, t, s[t], tau)
+                assert all(s[t] >= tau - lim for t in g)
+        assert n_kept > 0
+        given = oracle.attend_given_idx(p, x["q"], x["Kc"], x["Vc"], x["Pk"], x["Pv"], gidx)
+        assert max_rel_err(out, given["out"]) <= TOL[w.dtype]
 
 
 def _free_port():
