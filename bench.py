@@ -72,6 +72,10 @@ def parse_args():
                     help="time only the prefill compression GEMM and print its JSON object")
     ap.add_argument("--compress-rows", type=int, default=0,
                     help="rows of K and V for the compression GEMM (default: 16 x 4096)")
+    ap.add_argument("--no-side-workloads", action="store_true",
+                    help="time only the chosen workload (no `workloads` object)")
+    ap.add_argument("--side-steps", type=int, default=20,
+                    help="timed steps of each other decode workload")
     return ap.parse_args()
 
 
@@ -271,9 +275,22 @@ def oracle_time(inputs, n_threads: int) -> float:
     return time.perf_counter() - t0
 
 
-def cpu_baseline(w, n_threads, min_seconds: float = 10.0):
-    """The oracle on all units of sequence 0, repeated for at least
-    `min_seconds`, scaled to one layer-step of the whole batch."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline(w, n_threads, min_seconds: float = 10.0, single_seconds: float = 5.0):
+    """The oracle on all units of sequence 0 with every host core, repeated for at
+    least `min_seconds`, and on one unit single-threaded for at least
+    `single_seconds`; each extrapolated (units scaled linearly) to one
+    layer-step of the whole batch, and labelled as such."""
     total_units = w.batch * w.n_kv_heads
     inputs, units = oracle_inputs(w, w.n_kv_heads)
     secs = []
@@ -281,14 +298,35 @@ def cpu_baseline(w, n_threads, min_seconds: float = 10.0):
         secs.append(oracle_time(inputs, n_threads))
     scale = total_units / units
     mean = statistics.mean(secs)
+    inputs1, units1 = oracle_inputs(w, 1)
+    secs1 = []
+    while sum(secs1) < single_seconds:
+        secs1.append(oracle_time(inputs1, 1))
+    mean1 = statistics.mean(secs1)
+    scale1 = total_units / units1
     return {"value": mean * scale * 1e6, "unit": UNIT, "cores": n_threads, "kind": "oracle",
+            "cpu_model": cpu_model(),
             "sample": f"oracle.decode of sequence 0 ({units} of {total_units} selection units, "
                       f"n={w.seq_lens[0]}), {len(secs)} runs in {sum(secs):.1f} s, mean "
-                      f"{mean:.3f} s scaled x{scale:g} to one layer-step"}
+                      f"{mean:.3f} s, extrapolated x{scale:g} to one layer-step",
+            "extrapolated": {"sampled_units": units, "total_units": total_units,
+                             "scale": scale, "measured_s_per_sample": mean},
+            "single_thread": {"value": mean1 * scale1 * 1e6, "unit": UNIT, "cores": 1,
+                              "sample": f"oracle.decode of 1 of {total_units} units of sequence "
+                                        f"0, {len(secs1)} runs in {sum(secs1):.1f} s, mean "
+                                        f"{mean1:.3f} s, extrapolated x{scale1:g}",
+                              "extrapolated": {"sampled_units": units1,
+                                               "total_units": total_units, "scale": scale1,
+                                               "measured_s_per_sample": mean1}}}
 
 
 def run_reference(args, w):
-    """The oracle timed on the host cores: one bounded sample per step."""
+    """The oracle timed on the host cores: one bounded sample per step.
+
+    A timed step is the oracle on the first units of sequence 0 (as many as the
+    host has cores, at most all of the sequence's units); ``ms_per_step`` is
+    that sample's measured time, and ``value`` extrapolates it linearly in the
+    units to one layer-step of the whole batch (labelled in ``extrapolated``)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
@@ -298,18 +336,26 @@ def run_reference(args, w):
     for _ in range(args.warmup):
         oracle_time(inputs, n_threads)
     secs = [oracle_time(inputs, n_threads) for _ in range(args.steps)]
-    scale = w.batch * w.n_kv_heads / units
-    value = statistics.mean(secs) * scale * 1e6
+    total_units = w.batch * w.n_kv_heads
+    scale = total_units / units
+    mean = statistics.mean(secs)
+    value = mean * scale * 1e6
+    extrap = {"sampled_units": units, "total_units": total_units, "scale": scale,
+              "measured_s_per_sample": mean,
+              "how": "value = measured seconds per sample x scale, in us per layer-step; "
+                     "ms_per_step is the measured sample time"}
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": value * args.layers / 1e3, "higher_is_better": False, "scaling": "weak",
+        "ms_per_step": mean * 1e3, "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(args, w),
+        "extrapolated": extrap,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": n_threads, "kind": "oracle",
-                         "sample": f"per step: oracle.decode of {units} of "
-                                   f"{w.batch * w.n_kv_heads} units (sequence 0), scaled "
-                                   f"x{scale:g}"},
+                         "cpu_model": cpu_model(),
+                         "sample": f"per step: oracle.decode of {units} of {total_units} units "
+                                   f"(sequence 0), extrapolated x{scale:g}",
+                         "extrapolated": extrap},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -325,31 +371,86 @@ def config_of(args, w):
 
 # ------------------------------------------------------------------ main
 
-def main():
-    args = parse_args()
-    w = workloads.BY_NAME[args.workload]
-    if args.impl == "reference":
-        run_reference(args, w)
-        return
+# The other decode workloads timed beside the headline (the metric's 4K points
+# and the long-context ragged batch); each gets a `workloads` entry.
+SIDE_WORKLOADS = (workloads.LLAMA2_4K_B1.name, workloads.LLAMA2_4K_B16.name,
+                  workloads.LLAMA31_RAGGED_128K.name)
 
-    from latent_space_sparse_b200 import salsc
-    if args.compress_only:
-        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-        print(json.dumps(bench_compress(salsc, torch.device("cuda"), rows=args.compress_rows)),
-              flush=True)
-        return
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
-    L = args.layers
+def timeline_summary(tr, stages):
+    """Critical path of traced layer-steps.  tr: int64 [layers][stage][cta][3] global-timer
+    stamps (start, dependency wait returned, end; 0 = not recorded).  For each stage that
+    recorded: `critical_us` = its last CTA's end minus the previous recorded stage's last end
+    (the previous layer's last stage for the first), `wait_us` = its first returned
+    dependency wait minus that same previous end (the kernel boundary), and `span_us` = its
+    last end minus its first returned wait; means over the layers after the first."""
+    tr = np.asarray(tr, dtype=np.float64)
+    crit = {n: [] for n in stages}
+    wait = {n: [] for n in stages}
+    span = {n: [] for n in stages}
+    prev_end = None
+    step_us = []
+    for l in range(tr.shape[0]):
+        layer_start = prev_end
+        for k, n in enumerate(stages):
+            rows = tr[l, k]
+            ok = rows[:, 2] > 0
+            if not ok.any():
+                continue
+            end = rows[ok, 2].max()
+            waited = rows[ok & (rows[:, 1] > 0), 1].min() if (ok & (rows[:, 1] > 0)).any() \
+                else rows[ok, 0].min()
+            if prev_end is not None and l > 0:
+                crit[n].append((end - prev_end) / 1e3)
+                wait[n].append((waited - prev_end) / 1e3)
+                span[n].append((end - waited) / 1e3)
+            prev_end = end
+        if layer_start is not None and l > 0:
+            step_us.append((prev_end - layer_start) / 1e3)
+
+    def mean(d):
+        return {n: float(np.mean(v)) for n, v in d.items() if v}
+
+    return {"critical_us": mean(crit), "wait_us": mean(wait), "span_us": mean(span),
+            "layer_step_us": float(np.mean(step_us)) if step_us else None,
+            "how": "salsc_decode_step_traced in a CUDA graph of all layers; per-CTA "
+                   "%globaltimer stamps (start, dependency wait returned, end); critical_us = "
+                   "stage's last CTA end minus the previous stage's last end, wait_us = first "
+                   "returned dependency wait minus that end, span_us = last end minus first "
+                   "returned wait; means over layers 1..L-1"}
+
+
+def step_timeline(salsc, dec, layers, outs, idxs, stream, dev, reps=3):
+    """Per-stage critical path of the decode step from a traced graph replay."""
+    L = len(layers)
+    traces = [salsc.trace_buffer(dev) for _ in range(L)]
+
+    def traced():
+        for l, x in enumerate(layers):
+            salsc.salsc_decode_step_traced(dec.desc, x["q"], x["Kc"], x["Vc"], x["Pk"], x["Pv"],
+                                           outs[l], idxs[l], dec.ws, traces[l])
+
+    with torch.cuda.stream(stream):
+        traced()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+        traced()
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            g.replay()
+    torch.cuda.synchronize(dev)
+    del g
+    tr = torch.stack(traces).cpu().numpy()
+    return timeline_summary(tr, salsc.DECODE_KERNELS)
+
+
+def time_decode(salsc, w, L, steps, warmup, dev, local, dist, kernel_reps=None, e2e=False,
+                timeline=False):
+    """Times `steps` graph replays of one decoded token through L layers of
+    workload w (CUDA events on the replay stream, max over ranks).  Returns a
+    dict: us per layer-step, per-kernel event times, byte counts, clocks, and
+    (with e2e) the end-to-end time through the public API with host buffers."""
     dt = synth.torch_dtype(w.dtype)
     elem = 2 if w.dtype == "bf16" else 4
     layers = make_layers(w, L, dev)
@@ -383,107 +484,174 @@ def main():
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream, capture_error_mode="thread_local"):
         step()
-    nk = len(salsc.DECODE_KERNELS)
-    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(L)]
-    with torch.cuda.stream(stream):
-        for evs in kev:
-            for e in evs:
-                e.record(stream)
-    graph_t = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_t, stream=stream, capture_error_mode="thread_local"):
-        step(kev)
 
     def barrier():
         if dist is not None:
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    # ---- headline: K graph replays
     with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
+        for _ in range(warmup):
             graph.replay()
     barrier()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clocks:
         with torch.cuda.stream(stream):
             t0.record(stream)
-            for _ in range(args.steps):
+            for _ in range(steps):
                 graph.replay()
             t1.record(stream)
         torch.cuda.synchronize(dev)
     barrier()
     ms = max_over_ranks(t0.elapsed_time(t1), dev)
-    ms_per_step = ms / args.steps
-    us_layer = ms_per_step * 1e3 / L
+    res = {"ms_per_step": ms / steps, "us_layer": ms / steps * 1e3 / L,
+           "clocks": clocks.summary()}
+    del graph
 
-    # ---- per-kernel times (same work, with event marks between kernels)
-    reps = max(3, min(20, args.steps // 10))
-    per_kernel = np.zeros(nk)
-    for _ in range(reps):
+    # per-kernel times: the same work with event marks between the kernels (the
+    # marks end the programmatic-launch overlap, so each time includes its
+    # kernel's own launch latency)
+    nk = len(salsc.DECODE_KERNELS)
+    if kernel_reps:
+        kev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(L)]
         with torch.cuda.stream(stream):
-            graph_t.replay()
-        torch.cuda.synchronize(dev)
-        for evs in kev:
-            for i in range(nk):
-                per_kernel[i] += evs[i].elapsed_time(evs[i + 1])
-    per_kernel_us = per_kernel * 1e3 / (reps * L)
-    dominant = int(np.argmax(per_kernel_us))
+            for evs in kev:
+                for e in evs:
+                    e.record(stream)
+        graph_t = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_t, stream=stream, capture_error_mode="thread_local"):
+            step(kev)
+        per_kernel = np.zeros(nk)
+        for _ in range(kernel_reps):
+            with torch.cuda.stream(stream):
+                graph_t.replay()
+            torch.cuda.synchronize(dev)
+            for evs in kev:
+                for i in range(nk):
+                    per_kernel[i] += evs[i].elapsed_time(evs[i + 1])
+        res["per_kernel_us"] = per_kernel * 1e3 / (kernel_reps * L)
+        del graph_t
 
-    # ---- bytes
+    if timeline:
+        res["timeline"] = step_timeline(salsc, dec, layers, outs, idxs, stream, dev)
+
     assert dec.flags() == 0, "device-side anomaly flag set"
     idx_host = [i.cpu().numpy() for i in idxs]
-    step_bytes = algorithmic_bytes(w, idx_host, elem)
-    bytes_layer = float(np.mean(step_bytes))
+    res["bytes_layer"] = float(np.mean(algorithmic_bytes(w, idx_host, elem)))
+    res["kbytes"] = kernel_bytes(w, idx_host, elem)
+    res["launches"] = salsc.salsc_decode_launch_count(dec.desc)
+
+    if e2e:
+        # end to end through the public API with host buffers
+        q_host = q_all.cpu().pin_memory()
+        out_host = torch.empty(out_all.shape, dtype=out_all.dtype).pin_memory()
+        e2e_steps = max(3, min(steps, 50))
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(e2e_steps):
+                q_all.copy_(q_host, non_blocking=True)  # all layers' queries of this step
+                step()
+                out_host.copy_(out_all, non_blocking=True)
+                stream.synchronize()  # the host reads the step's result
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+        res["e2e"] = {"value": e_ms * 1e3 / (e2e_steps * L), "unit": UNIT,
+                      "h2d_bytes_per_step": q_host.numel() * q_host.element_size(),
+                      "d2h_bytes_per_step": out_host.numel() * out_host.element_size(),
+                      "steps": e2e_steps,
+                      "how": "eager salsc_decode_step per layer; every step copies all layers' "
+                             "q in from pinned host memory (one copy) and all outputs back (one "
+                             "copy); the host waits for each step"}
+    del layers, q_all, out_all, outs, idxs, dec
+    torch.cuda.empty_cache()
+    return res
+
+
+def step_roofline(res, peak):
+    gbs = res["bytes_layer"] / (res["us_layer"] * 1e-6) / 1e9
+    return {"bound": "hbm", "algorithmic_bytes_per_layer_step": res["bytes_layer"],
+            "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+            "frac_of_8tbs": gbs / 8000.0}
+
+
+def main():
+    args = parse_args()
+    w = workloads.BY_NAME[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    from latent_space_sparse_b200 import salsc
+    if args.compress_only:
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        print(json.dumps(bench_compress(salsc, torch.device("cuda"), rows=args.compress_rows)),
+              flush=True)
+        return
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    L = args.layers
     peak, peak_kind = measured_peaks()
-    launches = salsc.salsc_decode_launch_count(dec.desc)
-    kbytes = kernel_bytes(w, idx_host, elem)
+    # ---- headline: K graph replays of the default workload
+    reps = max(3, min(20, args.steps // 10))
+    res = time_decode(salsc, w, L, args.steps, args.warmup, dev, local, dist, kernel_reps=reps,
+                      e2e=True, timeline=True)
+    per_kernel_us = res["per_kernel_us"]
+    kbytes = res["kbytes"]
+    dominant = int(np.argmax(per_kernel_us))
     name = salsc.DECODE_KERNELS[dominant]
     ach = kbytes[name] / (per_kernel_us[dominant] * 1e-6) / 1e9
     roofline = {"kernel": name, "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
                 "frac": ach / peak, "traffic": PROFILED_TRAFFIC.get((w.name, name)),
-                "peak_kind": peak_kind, "algorithmic_bytes_per_launch": kbytes[name]}
-    step_gbs = bytes_layer / (us_layer * 1e-6) / 1e9
-
-    # ---- end to end through the public API with host buffers
-    q_host = q_all.cpu().pin_memory()
-    out_host = torch.empty(out_all.shape, dtype=out_all.dtype).pin_memory()
-    e2e_steps = max(3, min(args.steps, 50))
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            q_all.copy_(q_host, non_blocking=True)  # all layers' queries of this step
-            step()
-            out_host.copy_(out_all, non_blocking=True)
-            stream.synchronize()  # the host reads the step's result
-        e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
-    e2e_us = e_ms * 1e3 / (e2e_steps * L)
-    qbytes = q_host.numel() * q_host.element_size()
-    obytes = out_host.numel() * out_host.element_size()
+                "peak_kind": peak_kind, "algorithmic_bytes_per_launch": kbytes[name],
+                "time": "per_kernel_us (event-separated: includes the kernel's launch latency)"}
 
     line = {
-        "metric": METRIC, "value": us_layer, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "metric": METRIC, "value": res["us_layer"], "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic", "config": config_of(args, w),
-        "clocks": clocks.summary(),
-        "gpu_launches": launches * L * args.steps,
+        "clocks": res["clocks"],
+        "gpu_launches": res["launches"] * L * args.steps,
         "roofline": roofline,
-        "step_roofline": {"bound": "hbm", "algorithmic_bytes_per_layer_step": bytes_layer,
-                          "achieved": step_gbs, "peak": peak, "unit": "GB/s",
-                          "frac": step_gbs / peak, "frac_of_8tbs": step_gbs / 8000.0},
+        "step_roofline": step_roofline(res, peak),
         "per_kernel_us": {n: float(v) for n, v in zip(salsc.DECODE_KERNELS, per_kernel_us)},
         "per_kernel_gbs": {n: (kbytes[n] / (v * 1e-6) / 1e9 if kbytes[n] else 0.0)
                            for n, v in zip(salsc.DECODE_KERNELS, per_kernel_us)},
-        "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": qbytes,
-                "d2h_bytes_per_step": obytes, "steps": e2e_steps,
-                "how": "eager salsc_decode_step per layer; every step copies all layers' q in "
-                       "from pinned host memory (one copy) and all outputs back (one copy); "
-                       "the host waits for each step"},
+        "e2e": res["e2e"],
+        "timeline": res["timeline"],
     }
+    # ---- the other decode workloads (the metric's 4K points, long context)
+    if not args.no_side_workloads:
+        side = {}
+        for name_w in SIDE_WORKLOADS:
+            if name_w == w.name:
+                continue
+            ws = workloads.BY_NAME[name_w]
+            r2 = time_decode(salsc, ws, L, args.side_steps, args.warmup, dev, local, dist,
+                             kernel_reps=3, timeline=True)
+            side[name_w] = {
+                "value": r2["us_layer"], "unit": UNIT, "steps": args.side_steps,
+                "ms_per_step": r2["ms_per_step"], "clocks": r2["clocks"],
+                "step_roofline": step_roofline(r2, peak),
+                "per_kernel_us": {n: float(v)
+                                  for n, v in zip(salsc.DECODE_KERNELS, r2["per_kernel_us"])},
+                "gpu_launches": r2["launches"] * L * args.side_steps,
+                "timeline": r2["timeline"],
+                "config": config_of(args, ws)}
+        line["workloads"] = side
     if not args.no_compress:
         line["compress"] = bench_compress(salsc, dev, rows=args.compress_rows)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -491,7 +659,6 @@ def main():
         line["cpu_baseline"] = cpu_baseline(w, oracle.default_threads())
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graph, graph_t
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()

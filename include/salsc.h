@@ -206,6 +206,31 @@ salsc_status salsc_decode_step_timed(const salsc_decode_desc* desc, const void* 
                                      salsc_stream stream, void* const* events, int32_t n_events);
 
 /*
+ * salsc_decode_step with a timeline: the same work, and every kernel of the
+ * step records, per CTA, the global nanosecond timer (%globaltimer) when the
+ * CTA starts, when its dependency wait on the previous stage returns, and
+ * when it ends:
+ *   trace[((k * SALSC_TRACE_MAX_CTAS) + c) * 3 + {0, 1, 2}]
+ * for stage k < SALSC_DECODE_KERNELS (latent query, scoring, top-k,
+ * attention, merge) and CTA c = blockIdx.y * gridDim.x + blockIdx.x <
+ * SALSC_TRACE_MAX_CTAS.  Entries of CTAs that do not exist, and of kernels
+ * that do not record (the CUDA-core scoring and attention of fp32 storage, a
+ * merge stage that launches nothing), are left as they were: clear the buffer
+ * first.  trace: device memory of at least trace_bytes >= 3 * 8 *
+ * SALSC_DECODE_KERNELS * SALSC_TRACE_MAX_CTAS bytes, 8-byte aligned.  The
+ * kernels are the ones salsc_decode_step launches, with the same launch
+ * shapes and programmatic dependent launches; each stamp is one store.
+ * Errors: as salsc_decode_step; INVALID_ARG for a missing, misaligned or short
+ * trace buffer.
+ */
+#define SALSC_TRACE_MAX_CTAS 8192
+salsc_status salsc_decode_step_traced(const salsc_decode_desc* desc, const void* q,
+                                      const void* Kc, const void* Vc, const void* Pk,
+                                      const void* Pv, void* out, int32_t* idx_out, void* ws,
+                                      size_t ws_bytes, uint64_t* trace, size_t trace_bytes,
+                                      salsc_stream stream);
+
+/*
  * Decode step whose scratch is a fixed array inside the library, for callers
  * that cannot allocate device memory (no counterpart in the SALS paper).
  *

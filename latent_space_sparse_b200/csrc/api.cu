@@ -11,6 +11,10 @@
 
 namespace {
 
+// Unit-group partition of the attention tiles (CTA groups per unit, runs per
+// sequence) instead of one contiguous range of tile numbers per CTA.
+constexpr bool kUnitGroups = false;
+
 thread_local char g_last_cuda_error[256] = "no error";
 
 salsc_status cuda_fail(cudaError_t e) {
@@ -125,6 +129,8 @@ salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
     p.att_tiles = 0;
   }
   p.att_cluster = p.attend_tc ? salsc::attend_merge_cluster(p) : 0;
+  // unit groups need a CTA per unit at least
+  p.att_share = kUnitGroups && p.attend_tc && p.att_cluster == 0 && salsc::attend_tc_grid(p) >= p.U;
   if (!salsc::combine_supported(p)) return SALSC_ERR_UNSUPPORTED;
   p.scale = D->softmax_scale != 0.0f ? D->softmax_scale : (float)(1.0 / sqrt((double)p.d));
   p.rope_base = D->rope_base;
@@ -277,6 +283,7 @@ salsc::DecodeArgs make_args(const salsc::DecodePlan& p, const salsc_decode_desc*
   a.out = out;
   a.idx = idx_out ? idx_out : (int32_t*)(w + p.off_idx);
   a.seq_off = desc->seq_offsets_dev;
+  a.seq_off_host = desc->seq_offsets_host;
   a.q_pos = desc->q_pos_dev;
   a.flags = (uint32_t*)(w + p.off_flags);
   a.qlat = (float*)(w + p.off_qlat);
@@ -303,7 +310,8 @@ salsc_status decode_step_impl(const salsc_decode_desc* desc, const void* q, cons
                               const void* Vc, const void* Pk, const void* Pv, void* out,
                               int32_t* idx_out, void* ws, size_t ws_bytes, salsc_stream stream,
                               void* const* events, int32_t n_events,
-                              const AppendArgs* app = nullptr, bool clear_flags = false) {
+                              const AppendArgs* app = nullptr, bool clear_flags = false,
+                              uint64_t* trace = nullptr) {
   salsc::DecodePlan p;
   salsc_status st = make_plan(desc, &p);
   if (st != SALSC_OK) return st;
@@ -320,6 +328,7 @@ salsc_status decode_step_impl(const salsc_decode_desc* desc, const void* q, cons
   if ((st = check_ws(p, ws, ws_bytes)) != SALSC_OK) return st;
 
   salsc::DecodeArgs a = make_args(p, desc, q, Kc, Vc, Pk, Pv, out, idx_out, ws);
+  a.trace = trace;
 
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e0;
@@ -397,6 +406,18 @@ salsc_status salsc_decode_step_append(const salsc_decode_desc* desc, const void*
   const AppendArgs app{K_new, V_new, rows_dev};
   return decode_step_impl(desc, q, Kc, Vc, Pk, Pv, out, idx_out, ws, ws_bytes, stream, nullptr, 0,
                           &app);
+}
+
+salsc_status salsc_decode_step_traced(const salsc_decode_desc* desc, const void* q,
+                                      const void* Kc, const void* Vc, const void* Pk,
+                                      const void* Pv, void* out, int32_t* idx_out, void* ws,
+                                      size_t ws_bytes, uint64_t* trace, size_t trace_bytes,
+                                      salsc_stream stream) {
+  if (!trace || ((uintptr_t)trace & 7u) ||
+      trace_bytes < sizeof(uint64_t) * 3 * (size_t)SALSC_DECODE_KERNELS * SALSC_TRACE_MAX_CTAS)
+    return SALSC_ERR_INVALID_ARG;
+  return decode_step_impl(desc, q, Kc, Vc, Pk, Pv, out, idx_out, ws, ws_bytes, stream, nullptr, 0,
+                          nullptr, false, trace);
 }
 
 salsc_status salsc_decode_step_timed(const salsc_decode_desc* desc, const void* q, const void* Kc,
@@ -488,6 +509,7 @@ salsc_status salsc_shard_attend(const salsc_decode_desc* desc, const void* q, co
   // the shards' partials are merged after the exchange, so the attention
   // kernel does not merge (nor project) them itself
   p.att_cluster = 0;
+  p.att_share = kUnitGroups && p.attend_tc && salsc::attend_tc_grid(p) >= p.U;
   if (!desc->seq_offsets_dev || !desc->q_pos_dev || !q || !Kc || !Vc || !Pk || !idx_local ||
       !shard_off_dev || !part_out)
     return SALSC_ERR_INVALID_ARG;

@@ -74,17 +74,29 @@ struct AttendTcParams {
   __nv_bfloat16* out;
   int B, Hq, U, r, k, n_slots, n_tiles;
   int cluster;  // merged in the kernel: CTAs per unit (one thread-block cluster)
+  int share;    // 1: unit-group partition of the tiles (else a contiguous range)
+  uint64_t* trace;  // traced step: this kernel's rows, or null
   float scale;
   double base;
 };
 
-// Walks the tiles of all units in order (sequence, unit, slot); unit (b, u)
-// has ceil(min(k, n_b) / 128) tiles.
+// Walks the tiles of a CTA.  Tiles are numbered in the order (sequence,
+// unit, slot); unit (b, u) has tb = ceil(min(k, n_b) / 128) tiles.  Two
+// partitions over the grid of g CTAs:
+//   - a contiguous range of tile numbers (start);
+//   - unit groups (begin_group, for g >= U): the CTAs are split into U groups
+//     of m = floor((u+1)g/U) - floor(ug/U) consecutive CTAs, group u taking
+//     unit u of every sequence; in sequence b the unit's tb tiles are cut
+//     into m runs [floor(r*tb/m), floor((r+1)*tb/m)), and CTA i of the group
+//     takes run r = (i + floor(b*m/B)) mod m.  A CTA then keeps one unit
+//     (one Pk_u), works on the sequences in order, and the rotation spreads
+//     the empty runs (tb < m) over the CTAs.
 struct UnitTileCursor {
   const int64_t* so;
   int B, U, k;
   int b, u, slot, tb;
   int64_t off, nb, kb;
+  int gi, gm, hi;  // unit-group mode (gm > 0): CTA gi of the unit's gm, run end hi
   __device__ void load() {
     off = so[b];
     nb = so[b + 1] - off;
@@ -96,6 +108,7 @@ struct UnitTileCursor {
     B = B_;
     U = U_;
     k = k_;
+    gm = 0;
     int acc = 0;
     for (b = 0; b < B; ++b) {
       load();
@@ -108,7 +121,32 @@ struct UnitTileCursor {
       acc += U * tb;
     }
   }
+  // unit-group mode: the first tile of this CTA's run in sequence b0 or later
+  __device__ void seek(int b0) {
+    for (b = b0; b < B; ++b) {
+      load();
+      const int r = (gi + b * gm / B) % gm;
+      slot = r * tb / gm;
+      hi = (r + 1) * tb / gm;
+      if (slot < hi) return;
+    }
+  }
+  __device__ void begin_group(const int64_t* so_, int B_, int U_, int k_, int c, int g) {
+    so = so_;
+    B = B_;
+    U = U_;
+    k = k_;
+    u = (int)(((int64_t)(c + 1) * U - 1) / g);  // the group of CTA c
+    const int c0 = (int)((int64_t)u * g / U);
+    gm = (int)((int64_t)(u + 1) * g / U) - c0;
+    gi = c - c0;
+    seek(0);
+  }
   __device__ void next() {
+    if (gm > 0) {
+      if (++slot >= hi) seek(b + 1);
+      return;
+    }
     if (++slot >= tb) {
       slot = 0;
       if (++u >= U) {
@@ -119,6 +157,14 @@ struct UnitTileCursor {
   }
 };
 
+// Tiles of CTA c of g in the unit-group partition.
+__device__ __forceinline__ int group_tiles(const int64_t* so, int B, int U, int k, int c, int g) {
+  UnitTileCursor t;
+  t.begin_group(so, B, U, k, c, g);
+  int n = 0;
+  for (; t.b < B; t.seek(t.b + 1)) n += t.hi - t.slot;
+  return n;
+}
 
 // Token of row `row` of the cursor's tile, or -1 past the unit's k_b kept
 // tokens or on -1 (a slot threshold selection left empty); any other index
@@ -210,6 +256,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
   auto bar = [bar0](int i) { return bar0 + 8u * (uint32_t)i; };
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  if (tid == 0) trace_stamp(P.trace, TRACE_START);
   allow_dependent_launch();
   // Tile range: a contiguous share of all tiles, or (kMerge) the rank's share
   // of its unit's tiles, the unit being (blockIdx.x / cluster).
@@ -227,10 +274,20 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     const int lo = tu * m_rank / P.cluster, hi = tu * (m_rank + 1) / P.cluster;
     t_begin = before + (m_unit % P.U) * tu + lo;
     n = hi - lo;
+  } else if (P.share) {
+    t_begin = 0;
+    n = group_tiles(P.seq_off, P.B, P.U, P.k, (int)blockIdx.x, (int)gridDim.x);
   } else {
     t_begin = (int)((int64_t)blockIdx.x * P.n_tiles / gridDim.x);
     n = (int)((int64_t)(blockIdx.x + 1) * P.n_tiles / gridDim.x) - t_begin;
   }
+  // the CTA's first tile
+  auto first_tile = [&](UnitTileCursor& c) {
+    if (!kMerge && P.share)
+      c.begin_group(P.seq_off, P.B, P.U, P.k, (int)blockIdx.x, (int)gridDim.x);
+    else
+      c.start(P.seq_off, P.B, P.U, P.k, t_begin);
+  };
   // TMEM columns: K_sel [2][D], then acc [2][n_chunks * 16]
   const uint32_t o_col0 = 2 * D;
   const uint32_t o_cols = (uint32_t)n_chunks * 16;
@@ -267,8 +324,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     const uint32_t buf_s = tc::smem_u32(h ? s_buf1 : s_buf0);
     const uint32_t tile_bytes = (uint32_t)kTile * KB * 128;
     UnitTileCursor cur;
-    cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
+    first_tile(cur);
     grid_dependency_wait();  // the kept indices come from the previous kernel
+    if (gt == 0 && h == 0) trace_stamp(P.trace, TRACE_WAITED);
     int t_next[kGatherRows];
 #pragma unroll
     for (int j = 0; j < kGatherRows; ++j)
@@ -307,7 +365,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       const uint32_t idesc_v = tc::idesc_bf16_f32_amn(128, kPRows);
       const uint32_t pkb = tc::smem_u32(s_pk);
       UnitTileCursor cur;
-      cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
+      first_tile(cur);
       uint32_t pk_phase = 0, pkd_phase = 0;
       auto load_pk = [&](int u, int hh) {
         if (tc::elect_one()) {
@@ -400,9 +458,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     const uint32_t buf_s = tc::smem_u32(bi ? s_buf1 : s_buf0);
     const uint32_t tile_bytes = (uint32_t)kTile * P.r * 2;
     UnitTileCursor cur;
-    cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
+    first_tile(cur);
     if (bi == 1) cur.next();
     grid_dependency_wait();  // the kept indices come from the previous kernel
+    if (gt == 0 && bi == 0) trace_stamp(P.trace, TRACE_WAITED);
     int t_next[kGatherRows];
 #pragma unroll
     for (int j = 0; j < kGatherRows; ++j)
@@ -449,8 +508,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       const uint32_t idesc_k = tc::idesc_bf16_f32(kTile, D);
       const uint32_t idesc_v = tc::idesc_bf16_f32_amn(128, kPRows);
       UnitTileCursor cur;
-      cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
-      int cur_b = -1, cur_u = -1;
+      first_tile(cur);
+      int cur_u = -1;
       uint32_t pk_phase = 0;
       int pk_step = 0;  // 1: waiting to reload Pk, 2: Pk load in flight
       int nk = 0, np = 0;
@@ -462,7 +521,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       while (np < n) {
         bool progress = false;
         if (nk < n && nk <= np + 2) {
-          if (pk_step == 0 && (cur.b != cur_b || cur.u != cur_u)) pk_step = 1;
+          if (pk_step == 0 && cur.u != cur_u) pk_step = 1;  // Pk_u: the unit's rows of Pk
           // Pk_u of a new unit, once the previous reconstruction is done with Pk
           if (pk_step == 1 &&
               (nk == 0 || ready(bar(B_KDONE + ((nk - 1) & 1)), ((uint32_t)(nk - 1) >> 1) & 1u))) {
@@ -478,7 +537,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
           }
           if (pk_step == 2 && ready(bar(B_PK), pk_phase)) {
             pk_phase ^= 1u;
-            cur_b = cur.b;
             cur_u = cur.u;
             pk_step = 0;
             progress = true;
@@ -570,7 +628,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     const int quarter = warp & 3, part = warp >> 2;
     const int m = quarter * 32 + lane;  // token row = TMEM lane
     UnitTileCursor cur;
-    cur.start(P.seq_off, P.B, P.U, P.k, t_begin);
+    first_tile(cur);
     int cur_b = -1, cur_u = -1;
     uint32_t pos_b = 0;  // position of the sequence's token 0 (token-sharded caches)
     // the segment's running sums: slot s = part + kEpiParts*j (j < kSlots) holds latent
@@ -883,6 +941,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
   }
   tc::fence_before_sync();
   __syncthreads();
+  if (tid == 0) trace_stamp(P.trace, TRACE_END);
   if (warp == kMmaWarp) {
     __syncwarp();
     tc::fence_after_sync();
@@ -941,6 +1000,8 @@ cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s)
   P.n_slots = p.splits;
   P.n_tiles = p.att_tiles;
   P.cluster = kMerge ? p.att_cluster : 1;
+  P.share = kMerge ? 0 : (p.att_share ? 1 : 0);
+  P.trace = trace_of(a, 3);
   P.scale = p.scale;
   P.base = p.rope_base;
   if constexpr (!kMerge) {

@@ -36,7 +36,8 @@ constexpr int kThreads = 256;
 constexpr int kRows = 16;                      // output rows per CTA
 constexpr int kTpr = kThreads / kRows;         // threads per output row
 constexpr int kColsPer = kMaxRank / kThreads;  // latent columns per thread (r <= 512)
-constexpr uint32_t kRowBuf = 32u * 1024u;      // bytes of partial rows per batch
+constexpr uint32_t kRowBuf = 72u * 1024u;      // most bytes of partial rows per batch
+constexpr size_t kPairSmem = 100u * 1024u;     // dynamic shared memory that fits two CTAs per SM
 constexpr int kMaxSegs = kMaxShardCandidates / 64 > 128 ? kMaxShardCandidates / 64 : 128;
 
 struct CombineParams {
@@ -47,9 +48,12 @@ struct CombineParams {
   uint32_t* flags;
   int B, Hq, U, d, r, k, n_slots, chunk;
   int seg_grid, seg_tiles;  // tensor-core tile partition (seg_grid = 0: every slot used)
+  int share;                // 1: unit-group partition (CTA groups per unit, runs per sequence)
   int64_t bh_stride, slot_stride;  // partial row of (b, h, slot): (b*Hq + h)*bh_stride + slot*slot_stride
   float* part_out;  // non-null: write the merged partial row of every head, no projection
   int fixed_slots;  // > 0: every unit has this many slots (no tile count from the lengths)
+  uint64_t* trace;  // traced step: this kernel's rows, or null
+  uint32_t rowbuf;  // bytes of partial rows per batch (a multiple of one row per head)
 };
 
 template <typename T, int G>
@@ -59,7 +63,7 @@ combine_kernel(const CombineParams P) {
   const int rowf = part_row(P.r);  // floats per partial row
   T* const pv_s = (T*)smem;                                                 // [16][r]
   float* const rows_s = (float*)(smem + (size_t)kRows * P.r * sizeof(T));  // batch of rows
-  float* const acc_s = rows_s + kRowBuf / 4;                                // [G][r]
+  float* const acc_s = rows_s + P.rowbuf / 4;                               // [G][r]
   float* const w_s = acc_s + G * P.r;                                       // [G][32]
   __shared__ int s_seg[kMaxSegs];
   __shared__ int s_nseg, s_ok;
@@ -73,6 +77,7 @@ combine_kernel(const CombineParams P) {
   const int b = bu / P.U, u = bu % P.U;
   const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
   const uint32_t pv_bytes = (uint32_t)(kRows * P.r * sizeof(T));
+  if (tid == 0) trace_stamp(P.trace, TRACE_START);
   if (tid == 0) {
     tc::mbar_init(bar_pv, 1);
     tc::mbar_init(bar_rows, 1);
@@ -115,9 +120,16 @@ combine_kernel(const CombineParams P) {
       const int sl = s0 + lane;
       bool used = sl < tb;
       if (used && sl > 0 && P.seg_grid > 0) {
-        const int64_t t = unit_tile0 + sl;
-        const int64_t c = (t * P.seg_grid + P.seg_tiles - 1) / P.seg_tiles;  // first CTA at or after t
-        used = c < P.seg_grid && c * P.seg_tiles / P.seg_grid == t;
+        // tile t starts a CTA's range in a partition of T tiles over gc CTAs:
+        // all tiles over the grid, or (unit groups) the unit's tb tiles of
+        // this sequence over the unit's group of CTAs
+        const int64_t gc = P.share ? (int64_t)(u + 1) * P.seg_grid / P.U -
+                                         (int64_t)u * P.seg_grid / P.U
+                                   : P.seg_grid;
+        const int64_t t = P.share ? sl : unit_tile0 + sl;
+        const int64_t T = P.share ? tb : P.seg_tiles;
+        const int64_t c = (t * gc + T - 1) / T;  // first CTA at or after t
+        used = c < gc && c * T / gc == t;
       }
       const uint32_t mk = __ballot_sync(0xffffffffu, used);
       if (used) s_seg[cnt + __popc(mk & ((1u << lane) - 1u))] = sl;
@@ -130,6 +142,7 @@ combine_kernel(const CombineParams P) {
     }
   }
   grid_dependency_wait();  // the partials come from the attention kernel
+  if (tid == 0) trace_stamp(P.trace, TRACE_WAITED);
   __syncthreads();
   const int nseg = s_nseg;
   // this thread's latent columns tid, tid + 256 for every head
@@ -138,20 +151,20 @@ combine_kernel(const CombineParams P) {
   for (int g = 0; g < G; ++g)
 #pragma unroll
     for (int j = 0; j < kColsPer; ++j) acc[g][j] = 0.f;
-  int bs = (int)(kRowBuf / (uint32_t)(rowf * 4)) / G;  // slots per batch
-  if (bs * G > 32) bs = 32 / G;  // one row copy per lane of warp 0
+  int bs = (int)(P.rowbuf / (uint32_t)(rowf * 4)) / G;  // slots per batch
+  if (bs > 32) bs = 32;  // one weight per lane of a head's warp
   const float* part_u = P.part + ((int64_t)b * P.Hq + (int64_t)u * G) * P.bh_stride * rowf;
   uint32_t phase = 0;
   bool ok = true;
   for (int q0 = 0; q0 < nseg; q0 += bs, phase ^= 1u) {
     const int nq = nseg - q0 < bs ? nseg - q0 : bs;
     if (warp == 0) {
-      // lane e copies row e = (head e / nq, slot q0 + e % nq); one warp waits
+      // lanes copy rows e = (head e / nq, slot q0 + e % nq); one warp waits
       if (lane == 0) tc::mbar_expect_tx(bar_rows, (uint32_t)(G * nq * rowf * 4));
       __syncwarp();
-      if (lane < G * nq) {
-        const int g = lane / nq, j = lane % nq;
-        tc::bulk_load(tc::smem_u32(rows_s + (size_t)lane * rowf),
+      for (int e = lane; e < G * nq; e += 32) {
+        const int g = e / nq, j = e % nq;
+        tc::bulk_load(tc::smem_u32(rows_s + (size_t)e * rowf),
                       part_u + ((int64_t)g * P.bh_stride + s_seg[q0 + j] * P.slot_stride) * rowf,
                       (uint32_t)(rowf * 4), bar_rows);
       }
@@ -213,6 +226,7 @@ combine_kernel(const CombineParams P) {
       po[(int64_t)tid * rowf + 2] = 0.f;
       po[(int64_t)tid * rowf + 3] = 0.f;
     }
+    if (tid == 0) trace_stamp(P.trace, TRACE_END);
     return;
   }
 #pragma unroll
@@ -255,17 +269,75 @@ combine_kernel(const CombineParams P) {
 #pragma unroll
     for (int g = 0; g < G; ++g) out[(int64_t)g * P.d] = from_f32<T>(o[g]);
   }
+  if (tid == 0) trace_stamp(P.trace, TRACE_END);
 }
 
-size_t combine_smem(const DecodePlan& p) {
+size_t combine_smem(const DecodePlan& p, uint32_t rowbuf) {
   const size_t elem = p.dtype == SALSC_BF16 ? 2 : 4;
-  return (size_t)kRows * p.r * elem + kRowBuf + sizeof(float) * (size_t)p.G * (p.r + 32);
+  return (size_t)kRows * p.r * elem + rowbuf + sizeof(float) * (size_t)p.G * (p.r + 32);
+}
+
+// Most used slots of any unit: the CTAs of the tensor-core partition that meet
+// the unit's tiles, or every slot.
+int max_used_slots(const DecodePlan& p, const int64_t* seq_off_host, int seg_grid, int fixed) {
+  if (fixed > 0) return fixed;
+  if (seg_grid <= 0 || !seq_off_host || p.att_tiles <= 0) return p.splits;
+  int most = 1;
+  int64_t tile = 0;
+  for (int b = 0; b < p.B; ++b) {
+    const int64_t nb = seq_off_host[b + 1] - seq_off_host[b];
+    const int64_t kb = nb < p.k ? nb : p.k;
+    const int64_t tb = (kb + p.chunk - 1) / p.chunk;
+    for (int u = 0; u < p.U; ++u, tile += tb) {
+      // CTA c covers tiles [c*T/gc, (c+1)*T/gc) of a partition of T tiles over
+      // gc CTAs (all tiles over the grid; with unit groups, the unit's tb
+      // tiles of this sequence over its group): the CTA of tile t is
+      // ((t+1)*gc - 1) / T, and the unit's tiles meet at most the CTAs from
+      // its first tile's to its last tile's
+      const int64_t gc = p.att_share ? (int64_t)(u + 1) * seg_grid / p.U -
+                                           (int64_t)u * seg_grid / p.U
+                                     : seg_grid;
+      const int64_t T = p.att_share ? tb : p.att_tiles;
+      const int64_t t0 = p.att_share ? 0 : tile;
+      const int64_t n = ((t0 + tb) * gc - 1) / T - ((t0 + 1) * gc - 1) / T + 1;
+      if (n > most) most = (int)n;
+    }
+  }
+  return most < p.splits ? most : p.splits;
+}
+
+// Bytes of partial rows per batch: every used slot of a unit at once, within
+// kRowBuf.
+uint32_t rowbuf_bytes(const DecodePlan& p, int maxseg) {
+  const uint64_t row = (uint64_t)p.G * part_row(p.r) * 4;
+  uint64_t want = row * (uint64_t)maxseg;
+  if (want > kRowBuf) want = kRowBuf / row * row;
+  if (want < row) want = row;
+  return (uint32_t)want;
+}
+
+int num_sms_cb() {
+  static int cached[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
 }
 
 template <typename T, int G>
 cudaError_t launch_tg(const CombineParams& P, const DecodePlan& p, cudaStream_t s) {
   static int done[kMaxDevices] = {};
-  const size_t smem = combine_smem(p);
+  size_t smem = combine_smem(p, P.rowbuf);
+  // A grid of at most two CTAs per SM asks for enough shared memory that no
+  // more than two fit on an SM: the CTAs launched early, while the attention
+  // kernel still holds most SMs, would otherwise pile up on the few free SMs
+  // and run their share one after another.
+  const int64_t ctas = (int64_t)p.B * p.U * (P.part_out ? 1 : p.d / kRows);
+  if (ctas <= 2 * (int64_t)num_sms_cb() && smem < kPairSmem) smem = kPairSmem;
   cudaError_t e = ensure_smem(combine_kernel<T, G>, smem, done);
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)(p.B * p.U * (P.part_out ? 1 : p.d / kRows)));
@@ -311,14 +383,18 @@ CombineParams base_params(const DecodePlan& p, const DecodeArgs& a) {
   P.chunk = p.chunk;
   P.seg_grid = p.attend_tc ? attend_tc_grid(p) : 0;
   P.seg_tiles = p.att_tiles;
+  P.share = p.att_share ? 1 : 0;
   P.bh_stride = p.splits;
   P.slot_stride = 1;
   P.part_out = nullptr;
   P.fixed_slots = 0;
+  P.trace = trace_of(a, 4);
   return P;
 }
 
-cudaError_t launch_params(const CombineParams& P, const DecodePlan& p, cudaStream_t s) {
+cudaError_t launch_params(CombineParams P, const DecodePlan& p, const int64_t* seq_off_host,
+                          cudaStream_t s) {
+  P.rowbuf = rowbuf_bytes(p, max_used_slots(p, seq_off_host, P.seg_grid, P.fixed_slots));
   return p.dtype == SALSC_BF16 ? launch_t<__nv_bfloat16>(P, p, s) : launch_t<float>(P, p, s);
 }
 
@@ -327,7 +403,7 @@ cudaError_t launch_params(const CombineParams& P, const DecodePlan& p, cudaStrea
 cudaError_t launch_combine(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
   if (p.att_cluster > 0) return cudaSuccess;  // the attention kernel merged the partials
   if (!combine_supported(p)) return cudaErrorInvalidConfiguration;
-  return launch_params(base_params(p, a), p, s);
+  return launch_params(base_params(p, a), p, a.seq_off_host, s);
 }
 
 cudaError_t launch_combine_partial(const DecodePlan& p, const DecodeArgs& a, float* part_out,
@@ -335,7 +411,7 @@ cudaError_t launch_combine_partial(const DecodePlan& p, const DecodeArgs& a, flo
   if (p.att_cluster > 0 || !combine_supported(p)) return cudaErrorInvalidConfiguration;
   CombineParams P = base_params(p, a);
   P.part_out = part_out;
-  return launch_params(P, p, s);
+  return launch_params(P, p, a.seq_off_host, s);
 }
 
 cudaError_t launch_shard_merge(const DecodePlan& p, const float* part_all, int n_shards,
@@ -353,7 +429,7 @@ cudaError_t launch_shard_merge(const DecodePlan& p, const float* part_all, int n
   P.fixed_slots = n_shards;
   P.bh_stride = 1;
   P.slot_stride = (int64_t)p.B * p.Hq;
-  return launch_params(P, p, s);
+  return launch_params(P, p, nullptr, s);
 }
 
 }  // namespace salsc

@@ -51,6 +51,8 @@ struct DecodePlan {
   int att_tiles;        // sum over units of ceil(k_b / 128) (tensor-core path)
   int att_cluster;      // > 0: the attention kernel merges each unit's partials and projects
                         // them itself, one cluster of att_cluster CTAs per unit (no merge kernel)
+  bool att_share;       // tensor-core attention CTA c takes its share of every sequence's tiles
+                        // (else a contiguous range of all tiles)
   float scale;
   double rope_base;
   // workspace layout (byte offsets)
@@ -67,6 +69,7 @@ struct DecodeArgs {
   void* out;
   int32_t* idx;  // [B][U][k] (caller's or workspace)
   const int64_t* seq_off;
+  const int64_t* seq_off_host = nullptr;  // the same offsets on the host (launch shapes)
   const int32_t* q_pos;
   uint32_t* flags;
   float* qlat;                 // [B][U][r]
@@ -75,7 +78,27 @@ struct DecodeArgs {
   uint32_t* krange;            // [B][U][2] (min, max) order key of each unit's scores
   float* part;                 // [B][Hq][splits][part_row(r)]
   const int64_t* pos_off = nullptr;  // [B] or null: added to a kept token's index for RoPE
+  uint64_t* trace = nullptr;         // traced step: [kernel][cta][3] timestamps, or null
 };
+
+// Timeline of a traced step (salsc_decode_step_traced): kernel k of the step
+// writes, for CTA c < SALSC_TRACE_MAX_CTAS (c = blockIdx.y * gridDim.x +
+// blockIdx.x), the global nanosecond timer at three points into
+// trace[(k * SALSC_TRACE_MAX_CTAS + c) * 3 + {0, 1, 2}]: its start, the
+// return of its dependency wait, and its end.  Untraced steps pass null.
+enum { TRACE_START = 0, TRACE_WAITED = 1, TRACE_END = 2 };
+__device__ __forceinline__ void trace_stamp(uint64_t* kernel_trace, int which) {
+  if (!kernel_trace) return;
+  const unsigned c = blockIdx.y * gridDim.x + blockIdx.x;
+  if (c >= (unsigned)SALSC_TRACE_MAX_CTAS) return;
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  kernel_trace[(size_t)c * 3 + which] = t;
+}
+// The trace rows of stage k (null when the step is not traced).
+inline uint64_t* trace_of(const DecodeArgs& a, int k) {
+  return a.trace ? a.trace + (size_t)k * SALSC_TRACE_MAX_CTAS * 3 : nullptr;
+}
 
 // Record a CUDA error for salsc_last_cuda_error() and return SALSC_ERR_CUDA.
 salsc_status record_cuda_error(cudaError_t e);

@@ -39,8 +39,9 @@ template <typename T, int COLS>
 __device__ __forceinline__ void latent_q_body(const T* __restrict__ q, const T* __restrict__ Pk,
                                               float* __restrict__ qlat,
                                               __nv_bfloat16* __restrict__ qsplit,
-                                              uint32_t* __restrict__ krange, int B, int Hq, int U,
-                                              int G, int d, int r, int npad) {
+                                              uint32_t* __restrict__ krange,
+                                              uint64_t* trace, int B, int Hq, int U, int G,
+                                              int d, int r, int npad) {
   constexpr int kThreads = lq_threads<COLS>();
   constexpr int SLICES = kThreads / COLS;
   constexpr int kRowsMax = (kMaxHeadDim + SLICES - 1) / SLICES;
@@ -48,6 +49,7 @@ __device__ __forceinline__ void latent_q_body(const T* __restrict__ q, const T* 
   __shared__ float red[SLICES][kBatchChunk][COLS];
   const int u = blockIdx.x;
   const int tid = threadIdx.x;
+  if (tid == 0) trace_stamp(trace, TRACE_START);
   const int col = tid % COLS, slice = tid / COLS;
   const int c = blockIdx.y * COLS + col;
   const int rows = (d + SLICES - 1) / SLICES, i0 = slice * rows;
@@ -56,6 +58,7 @@ __device__ __forceinline__ void latent_q_body(const T* __restrict__ q, const T* 
   for (int j = 0; j < kRowsMax; ++j)
     pk[j] = (j < rows && i0 + j < d && c < r) ? to_f32(Pk[((size_t)u * d + i0 + j) * r + c]) : 0.f;
   grid_dependency_wait();  // q and the workspace belong to the previous kernel until now
+  if (tid == 0) trace_stamp(trace, TRACE_WAITED);
   // Only now may the step's later kernels start: they read step inputs (Kc,
   // the sequence offsets) before their own dependency waits, and everything
   // the stream did before this step is complete once the wait above returns.
@@ -116,22 +119,23 @@ __device__ __forceinline__ void latent_q_body(const T* __restrict__ q, const T* 
     }
     __syncthreads();  // qsum and red are reused by the next chunk
   }
+  if (tid == 0) trace_stamp(trace, TRACE_END);
 }
 
 template <typename T>
 __global__ void __maxnreg__(48)
 latent_q16_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __restrict__ qlat,
-                  __nv_bfloat16* __restrict__ qsplit, uint32_t* __restrict__ krange, int B, int Hq,
-                  int U, int G, int d, int r, int npad) {
-  latent_q_body<T, 16>(q, Pk, qlat, qsplit, krange, B, Hq, U, G, d, r, npad);
+                  __nv_bfloat16* __restrict__ qsplit, uint32_t* __restrict__ krange,
+                  uint64_t* trace, int B, int Hq, int U, int G, int d, int r, int npad) {
+  latent_q_body<T, 16>(q, Pk, qlat, qsplit, krange, trace, B, Hq, U, G, d, r, npad);
 }
 
 template <typename T>
 __global__ void __launch_bounds__(lq_threads<64>())
 latent_q64_kernel(const T* __restrict__ q, const T* __restrict__ Pk, float* __restrict__ qlat,
-                  __nv_bfloat16* __restrict__ qsplit, uint32_t* __restrict__ krange, int B, int Hq,
-                  int U, int G, int d, int r, int npad) {
-  latent_q_body<T, 64>(q, Pk, qlat, qsplit, krange, B, Hq, U, G, d, r, npad);
+                  __nv_bfloat16* __restrict__ qsplit, uint32_t* __restrict__ krange,
+                  uint64_t* trace, int B, int Hq, int U, int G, int d, int r, int npad) {
+  latent_q_body<T, 64>(q, Pk, qlat, qsplit, krange, trace, B, Hq, U, G, d, r, npad);
 }
 
 template <typename T, int COLS>
@@ -139,8 +143,8 @@ cudaError_t launch_cols(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s
   dim3 grid(p.U, (p.r + COLS - 1) / COLS);
   auto kernel = COLS == 16 ? latent_q16_kernel<T> : latent_q64_kernel<T>;
   return launch_k(kernel, grid, dim3(lq_threads<COLS>()), 0, s, true, (const T*)a.q,
-                  (const T*)a.Pk, a.qlat, a.qsplit, a.krange, p.B, p.Hq, p.U, p.G, p.d, p.r,
-                  p.npad);
+                  (const T*)a.Pk, a.qlat, a.qsplit, a.krange, trace_of(a, 0), p.B, p.Hq,
+                  p.U, p.G, p.d, p.r, p.npad);
 }
 
 template <typename T>

@@ -100,6 +100,7 @@ struct ScoreTcParams {
   uint32_t* flags;
   int B, U, npad, r, n_tiles, stages, tmem_cols;
   int ng, ncol;  // unit groups, and the 2 * units-per-group query rows of one group
+  uint64_t* trace;  // traced step: this kernel's rows, or null
 };
 
 // Walks the work items of a CTA: item w is tile w % n_tiles of unit group
@@ -150,6 +151,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
   __shared__ uint32_t s_kr[kRangeSeqs][kMaxUnits][2];
   __shared__ int s_krb[kRangeSeqs], s_nkr;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) trace_stamp(P.trace, TRACE_START);
   for (int e = threadIdx.x; e < kRangeSeqs * P.U; e += kTcThreads) {
     s_kr[e / P.U][e % P.U][0] = 0xffffffffu;
     s_kr[e / P.U][e % P.U][1] = 0u;
@@ -207,6 +209,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
             }
           }
           grid_dependency_wait();
+          trace_stamp(P.trace, TRACE_WAITED);
         }
         tc::mbar_expect_tx(bfull, (uint32_t)KB * b_kblock_bytes);
         for (int kb = 0; kb < KB; ++kb)
@@ -338,6 +341,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
   }
   tc::fence_before_sync();
   __syncthreads();
+  if (threadIdx.x == 0) trace_stamp(P.trace, TRACE_END);
   for (int e = threadIdx.x; e < s_nkr * P.U; e += kTcThreads) {
     const int q = e / P.U, u = e % P.U;
     atomicMin(&P.krange[2 * ((int64_t)s_krb[q] * P.U + u)], s_kr[q][u][0]);
@@ -401,6 +405,7 @@ cudaError_t launch_score_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream
   P.scores = a.scores;
   P.krange = a.krange;
   P.flags = a.flags;
+  P.trace = trace_of(a, 1);
   P.B = p.B;
   P.U = p.U;
   P.npad = p.npad;

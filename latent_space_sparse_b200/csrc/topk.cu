@@ -112,7 +112,7 @@ template <bool kCluster, int kThreads>
 __global__ void __launch_bounds__(kThreads)
 topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_off,
             const uint32_t* __restrict__ krange, int32_t* __restrict__ idx_out, int U, int k,
-            uint32_t kthr) {
+            uint32_t kthr, uint64_t* trace) {
   constexpr int kWarps = kThreads / 32;
   cg::cluster_group cluster = cg::this_cluster();
   const int C = kCluster ? (int)cluster.num_blocks() : 1;
@@ -131,6 +131,7 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
   __shared__ uint32_t s_digit, s_above, s_count, s_base_gt, s_base_eq, s_ncand, s_ngt;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) trace_stamp(trace, TRACE_START);
   // shared memory of cluster rank q (this CTA's own when not a cluster)
   auto remote = [&](uint32_t* ptr, int q) -> uint32_t* {
     return kCluster ? cluster.map_shared_rank(ptr, q) : ptr;
@@ -162,11 +163,13 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
   // cluster histogram (they wait for this arrival before they do).
   if (kCluster && !keep_all) cluster_arrive();
   grid_dependency_wait();  // the scores and their range come from the previous kernel
+  if (tid == 0) trace_stamp(trace, TRACE_WAITED);
   if (keep_all) {
     // keep every token, in index order
     for (int i = tid; i < n_loc; i += kThreads) out[lo + i] = (int32_t)(lo + i);
     if (rank == 0)
       for (int64_t j = kb + tid; j < k; j += kThreads) out[j] = -1;
+    if (tid == 0) trace_stamp(trace, TRACE_END);
     return;
   }
   // the slice's first batch of scores is requested together with the unit's
@@ -326,6 +329,7 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
     }
     if (rank == 0)
       for (int64_t j = kb + tid; j < k; j += kThreads) out[j] = -1;
+    if (tid == 0) trace_stamp(trace, TRACE_END);
     // nothing reads or writes this CTA's shared memory from other CTAs any more
     return;
   }
@@ -457,6 +461,7 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
   if (rank == 0)
     for (int64_t j = kb + tid; j < k; j += kThreads) out[j] = -1;
   if (kCluster) cluster.sync();  // no CTA leaves while another may still read its counts
+  if (tid == 0) trace_stamp(trace, TRACE_END);
 }
 
 template <bool kCluster, int kThreads>
@@ -483,7 +488,7 @@ cudaError_t launch_tk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) 
   cfg.numAttrs = kCluster ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, topk_kernel<kCluster, kThreads>, (const float*)a.scores,
                             (const int64_t*)a.seq_off, (const uint32_t*)a.krange, a.idx, p.U, p.k,
-                            p.topk_kthr);
+                            p.topk_kthr, trace_of(a, 2));
 }
 
 }  // namespace

@@ -23,7 +23,8 @@ WS_ALIGN = 256
 
 EXPORTS = (
     "salsc_compress", "salsc_decode_workspace_size", "salsc_decode_prepare", "salsc_decode_step",
-    "salsc_decode_step_timed", "salsc_decode_step_static_ws", "salsc_static_workspace_bytes",
+    "salsc_decode_step_timed", "salsc_decode_step_traced", "salsc_decode_step_static_ws",
+    "salsc_static_workspace_bytes",
     "salsc_decode_launch_count", "salsc_append", "salsc_decode_step_append",
     "salsc_fit_workspace_size",
     "salsc_fit_projection", "salsc_shard_candidates", "salsc_shard_select", "salsc_shard_attend",
@@ -101,6 +102,8 @@ def _lib():
         lib.salsc_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, ctypes.c_int, vp]
         lib.salsc_decode_launch_count.restype = ctypes.c_int32
         lib.salsc_decode_launch_count.argtypes = [dp]
+        lib.salsc_decode_step_traced.restype = ctypes.c_int
+        lib.salsc_decode_step_traced.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, sz, vp]
         lib.salsc_decode_step_timed.restype = ctypes.c_int
         lib.salsc_decode_step_timed.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
                                                 ctypes.POINTER(ctypes.c_void_p), i32]
@@ -311,6 +314,26 @@ def salsc_decode_step_timed(desc: DecodeDesc, q, Kc, Vc, Pk, Pv, out, idx_out, w
                                         ws.numel() * ws.element_size(), _stream(stream), arr,
                                         len(events))
     _check(st, "salsc_decode_step_timed")
+
+
+TRACE_MAX_CTAS = 8192  # SALSC_TRACE_MAX_CTAS
+
+
+def trace_buffer(device) -> torch.Tensor:
+    """A zeroed int64 timeline buffer for salsc_decode_step_traced: [stage][cta][3]."""
+    return torch.zeros((len(DECODE_KERNELS), TRACE_MAX_CTAS, 3), dtype=torch.int64,
+                       device=device)
+
+
+def salsc_decode_step_traced(desc: DecodeDesc, q, Kc, Vc, Pk, Pv, out, idx_out, ws, trace,
+                             stream=None):
+    """salsc_decode_step that records per-CTA timestamps (start, dependency wait done,
+    end; global ns timer) of every stage into ``trace`` (see trace_buffer)."""
+    st = _lib().salsc_decode_step_traced(ctypes.byref(desc), _ptr(q), _ptr(Kc), _ptr(Vc),
+                                         _ptr(Pk), _ptr(Pv), _ptr(out), _ptr(idx_out), _ptr(ws),
+                                         ws.numel() * ws.element_size(), _ptr(trace),
+                                         trace.numel() * trace.element_size(), _stream(stream))
+    _check(st, "salsc_decode_step_traced")
 
 
 def static_workspace_bytes() -> int:

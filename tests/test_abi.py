@@ -29,6 +29,30 @@ def test_library_exports_every_declared_symbol():
     assert salsc.version().startswith("salsc")
 
 
+def test_header_constants_match_the_binding():
+    text = open(os.path.join(ROOT, "include", "salsc.h")).read()
+    assert int(re.search(r"#define SALSC_DECODE_KERNELS (\d+)", text).group(1)) == \
+        len(salsc.DECODE_KERNELS)
+    assert int(re.search(r"#define SALSC_TRACE_MAX_CTAS (\d+)", text).group(1)) == \
+        salsc.TRACE_MAX_CTAS
+
+
+def test_traced_step_checks_its_buffer_before_launch():
+    lib = salsc.load()
+    vp = ctypes.c_void_p
+    d = desc([0, 1000])
+    need = 3 * 8 * len(salsc.DECODE_KERNELS) * salsc.TRACE_MAX_CTAS
+    a = vp(1 << 20)
+
+    def traced(tr=vp(1 << 24), nb=need):
+        return lib.salsc_decode_step_traced(ctypes.byref(d), a, a, a, a, a, a, None, vp(1 << 28),
+                                            1 << 30, tr, nb, None)
+
+    assert traced(tr=None) == salsc.SALSC_ERR_INVALID_ARG
+    assert traced(tr=vp((1 << 24) + 4)) == salsc.SALSC_ERR_INVALID_ARG  # not 8-byte aligned
+    assert traced(nb=need - 8) == salsc.SALSC_ERR_INVALID_ARG
+
+
 def test_status_strings():
     for code in range(5):
         assert salsc.status_string(code)

@@ -129,3 +129,26 @@ def test_max_over_ranks_gloo(tmp_path):
     for r in range(world):
         assert float(open(f"{path}.{r}").read()) == 2.25  # every rank gets the slowest time
     assert bench.max_over_ranks(0.5, "cpu") == 0.5  # no process group: the value itself
+
+
+def test_timeline_summary_on_hand_made_stamps():
+    # two layers, stages (a, b, c); stage c records nothing (a merge that launches nothing)
+    stages = ("a", "b", "c")
+    tr = np.zeros((2, 3, 4, 3), dtype=np.int64)
+
+    def layer(l, t0):
+        # stage a: CTAs 0-1 start t0, wait returns t0+1000, end t0+3000 / t0+3500
+        tr[l, 0, 0] = (t0, t0 + 1000, t0 + 3000)
+        tr[l, 0, 1] = (t0, t0 + 1100, t0 + 3500)
+        # stage b: wait returns 500 ns after a's last end, ends 4000 ns after that end
+        tr[l, 1, 0] = (t0 + 500, t0 + 4000, t0 + 7500)
+        tr[l, 1, 2] = (t0 + 600, t0 + 4100, t0 + 6000)
+        return t0 + 7500
+
+    end0 = layer(0, 10_000)
+    layer(1, end0 + 200)  # layer 1's first stage waits 200 ns + 1000 ns after layer 0's end
+    s = bench.timeline_summary(tr, stages)
+    assert s["critical_us"] == pytest.approx({"a": 3.7, "b": 4.0})
+    assert s["wait_us"] == pytest.approx({"a": 1.2, "b": 0.5})
+    assert s["span_us"] == pytest.approx({"a": 2.5, "b": 3.5})
+    assert s["layer_step_us"] == pytest.approx(7.7)
