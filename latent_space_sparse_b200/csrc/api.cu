@@ -11,10 +11,6 @@
 
 namespace {
 
-// Unit-group partition of the attention tiles (CTA groups per unit, runs per
-// sequence) instead of one contiguous range of tile numbers per CTA.
-constexpr bool kUnitGroups = false;
-
 thread_local char g_last_cuda_error[256] = "no error";
 
 salsc_status cuda_fail(cudaError_t e) {
@@ -47,12 +43,13 @@ salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
   if (!(D->softmax_scale >= 0.0f) || !isfinite(D->softmax_scale)) return SALSC_ERR_INVALID_ARG;
   if (D->seq_offsets_host[0] != 0) return SALSC_ERR_INVALID_ARG;
   int64_t n_max = 0;
-  int n_tiles = 0;
+  int n_tiles = 0, n_chunks = 0;
   for (int b = 0; b < D->batch; ++b) {
     const int64_t nb = D->seq_offsets_host[b + 1] - D->seq_offsets_host[b];
     if (nb < 1 || nb > (int64_t)INT32_MAX) return SALSC_ERR_INVALID_ARG;
     if (nb > n_max) n_max = nb;
     n_tiles += (int)((nb + kScoreTile - 1) / kScoreTile);
+    n_chunks += (int)((nb + 31) / 32);
   }
   // shapes with kernels
   if (D->head_dim != 64 && D->head_dim != 128) return SALSC_ERR_UNSUPPORTED;
@@ -77,6 +74,7 @@ salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
   p.n_max = n_max;
   p.score_tile = kScoreTile;
   p.n_score_tiles = n_tiles;
+  p.n_score_chunks = n_chunks;
   // Top-k: C CTAs per unit, about one CTA per SM in all (up to 8 per unit, and
   // enough for a slice of the scores to fit shared memory); many small units
   // take 256-thread CTAs, several resident per SM.
@@ -129,8 +127,6 @@ salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
     p.att_tiles = 0;
   }
   p.att_cluster = p.attend_tc ? salsc::attend_merge_cluster(p) : 0;
-  // unit groups need a CTA per unit at least
-  p.att_share = kUnitGroups && p.attend_tc && p.att_cluster == 0 && salsc::attend_tc_grid(p) >= p.U;
   if (!salsc::combine_supported(p)) return SALSC_ERR_UNSUPPORTED;
   p.scale = D->softmax_scale != 0.0f ? D->softmax_scale : (float)(1.0 / sqrt((double)p.d));
   p.rope_base = D->rope_base;
@@ -509,7 +505,6 @@ salsc_status salsc_shard_attend(const salsc_decode_desc* desc, const void* q, co
   // the shards' partials are merged after the exchange, so the attention
   // kernel does not merge (nor project) them itself
   p.att_cluster = 0;
-  p.att_share = kUnitGroups && p.attend_tc && salsc::attend_tc_grid(p) >= p.U;
   if (!desc->seq_offsets_dev || !desc->q_pos_dev || !q || !Kc || !Vc || !Pk || !idx_local ||
       !shard_off_dev || !part_out)
     return SALSC_ERR_INVALID_ARG;

@@ -74,79 +74,40 @@ struct AttendTcParams {
   __nv_bfloat16* out;
   int B, Hq, U, r, k, n_slots, n_tiles;
   int cluster;  // merged in the kernel: CTAs per unit (one thread-block cluster)
-  int share;    // 1: unit-group partition of the tiles (else a contiguous range)
   uint64_t* trace;  // traced step: this kernel's rows, or null
   float scale;
   double base;
 };
 
 // Walks the tiles of a CTA.  Tiles are numbered in the order (sequence,
-// unit, slot); unit (b, u) has tb = ceil(min(k, n_b) / 128) tiles.  Two
-// partitions over the grid of g CTAs:
-//   - a contiguous range of tile numbers (start);
-//   - unit groups (begin_group, for g >= U): the CTAs are split into U groups
-//     of m = floor((u+1)g/U) - floor(ug/U) consecutive CTAs, group u taking
-//     unit u of every sequence; in sequence b the unit's tb tiles are cut
-//     into m runs [floor(r*tb/m), floor((r+1)*tb/m)), and CTA i of the group
-//     takes run r = (i + floor(b*m/B)) mod m.  A CTA then keeps one unit
-//     (one Pk_u), works on the sequences in order, and the rotation spreads
-//     the empty runs (tb < m) over the CTAs.
+// unit, slot); unit (b, u) has tb = ceil(min(k, n_b) / 128) tiles.  A CTA's
+// first tile is found once per CTA (find_first_tile) and set with at().
 struct UnitTileCursor {
   const int64_t* so;
   int B, U, k;
   int b, u, slot, tb;
   int64_t off, nb, kb;
-  int gi, gm, hi;  // unit-group mode (gm > 0): CTA gi of the unit's gm, run end hi
   __device__ void load() {
     off = so[b];
     nb = so[b + 1] - off;
     kb = nb < k ? nb : k;
     tb = (int)((kb + kTile - 1) / kTile);
   }
-  __device__ void start(const int64_t* so_, int B_, int U_, int k_, int tile) {
+  __device__ void at(const int64_t* so_, int B_, int U_, int k_, int b_, int u_, int slot_,
+                     int64_t off_, int64_t nb_) {
     so = so_;
     B = B_;
     U = U_;
     k = k_;
-    gm = 0;
-    int acc = 0;
-    for (b = 0; b < B; ++b) {
-      load();
-      if (tile < acc + U * tb) {
-        const int rem = tile - acc;
-        u = rem / tb;
-        slot = rem % tb;
-        return;
-      }
-      acc += U * tb;
-    }
-  }
-  // unit-group mode: the first tile of this CTA's run in sequence b0 or later
-  __device__ void seek(int b0) {
-    for (b = b0; b < B; ++b) {
-      load();
-      const int r = (gi + b * gm / B) % gm;
-      slot = r * tb / gm;
-      hi = (r + 1) * tb / gm;
-      if (slot < hi) return;
-    }
-  }
-  __device__ void begin_group(const int64_t* so_, int B_, int U_, int k_, int c, int g) {
-    so = so_;
-    B = B_;
-    U = U_;
-    k = k_;
-    u = (int)(((int64_t)(c + 1) * U - 1) / g);  // the group of CTA c
-    const int c0 = (int)((int64_t)u * g / U);
-    gm = (int)((int64_t)(u + 1) * g / U) - c0;
-    gi = c - c0;
-    seek(0);
+    b = b_;
+    u = u_;
+    slot = slot_;
+    off = off_;
+    nb = nb_;
+    kb = nb < k ? nb : k;
+    tb = (int)((kb + kTile - 1) / kTile);
   }
   __device__ void next() {
-    if (gm > 0) {
-      if (++slot >= hi) seek(b + 1);
-      return;
-    }
     if (++slot >= tb) {
       slot = 0;
       if (++u >= U) {
@@ -157,13 +118,93 @@ struct UnitTileCursor {
   }
 };
 
-// Tiles of CTA c of g in the unit-group partition.
-__device__ __forceinline__ int group_tiles(const int64_t* so, int B, int U, int k, int c, int g) {
-  UnitTileCursor t;
-  t.begin_group(so, B, U, k, c, g);
-  int n = 0;
-  for (; t.b < B; t.seek(t.b + 1)) n += t.hi - t.slot;
-  return n;
+// The CTA's tile range and its first tile, found by one warp: every lane reads
+// the offsets of one sequence (32 at a time), and a warp scan of the tiles
+// per sequence locates tile t_begin with one round trip of loads.  Merging
+// CTAs (cluster > 0) take their rank's share of unit m_unit's tiles; the
+// others take tiles [c*T/g, (c+1)*T/g).  Lane 0 writes (t_begin, n, b, u,
+// slot) to st[0..4] and (off, nb) of sequence b to st64[0..1]; b = B when the
+// range is empty.
+__device__ __forceinline__ void find_first_tile(const int64_t* so, int B, int U, int k,
+                                                int n_tiles, int cluster, int* st,
+                                                int64_t* st64) {
+  const int lane = threadIdx.x % 32;
+  int t_begin = 0, n = 0, mb = -1;
+  if (cluster > 0) {
+    mb = (int)(blockIdx.x / (unsigned)cluster) / U;  // the unit's sequence
+  } else {
+    t_begin = (int)((int64_t)blockIdx.x * n_tiles / gridDim.x);
+    n = (int)((int64_t)(blockIdx.x + 1) * n_tiles / gridDim.x) - t_begin;
+  }
+  int64_t before = 0;  // tiles of the sequences before this group of 32
+  int fb = B, fu = 0, fslot = 0;
+  int64_t foff = 0, fnb = 0;
+  for (int b0 = 0; b0 < B; b0 += 32) {
+    const int bb = b0 + lane;
+    int64_t offb = 0, nbb = 0;
+    int tbb = 0;
+    if (bb < B) {
+      offb = so[bb];
+      nbb = so[bb + 1] - offb;
+      const int64_t kbb = nbb < k ? nbb : k;
+      tbb = (int)((kbb + kTile - 1) / kTile);
+    }
+    const int64_t x = (int64_t)U * tbb;
+    int64_t incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const int64_t excl = before + incl - x;
+    if (cluster > 0) {
+      // unit m_unit = (mb, u): the rank's share [lo, hi) of its tb tiles
+      const uint32_t m = __ballot_sync(0xffffffffu, bb == mb);
+      if (m) {
+        const int src = __ffs(m) - 1;
+        const int64_t e = __shfl_sync(0xffffffffu, excl, src);
+        const int tu = __shfl_sync(0xffffffffu, tbb, src);
+        const int64_t o2 = __shfl_sync(0xffffffffu, offb, src);
+        const int64_t n2 = __shfl_sync(0xffffffffu, nbb, src);
+        const int m_rank = (int)(blockIdx.x % (unsigned)cluster);
+        const int u = (int)(blockIdx.x / (unsigned)cluster) % U;
+        const int l0 = tu * m_rank / cluster, h0 = tu * (m_rank + 1) / cluster;
+        t_begin = (int)(e + (int64_t)u * tu + l0);
+        n = h0 - l0;
+        if (n > 0) {
+          fb = mb;
+          fu = u;
+          fslot = l0;
+          foff = o2;
+          fnb = n2;
+        }
+      }
+    } else {
+      const bool here = bb < B && tbb > 0 && excl <= t_begin && t_begin < excl + x;
+      const uint32_t m = __ballot_sync(0xffffffffu, here);
+      if (m && fb == B && n > 0) {
+        const int src = __ffs(m) - 1;
+        const int64_t e = __shfl_sync(0xffffffffu, excl, src);
+        const int tu = __shfl_sync(0xffffffffu, tbb, src);
+        fb = b0 + src;
+        foff = __shfl_sync(0xffffffffu, offb, src);
+        fnb = __shfl_sync(0xffffffffu, nbb, src);
+        const int rem = (int)(t_begin - e);
+        fu = rem / tu;
+        fslot = rem % tu;
+      }
+    }
+    before += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) {
+    st[0] = t_begin;
+    st[1] = n;
+    st[2] = fb;
+    st[3] = fu;
+    st[4] = fslot;
+    st64[0] = foff;
+    st64[1] = fnb;
+  }
 }
 
 // Token of row `row` of the cursor's tile, or -1 past the unit's k_b kept
@@ -252,41 +293,24 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
   float* const s_ab = s_run + 2 * G;                         // [G][2] rescale factors
   uint64_t* const s_bars = (uint64_t*)(((uintptr_t)(s_ab + 2 * G) + 7) & ~(uintptr_t)7);
   uint32_t* const s_tmem_slot = (uint32_t*)(s_bars + B_COUNT);
+  int64_t* const s_start64 = (int64_t*)(s_bars + B_COUNT + 1);  // first tile's (off, n_b)
+  int* const s_start = (int*)(s_start64 + 2);                    // t_begin, n, b, u, slot
   const uint32_t bar0 = tc::smem_u32(s_bars);
   auto bar = [bar0](int i) { return bar0 + 8u * (uint32_t)i; };
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   if (tid == 0) trace_stamp(P.trace, TRACE_START);
   allow_dependent_launch();
-  // Tile range: a contiguous share of all tiles, or (kMerge) the rank's share
-  // of its unit's tiles, the unit being (blockIdx.x / cluster).
-  int t_begin, n, m_unit = 0, m_rank = 0;
-  if constexpr (kMerge) {
-    m_rank = (int)(blockIdx.x % (unsigned)P.cluster);
-    m_unit = (int)(blockIdx.x / (unsigned)P.cluster);
-    const int mb = m_unit / P.U;
-    int before = 0, tu = 0;
-    for (int bb = 0; bb <= mb; ++bb) {
-      const int64_t nbb = P.seq_off[bb + 1] - P.seq_off[bb];
-      const int t = (int)(((nbb < P.k ? nbb : (int64_t)P.k) + kTile - 1) / kTile);
-      if (bb < mb) before += P.U * t; else tu = t;
-    }
-    const int lo = tu * m_rank / P.cluster, hi = tu * (m_rank + 1) / P.cluster;
-    t_begin = before + (m_unit % P.U) * tu + lo;
-    n = hi - lo;
-  } else if (P.share) {
-    t_begin = 0;
-    n = group_tiles(P.seq_off, P.B, P.U, P.k, (int)blockIdx.x, (int)gridDim.x);
-  } else {
-    t_begin = (int)((int64_t)blockIdx.x * P.n_tiles / gridDim.x);
-    n = (int)((int64_t)(blockIdx.x + 1) * P.n_tiles / gridDim.x) - t_begin;
-  }
-  // the CTA's first tile
+  const int m_rank = kMerge ? (int)(blockIdx.x % (unsigned)P.cluster) : 0;
+  const int m_unit = kMerge ? (int)(blockIdx.x / (unsigned)P.cluster) : 0;
+  // Tile range and first tile (set before the block-wide barrier below).
+  if (warp == kLoadWarp0)
+    find_first_tile(P.seq_off, P.B, P.U, P.k, P.n_tiles, kMerge ? P.cluster : 0, s_start,
+                    s_start64);
+  int n = 0;  // tiles of this CTA
   auto first_tile = [&](UnitTileCursor& c) {
-    if (!kMerge && P.share)
-      c.begin_group(P.seq_off, P.B, P.U, P.k, (int)blockIdx.x, (int)gridDim.x);
-    else
-      c.start(P.seq_off, P.B, P.U, P.k, t_begin);
+    c.at(P.seq_off, P.B, P.U, P.k, s_start[2], s_start[3], s_start[4], s_start64[0],
+         s_start64[1]);
   };
   // TMEM columns: K_sel [2][D], then acc [2][n_chunks * 16]
   const uint32_t o_col0 = 2 * D;
@@ -300,17 +324,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     tc::tma_prefetch_desc(&tmap_vc);
   }
   if (warp == kMmaWarp) tc::tmem_alloc(tc::smem_u32(s_tmem_slot), 512);
-  for (int i = tid; i < HALF; i += kThreads) {
-    const double th = pow(P.base, -2.0 * (double)i / (double)D);
-    s_theta[i] = th;
-    s_fturn[i] = __double2ull_rn(th / kTwoPi * 18446744073709551616.0);
-  }
   // the p operand's unused rows (2G..15) stay zero
   for (int e = tid; e < 2 * 4096 / 4; e += kThreads) ((uint32_t*)s_pbuf0)[e] = 0u;
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem_base = *s_tmem_slot;
+  n = s_start[1];
 
   if (W == 2 && warp >= kLoadWarp0) {
     // ======================= gather warps, two latent halves =================
@@ -627,6 +647,14 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     // e%128 for the tile's softmax.
     const int quarter = warp & 3, part = warp >> 2;
     const int m = quarter * 32 + lane;  // token row = TMEM lane
+    // RoPE frequencies theta_i = base^(-2i/d) and their fixed-point turns
+    // (here, not before the block-wide barrier: the gathers need neither)
+    for (int i = tid; i < HALF; i += kEpiThreads) {
+      const double th = pow(P.base, -2.0 * (double)i / (double)D);
+      s_theta[i] = th;
+      s_fturn[i] = __double2ull_rn(th / kTwoPi * 18446744073709551616.0);
+    }
+    tc::named_sync(kEpiBar, kEpiThreads);
     UnitTileCursor cur;
     first_tile(cur);
     int cur_b = -1, cur_u = -1;
@@ -966,7 +994,7 @@ size_t smem_bytes(int r) {
   const int KB = r / 64 / W;
   return 1024 + (size_t)KB * D * 128 + 2 * (size_t)KB * 16384 + 2 * 4096 + 8 * (D / 2) * 2 +
          4 * (G * D + kEpiParts * G * kTile + 16 * G + 2 * kTile + 4 * G) + 8 +
-         8 * B_COUNT + 16;
+         8 * B_COUNT + 16 + 16 + 24;
 }
 
 template <int G, int D, int W, bool kMerge>
@@ -1000,7 +1028,6 @@ cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s)
   P.n_slots = p.splits;
   P.n_tiles = p.att_tiles;
   P.cluster = kMerge ? p.att_cluster : 1;
-  P.share = kMerge ? 0 : (p.att_share ? 1 : 0);
   P.trace = trace_of(a, 3);
   P.scale = p.scale;
   P.base = p.rope_base;

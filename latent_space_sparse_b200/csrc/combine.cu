@@ -48,7 +48,6 @@ struct CombineParams {
   uint32_t* flags;
   int B, Hq, U, d, r, k, n_slots, chunk;
   int seg_grid, seg_tiles;  // tensor-core tile partition (seg_grid = 0: every slot used)
-  int share;                // 1: unit-group partition (CTA groups per unit, runs per sequence)
   int64_t bh_stride, slot_stride;  // partial row of (b, h, slot): (b*Hq + h)*bh_stride + slot*slot_stride
   float* part_out;  // non-null: write the merged partial row of every head, no projection
   int fixed_slots;  // > 0: every unit has this many slots (no tile count from the lengths)
@@ -120,14 +119,8 @@ combine_kernel(const CombineParams P) {
       const int sl = s0 + lane;
       bool used = sl < tb;
       if (used && sl > 0 && P.seg_grid > 0) {
-        // tile t starts a CTA's range in a partition of T tiles over gc CTAs:
-        // all tiles over the grid, or (unit groups) the unit's tb tiles of
-        // this sequence over the unit's group of CTAs
-        const int64_t gc = P.share ? (int64_t)(u + 1) * P.seg_grid / P.U -
-                                         (int64_t)u * P.seg_grid / P.U
-                                   : P.seg_grid;
-        const int64_t t = P.share ? sl : unit_tile0 + sl;
-        const int64_t T = P.share ? tb : P.seg_tiles;
+        // tile t starts a CTA's range [c*T/grid, (c+1)*T/grid)
+        const int64_t t = unit_tile0 + sl, T = P.seg_tiles, gc = P.seg_grid;
         const int64_t c = (t * gc + T - 1) / T;  // first CTA at or after t
         used = c < gc && c * T / gc == t;
       }
@@ -289,17 +282,13 @@ int max_used_slots(const DecodePlan& p, const int64_t* seq_off_host, int seg_gri
     const int64_t kb = nb < p.k ? nb : p.k;
     const int64_t tb = (kb + p.chunk - 1) / p.chunk;
     for (int u = 0; u < p.U; ++u, tile += tb) {
-      // CTA c covers tiles [c*T/gc, (c+1)*T/gc) of a partition of T tiles over
-      // gc CTAs (all tiles over the grid; with unit groups, the unit's tb
-      // tiles of this sequence over its group): the CTA of tile t is
-      // ((t+1)*gc - 1) / T, and the unit's tiles meet at most the CTAs from
-      // its first tile's to its last tile's
-      const int64_t gc = p.att_share ? (int64_t)(u + 1) * seg_grid / p.U -
-                                           (int64_t)u * seg_grid / p.U
-                                     : seg_grid;
-      const int64_t T = p.att_share ? tb : p.att_tiles;
-      const int64_t t0 = p.att_share ? 0 : tile;
-      const int64_t n = ((t0 + tb) * gc - 1) / T - ((t0 + 1) * gc - 1) / T + 1;
+      // CTA c covers tiles [c*T/gc, (c+1)*T/gc) of the T tiles over gc CTAs:
+      // the CTA of tile t is ((t+1)*gc - 1) / T, and the unit's tiles meet at
+      // most the CTAs from its first tile's to its last tile's
+      const int64_t gc = seg_grid, T = p.att_tiles, t0 = tile;
+      if (tb == 0) continue;
+      int64_t n = ((t0 + tb) * gc - 1) / T - ((t0 + 1) * gc - 1) / T + 1;
+      if (n > tb) n = tb;  // a segment holds one tile at least
       if (n > most) most = (int)n;
     }
   }
@@ -383,7 +372,6 @@ CombineParams base_params(const DecodePlan& p, const DecodeArgs& a) {
   P.chunk = p.chunk;
   P.seg_grid = p.attend_tc ? attend_tc_grid(p) : 0;
   P.seg_tiles = p.att_tiles;
-  P.share = p.att_share ? 1 : 0;
   P.bh_stride = p.splits;
   P.slot_stride = 1;
   P.part_out = nullptr;

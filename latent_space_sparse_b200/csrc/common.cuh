@@ -41,6 +41,7 @@ struct DecodePlan {
   int64_t N, n_max;
   int n_score_tiles;    // sum_b ceil(n_b / score tile)
   int score_tile;       // tokens per scoring CTA
+  int n_score_chunks;   // sum_b ceil(n_b / 32): the tensor-core scoring kernel's work items
   int topk_cluster;     // CTAs per selection unit in the top-k kernel
   int topk_slice;       // max keys per top-k CTA
   int topk_threads;     // threads per top-k CTA (1024, or 256 for many small units)
@@ -51,7 +52,6 @@ struct DecodePlan {
   int att_tiles;        // sum over units of ceil(k_b / 128) (tensor-core path)
   int att_cluster;      // > 0: the attention kernel merges each unit's partials and projects
                         // them itself, one cluster of att_cluster CTAs per unit (no merge kernel)
-  bool att_share;       // tensor-core attention CTA c takes its share of every sequence's tiles
                         // (else a contiguous range of all tiles)
   float scale;
   double rope_base;

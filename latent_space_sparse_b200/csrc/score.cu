@@ -86,44 +86,116 @@ score_simt_kernel(const T* __restrict__ Kc, const float* __restrict__ qlat,
 // when the sequence changes); warp 1 = TMEM owner and (lane 0) MMA issuer,
 // accumulating into one of two TMEM buffers; warps 2-5 = epilogue: TMEM ->
 // registers, s_u = D[:, 2u] + D[:, 2u+1], coalesced fp32 stores.
-// Each CTA owns a contiguous range of tiles (persistent, grid <= #SMs), so
-// Qs is reloaded only at sequence boundaries.
+// Each CTA owns a contiguous range of 32-row chunks (persistent, grid <= #SMs),
+// taken as pieces of up to four chunks (one 128-row MMA tile) inside one
+// sequence, so the CTAs' shares differ by at most one chunk and Qs is
+// reloaded only at sequence boundaries.
 constexpr int kTcThreads = 192;
 constexpr int kRangeSeqs = 4;  // sequences per CTA whose score ranges are kept in shared memory
 constexpr int kTileM = 128;
+constexpr int kChunk = 32;                          // rows of a work item (one TMA box)
+constexpr int kChunksPerTile = kTileM / kChunk;
 constexpr uint32_t kStageBytes = kTileM * 64 * 2;  // one [128 x 64] bf16 k-block
+constexpr uint32_t kChunkBytes = kChunk * 64 * 2;  // one [32 x 64] box of it
 
 struct ScoreTcParams {
   const int64_t* seq_off;
   float* scores;
   uint32_t* krange;
   uint32_t* flags;
-  int B, U, npad, r, n_tiles, stages, tmem_cols;
+  int B, U, npad, r, n_chunks, stages, tmem_cols;
   int ng, ncol;  // unit groups, and the 2 * units-per-group query rows of one group
   uint64_t* trace;  // traced step: this kernel's rows, or null
 };
 
-// Walks the work items of a CTA: item w is tile w % n_tiles of unit group
-// w / n_tiles (groups outermost, so the CTAs that read the same tile for
-// different groups run at about the same time and share it through L2).
-struct ItemCursor {
-  TileCursor tc_;
-  int n_tiles, tile, g;
-  __device__ void start(const int64_t* so, int B, int n_tiles_, int w) {
-    n_tiles = n_tiles_;
-    g = w / n_tiles;
-    tile = w % n_tiles;
-    tc_.start(so, B, kTileM, tile);
-  }
-  __device__ void next(const int64_t* so, int B) {
-    if (++tile == n_tiles) {
-      tile = 0;
-      ++g;
-      tc_.start(so, B, kTileM, 0);
-    } else {
-      tc_.next();
+// Item w's group, sequence and chunk, found by one warp: every lane reads the
+// offsets of one sequence (32 at a time) and a warp scan of the chunks per
+// sequence locates the item with one round trip of loads.  Lane 0 writes
+// (g, b, q) to st[0..2] and (off, n_b) of sequence b to st64[0..1].
+__device__ __forceinline__ void find_first_chunk(const int64_t* so, int B, int nq_all, int w,
+                                                 int* st, int64_t* st64) {
+  const int lane = threadIdx.x % 32;
+  const int g = w / nq_all, c = w % nq_all;
+  int64_t before = 0;
+  bool found = false;
+  for (int b0 = 0; b0 < B && !found; b0 += 32) {
+    const int bb = b0 + lane;
+    int64_t offb = 0, nbb = 0;
+    if (bb < B) {
+      offb = so[bb];
+      nbb = so[bb + 1] - offb;
     }
+    const int64_t x = (nbb + kChunk - 1) / kChunk;
+    int64_t incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const int64_t excl = before + incl - x;
+    const uint32_t m = __ballot_sync(0xffffffffu, bb < B && excl <= c && c < excl + x);
+    if (m) {
+      const int src = __ffs(m) - 1;
+      if (lane == src) {
+        st[0] = g;
+        st[1] = bb;
+        st[2] = (int)(c - excl);
+        st64[0] = offb;
+        st64[1] = nbb;
+      }
+      found = true;
+    }
+    before += __shfl_sync(0xffffffffu, incl, 31);
   }
+}
+
+// Walks the work items of a CTA as pieces.  Item w is chunk w % nq_all of
+// unit group w / nq_all (groups outermost, so the CTAs that read the same rows
+// for different groups run at about the same time and share them through
+// L2); sequence b has nq = ceil(n_b / 32) chunks.  A piece is up to four
+// consecutive chunks of one sequence and group within the CTA's range.
+struct PieceCursor {
+  const int64_t* so;
+  int B;
+  int g, b, q, nq, len, left;  // group, sequence, first chunk, chunks of b, of the piece, left in the range
+  int64_t off, nb;
+  __device__ void load() {
+    off = so[b];
+    nb = so[b + 1] - off;
+    nq = (int)((nb + kChunk - 1) / kChunk);
+  }
+  __device__ void fit() { len = min(min(kChunksPerTile, nq - q), left); }
+  // first piece: chunk q of sequence b in group g (from find_first_chunk)
+  __device__ void at(const int64_t* so_, int B_, int n, int g_, int b_, int q_, int64_t off_,
+                     int64_t nb_) {
+    so = so_;
+    B = B_;
+    left = n;
+    len = 0;
+    g = g_;
+    b = b_;
+    q = q_;
+    off = off_;
+    nb = nb_;
+    nq = (int)((nb + kChunk - 1) / kChunk);
+    if (left > 0) fit();
+  }
+  __device__ void next() {
+    left -= len;
+    q += len;
+    if (left <= 0) return;
+    while (q >= nq) {  // the range goes on in the next sequence (or group)
+      q = 0;
+      if (++b == B) {
+        b = 0;
+        ++g;
+      }
+      load();
+    }
+    fit();
+  }
+  __device__ bool done() const { return left <= 0; }
+  __device__ int64_t row0() const { return off + (int64_t)q * kChunk; }
 };
 
 __global__ void __launch_bounds__(kTcThreads)
@@ -134,7 +206,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
   const int KB = P.r / 64;
   const int S = P.stages;
   const uint32_t b_kblock_bytes = (uint32_t)P.ncol * 128u;
-  const int n_items = P.n_tiles * P.ng;
+  const int n_items = P.n_chunks * P.ng;
   uint8_t* a_ring = smem;
   uint8_t* b_buf = a_ring + (size_t)S * kStageBytes;
   uint64_t* bars = (uint64_t*)(b_buf + (size_t)KB * b_kblock_bytes);
@@ -150,6 +222,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
   // CTA's tile range
   __shared__ uint32_t s_kr[kRangeSeqs][kMaxUnits][2];
   __shared__ int s_krb[kRangeSeqs], s_nkr;
+  __shared__ int s_first[3];        // the CTA's first item: group, sequence, chunk
+  __shared__ int64_t s_first64[2];  // and that sequence's (offset, length)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) trace_stamp(P.trace, TRACE_START);
   for (int e = threadIdx.x; e < kRangeSeqs * P.U; e += kTcThreads) {
@@ -160,6 +234,12 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
   const int t_begin = (int)((int64_t)blockIdx.x * n_items / gridDim.x);
   const int t_end = (int)((int64_t)(blockIdx.x + 1) * n_items / gridDim.x);
   allow_dependent_launch();
+  if (warp == 2 && t_end > t_begin)
+    find_first_chunk(P.seq_off, P.B, P.n_chunks, t_begin, s_first, s_first64);
+  auto first_piece = [&](PieceCursor& c) {
+    c.at(P.seq_off, P.B, t_end - t_begin, s_first[0], s_first[1], s_first[2], s_first64[0],
+         s_first64[1]);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -187,12 +267,18 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
     uint32_t it = 0, bpar = 0;
     int cur_bg = -1;
     bool ok = true;
-    ItemCursor ic;
-    ic.start(P.seq_off, P.B, P.n_tiles, t_begin);
-    for (int tile = t_begin; tile < t_end && ok; ++tile, ic.next(P.seq_off, P.B)) {
-      const TileCursor& cur = ic.tc_;
-      const int b = cur.b;
-      const int bg = b * P.ng + ic.g;
+    PieceCursor pc;
+    first_piece(pc);
+    // k-block kb of the piece: its chunks, one 32-row box each, into stage s
+    auto load_kblock = [&](int s, int kb) {
+      tc::mbar_expect_tx(full(s), (uint32_t)pc.len * kChunkBytes);
+      for (int j = 0; j < pc.len; ++j)
+        tc::tma_load_2d(tc::smem_u32(a_ring + (size_t)s * kStageBytes + (size_t)j * kChunkBytes),
+                        &tmap_kc, kb * 64, (int)(pc.row0() + (int64_t)j * kChunk), full(s));
+    };
+    for (int i = 0; !pc.done() && ok; ++i, pc.next()) {
+      const int b = pc.b;
+      const int bg = b * P.ng + pc.g;
       if (bg != cur_bg) {
         if (cur_bg >= 0) {
           ok = tc::mbar_wait(bempty, bpar, P.flags);
@@ -201,34 +287,26 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
         } else {
           // the latent cache streams in already; the split query comes from the
           // previous kernel
-          if (tile == t_begin) {
-            for (int kb = 0; kb < KB && kb < S; ++kb) {
-              tc::mbar_expect_tx(full(kb), kStageBytes);
-              tc::tma_load_2d(tc::smem_u32(a_ring + (size_t)kb * kStageBytes), &tmap_kc, kb * 64,
-                              (int)(cur.off + cur.t0), full(kb));
-            }
-          }
+          if (i == 0)
+            for (int kb = 0; kb < KB && kb < S; ++kb) load_kblock(kb, kb);
           grid_dependency_wait();
           trace_stamp(P.trace, TRACE_WAITED);
         }
         tc::mbar_expect_tx(bfull, (uint32_t)KB * b_kblock_bytes);
         for (int kb = 0; kb < KB; ++kb)
           tc::tma_load_2d(tc::smem_u32(b_buf + (size_t)kb * b_kblock_bytes), &tmap_q, kb * 64,
-                          b * P.npad + ic.g * P.ncol, bfull);
+                          b * P.npad + pc.g * P.ncol, bfull);
         cur_bg = bg;
       }
-      const int row0 = (int)(cur.off + cur.t0);
       for (int kb = 0; kb < KB; ++kb, ++it) {
         const int s = (int)(it % (uint32_t)S);
         const uint32_t ph = (it / (uint32_t)S) & 1u;
-        if (tile == t_begin && kb < S) continue;  // issued before the dependency wait
+        if (i == 0 && kb < S) continue;  // issued before the dependency wait
         if (!tc::mbar_wait(empty(s), ph ^ 1u, P.flags)) {
           ok = false;
           break;
         }
-        tc::mbar_expect_tx(full(s), kStageBytes);
-        tc::tma_load_2d(tc::smem_u32(a_ring + (size_t)s * kStageBytes), &tmap_kc, kb * 64, row0,
-                        full(s));
+        load_kblock(s, kb);
       }
     }
     // every issued load has landed before the CTA may exit
@@ -240,11 +318,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
     uint32_t it = 0, bpar = 0;
     int cur_bg = -1, nseq = 0, i = 0;
     bool ok = true;
-    ItemCursor ic;
-    ic.start(P.seq_off, P.B, P.n_tiles, t_begin);
-    for (int tile = t_begin; tile < t_end && ok; ++tile, ++i, ic.next(P.seq_off, P.B)) {
-      const TileCursor& cur = ic.tc_;
-      const int bg = cur.b * P.ng + ic.g;
+    PieceCursor pc;
+    first_piece(pc);
+    for (; !pc.done() && ok; ++i) {
+      const int bg = pc.b * P.ng + pc.g;
       if (bg != cur_bg) {
         if (!tc::mbar_wait(bfull, bpar, P.flags)) break;
         bpar ^= 1u;
@@ -273,9 +350,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
       }
       if (!ok) break;
       tc::mma_commit(tfull(acc));
-      // last item of this (sequence, group) in the CTA's range: its Qs is then free
-      const bool last_of_seq = tile + 1 == t_end || cur.t0 + kTileM >= cur.nb;
-      if (last_of_seq) tc::mma_commit(bempty);
+      // last piece of this (sequence, group) in the CTA's range: its Qs is then free
+      const int pb = pc.b, pg = pc.g;
+      pc.next();
+      if (pc.done() || pc.b != pb || pc.g != pg) tc::mma_commit(bempty);
     }
     // the last release of Qs lands before the CTA may exit
     if (ok && nseq > 0) tc::mbar_wait(bempty, (uint32_t)(nseq - 1) & 1u, P.flags);
@@ -287,12 +365,11 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
     int i = 0, eb = -1, so = -1;  // sequence and its ordinal in this CTA's range
-    ItemCursor ic;
-    ic.start(P.seq_off, P.B, P.n_tiles, t_begin);
-    for (int tile = t_begin; tile < t_end; ++tile, ++i, ic.next(P.seq_off, P.B)) {
-      const TileCursor& cur = ic.tc_;
-      if (cur.b != eb) {
-        eb = cur.b;
+    PieceCursor pc;
+    first_piece(pc);
+    for (; !pc.done(); ++i, pc.next()) {
+      if (pc.b != eb) {
+        eb = pc.b;
         ++so;
         if (so < kRangeSeqs && threadIdx.x == 64) {
           s_krb[so] = eb;
@@ -305,11 +382,13 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
                                                             P.flags));
       if (!ok) break;
       tc::fence_after_sync();
-      const int64_t off = cur.off;
-      const int64_t nb = cur.nb;
-      const int64_t t = cur.t0 + row;
+      const int64_t off = pc.off;
+      const int64_t nb = pc.nb;
+      const int64_t t = (int64_t)pc.q * kChunk + row;
+      // rows past the piece hold stale ring data: neither stored nor ranged
+      const bool live = row < pc.len * kChunk && t < nb;
       float* sbase = P.scores + off * P.U + t;
-      const int u0 = ic.g * (P.ncol / 2);  // first unit of the group
+      const int u0 = pc.g * (P.ncol / 2);  // first unit of the group
       for (int c0 = 0; c0 < P.ncol; c0 += 16) {
         uint32_t v[16];
         tc::tmem_ld16(lane_addr + (uint32_t)(acc * P.ncol + c0), v);
@@ -319,10 +398,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_kc,
           const int u = u0 + c0 / 2 + j;
           const float sv = __uint_as_float(v[2 * j]) + __uint_as_float(v[2 * j + 1]);
           const uint32_t key = order_key(sv);
-          const uint32_t kmn = __reduce_min_sync(0xffffffffu, t < nb ? key : 0xffffffffu);
-          const uint32_t kmx = __reduce_max_sync(0xffffffffu, t < nb ? key : 0u);
+          const uint32_t kmn = __reduce_min_sync(0xffffffffu, live ? key : 0xffffffffu);
+          const uint32_t kmx = __reduce_max_sync(0xffffffffu, live ? key : 0u);
           if (u < P.U) {
-            if (t < nb) sbase[(int64_t)u * nb] = sv;
+            if (live) sbase[(int64_t)u * nb] = sv;
             if (lane == 0) {
               if (so < kRangeSeqs) {
                 atomicMin(&s_kr[so][u][0], kmn);
@@ -394,7 +473,7 @@ cudaError_t launch_score_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream
   if (stages < 2) return cudaErrorInvalidConfiguration;
   const size_t smem = 1024 + (size_t)stages * kStageBytes + b_bytes + (2 * stages + 6) * 8 + 16;
   CUtensorMap tk, tq;
-  if (!make_tmap_bf16_2d(&tk, a.Kc, (uint64_t)p.N, (uint64_t)p.r, kTileM, 64) ||
+  if (!make_tmap_bf16_2d(&tk, a.Kc, (uint64_t)p.N, (uint64_t)p.r, kChunk, 64) ||
       !make_tmap_bf16_2d(&tq, a.qsplit, (uint64_t)p.B * p.npad, (uint64_t)p.r, ncol, 64))
     return cudaErrorInvalidValue;
   static int done[kMaxDevices] = {};
@@ -410,16 +489,17 @@ cudaError_t launch_score_tc(const DecodePlan& p, const DecodeArgs& a, cudaStream
   P.U = p.U;
   P.npad = p.npad;
   P.r = p.r;
-  P.n_tiles = p.n_score_tiles;
+  P.n_chunks = p.n_score_chunks;
   P.stages = stages;
   P.ng = ng;
   P.ncol = ncol;
   int cols = 32;
   while (cols < 2 * ncol) cols *= 2;
   P.tmem_cols = cols;
+  // at most one CTA per 128 rows of work
   const int max_ctas = num_sms() * ctas_per_sm;
-  const int64_t items = (int64_t)p.n_score_tiles * ng;
-  const int grid = items < max_ctas ? (int)items : max_ctas;
+  const int64_t pieces = ((int64_t)p.n_score_chunks * ng + kChunksPerTile - 1) / kChunksPerTile;
+  const int grid = pieces < max_ctas ? (int)pieces : max_ctas;
   return launch_k(score_tc_kernel, dim3(grid), dim3(kTcThreads), smem, s, true, tk, tq, P);
 }
 
