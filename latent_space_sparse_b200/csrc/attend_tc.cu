@@ -224,20 +224,36 @@ __device__ __forceinline__ int row_token(const AttendTcParams& P, const UnitTile
   return t;
 }
 
+// The same in two steps, so that the load is not waited for until the token
+// is used: the raw index of the row, and its check against n_b.
+__device__ __forceinline__ int row_raw(const AttendTcParams& P, const UnitTileCursor& c, int row) {
+  const int64_t jj = (int64_t)c.slot * kTile + row;
+  return jj < c.kb ? P.idx[((int64_t)c.b * P.U + c.u) * P.k + jj] : -1;
+}
+__device__ __forceinline__ int row_checked(const AttendTcParams& P, int t, int64_t nb) {
+  if (t < -1 || t >= nb) {
+    atomicOr(P.flags, FLAG_BAD_INDEX);
+    t = -1;
+  }
+  return t;
+}
+
 constexpr int kGatherRows = (kTile + kGatherThreads - 1) / kGatherThreads;  // token rows per gather thread
 
-// Gather thread gt's share of one tile's latent rows: items e = gt + 128j
+// Gather thread gt's share (of kW warps) of one tile's latent rows: items
 // over 32 row groups x KB k-blocks; item e copies rows tk[4g .. 4g+3]
 // (g = e % 32), latent columns (kb0 + kb)*64 .. +63 (kb = e / 32), by TMA
 // gather4 into k-block kb of the buffer (128-byte swizzled [128 x 64] blocks,
 // rows 4g .. 4g+3 at byte (g/2)*1024 + (g%2)*512).  A row without a token
 // (-1) copies row `off`, which gets weight 0.
+template <int kW>
 __device__ __forceinline__ void gather_rows(const int* tk, int64_t off, uint32_t buf_s,
                                             const CUtensorMap* tmap, int kb0, int KB, int gt,
                                             uint32_t mbar) {
-  // ops dealt round-robin over the group's warps (a warp issues its ops one
-  // after another)
-  for (int e = (gt % 32) * kGatherWarps + gt / 32; e < 32 * KB; e += kGatherThreads) {
+  // ops dealt round-robin over the warps: a warp's lanes issue their copies
+  // one after another, so the issue time of a tile falls with the warps
+  // that share it
+  for (int e = (gt % 32) * kW + gt / 32; e < 32 * KB; e += kW * 32) {
     const int g4 = e & 31, kb = e >> 5;
     int rows[4];
 #pragma unroll
@@ -361,7 +377,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
         if (gt + j * kGatherThreads < kTile) tk[gt + j * kGatherThreads] = t_next[j];
       if (gt == 0) tc::mbar_expect_tx(bar(B_KFULL + h), tile_bytes);
       tc::named_sync(gbar, kGatherThreads);
-      gather_rows(tk, off, buf_s, &tmap_kc, h * KB, KB, gt, bar(B_KFULL + h));
+      gather_rows<kGatherWarps>(tk, off, buf_s, &tmap_kc, h * KB, KB, gt, bar(B_KFULL + h));
       cur.next();
 #pragma unroll
       for (int j = 0; j < kGatherRows; ++j)
@@ -370,7 +386,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       if (!tc::mbar_wait(bar(B_KDONE + (i & 1)), ((uint32_t)i >> 1) & 1u, P.flags)) break;
       if (gt == 0) tc::mbar_expect_tx(bar(B_VFULL + h), tile_bytes);
       tc::named_sync(gbar, kGatherThreads);
-      gather_rows(tk, off, buf_s, &tmap_vc, h * KB, KB, gt, bar(B_VFULL + h));
+      gather_rows<kGatherWarps>(tk, off, buf_s, &tmap_vc, h * KB, KB, gt, bar(B_VFULL + h));
     }
   } else if (W == 2 && warp == kMmaWarp) {
     // ======================= MMA issuer, two latent halves ===================
@@ -467,51 +483,66 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     }
   } else if (warp >= kLoadWarp0) {
     // ======================= gather warps =======================
-    // Warp bi fills buffer bi with tiles bi, bi+2, ...: first the latent key
-    // rows Kc_b[idx], then, once the reconstruction is done with them, the
-    // same rows of Vc (gather_rows).  Thread gt looks up the token of row gt;
-    // the next tile's is loaded while the current tile is in flight.
-    const int bi = (warp - kLoadWarp0) / kGatherWarps;
-    const int gt = tid - (kLoadWarp0 + bi * kGatherWarps) * 32;  // 0..127
-    const uint32_t gbar = 2 + bi;  // named barrier of the group
-    int* tk = s_tok + bi * kTile;
-    const uint32_t buf_s = tc::smem_u32(bi ? s_buf1 : s_buf0);
+    // The eight gather warps issue the copies of every tile together, in the
+    // order K(i), K(i+1), V(i), V(i+1), K(i+2), ...: tile i goes to buffer
+    // i % 2, its latent key rows Kc_b[idx] once the value MMA of tile i-2 is
+    // done with the buffer, the same rows of Vc once the reconstruction of
+    // tile i is done with the key rows (gather_rows).  Thread gt < 128 looks
+    // up row gt of the pair's even tile, thread gt >= 128 row gt - 128 of the
+    // odd one; the next pair's indices are loaded while this pair is in
+    // flight, and checked when stored.  Every wait ends in a team-wide vote,
+    // so the team leaves together when one gives up.
+    constexpr int kTeamWarps = 2 * kGatherWarps;
+    constexpr int kTeam = kTeamWarps * 32;
+    const int gt = tid - kLoadWarp0 * 32;  // 0..255
+    const int half = gt >> 7, row = gt & (kTile - 1);
+    constexpr uint32_t kTeamBar = 2;
+    const uint32_t buf0 = tc::smem_u32(s_buf0), buf1 = tc::smem_u32(s_buf1);
     const uint32_t tile_bytes = (uint32_t)kTile * P.r * 2;
-    UnitTileCursor cur;
-    first_tile(cur);
-    if (bi == 1) cur.next();
+    UnitTileCursor ca, cb;  // tiles i and i+1
+    first_tile(ca);
+    cb = ca;
+    cb.next();
     grid_dependency_wait();  // the kept indices come from the previous kernel
-    if (gt == 0 && bi == 0) trace_stamp(P.trace, TRACE_WAITED);
-    int t_next[kGatherRows];
-#pragma unroll
-    for (int j = 0; j < kGatherRows; ++j)
-      t_next[j] = bi < n && gt + j * kGatherThreads < kTile ? row_token(P, cur, gt + j * kGatherThreads) : -1;
-    bool ok = true;
-    for (int i = bi; i < n && ok; i += 2) {
+    if (gt == 0) trace_stamp(P.trace, TRACE_WAITED);
+    int t_next = half < n ? row_raw(P, half ? cb : ca, row) : -1;
+    for (int i = 0; i < n; i += 2) {
+      const bool two = i + 1 < n;
       const uint32_t ph = ((uint32_t)i >> 1) & 1u;
-      const int64_t off = cur.off;
-      // the buffer is free once the value MMA of tile i-2 is done
-      if (i >= 2) {
-        ok = tc::mbar_wait(bar(B_PDONE + bi), ph ^ 1u, P.flags);
+      const int64_t off0 = ca.off, off1 = cb.off;
+      // K(i): buffer 0 is free once the value MMA of tile i-2 is done
+      bool okl = i < 2 || tc::mbar_wait(bar(B_PDONE + 0), ph ^ 1u, P.flags);
+      if (okl && half == 0) s_tok[row] = row_checked(P, t_next, ca.nb);
+      if (!tc::named_sync_and(kTeamBar, kTeam, okl)) break;
+      if (gt == 0) tc::mbar_expect_tx(bar(B_KFULL + 0), tile_bytes);
+      gather_rows<kTeamWarps>(s_tok, off0, buf0, &tmap_kc, 0, KB, gt, bar(B_KFULL + 0));
+      // K(i+1) into buffer 1, free once the value MMA of tile i-1 is done
+      if (two) {
+        okl = i < 2 || tc::mbar_wait(bar(B_PDONE + 1), ph ^ 1u, P.flags);
+        if (okl && half == 1) s_tok[kTile + row] = row_checked(P, t_next, cb.nb);
+        if (!tc::named_sync_and(kTeamBar, kTeam, okl)) break;
+        if (gt == 0) tc::mbar_expect_tx(bar(B_KFULL + 1), tile_bytes);
+        gather_rows<kTeamWarps>(s_tok + kTile, off1, buf1, &tmap_kc, 0, KB, gt,
+                                bar(B_KFULL + 1));
       }
-#pragma unroll
-      for (int j = 0; j < kGatherRows; ++j)
-        if (gt + j * kGatherThreads < kTile) tk[gt + j * kGatherThreads] = t_next[j];
-      if (gt == 0) tc::mbar_expect_tx(bar(B_KFULL + bi), tile_bytes);
-      tc::named_sync(gbar, kGatherThreads);
-      gather_rows(tk, off, buf_s, &tmap_kc, 0, KB, gt, bar(B_KFULL + bi));
-      // next tile of this group: its tokens arrive during this tile
-      cur.next();
-      cur.next();
-#pragma unroll
-      for (int j = 0; j < kGatherRows; ++j)
-        t_next[j] = i + 2 < n && gt + j * kGatherThreads < kTile
-                        ? row_token(P, cur, gt + j * kGatherThreads) : -1;
-      // the reconstruction is done with the key rows: bring the value rows
-      if (!tc::mbar_wait(bar(B_KDONE + bi), ph, P.flags)) break;
-      if (gt == 0) tc::mbar_expect_tx(bar(B_VFULL + bi), tile_bytes);
-      tc::named_sync(gbar, kGatherThreads);
-      gather_rows(tk, off, buf_s, &tmap_vc, 0, KB, gt, bar(B_VFULL + bi));
+      // the next pair's indices: loaded now, used at its key gathers
+      ca.next();
+      ca.next();
+      cb.next();
+      cb.next();
+      t_next = i + 2 + half < n ? row_raw(P, half ? cb : ca, row) : -1;
+      // V(i), V(i+1): the reconstruction is done with the key rows
+      okl = tc::mbar_wait(bar(B_KDONE + 0), ph, P.flags);
+      if (!tc::named_sync_and(kTeamBar, kTeam, okl)) break;
+      if (gt == 0) tc::mbar_expect_tx(bar(B_VFULL + 0), tile_bytes);
+      gather_rows<kTeamWarps>(s_tok, off0, buf0, &tmap_vc, 0, KB, gt, bar(B_VFULL + 0));
+      if (two) {
+        okl = tc::mbar_wait(bar(B_KDONE + 1), ph, P.flags);
+        if (!tc::named_sync_and(kTeamBar, kTeam, okl)) break;
+        if (gt == 0) tc::mbar_expect_tx(bar(B_VFULL + 1), tile_bytes);
+        gather_rows<kTeamWarps>(s_tok + kTile, off1, buf1, &tmap_vc, 0, KB, gt,
+                                bar(B_VFULL + 1));
+      }
     }
   } else if (warp == kMmaWarp) {
     // ======================= MMA issuer =======================
