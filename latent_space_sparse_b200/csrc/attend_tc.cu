@@ -51,10 +51,14 @@ constexpr int kEpiWarps = 16;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kEpiParts = kEpiWarps / 4;  // threads per token row
 constexpr int kMmaWarp = 16;
-constexpr int kLoadWarp0 = 17;  // warps 17-20 fill buffer 0 (even tiles), 21-24 buffer 1
-constexpr int kGatherWarps = 4;
+constexpr int kLoadWarp0 = 17;  // the gather warps follow the MMA warp
+constexpr int kGatherWarps = 4;  // per latent half (W = 2)
 constexpr int kGatherThreads = kGatherWarps * 32;
-constexpr int kThreads = (kLoadWarp0 + 2 * kGatherWarps) * 32;  // 800
+// Gather warps: one team of seven (W = 1), or four per latent half (W = 2).
+// Seven keep the block at 24 warps, six per scheduler, which leaves 80
+// registers a thread (25 warps put seven on one scheduler: 72 registers).
+template <int W> constexpr int gather_warps() { return W == 1 ? 7 : 2 * kGatherWarps; }
+template <int W> constexpr int block_threads() { return (kLoadWarp0 + gather_warps<W>()) * 32; }
 constexpr int kTile = 128;
 constexpr int kPRows = 16;  // rows of the p operand (2G <= 16)
 constexpr uint32_t kEpiBar = 1;
@@ -277,7 +281,7 @@ enum { B_PK = 0, B_KFULL = 1, B_VFULL = 3, B_KDONE = 5, B_PDONE = 7, B_PREADY = 
 // reconstruction accumulates over the halves), and tiles run one after the
 // other.
 template <int G, int D, int W, bool kMerge>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(block_threads<W>(), 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
                  const __grid_constant__ CUtensorMap tmap_kc,
                  const __grid_constant__ CUtensorMap tmap_vc, const AttendTcParams P) {
@@ -341,7 +345,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
   }
   if (warp == kMmaWarp) tc::tmem_alloc(tc::smem_u32(s_tmem_slot), 512);
   // the p operand's unused rows (2G..15) stay zero
-  for (int e = tid; e < 2 * 4096 / 4; e += kThreads) ((uint32_t*)s_pbuf0)[e] = 0u;
+  for (int e = tid; e < 2 * 4096 / 4; e += block_threads<W>()) ((uint32_t*)s_pbuf0)[e] = 0u;
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -483,19 +487,20 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     }
   } else if (warp >= kLoadWarp0) {
     // ======================= gather warps =======================
-    // The eight gather warps issue the copies of every tile together, in the
+    // The seven gather warps issue the copies of every tile together, in the
     // order K(i), K(i+1), V(i), V(i+1), K(i+2), ...: tile i goes to buffer
     // i % 2, its latent key rows Kc_b[idx] once the value MMA of tile i-2 is
     // done with the buffer, the same rows of Vc once the reconstruction of
-    // tile i is done with the key rows (gather_rows).  Thread gt < 128 looks
-    // up row gt of the pair's even tile, thread gt >= 128 row gt - 128 of the
-    // odd one; the next pair's indices are loaded while this pair is in
+    // tile i is done with the key rows (gather_rows).  A pair's 256 token
+    // slots (slot s: row s % 128 of tile i + s / 128) are dealt to the team's
+    // threads; the next pair's indices are loaded while this pair is in
     // flight, and checked when stored.  Every wait ends in a team-wide vote,
     // so the team leaves together when one gives up.
-    constexpr int kTeamWarps = 2 * kGatherWarps;
+    constexpr int kTeamWarps = gather_warps<1>();
     constexpr int kTeam = kTeamWarps * 32;
-    const int gt = tid - kLoadWarp0 * 32;  // 0..255
-    const int half = gt >> 7, row = gt & (kTile - 1);
+    // token slots s = gt + j*kTeam < 256 of a pair: tile s / 128, row s % 128
+    constexpr int kTokSlots = (2 * kTile + kTeam - 1) / kTeam;
+    const int gt = tid - kLoadWarp0 * 32;
     constexpr uint32_t kTeamBar = 2;
     const uint32_t buf0 = tc::smem_u32(s_buf0), buf1 = tc::smem_u32(s_buf1);
     const uint32_t tile_bytes = (uint32_t)kTile * P.r * 2;
@@ -505,21 +510,34 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     cb.next();
     grid_dependency_wait();  // the kept indices come from the previous kernel
     if (gt == 0) trace_stamp(P.trace, TRACE_WAITED);
-    int t_next = half < n ? row_raw(P, half ? cb : ca, row) : -1;
+    int t_next[kTokSlots];
+#pragma unroll
+    for (int j = 0; j < kTokSlots; ++j) {
+      const int sl = gt + j * kTeam;
+      t_next[j] = sl < 2 * kTile && (sl >> 7) < n ? row_raw(P, (sl >> 7) ? cb : ca, sl & 127) : -1;
+    }
     for (int i = 0; i < n; i += 2) {
       const bool two = i + 1 < n;
       const uint32_t ph = ((uint32_t)i >> 1) & 1u;
       const int64_t off0 = ca.off, off1 = cb.off;
       // K(i): buffer 0 is free once the value MMA of tile i-2 is done
       bool okl = i < 2 || tc::mbar_wait(bar(B_PDONE + 0), ph ^ 1u, P.flags);
-      if (okl && half == 0) s_tok[row] = row_checked(P, t_next, ca.nb);
+#pragma unroll
+      for (int j = 0; j < kTokSlots; ++j) {
+        const int sl = gt + j * kTeam;
+        if (okl && sl < kTile) s_tok[sl] = row_checked(P, t_next[j], ca.nb);
+      }
       if (!tc::named_sync_and(kTeamBar, kTeam, okl)) break;
       if (gt == 0) tc::mbar_expect_tx(bar(B_KFULL + 0), tile_bytes);
       gather_rows<kTeamWarps>(s_tok, off0, buf0, &tmap_kc, 0, KB, gt, bar(B_KFULL + 0));
       // K(i+1) into buffer 1, free once the value MMA of tile i-1 is done
       if (two) {
         okl = i < 2 || tc::mbar_wait(bar(B_PDONE + 1), ph ^ 1u, P.flags);
-        if (okl && half == 1) s_tok[kTile + row] = row_checked(P, t_next, cb.nb);
+#pragma unroll
+        for (int j = 0; j < kTokSlots; ++j) {
+          const int sl = gt + j * kTeam;
+          if (okl && sl >= kTile && sl < 2 * kTile) s_tok[sl] = row_checked(P, t_next[j], cb.nb);
+        }
         if (!tc::named_sync_and(kTeamBar, kTeam, okl)) break;
         if (gt == 0) tc::mbar_expect_tx(bar(B_KFULL + 1), tile_bytes);
         gather_rows<kTeamWarps>(s_tok + kTile, off1, buf1, &tmap_kc, 0, KB, gt,
@@ -530,7 +548,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
       ca.next();
       cb.next();
       cb.next();
-      t_next = i + 2 + half < n ? row_raw(P, half ? cb : ca, row) : -1;
+#pragma unroll
+      for (int j = 0; j < kTokSlots; ++j) {
+        const int sl = gt + j * kTeam;
+        t_next[j] = sl < 2 * kTile && i + 2 + (sl >> 7) < n
+                        ? row_raw(P, (sl >> 7) ? cb : ca, sl & 127) : -1;
+      }
       // V(i), V(i+1): the reconstruction is done with the key rows
       okl = tc::mbar_wait(bar(B_KDONE + 0), ph, P.flags);
       if (!tc::named_sync_and(kTeamBar, kTeam, okl)) break;
@@ -1063,7 +1086,8 @@ cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s)
   P.scale = p.scale;
   P.base = p.rope_base;
   if constexpr (!kMerge) {
-    return launch_k(attend_tc_kernel<G, D, W, false>, dim3(attend_tc_grid(p)), dim3(kThreads),
+    return launch_k(attend_tc_kernel<G, D, W, false>, dim3(attend_tc_grid(p)),
+                    dim3(block_threads<W>()),
                     smem, s, true, tpk, tkc, tvc, P);
   } else {
     // one cluster of att_cluster CTAs per unit
@@ -1071,7 +1095,7 @@ cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s)
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(p.B * p.U * p.att_cluster));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(block_threads<W>());
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
