@@ -89,17 +89,19 @@ __device__ __forceinline__ void latent_q_body(const T* __restrict__ q, const T* 
                              ((v[j][4] + v[j][5]) + (v[j][6] + v[j][7]));
     }
     __syncthreads();
-#pragma unroll
-    for (int bb = 0; bb < kBatchChunk; ++bb) {
+    // the chunk's live sequences only (a chain of shared-memory loads and
+    // FMAs per sequence: at B = 1 one pass, not kBatchChunk)
+#pragma unroll 1
+    for (int bb = 0; bb < nb; ++bb) {
       float acc = 0.f;
 #pragma unroll
       for (int j = 0; j < kRowsMax; ++j)
-        if (j < rows && i0 + j < d && bb < nb) acc = fmaf(qsum[bb][i0 + j], pk[j], acc);
+        if (j < rows && i0 + j < d) acc = fmaf(qsum[bb][i0 + j], pk[j], acc);
       red[slice][bb][col] = acc;
     }
     __syncthreads();
-    if (tid < nb * COLS) {
-      const int bb = tid / COLS, cl = tid % COLS;
+    for (int e = tid; e < nb * COLS; e += kThreads) {
+      const int bb = e / COLS, cl = e % COLS;
       const int cc = blockIdx.y * COLS + cl;
       float sum = 0.f;
 #pragma unroll
