@@ -88,13 +88,17 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def measured_bf16_peak():
-    """Burst bf16 dense GEMM TFLOP/s (a kernel timed alone)."""
+def measured_bf16_peak(sustained: bool = False):
+    """bf16 dense GEMM TFLOP/s: the burst figure (a kernel timed alone), or the
+    sustained one (GEMMs back to back under the power cap)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as f:
-            return float(json.load(f)["bf16_tflops"]), "measured"
-    return 1590.0, "fallback"
+            peaks = json.load(f)
+        key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+        if key in peaks:
+            return float(peaks[key]), "measured"
+    return (1400.0 if sustained else 1590.0), "fallback"
 
 
 def bench_compress(salsc, dev, reps: int = 20, warmup: int = 3, rows: int = 0):
@@ -126,15 +130,46 @@ def bench_compress(salsc, dev, reps: int = 20, warmup: int = 3, rows: int = 0):
         ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(reps)]
         return statistics.median(ms)
 
-    ms = timed(lambda: salsc.salsc_compress(K, V, Pk, Pv, Kc, Vc))
-    ms_lib = timed(lambda: (torch.matmul(K, Pk, out=Kc), torch.matmul(V, Pv, out=Vc)))
+    def isolated(fn):
+        # each launch after the GPU has idled for a few ms, so that it runs at
+        # the clocks a kernel timed alone gets (the back-to-back loop above
+        # settles under the power cap)
+        for _ in range(warmup):
+            fn()
+        ms = []
+        for _ in range(reps):
+            torch.cuda.synchronize(dev)
+            time.sleep(0.004)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        return statistics.median(ms)
+
+    ours = lambda: salsc.salsc_compress(K, V, Pk, Pv, Kc, Vc)  # noqa: E731
+    lib = lambda: (torch.matmul(K, Pk, out=Kc), torch.matmul(V, Pv, out=Vc))  # noqa: E731
+    with ClockSampler(dev.index if dev.index is not None else 0) as sampler:
+        ms = timed(ours)
+        ms_lib = timed(lib)
+    ms_iso, ms_iso_lib = isolated(ours), isolated(lib)
     peak, kind = measured_bf16_peak()
+    peak_s, kind_s = measured_bf16_peak(sustained=True)
     tf = flop / (ms * 1e-3) / 1e12
+    tf_iso = flop / (ms_iso * 1e-3) / 1e12
     return {"workload": f"{w.name} prefill: 2 x [{n} x {hid}] . [{hid} x {r}] bf16",
-            "us": ms * 1e3, "achieved": tf, "peak": peak, "unit": "TFLOP/s", "bound": "tensor",
-            "frac": tf / peak, "peak_kind": kind,
-            "torch_matmul_us": ms_lib * 1e3,
-            "torch_matmul_tflops": flop / (ms_lib * 1e-3) / 1e12}
+            "us": ms_iso * 1e3, "achieved": tf_iso, "peak": peak, "unit": "TFLOP/s",
+            "bound": "tensor", "frac": tf_iso / peak, "peak_kind": kind,
+            "torch_matmul_us": ms_iso_lib * 1e3,
+            "torch_matmul_tflops": flop / (ms_iso_lib * 1e-3) / 1e12,
+            "how": f"median of {reps} launches, each after {4} ms of idle GPU (a kernel timed "
+                   "alone, against the burst peak); back_to_back: the same launches in a loop, "
+                   "against the sustained peak",
+            "back_to_back": {"us": ms * 1e3, "achieved": tf, "peak": peak_s, "frac": tf / peak_s,
+                             "peak_kind": kind_s, "torch_matmul_us": ms_lib * 1e3,
+                             "torch_matmul_tflops": flop / (ms_lib * 1e-3) / 1e12,
+                             "clocks": sampler.summary()}}
 
 
 # ------------------------------------------------------------------ clocks
