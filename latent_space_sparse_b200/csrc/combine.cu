@@ -55,6 +55,49 @@ struct CombineParams {
   uint32_t rowbuf;  // bytes of partial rows per batch (a multiple of one row per head)
 };
 
+// Used slots of unit (b, u), in slot order, into seg[]; by one whole warp,
+// every lane returns the count.  Slots follow from the sequence lengths and
+// the tile partition alone (inputs of the step, not outputs of the attention
+// kernel), so they are found before the dependency wait.
+__device__ __forceinline__ int used_slots(const CombineParams& P, int b, int u, int* seg) {
+  const int lane = threadIdx.x % 32;
+  // slots of unit (b, u) and, with the tile partition, the unit's first tile:
+  // every lane reads one sequence's offsets, a warp scan sums the tiles
+  int64_t before = 0;  // tiles of the sequences before b
+  int tb = P.fixed_slots;
+  for (int b0 = 0; b0 <= b && P.fixed_slots == 0; b0 += 32) {
+    const int bb = b0 + lane;
+    int64_t t = 0;
+    if (bb <= b && bb < P.B) {
+      const int64_t n2 = P.seq_off[bb + 1] - P.seq_off[bb];
+      const int64_t k2 = n2 < P.k ? n2 : P.k;
+      t = (k2 + P.chunk - 1) / P.chunk;
+      if (bb == b) tb = (int)t;
+    }
+    int64_t x = bb < b ? t : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    before += x;
+  }
+  if (P.fixed_slots == 0) tb = __reduce_max_sync(0xffffffffu, tb);  // set by the lane of sequence b only
+  const int64_t unit_tile0 = before * P.U + (int64_t)u * tb;
+  int cnt = 0;
+  for (int s0 = 0; s0 < tb; s0 += 32) {
+    const int sl = s0 + lane;
+    bool used = sl < tb;
+    if (used && sl > 0 && P.seg_grid > 0) {
+      // tile t starts a CTA's range [c*T/grid, (c+1)*T/grid)
+      const int64_t t = unit_tile0 + sl, T = P.seg_tiles, gc = P.seg_grid;
+      const int64_t c = (t * gc + T - 1) / T;  // first CTA at or after t
+      used = c < gc && c * T / gc == t;
+    }
+    const uint32_t mk = __ballot_sync(0xffffffffu, used);
+    if (used) seg[cnt + __popc(mk & ((1u << lane) - 1u))] = sl;
+    cnt += __popc(mk);
+  }
+  return cnt;
+}
+
 template <typename T, int G>
 __global__ void __launch_bounds__(kThreads)
 combine_kernel(const CombineParams P) {
@@ -94,40 +137,7 @@ combine_kernel(const CombineParams P) {
   // alone (inputs of the step, not outputs of the attention kernel), so they
   // are found before the dependency wait.
   if (warp == 0) {
-    // slots of unit (b, u) and, with the tile partition, the unit's first tile:
-    // every lane reads one sequence's offsets, a warp scan sums the tiles
-    int64_t before = 0;  // tiles of the sequences before b
-    int tb = P.fixed_slots;
-    for (int b0 = 0; b0 <= b && P.fixed_slots == 0; b0 += 32) {
-      const int bb = b0 + lane;
-      int64_t t = 0;
-      if (bb <= b && bb < P.B) {
-        const int64_t n2 = P.seq_off[bb + 1] - P.seq_off[bb];
-        const int64_t k2 = n2 < P.k ? n2 : P.k;
-        t = (k2 + P.chunk - 1) / P.chunk;
-        if (bb == b) tb = (int)t;
-      }
-      int64_t x = bb < b ? t : 0;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-      before += x;
-    }
-    if (P.fixed_slots == 0) tb = __reduce_max_sync(0xffffffffu, tb);  // set by the lane of sequence b only
-    const int64_t unit_tile0 = before * P.U + (int64_t)u * tb;
-    int cnt = 0;
-    for (int s0 = 0; s0 < tb; s0 += 32) {
-      const int sl = s0 + lane;
-      bool used = sl < tb;
-      if (used && sl > 0 && P.seg_grid > 0) {
-        // tile t starts a CTA's range [c*T/grid, (c+1)*T/grid)
-        const int64_t t = unit_tile0 + sl, T = P.seg_tiles, gc = P.seg_grid;
-        const int64_t c = (t * gc + T - 1) / T;  // first CTA at or after t
-        used = c < gc && c * T / gc == t;
-      }
-      const uint32_t mk = __ballot_sync(0xffffffffu, used);
-      if (used) s_seg[cnt + __popc(mk & ((1u << lane) - 1u))] = sl;
-      cnt += __popc(mk);
-    }
+    const int cnt = used_slots(P, b, u, s_seg);
     if (lane == 0) s_nseg = cnt;
     if (lane < G) {
       s_M[lane] = -INFINITY;
@@ -265,6 +275,119 @@ combine_kernel(const CombineParams P) {
   if (tid == 0) trace_stamp(P.trace, TRACE_END);
 }
 
+// Many units (a grid of the kernel above beyond two CTAs per SM, e.g. 16
+// sequences x 32 MHA heads): one warp per (sequence, unit, 16 output rows),
+// eight sequences per CTA sharing the CTA's 16 rows of Pv_u.  A warp merges
+// its unit's used slots in registers (lane j holds latent columns 2j + 64i,
+// +1 of every head), then projects: each lane forms its columns' share of
+// the 16 x G output dots, and a shuffle reduce-scatter leaves the sums of
+// row i on lanes 2i, 2i+1.  Same merge as above, slot by slot in slot order.
+constexpr int kSeqWarps = 8;
+__device__ __forceinline__ float2 pv2_f32(const __nv_bfloat16* p) {
+  return __bfloat1622float2(*(const __nv_bfloat162*)p);
+}
+__device__ __forceinline__ float2 pv2_f32(const float* p) { return *(const float2*)p; }
+template <typename T, int G, int R64>  // R64 = r / 64
+__global__ void __launch_bounds__(kSeqWarps * 32)
+combine_seq_kernel(const CombineParams P) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  T* const pv_s = (T*)smem;  // [16][r]
+  __shared__ int s_seg[kSeqWarps][kMaxSegs];
+  const int n_slices = P.d / kRows;
+  const int slice = blockIdx.x % n_slices;
+  const int rest = blockIdx.x / n_slices;
+  const int u = rest % P.U, bg = rest / P.U;
+  const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+  const int b = bg * kSeqWarps + warp;
+  const int r = R64 * 64;
+  if (tid == 0) trace_stamp(P.trace, TRACE_START);
+  allow_dependent_launch();
+  // the 16 rows of Pv_u (a weight) and the used slots, before the wait
+  {
+    const uint4* src = (const uint4*)((const T*)P.Pv + ((int64_t)u * P.d + (int64_t)slice * kRows) * r);
+    uint4* dst = (uint4*)pv_s;
+    const int n16 = kRows * r * (int)sizeof(T) / 16;
+    for (int e = tid; e < n16; e += kSeqWarps * 32) dst[e] = src[e];
+  }
+  const int nseg = b < P.B ? used_slots(P, b, u, s_seg[warp]) : 0;
+  grid_dependency_wait();  // the partials come from the attention kernel
+  if (tid == 0) trace_stamp(P.trace, TRACE_WAITED);
+  __syncthreads();  // the Pv rows
+  if (b < P.B) {
+    const int rowf = part_row(r);
+    float acc[G][2 * R64];
+    float M[G], L[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      M[g] = -INFINITY;
+      L[g] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 2 * R64; ++j) acc[g][j] = 0.f;
+    }
+    const float* part_u = P.part + ((int64_t)b * P.Hq + (int64_t)u * G) * P.bh_stride * rowf;
+    for (int q = 0; q < nseg; ++q) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float* row = part_u + ((int64_t)g * P.bh_stride + s_seg[warp][q] * P.slot_stride) * rowf;
+        const float m = row[0], l = row[1];
+        float2 v[R64];
+#pragma unroll
+        for (int i = 0; i < R64; ++i) v[i] = *(const float2*)(row + kPartAcc + 2 * lane + 64 * i);
+        const float Mn = fmaxf(M[g], m);
+        const float sc = M[g] == -INFINITY ? 0.f : expf(M[g] - Mn);
+        const float w = m == -INFINITY ? 0.f : expf(m - Mn);
+        L[g] = L[g] * sc + w * l;
+        M[g] = Mn;
+#pragma unroll
+        for (int i = 0; i < R64; ++i) {
+          acc[g][2 * i] = fmaf(w, v[i].x, acc[g][2 * i] * sc);
+          acc[g][2 * i + 1] = fmaf(w, v[i].y, acc[g][2 * i + 1] * sc);
+        }
+      }
+    }
+    // projection: o[g][i] = sum over this lane's columns of Pv row i . acc
+    float o[G][kRows];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float inv = L[g] > 0.f ? 1.f / L[g] : 0.f;
+#pragma unroll
+      for (int i = 0; i < kRows; ++i) o[g][i] = 0.f;
+#pragma unroll
+      for (int c = 0; c < R64; ++c) {
+        const float a0 = acc[g][2 * c] * inv, a1 = acc[g][2 * c + 1] * inv;
+#pragma unroll
+        for (int i = 0; i < kRows; ++i) {
+          const float2 pv = pv2_f32(pv_s + (size_t)i * r + 2 * lane + 64 * c);
+          o[g][i] = fmaf(pv.x, a0, fmaf(pv.y, a1, o[g][i]));
+        }
+      }
+    }
+    // reduce-scatter over the 32 lanes: after the step with offset 16 >> s,
+    // a lane keeps the rows whose bit (3 - s) matches its lane bit (4 - s)
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+#pragma unroll
+      for (int half = 8, off = 16; half >= 1; half >>= 1, off >>= 1) {
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+          const float send = upper ? o[g][i] : o[g][i + half];
+          const float keep = upper ? o[g][i + half] : o[g][i];
+          o[g][i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
+      // lanes 2i, 2i+1 hold row i's sums over lanes of equal bit 0: add the pair
+      const float tot = o[g][0] + __shfl_xor_sync(0xffffffffu, o[g][0], 1);
+      const int i = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
+                    ((lane >> 1) & 1);
+      if ((lane & 1) == 0)
+        ((T*)P.out)[((int64_t)b * P.Hq + (int64_t)u * G + g) * P.d + slice * kRows + i] =
+            from_f32<T>(tot);
+    }
+  }
+  if (tid == 0) trace_stamp(P.trace, TRACE_END);
+}
+
 size_t combine_smem(const DecodePlan& p, uint32_t rowbuf) {
   const size_t elem = p.dtype == SALSC_BF16 ? 2 : 4;
   return (size_t)kRows * p.r * elem + rowbuf + sizeof(float) * (size_t)p.G * (p.r + 32);
@@ -317,9 +440,27 @@ int num_sms_cb() {
   return cached[dev];
 }
 
+template <typename T, int G, int R64>
+cudaError_t launch_seq(const CombineParams& P, const DecodePlan& p, cudaStream_t s) {
+  static int done[kMaxDevices] = {};
+  const size_t smem = (size_t)kRows * p.r * sizeof(T);
+  cudaError_t e = ensure_smem(combine_seq_kernel<T, G, R64>, smem, done);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)((p.d / kRows) * p.U * ((p.B + kSeqWarps - 1) / kSeqWarps)));
+  return launch_k(combine_seq_kernel<T, G, R64>, grid, dim3(kSeqWarps * 32), smem, s, true, P);
+}
+
 template <typename T, int G>
 cudaError_t launch_tg(const CombineParams& P, const DecodePlan& p, cudaStream_t s) {
   static int done[kMaxDevices] = {};
+  // many units, one head per unit: a warp per (sequence, unit, slice)
+  if constexpr (G == 1) {
+    if (!P.part_out && P.fixed_slots == 0 &&
+        (int64_t)p.B * p.U * (p.d / kRows) > 2 * (int64_t)num_sms_cb()) {
+      if (p.r == 512) return launch_seq<T, 1, 8>(P, p, s);
+      if (p.r == 256) return launch_seq<T, 1, 4>(P, p, s);
+    }
+  }
   size_t smem = combine_smem(p, P.rowbuf);
   // A grid of at most two CTAs per SM asks for enough shared memory that no
   // more than two fit on an SM: the CTAs launched early, while the attention
