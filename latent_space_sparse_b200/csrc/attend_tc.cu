@@ -5,9 +5,9 @@
 // SALS technical framework, stages 3-4, with RoPE applied after
 // reconstruction (abstract).  Work unit: a tile of 128 kept tokens of one
 // selection unit (b, u):
-//   1. a gather warp copies the 128 latent key rows Kc_b[idx] into shared
-//      memory (cp.async, 16 bytes a lane, into the 128-byte swizzled K-major
-//      layout);
+//   1. the gather warps copy the 128 latent key rows Kc_b[idx] into shared
+//      memory by TMA gather4 (four rows of 64 latent columns per copy, into
+//      the 128-byte swizzled K-major layout);
 //   2. tcgen05: K_sel[128 x d] = Kc_tile . Pk_u^T into TMEM (fp32; Pk_u comes
 //      by TMA once per unit and stays in shared memory);
 //   3. the same rows of Vc are copied into the buffer the MMA has finished
@@ -29,13 +29,15 @@
 //      so the combine kernel finds the used slots from the tile partition
 //      alone; it merges the few segments of a unit and applies the deferred
 //      Pv_u^T.
-// Warp roles (800 threads): warps 0-15 epilogue, warp 16 TMEM owner and MMA
-// issuer, warps 17-20 and 21-24 row gathers (four per tile buffer: the issue
-// of TMA gather4 copies bounds the gather chain).  The epilogue is the
-// busiest role (RoPE needs a sine and a cosine per pair and token), so it has
-// four warps per scheduler; 25 warps keep 72 registers per thread (the
-// register file is split per scheduler).  Each CTA walks a contiguous range
-// of tiles;
+// Warp roles: warps 0-15 epilogue, warp 16 TMEM owner and MMA issuer, then
+// the gather warps: r <= 256, a team of seven (768 threads, 24 warps, 80
+// registers a thread) that issues every tile's copies together (a warp's
+// lanes issue their TMA copies one after another, so a tile's issue time
+// falls with the warps sharing it); r > 256, two groups of four, one per
+// latent half (800 threads, 72 registers: 25 warps put seven on one
+// scheduler, whose register file is a quarter of the SM's).  The epilogue is
+// the busiest role (RoPE needs a sine and a cosine per pair and token), so it
+// has four warps per scheduler.  Each CTA walks a contiguous range of tiles;
 // the two tile buffers alternate (Kc(i) -> Vc(i) -> Kc(i+2)), so the
 // reconstruction of tile i+1 runs during the epilogue of tile i.
 //
