@@ -109,10 +109,11 @@ __device__ __forceinline__ void find_digit(Cnt cnt, uint32_t target, int nbins, 
 }
 
 template <bool kCluster, int kThreads>
-__global__ void __launch_bounds__(kThreads)
-topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_off,
-            const uint32_t* __restrict__ krange, int32_t* __restrict__ idx_out, int U, int k,
-            uint32_t kthr, uint64_t* trace) {
+__device__ __forceinline__ void topk_body(const float* __restrict__ scores,
+                                          const int64_t* __restrict__ seq_off,
+                                          const uint32_t* __restrict__ krange,
+                                          int32_t* __restrict__ idx_out, int U, int k,
+                                          uint32_t kthr, uint64_t* trace) {
   constexpr int kWarps = kThreads / 32;
   cg::cluster_group cluster = cg::this_cluster();
   const int C = kCluster ? (int)cluster.num_blocks() : 1;
@@ -464,13 +465,39 @@ topk_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_of
   if (tid == 0) trace_stamp(trace, TRACE_END);
 }
 
+// 1024-thread CTAs, at most 48 registers a thread: a CTA (49K registers) then
+// fits beside one scoring CTA (10.8K), so the top-k CTAs, launched early,
+// take an SM as soon as one of its two scoring CTAs has finished, not both.
+template <bool kCluster>
+__global__ void __maxnreg__(48)
+topk1024_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_off,
+                const uint32_t* __restrict__ krange, int32_t* __restrict__ idx_out, int U,
+                int k, uint32_t kthr, uint64_t* trace) {
+  topk_body<kCluster, 1024>(scores, seq_off, krange, idx_out, U, k, kthr, trace);
+}
+
+// 256-thread CTAs (many small units, several CTAs per SM)
+template <bool kCluster>
+__global__ void __launch_bounds__(256)
+topk256_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_off,
+               const uint32_t* __restrict__ krange, int32_t* __restrict__ idx_out, int U, int k,
+               uint32_t kthr, uint64_t* trace) {
+  topk_body<kCluster, 256>(scores, seq_off, krange, idx_out, U, k, kthr, trace);
+}
+
+template <bool kCluster, int kThreads>
+constexpr auto topk_kernel_of() {
+  if constexpr (kThreads == 1024) return topk1024_kernel<kCluster>;
+  else return topk256_kernel<kCluster>;
+}
+
 template <bool kCluster, int kThreads>
 cudaError_t launch_tk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) {
   const size_t smem = sizeof(uint32_t) * (size_t)p.topk_slice;
   static int done[kMaxDevices] = {};
-  cudaError_t e = ensure_smem(topk_kernel<kCluster, kThreads>, smem, done);
+  cudaError_t e = ensure_smem(topk_kernel_of<kCluster, kThreads>(), smem, done);
   if (e != cudaSuccess) return e;
-  e = prefer_max_shared((const void*)topk_kernel<kCluster, kThreads>);
+  e = prefer_max_shared((const void*)topk_kernel_of<kCluster, kThreads>());
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(p.B * p.U * p.topk_cluster));
@@ -486,7 +513,7 @@ cudaError_t launch_tk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) 
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = kCluster ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, topk_kernel<kCluster, kThreads>, (const float*)a.scores,
+  return cudaLaunchKernelEx(&cfg, topk_kernel_of<kCluster, kThreads>(), (const float*)a.scores,
                             (const int64_t*)a.seq_off, (const uint32_t*)a.krange, a.idx, p.U, p.k,
                             p.topk_kthr, trace_of(a, 2));
 }
