@@ -75,6 +75,9 @@ salsc_status make_plan(const salsc_decode_desc* D, salsc::DecodePlan* P) {
   p.score_tile = kScoreTile;
   p.n_score_tiles = n_tiles;
   p.n_score_chunks = n_chunks;
+  p.uni_nb = D->seq_offsets_host[1];
+  for (int b = 1; b < D->batch; ++b)
+    if (D->seq_offsets_host[b + 1] - D->seq_offsets_host[b] != p.uni_nb) p.uni_nb = 0;
   // Top-k: C CTAs per unit, about one CTA per SM in all (up to 8 per unit, and
   // enough for a slice of the scores to fit shared memory); many small units
   // take 256-thread CTAs, several resident per SM.

@@ -79,6 +79,7 @@ struct AttendTcParams {
   const __nv_bfloat16* Pv;  // merged in the kernel: the value projection
   __nv_bfloat16* out;
   int B, Hq, U, r, k, n_slots, n_tiles;
+  int64_t uni_nb;  // every sequence's length when they are equal, else 0
   int cluster;  // merged in the kernel: CTAs per unit (one thread-block cluster)
   uint64_t* trace;  // traced step: this kernel's rows, or null
   float scale;
@@ -132,9 +133,40 @@ struct UnitTileCursor {
 // slot) to st[0..4] and (off, nb) of sequence b to st64[0..1]; b = B when the
 // range is empty.
 __device__ __forceinline__ void find_first_tile(const int64_t* so, int B, int U, int k,
-                                                int n_tiles, int cluster, int* st,
-                                                int64_t* st64) {
+                                                int n_tiles, int cluster, int64_t uni_nb,
+                                                int* st, int64_t* st64) {
   const int lane = threadIdx.x % 32;
+  if (uni_nb > 0) {
+    // every sequence has uni_nb tokens: the first tile is arithmetic, no loads
+    const int tu = (int)(((uni_nb < k ? uni_nb : (int64_t)k) + kTile - 1) / kTile);
+    int t_begin, n, fb, fu = 0, fslot = 0;
+    if (cluster > 0) {
+      const int m_unit = (int)(blockIdx.x / (unsigned)cluster);
+      const int m_rank = (int)(blockIdx.x % (unsigned)cluster);
+      const int l0 = tu * m_rank / cluster, h0 = tu * (m_rank + 1) / cluster;
+      t_begin = m_unit * tu + l0;
+      n = h0 - l0;
+    } else {
+      t_begin = (int)((int64_t)blockIdx.x * n_tiles / gridDim.x);
+      n = (int)((int64_t)(blockIdx.x + 1) * n_tiles / gridDim.x) - t_begin;
+    }
+    fb = n > 0 && tu > 0 ? t_begin / (U * tu) : B;
+    if (fb < B) {
+      const int rem = t_begin - fb * U * tu;
+      fu = rem / tu;
+      fslot = rem % tu;
+    }
+    if (lane == 0) {
+      st[0] = t_begin;
+      st[1] = n;
+      st[2] = fb;
+      st[3] = fu;
+      st[4] = fslot;
+      st64[0] = (int64_t)fb * uni_nb;
+      st64[1] = uni_nb;
+    }
+    return;
+  }
   int t_begin = 0, n = 0, mb = -1;
   if (cluster > 0) {
     mb = (int)(blockIdx.x / (unsigned)cluster) / U;  // the unit's sequence
@@ -327,8 +359,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
   const int m_unit = kMerge ? (int)(blockIdx.x / (unsigned)P.cluster) : 0;
   // Tile range and first tile (set before the block-wide barrier below).
   if (warp == kLoadWarp0)
-    find_first_tile(P.seq_off, P.B, P.U, P.k, P.n_tiles, kMerge ? P.cluster : 0, s_start,
-                    s_start64);
+    find_first_tile(P.seq_off, P.B, P.U, P.k, P.n_tiles, kMerge ? P.cluster : 0, P.uni_nb,
+                    s_start, s_start64);
   int n = 0;  // tiles of this CTA
   auto first_tile = [&](UnitTileCursor& c) {
     c.at(P.seq_off, P.B, P.U, P.k, s_start[2], s_start[3], s_start[4], s_start64[0],
@@ -1083,6 +1115,7 @@ cudaError_t launch_g_d(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s)
   P.k = p.k;
   P.n_slots = p.splits;
   P.n_tiles = p.att_tiles;
+  P.uni_nb = p.uni_nb;
   P.cluster = kMerge ? p.att_cluster : 1;
   P.trace = trace_of(a, 3);
   P.scale = p.scale;

@@ -42,6 +42,7 @@ struct DecodePlan {
   int n_score_tiles;    // sum_b ceil(n_b / score tile)
   int score_tile;       // tokens per scoring CTA
   int n_score_chunks;   // sum_b ceil(n_b / 32): the tensor-core scoring kernel's work items
+  int64_t uni_nb;       // the common length when every sequence has it, else 0
   int topk_cluster;     // CTAs per selection unit in the top-k kernel
   int topk_slice;       // max keys per top-k CTA
   int topk_threads;     // threads per top-k CTA (1024, or 256 for many small units)

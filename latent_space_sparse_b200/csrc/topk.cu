@@ -113,7 +113,7 @@ __device__ __forceinline__ void topk_body(const float* __restrict__ scores,
                                           const int64_t* __restrict__ seq_off,
                                           const uint32_t* __restrict__ krange,
                                           int32_t* __restrict__ idx_out, int U, int k,
-                                          uint32_t kthr, uint64_t* trace) {
+                                          uint32_t kthr, int64_t uni_nb, uint64_t* trace) {
   constexpr int kWarps = kThreads / 32;
   cg::cluster_group cluster = cg::this_cluster();
   const int C = kCluster ? (int)cluster.num_blocks() : 1;
@@ -146,8 +146,9 @@ __device__ __forceinline__ void topk_body(const float* __restrict__ scores,
   }
   if (tid == 0) s_ncand = 0u;
   allow_dependent_launch();
-  const int64_t off = seq_off[b];
-  const int64_t nb = seq_off[b + 1] - off;
+  // equal lengths: the unit's scores are found without a load
+  const int64_t off = uni_nb > 0 ? (int64_t)b * uni_nb : seq_off[b];
+  const int64_t nb = uni_nb > 0 ? uni_nb : seq_off[b + 1] - off;
   const int64_t kb = nb < k ? nb : k;
   const float* s = scores + off * U + (int64_t)u * nb;
   const int64_t lo = nb * rank / C, hi = nb * (rank + 1) / C;
@@ -472,8 +473,8 @@ template <bool kCluster>
 __global__ void __maxnreg__(48)
 topk1024_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_off,
                 const uint32_t* __restrict__ krange, int32_t* __restrict__ idx_out, int U,
-                int k, uint32_t kthr, uint64_t* trace) {
-  topk_body<kCluster, 1024>(scores, seq_off, krange, idx_out, U, k, kthr, trace);
+                int k, uint32_t kthr, int64_t uni_nb, uint64_t* trace) {
+  topk_body<kCluster, 1024>(scores, seq_off, krange, idx_out, U, k, kthr, uni_nb, trace);
 }
 
 // 256-thread CTAs (many small units, several CTAs per SM)
@@ -481,8 +482,8 @@ template <bool kCluster>
 __global__ void __launch_bounds__(256)
 topk256_kernel(const float* __restrict__ scores, const int64_t* __restrict__ seq_off,
                const uint32_t* __restrict__ krange, int32_t* __restrict__ idx_out, int U, int k,
-               uint32_t kthr, uint64_t* trace) {
-  topk_body<kCluster, 256>(scores, seq_off, krange, idx_out, U, k, kthr, trace);
+               uint32_t kthr, int64_t uni_nb, uint64_t* trace) {
+  topk_body<kCluster, 256>(scores, seq_off, krange, idx_out, U, k, kthr, uni_nb, trace);
 }
 
 template <bool kCluster, int kThreads>
@@ -515,7 +516,7 @@ cudaError_t launch_tk(const DecodePlan& p, const DecodeArgs& a, cudaStream_t s) 
   cfg.numAttrs = kCluster ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, topk_kernel_of<kCluster, kThreads>(), (const float*)a.scores,
                             (const int64_t*)a.seq_off, (const uint32_t*)a.krange, a.idx, p.U, p.k,
-                            p.topk_kthr, trace_of(a, 2));
+                            p.topk_kthr, p.uni_nb, trace_of(a, 2));
 }
 
 }  // namespace
