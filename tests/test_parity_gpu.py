@@ -153,6 +153,19 @@ def test_wide_rank_512_mha_many_tiles():
     check(w, synth.decode_inputs(w, seq_lens=(4096,)), top_k=1000)
 
 
+@pytest.mark.parametrize("batch,heads,rank,lens", [
+    (11, 32, 512, (300, 517, 900, 128, 640, 777, 256, 1000, 333, 129, 450)),  # ragged, B % 8 != 0
+    (9, 16, 256, (500,) * 9),                                                # equal lengths, r = 256
+])
+def test_merge_one_warp_per_sequence(batch, heads, rank, lens):
+    # many single-head units: the merge runs one warp per (sequence, unit, 16
+    # output rows), eight sequences per CTA (the last CTA's spare warps idle)
+    w = W.Workload(name="mha_many_units", batch=batch, n_q_heads=heads, n_kv_heads=heads,
+                   head_dim=128, rank=rank, top_k=256, seq_lens=lens, dtype="bf16",
+                   rope_base=10000.0, low_rank=32, seed=93 + batch)
+    check(w, synth.decode_inputs(w))
+
+
 def launches(w, top_k=None):
     lens = w.seq_lens
     dec = salsc.Decoder(len(lens), w.n_q_heads, w.n_kv_heads, w.head_dim, w.rank,
