@@ -110,6 +110,15 @@ def test_single_token_sequences_and_k_above_n():
     check(w, x, top_k=64)
 
 
+def test_equal_lengths_k_above_n():
+    # every sequence has the same length (the kernels' equal-length path),
+    # shorter than k: every token is kept and the tail slots are -1
+    w = W.Workload(name="equal_short", batch=3, n_q_heads=8, n_kv_heads=2, head_dim=128,
+                   rank=256, top_k=300, seq_lens=(100, 100, 100), dtype="bf16",
+                   rope_base=10000.0, low_rank=16, seed=91)
+    check(w, synth.decode_inputs(w))
+
+
 def test_k_equals_one():
     w = W.LLAMA2_4K_B1
     check(w, synth.decode_inputs(w, seq_lens=(700,)), top_k=1)
@@ -355,6 +364,7 @@ def test_compress_one_half_only():
 
 
 @pytest.mark.parametrize("rows,hid,r", [
+    (100, 256, 256),     # CTA pairs: the second CTA's 128 rows all lie past the last row
     (1000, 1024, 256),   # 256-column tiles, two 128-row sub-tiles, ragged last row block
     (300, 512, 512),     # two latent column tiles
     (130, 256, 128),     # 128-column tiles, one sub-tile
