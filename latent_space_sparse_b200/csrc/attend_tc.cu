@@ -428,10 +428,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
     }
   } else if (W == 2 && warp == kMmaWarp) {
     // ======================= MMA issuer, two latent halves ===================
-    // Per tile: Pk_u half 0 -> reconstruction over half 0 -> Pk_u half 1 ->
-    // reconstruction over half 1 (accumulating) -> value MMA over the four
-    // 128-column chunks of the latent width.  Half 0 of the next tile's Pk_u
-    // is loaded while the epilogue works on this tile.  The whole warp runs
+    // Per tile: reconstruction over the latent half of Pk_u in the buffer ->
+    // the other half of Pk_u -> reconstruction over it (accumulating) -> value
+    // MMA over the four 128-column chunks of the latent width.  The next tile
+    // of the same unit starts with the half left in the buffer; a new unit's
+    // half 0 is loaded while the epilogue works on this tile.  The whole warp runs
     // the sequence (warp-uniform state and descriptors); one elected lane
     // issues each group of loads, MMAs and its commit.
     {
@@ -467,31 +468,58 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tmap_pk,
         return __all_sync(0xffffffffu, tc::mbar_wait(b, parity, P.flags));
       };
       bool ok = true;
-      if (n > 0) load_pk(cur.u, 0);
+      // the Pk buffer holds latent half pk_h of Pk_{pk_u} (pk_u < 0: nothing
+      // yet); a load into it is in flight while pk_pending
+      int pk_u = -1, pk_h = 0;
+      bool pk_pending = false;
+      auto fetch_pk = [&](int u, int hh) {
+        load_pk(u, hh);
+        pk_u = u;
+        pk_h = hh;
+        pk_pending = true;
+      };
+      auto have_pk = [&]() -> bool {
+        if (!pk_pending) return true;
+        if (!wait(bar(B_PK), pk_phase)) return false;
+        pk_phase ^= 1u;
+        pk_pending = false;
+        return true;
+      };
+      if (n > 0) fetch_pk(cur.u, 0);
       for (int i = 0; i < n && ok; ++i, cur.next()) {
         const int bi = i & 1;
         const uint32_t ph = ((uint32_t)i >> 1) & 1u;
         const uint32_t d_tmem = tmem_base + (uint32_t)bi * D;
-        ok = wait(bar(B_PK), pk_phase) && wait(bar(B_KFULL + 0), (uint32_t)i & 1u) &&
+        // The half of Pk_u already in the buffer goes first: consecutive tiles
+        // of a unit take the halves in alternate order (the sum over halves
+        // does not depend on it), so one load of Pk per tile, not two.
+        const int h0 = pk_u == cur.u ? pk_h : 0, h1 = 1 - h0;
+        if (pk_u != cur.u || pk_h != h0) {
+          // not reached with the prefetch below; kept for any other order
+          if (i > 0 && !(ok = wait(bar(B_KDONE + (bi ^ 1)), (((uint32_t)(i - 1)) >> 1) & 1u)))
+            break;
+          fetch_pk(cur.u, h0);
+        }
+        ok = have_pk() && wait(bar(B_KFULL + h0), (uint32_t)i & 1u) &&
              wait(bar(B_TKFREE + bi), ph ^ 1u);
         if (!ok) break;
-        pk_phase ^= 1u;
         tc::fence_after_sync();
-        kmma(tc::smem_u32(s_buf0), d_tmem, false, bar(B_PKDONE));
+        kmma(tc::smem_u32(h0 ? s_buf1 : s_buf0), d_tmem, false, bar(B_PKDONE));
         if (!(ok = wait(bar(B_PKDONE), pkd_phase))) break;
         pkd_phase ^= 1u;
-        load_pk(cur.u, 1);
-        ok = wait(bar(B_PK), pk_phase) && wait(bar(B_KFULL + 1), (uint32_t)i & 1u);
+        fetch_pk(cur.u, h1);
+        ok = have_pk() && wait(bar(B_KFULL + h1), (uint32_t)i & 1u);
         if (!ok) break;
-        pk_phase ^= 1u;
         tc::fence_after_sync();
-        kmma(tc::smem_u32(s_buf1), d_tmem, true, bar(B_KDONE + bi));
+        kmma(tc::smem_u32(h1 ? s_buf1 : s_buf0), d_tmem, true, bar(B_KDONE + bi));
         if (i + 1 < n) {
-          // half 0 of the next tile's Pk_u, once this reconstruction is done with Pk
-          if (!(ok = wait(bar(B_KDONE + bi), ph))) break;
           UnitTileCursor nx = cur;
           nx.next();
-          load_pk(nx.u, 0);
+          if (nx.u != cur.u) {
+            // half 0 of the next unit's Pk_u, once this reconstruction is done with Pk
+            if (!(ok = wait(bar(B_KDONE + bi), ph))) break;
+            fetch_pk(nx.u, 0);
+          }
         }
         // value MMA: acc^T[r x 2G] = Vc_tile^T . p.  The two buffers are adjacent,
         // so latent k-block j of the tile is at s_buf0 + j * 16 KiB and chunk ch
