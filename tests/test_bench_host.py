@@ -152,3 +152,23 @@ def test_timeline_summary_on_hand_made_stamps():
     assert s["wait_us"] == pytest.approx({"a": 1.2, "b": 0.5})
     assert s["span_us"] == pytest.approx({"a": 2.5, "b": 3.5})
     assert s["layer_step_us"] == pytest.approx(7.7)
+
+
+def test_peak_lookup_burst_sustained_and_fallback(tmp_path, monkeypatch):
+    """The roofline denominators: the measured file's burst and sustained bf16
+    figures and its copy bandwidth; the stated fallback figures when the file,
+    or one key of it, is absent."""
+    import json
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_peaks() == (6650.0, "fallback")
+    assert bench.measured_bf16_peak() == (1590.0, "fallback")
+    assert bench.measured_bf16_peak(sustained=True) == (1400.0, "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6500.5,
+                                                              "bf16_tflops": 1650.0}))
+    assert bench.measured_peaks() == (6500.5, "measured")
+    assert bench.measured_bf16_peak() == (1650.0, "measured")
+    assert bench.measured_bf16_peak(sustained=True) == (1400.0, "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6500.5,
+                                                              "bf16_tflops": 1650.0,
+                                                              "bf16_tflops_sustained": 1390.0}))
+    assert bench.measured_bf16_peak(sustained=True) == (1390.0, "measured")
