@@ -275,30 +275,36 @@ combine_kernel(const CombineParams P) {
   if (tid == 0) trace_stamp(P.trace, TRACE_END);
 }
 
-// Many units (a grid of the kernel above beyond two CTAs per SM, e.g. 16
-// sequences x 32 MHA heads): one warp per (sequence, unit, 16 output rows),
-// eight sequences per CTA sharing the CTA's 16 rows of Pv_u.  A warp merges
-// its unit's used slots in registers (lane j holds latent columns 2j + 64i,
-// +1 of every head), then projects: each lane forms its columns' share of
-// the 16 x G output dots, and a shuffle reduce-scatter leaves the sums of
-// row i on lanes 2i, 2i+1.  Same merge as above, slot by slot in slot order.
+// Low-latency merge: one warp per (sequence, query head, 16 output rows), eight
+// such heads per CTA, all of one unit and one slice so that they share the
+// CTA's 16 rows of Pv_u.  Everything that does not depend on the attention
+// kernel (the Pv rows, the used slots) is done before the dependency wait;
+// after it a warp runs alone, with no block barrier: it loads the rows of NB
+// of its head's used slots at once (lane j holds latent columns 2j + 64i,
+// +1), merges them in registers, then projects: each lane forms its columns'
+// share of the 16 output dots, and a shuffle reduce-scatter leaves the sum of
+// row i on lanes 2i, 2i+1.  Same merge as above, NB slots at a time in slot
+// order.  NB > 1 takes the slot loads' latency once for several slots (few
+// CTAs, each warp's chain is the kernel's time); NB = 1 keeps the registers,
+// and so the CTAs resident per SM, for grids of several CTAs per SM.
 constexpr int kSeqWarps = 8;
 __device__ __forceinline__ float2 pv2_f32(const __nv_bfloat16* p) {
   return __bfloat1622float2(*(const __nv_bfloat162*)p);
 }
 __device__ __forceinline__ float2 pv2_f32(const float* p) { return *(const float2*)p; }
-template <typename T, int G, int R64>  // R64 = r / 64
+template <typename T, int G, int R64, int NB>  // R64 = r / 64, NB slots a batch
 __global__ void __launch_bounds__(kSeqWarps * 32)
-combine_seq_kernel(const CombineParams P) {
+combine_head_kernel(const CombineParams P) {
   extern __shared__ __align__(16) uint8_t smem[];
   T* const pv_s = (T*)smem;  // [16][r]
   __shared__ int s_seg[kSeqWarps][kMaxSegs];
   const int n_slices = P.d / kRows;
   const int slice = blockIdx.x % n_slices;
   const int rest = blockIdx.x / n_slices;
-  const int u = rest % P.U, bg = rest / P.U;
+  const int u = rest % P.U, hgroup = rest / P.U;
   const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
-  const int b = bg * kSeqWarps + warp;
+  const int head = hgroup * kSeqWarps + warp;  // (sequence, head of the unit)
+  const int b = head / G, g = head % G;
   const int r = R64 * 64;
   if (tid == 0) trace_stamp(P.trace, TRACE_START);
   allow_dependent_launch();
@@ -310,80 +316,87 @@ combine_seq_kernel(const CombineParams P) {
     for (int e = tid; e < n16; e += kSeqWarps * 32) dst[e] = src[e];
   }
   const int nseg = b < P.B ? used_slots(P, b, u, s_seg[warp]) : 0;
+  __syncthreads();  // the Pv rows
   grid_dependency_wait();  // the partials come from the attention kernel
   if (tid == 0) trace_stamp(P.trace, TRACE_WAITED);
-  __syncthreads();  // the Pv rows
   if (b < P.B) {
     const int rowf = part_row(r);
-    float acc[G][2 * R64];
-    float M[G], L[G];
+    const float* part_h =
+        P.part + ((int64_t)b * P.Hq + (int64_t)u * G + g) * P.bh_stride * rowf;
+    float acc[2 * R64];
+    float M = -INFINITY, L = 0.f;
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      M[g] = -INFINITY;
-      L[g] = 0.f;
+    for (int j = 0; j < 2 * R64; ++j) acc[j] = 0.f;
+    for (int q0 = 0; q0 < nseg; q0 += NB) {
+      float m[NB], l[NB];
+      float2 v[NB][R64];
 #pragma unroll
-      for (int j = 0; j < 2 * R64; ++j) acc[g][j] = 0.f;
-    }
-    const float* part_u = P.part + ((int64_t)b * P.Hq + (int64_t)u * G) * P.bh_stride * rowf;
-    for (int q = 0; q < nseg; ++q) {
+      for (int q = 0; q < NB; ++q) {
+        m[q] = -INFINITY;
+        l[q] = 0.f;
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float* row = part_u + ((int64_t)g * P.bh_stride + s_seg[warp][q] * P.slot_stride) * rowf;
-        const float m = row[0], l = row[1];
-        float2 v[R64];
+        for (int i = 0; i < R64; ++i) v[q][i] = make_float2(0.f, 0.f);
+        if (q0 + q < nseg) {
+          const float* row = part_h + (int64_t)s_seg[warp][q0 + q] * P.slot_stride * rowf;
+          m[q] = row[0];
+          l[q] = row[1];
 #pragma unroll
-        for (int i = 0; i < R64; ++i) v[i] = *(const float2*)(row + kPartAcc + 2 * lane + 64 * i);
-        const float Mn = fmaxf(M[g], m);
-        const float sc = M[g] == -INFINITY ? 0.f : expf(M[g] - Mn);
-        const float w = m == -INFINITY ? 0.f : expf(m - Mn);
-        L[g] = L[g] * sc + w * l;
-        M[g] = Mn;
-#pragma unroll
-        for (int i = 0; i < R64; ++i) {
-          acc[g][2 * i] = fmaf(w, v[i].x, acc[g][2 * i] * sc);
-          acc[g][2 * i + 1] = fmaf(w, v[i].y, acc[g][2 * i + 1] * sc);
+          for (int i = 0; i < R64; ++i) v[q][i] = *(const float2*)(row + kPartAcc + 2 * lane + 64 * i);
         }
       }
-    }
-    // projection: o[g][i] = sum over this lane's columns of Pv row i . acc
-    float o[G][kRows];
+      float Mn = M;
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float inv = L[g] > 0.f ? 1.f / L[g] : 0.f;
+      for (int q = 0; q < NB; ++q) Mn = fmaxf(Mn, m[q]);
+      const float sc = M == -INFINITY ? 0.f : expf(M - Mn);
+      L *= sc;
 #pragma unroll
-      for (int i = 0; i < kRows; ++i) o[g][i] = 0.f;
+      for (int j = 0; j < 2 * R64; ++j) acc[j] *= sc;
 #pragma unroll
-      for (int c = 0; c < R64; ++c) {
-        const float a0 = acc[g][2 * c] * inv, a1 = acc[g][2 * c + 1] * inv;
+      for (int q = 0; q < NB; ++q) {
+        if (q0 + q >= nseg) break;  // the same for the whole warp
+        const float w = m[q] == -INFINITY ? 0.f : expf(m[q] - Mn);
+        L = fmaf(w, l[q], L);
 #pragma unroll
-        for (int i = 0; i < kRows; ++i) {
-          const float2 pv = pv2_f32(pv_s + (size_t)i * r + 2 * lane + 64 * c);
-          o[g][i] = fmaf(pv.x, a0, fmaf(pv.y, a1, o[g][i]));
+        for (int i = 0; i < R64; ++i) {
+          acc[2 * i] = fmaf(w, v[q][i].x, acc[2 * i]);
+          acc[2 * i + 1] = fmaf(w, v[q][i].y, acc[2 * i + 1]);
         }
+      }
+      M = Mn;
+    }
+    // projection: o[i] = sum over this lane's columns of Pv row i . acc / L
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    float o[kRows];
+#pragma unroll
+    for (int i = 0; i < kRows; ++i) o[i] = 0.f;
+#pragma unroll
+    for (int c = 0; c < R64; ++c) {
+      const float a0 = acc[2 * c] * inv, a1 = acc[2 * c + 1] * inv;
+#pragma unroll
+      for (int i = 0; i < kRows; ++i) {
+        const float2 pv = pv2_f32(pv_s + (size_t)i * r + 2 * lane + 64 * c);
+        o[i] = fmaf(pv.x, a0, fmaf(pv.y, a1, o[i]));
       }
     }
     // reduce-scatter over the 32 lanes: after the step with offset 16 >> s,
     // a lane keeps the rows whose bit (3 - s) matches its lane bit (4 - s)
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
+    for (int half = 8, off = 16; half >= 1; half >>= 1, off >>= 1) {
+      const bool upper = (lane & off) != 0;
 #pragma unroll
-      for (int half = 8, off = 16; half >= 1; half >>= 1, off >>= 1) {
-        const bool upper = (lane & off) != 0;
-#pragma unroll
-        for (int i = 0; i < half; ++i) {
-          const float send = upper ? o[g][i] : o[g][i + half];
-          const float keep = upper ? o[g][i + half] : o[g][i];
-          o[g][i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-        }
+      for (int i = 0; i < half; ++i) {
+        const float send = upper ? o[i] : o[i + half];
+        const float keep = upper ? o[i + half] : o[i];
+        o[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
       }
-      // lanes 2i, 2i+1 hold row i's sums over lanes of equal bit 0: add the pair
-      const float tot = o[g][0] + __shfl_xor_sync(0xffffffffu, o[g][0], 1);
-      const int i = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
-                    ((lane >> 1) & 1);
-      if ((lane & 1) == 0)
-        ((T*)P.out)[((int64_t)b * P.Hq + (int64_t)u * G + g) * P.d + slice * kRows + i] =
-            from_f32<T>(tot);
     }
+    // lanes 2i, 2i+1 hold row i's sums over lanes of equal bit 0: add the pair
+    const float tot = o[0] + __shfl_xor_sync(0xffffffffu, o[0], 1);
+    const int i = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
+                  ((lane >> 1) & 1);
+    if ((lane & 1) == 0)
+      ((T*)P.out)[((int64_t)b * P.Hq + (int64_t)u * G + g) * P.d + slice * kRows + i] =
+          from_f32<T>(tot);
   }
   if (tid == 0) trace_stamp(P.trace, TRACE_END);
 }
@@ -441,25 +454,29 @@ int num_sms_cb() {
 }
 
 template <typename T, int G, int R64>
-cudaError_t launch_seq(const CombineParams& P, const DecodePlan& p, cudaStream_t s) {
+cudaError_t launch_head(const CombineParams& P, const DecodePlan& p, cudaStream_t s) {
+  // one head a unit: the grid is several CTAs per SM (the rule below), one
+  // slot at a time; several heads: a few CTAs per SM at most, a batch of slots
+  constexpr int NB = G == 1 ? 1 : 32 / R64;
   static int done[kMaxDevices] = {};
   const size_t smem = (size_t)kRows * p.r * sizeof(T);
-  cudaError_t e = ensure_smem(combine_seq_kernel<T, G, R64>, smem, done);
+  cudaError_t e = ensure_smem(combine_head_kernel<T, G, R64, NB>, smem, done);
   if (e != cudaSuccess) return e;
-  const dim3 grid((unsigned)((p.d / kRows) * p.U * ((p.B + kSeqWarps - 1) / kSeqWarps)));
-  return launch_k(combine_seq_kernel<T, G, R64>, grid, dim3(kSeqWarps * 32), smem, s, true, P);
+  const int64_t groups = ((int64_t)p.B * G + kSeqWarps - 1) / kSeqWarps;
+  const dim3 grid((unsigned)((p.d / kRows) * p.U * groups));
+  return launch_k(combine_head_kernel<T, G, R64, NB>, grid, dim3(kSeqWarps * 32), smem, s, true,
+                  P);
 }
 
 template <typename T, int G>
 cudaError_t launch_tg(const CombineParams& P, const DecodePlan& p, cudaStream_t s) {
   static int done[kMaxDevices] = {};
-  // many units, one head per unit: a warp per (sequence, unit, slice)
-  if constexpr (G == 1) {
-    if (!P.part_out && P.fixed_slots == 0 &&
-        (int64_t)p.B * p.U * (p.d / kRows) > 2 * (int64_t)num_sms_cb()) {
-      if (p.r == 512) return launch_seq<T, 1, 8>(P, p, s);
-      if (p.r == 256) return launch_seq<T, 1, 4>(P, p, s);
-    }
+  // a warp per (sequence, head, slice): with several heads per unit always,
+  // with one head per unit when the grid above would exceed two CTAs per SM
+  if (!P.part_out && P.fixed_slots == 0 &&
+      (G > 1 || (int64_t)p.B * p.U * (p.d / kRows) > 2 * (int64_t)num_sms_cb())) {
+    if (p.r == 512) return launch_head<T, G, 8>(P, p, s);
+    if (p.r == 256) return launch_head<T, G, 4>(P, p, s);
   }
   size_t smem = combine_smem(p, P.rowbuf);
   // A grid of at most two CTAs per SM asks for enough shared memory that no

@@ -9,7 +9,7 @@
 // loads a contiguous slice of the unit's scores into shared memory once, as
 // 32-bit keys whose unsigned order is the float order; the unit's score range
 // [min, max] comes from the scoring kernel.  Each CTA histograms its slice
-// into 2048 bins of equal width over that range (the bin is a monotone
+// into 1024 bins of equal width over that range (the bin is a monotone
 // function of the score, and scores spread over many bins, so the
 // shared-memory atomics barely contend) and adds it into every CTA's copy of
 // the cluster histogram through distributed shared memory; every CTA then
@@ -47,7 +47,7 @@ __device__ __forceinline__ float key_float(uint32_t key) {
 
 constexpr int kBins = 2048;  // 11-bit digits of the radix fallback
 constexpr int kDigit = 11;
-constexpr int kLinBins = 2048;  // bins of the linear pass
+constexpr int kLinBins = 1024;  // bins of the linear pass
 constexpr int kCand = 1024;    // most candidates the boundary bin may hold for the fast path
 
 // Bin of a key in the linear partition of [fmin, fmax] into kLinBins bins: a

@@ -162,16 +162,21 @@ def test_wide_rank_512_mha_many_tiles():
     check(w, synth.decode_inputs(w, seq_lens=(4096,)), top_k=1000)
 
 
-@pytest.mark.parametrize("batch,heads,rank,lens", [
-    (11, 32, 512, (300, 517, 900, 128, 640, 777, 256, 1000, 333, 129, 450)),  # ragged, B % 8 != 0
-    (9, 16, 256, (500,) * 9),                                                # equal lengths, r = 256
+@pytest.mark.parametrize("batch,heads,kv_heads,rank,top_k,lens", [
+    (11, 32, 32, 512, 256, (300, 517, 900, 128, 640, 777, 256, 1000, 333, 129, 450)),  # ragged
+    (9, 16, 16, 256, 256, (500,) * 9),               # equal lengths, r = 256
+    (3, 16, 2, 256, 2048, (2100, 3000, 2500)),       # 8 heads a unit: three full CTAs of heads
+    (5, 8, 4, 512, 256, (900, 1200, 64, 2000, 517)),  # 2 heads a unit, r = 512: a CTA part idle
 ])
-def test_merge_one_warp_per_sequence(batch, heads, rank, lens):
-    # many single-head units: the merge runs one warp per (sequence, unit, 16
-    # output rows), eight sequences per CTA (the last CTA's spare warps idle)
-    w = W.Workload(name="mha_many_units", batch=batch, n_q_heads=heads, n_kv_heads=heads,
-                   head_dim=128, rank=rank, top_k=256, seq_lens=lens, dtype="bf16",
+def test_merge_one_warp_per_head(batch, heads, kv_heads, rank, top_k, lens):
+    # the merge runs one warp per (sequence, query head, 16 output rows),
+    # eight heads of one unit per CTA (the last CTA's spare warps idle); the
+    # attention kernel leaves the merge to it (too many tiles a unit for the
+    # in-kernel merge, or r > 256)
+    w = W.Workload(name="merge_per_head", batch=batch, n_q_heads=heads, n_kv_heads=kv_heads,
+                   head_dim=128, rank=rank, top_k=top_k, seq_lens=lens, dtype="bf16",
                    rope_base=10000.0, low_rank=32, seed=93 + batch)
+    assert launches(w) == len(salsc.DECODE_KERNELS)
     check(w, synth.decode_inputs(w))
 
 
