@@ -44,12 +44,18 @@ UNIT = "us/layer-step"
 
 # DRAM bytes (read + write) of one launch, from an ncu capture of the named
 # kernel on the named workload (the summary under profiles/ gives the command).
-# An entry is removed whenever its kernel changes after the capture.
+# The capture keeps the caches as the bench's own kernel order leaves them
+# (--cache-control none), as in the timed step. An entry is removed whenever
+# its kernel changes after the capture.
 PROFILED_TRAFFIC: dict[tuple[str, str], float] = {
-    # dram__bytes.sum.per_second x gpu__time_duration.sum of two captured
-    # launches: 54.96 and 55.04 MB
-    ("mistral_7b_gqa32x8_d128_r256_n32768_b4_k2048_bf16", "attend"): 55.00e6,
+    # dram__bytes_read.sum + dram__bytes_write.sum of two captured launches:
+    # 33.30 and 30.48 MB (the kept Kc rows come from L2, where the scoring
+    # kernel has just streamed them; with flushed caches the launch reads and
+    # writes 55.0 MB)
+    ("mistral_7b_gqa32x8_d128_r256_n32768_b4_k2048_bf16", "attend"): 31.89e6,
 }
+TRAFFIC_HOW = ("ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, mean of two launches "
+               "in the bench's own kernel order, --cache-control none")
 DEFAULT_WORKLOAD = workloads.MISTRAL_32K_B4.name
 THROTTLE_BITS = {
     0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -651,6 +657,7 @@ def main():
     ach = kbytes[name] / (per_kernel_us[dominant] * 1e-6) / 1e9
     roofline = {"kernel": name, "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
                 "frac": ach / peak, "traffic": PROFILED_TRAFFIC.get((w.name, name)),
+                "traffic_how": TRAFFIC_HOW if (w.name, name) in PROFILED_TRAFFIC else None,
                 "peak_kind": peak_kind, "algorithmic_bytes_per_launch": kbytes[name],
                 "time": "per_kernel_us (event-separated: includes the kernel's launch latency)"}
 
