@@ -11,11 +11,15 @@
 // the value projection is applied once, after the weighted sum of latent
 // rows, which is exact by associativity).
 //
-// CTA (b, u, slice) produces output rows slice*16 .. slice*16+15 of the G
-// heads of unit u.  Its loads are whole-row bulk copies into shared memory,
-// so that they are in flight together while the code stays short (the
-// kernel runs once per SM and layer-step; every instruction it executes once
-// is a cold instruction fetch): the 32 rows of Pv_u are copied before the
+// Two kernels compute it.  combine_head_kernel (several query heads per unit,
+// or a grid of several CTAs per SM): one warp per (sequence, head, 16 output
+// rows), merging in registers with no block barrier after the dependency
+// wait.  combine_kernel (otherwise, and for the shard merge below): CTA
+// (b, u, slice) produces output rows slice*16 .. slice*16+15 of the G heads
+// of unit u.  Its loads are whole-row bulk copies into shared memory, so that
+// they are in flight together while the code stays short (the kernel runs
+// once per SM and layer-step; every instruction it executes once is a cold
+// instruction fetch).  In both, the 16 rows of Pv_u are loaded before the
 // dependency wait (Pv is a weight, not an output of the attention kernel),
 // the used partial rows after it.  Used slots: with the tensor-core
 // attention, a slot holds a partial when a CTA's contiguous range of tiles
@@ -23,10 +27,11 @@
 // partition; with the CUDA-core attention every slot of the unit is used.
 // The sums run over slots in slot order, so the result is deterministic.
 //
-// Two more uses for token-sharded decode: with part_out set, the kernel stops
-// after the merge and writes the merged (M, L, acc) of every head as one
-// partial row (one CTA per unit, no projection); with the row strides set to
-// (1, B*Hq), it merges one such row per shard (every slot used) and projects.
+// Two more uses for token-sharded decode, both by combine_kernel: with
+// part_out set, it stops after the merge and writes the merged (M, L, acc) of
+// every head as one partial row (one CTA per unit, no projection); with the
+// row strides set to (1, B*Hq), it merges one such row per shard (every slot
+// used) and projects.
 #include "tc.cuh"
 
 namespace salsc {
