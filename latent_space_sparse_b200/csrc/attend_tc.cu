@@ -129,7 +129,7 @@ struct UnitTileCursor {
 // the offsets of one sequence (32 at a time), and a warp scan of the tiles
 // per sequence locates tile t_begin with one round trip of loads.  Merging
 // CTAs (cluster > 0) take their rank's share of unit m_unit's tiles; the
-// others take tiles [c*T/g, (c+1)*T/g).  Lane 0 writes (t_begin, n, b, u,
+// others take tiles [share_begin(c), share_begin(c + 1)).  Lane 0 writes (t_begin, n, b, u,
 // slot) to st[0..4] and (off, nb) of sequence b to st64[0..1]; b = B when the
 // range is empty.
 __device__ __forceinline__ void find_first_tile(const int64_t* so, int B, int U, int k,
@@ -147,8 +147,8 @@ __device__ __forceinline__ void find_first_tile(const int64_t* so, int B, int U,
       t_begin = m_unit * tu + l0;
       n = h0 - l0;
     } else {
-      t_begin = (int)((int64_t)blockIdx.x * n_tiles / gridDim.x);
-      n = (int)((int64_t)(blockIdx.x + 1) * n_tiles / gridDim.x) - t_begin;
+      t_begin = (int)share_begin(blockIdx.x, n_tiles, gridDim.x);
+      n = (int)share_begin(blockIdx.x + 1, n_tiles, gridDim.x) - t_begin;
     }
     fb = n > 0 && tu > 0 ? t_begin / (U * tu) : B;
     if (fb < B) {
@@ -171,8 +171,8 @@ __device__ __forceinline__ void find_first_tile(const int64_t* so, int B, int U,
   if (cluster > 0) {
     mb = (int)(blockIdx.x / (unsigned)cluster) / U;  // the unit's sequence
   } else {
-    t_begin = (int)((int64_t)blockIdx.x * n_tiles / gridDim.x);
-    n = (int)((int64_t)(blockIdx.x + 1) * n_tiles / gridDim.x) - t_begin;
+    t_begin = (int)share_begin(blockIdx.x, n_tiles, gridDim.x);
+    n = (int)share_begin(blockIdx.x + 1, n_tiles, gridDim.x) - t_begin;
   }
   int64_t before = 0;  // tiles of the sequences before this group of 32
   int fb = B, fu = 0, fslot = 0;

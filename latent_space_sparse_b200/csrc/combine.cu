@@ -91,10 +91,9 @@ __device__ __forceinline__ int used_slots(const CombineParams& P, int b, int u, 
     const int sl = s0 + lane;
     bool used = sl < tb;
     if (used && sl > 0 && P.seg_grid > 0) {
-      // tile t starts a CTA's range [c*T/grid, (c+1)*T/grid)
+      // tile t starts the range of the CTA that holds it
       const int64_t t = unit_tile0 + sl, T = P.seg_tiles, gc = P.seg_grid;
-      const int64_t c = (t * gc + T - 1) / T;  // first CTA at or after t
-      used = c < gc && c * T / gc == t;
+      used = share_begin(share_of_tile(t, T, gc), T, gc) == t;
     }
     const uint32_t mk = __ballot_sync(0xffffffffu, used);
     if (used) seg[cnt + __popc(mk & ((1u << lane) - 1u))] = sl;
@@ -423,12 +422,12 @@ int max_used_slots(const DecodePlan& p, const int64_t* seq_off_host, int seg_gri
     const int64_t kb = nb < p.k ? nb : p.k;
     const int64_t tb = (kb + p.chunk - 1) / p.chunk;
     for (int u = 0; u < p.U; ++u, tile += tb) {
-      // CTA c covers tiles [c*T/gc, (c+1)*T/gc) of the T tiles over gc CTAs:
-      // the CTA of tile t is ((t+1)*gc - 1) / T, and the unit's tiles meet at
-      // most the CTAs from its first tile's to its last tile's
+      // the unit's tiles meet the CTAs from its first tile's to its last
+      // tile's (share_of_tile: the contiguous partition of the T tiles over
+      // gc CTAs)
       const int64_t gc = seg_grid, T = p.att_tiles, t0 = tile;
       if (tb == 0) continue;
-      int64_t n = ((t0 + tb) * gc - 1) / T - ((t0 + 1) * gc - 1) / T + 1;
+      int64_t n = share_of_tile(t0 + tb - 1, T, gc) - share_of_tile(t0, T, gc) + 1;
       if (n > tb) n = tb;  // a segment holds one tile at least
       if (n > most) most = (int)n;
     }

@@ -28,6 +28,19 @@ constexpr int kMaxRank = 512;
 // starts on a 16-byte boundary (rows are copied whole with cp.async.bulk).
 constexpr int kPartAcc = 4;
 __host__ __device__ constexpr int part_row(int r) { return r + kPartAcc; }
+
+// Tile partition of the tensor-core attention: T tiles over g CTAs in
+// contiguous ranges, CTA c from share_begin(c) to share_begin(c + 1).  The
+// first T % g CTAs take one tile more: CTAs are dispatched in index order,
+// so the longer ranges go to the CTAs that start first.
+__host__ __device__ constexpr int64_t share_begin(int64_t c, int64_t T, int64_t g) {
+  return c * (T / g) + (c < T % g ? c : T % g);
+}
+// The CTA whose range holds tile t (0 <= t < T).
+__host__ __device__ constexpr int64_t share_of_tile(int64_t t, int64_t T, int64_t g) {
+  return t < (T % g) * (T / g + 1) ? t / (T / g + 1)
+                                   : T % g + (t - (T % g) * (T / g + 1)) / (T / g);
+}
 constexpr int kMaxHeadDim = 128;
 constexpr int kMaxUnits = 256;  // KV heads per layer
 constexpr size_t kWsAlign = 256;
