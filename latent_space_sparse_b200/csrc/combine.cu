@@ -299,8 +299,8 @@ __device__ __forceinline__ float2 pv2_f32(const float* p) { return *(const float
 template <typename T, int G, int R64, int NB>  // R64 = r / 64, NB slots a batch
 __global__ void __launch_bounds__(kSeqWarps * 32)
 combine_head_kernel(const CombineParams P) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  T* const pv_s = (T*)smem;  // [16][r]
+  extern __shared__ __align__(16) uint8_t smem_pv[];
+  T* const pv_s = (T*)smem_pv;  // [16][r]
   __shared__ int s_seg[kSeqWarps][kMaxSegs];
   const int n_slices = P.d / kRows;
   const int slice = blockIdx.x % n_slices;
